@@ -1,0 +1,126 @@
+/*
+ * flint_oracle.h -- plain fp64 CPU oracle of one Flint MoE layer's decode step.
+ *
+ * TEST INFRASTRUCTURE. Only tests/, __graft_entry__.smoke() and bench.py's
+ * cpu_baseline / reference leg may load or call this library. The product path
+ * (libflint_moe.so and its Python binding) never links, imports or runs it, and
+ * the two share no code, header, table or constant generator.
+ *
+ * What it computes, and where the definition comes from:
+ *  - Mixture of experts with 256 routed experts, 6 picked per token, plus one
+ *    always-on shared expert: "Recursive Flint: 40B Local Coding Model,
+ *    Benchmarks", architecture table (Experts row); "Run the Flint coding model
+ *    on a CPU VPS", section "What Flint is, from the model card".
+ *  - Weight-only NVFP4 (W4A16) experts: "[Model] Add Flint (RecursiveSI/flint)",
+ *    section "What happened" (NVFP4 checkpoint served weight-only as W4A16);
+ *    NVFP4 is NVIDIA's 4-bit floating-point format ("Run the Flint coding model
+ *    on a CPU VPS", section "Which Flint tag to pull on a CPU VPS").
+ *  - The pages fix no bit layout, gating, FFN type or shapes. The layer
+ *    contract supplies them: E2M1 values, one E4M3 scale per 16 elements along
+ *    K, one FP32 tensor scale; softmax over all routed logits, top-k with ties
+ *    to the lower index, gates renormalised to sum 1, shared expert weight 1;
+ *    SwiGLU experts (gate/up d->I, down I->d, no biases).
+ *  - E2M1 / E4M3 bit meanings follow the public OCP Microscaling (MX) v1.0
+ *    element formats (FP4 E2M1; FP8 E4M3 "fn": no infinities, S.1111.111 NaN).
+ *
+ * Precision: every arithmetic step of the forward pass runs in fp64; weights
+ * are decoded exactly (e2m1 * e4m3 * fp32 tensor scale fits in 53 bits).
+ * The quantiser runs in IEEE fp32 round-to-nearest (the recipe fixes fp32),
+ * built with -ffp-contract=off so no multiply-add is fused.
+ */
+#ifndef FLINT_ORACLE_H
+#define FLINT_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* One weight matrix in the oracle's plain ("natural") layout.
+ *   kind 0 (NVFP4): codes [rows][cols/2], element 2j in the low nibble of byte j,
+ *                   scales [rows][cols/16] E4M3 bytes, block b = elements 16b..16b+15,
+ *                   tensor_scale = the fp32 per-tensor scale.
+ *   kind 1 (BF16):  bf16 [rows][cols] bit patterns.
+ * Unused experts may be left with NULL pointers. */
+typedef struct oracle_matrix {
+  int32_t kind;
+  int32_t rows;
+  int32_t cols;
+  float tensor_scale;
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const uint16_t* bf16;
+} oracle_matrix;
+
+/* ---- element codecs (OCP MX v1.0 element formats) ---- */
+double oracle_e2m1_decode(uint8_t code);
+double oracle_e4m3_decode(uint8_t code);
+/* Round-to-nearest-even, saturating to +-6; the sign of v is kept (so -0 -> 0x8). */
+uint8_t oracle_e2m1_encode(float v);
+/* Round-to-nearest-even, saturating to +-448; the sign of v is kept. */
+uint8_t oracle_e4m3_encode(float v);
+/* Round-to-nearest-even fp64 -> bf16 bit pattern (finite inputs). */
+uint16_t oracle_bf16_from_double(double v);
+double oracle_bf16_to_double(uint16_t bits);
+
+/* ---- NVFP4 quantiser (the recipe, fp32) ----
+ * s_t = amax/2688 (1 if amax == 0); per block sb = E4M3((amax_b/6)/s_t);
+ * q = E2M1(w / (dec(sb)*s_t)), and q = 0 for every element of a block whose
+ * scale decodes to 0. Writes natural-layout planes. Returns 0, or -1 when the
+ * shape is not a multiple of 16 along cols or w holds a non-finite value. */
+int oracle_quantize_nvfp4(const float* w, int32_t rows, int32_t cols,
+                          uint8_t* codes, uint8_t* scales, float* tensor_scale);
+
+/* Decode one matrix to fp64 [rows][cols] (NVFP4: e2m1*e4m3*s_t; BF16: exact). */
+int oracle_decode_matrix(const oracle_matrix* m, double* out);
+
+/* ---- the product's packed HBM layout, restated from its definition ----
+ * Expert e (routed 0..E-1, then the n_shared shared experts) owns a contiguous
+ * region in each array. Codes: I units of [gate row u | up row u] (d/2 bytes
+ * each), then d down rows of I/2 bytes. Scales: the same rows in the same
+ * order, d/16 resp. I/16 bytes per row. Tensor scales: [expert][gate,up,down].
+ * mats holds (E+S)*3 natural-layout NVFP4 matrices: gate [I][d], up [I][d],
+ * down [d][I] per expert. */
+int oracle_pack_layout(const oracle_matrix* mats, int32_t n_experts_total,
+                       int32_t d, int32_t inter, uint8_t* packed_codes,
+                       uint8_t* packed_scales, float* tensor_scales);
+/* The same row order for bf16 weights: [gate row u | up row u] (d bf16 each),
+ * then d down rows of I bf16. */
+int oracle_pack_layout_bf16(const oracle_matrix* mats, int32_t n_experts_total,
+                            int32_t d, int32_t inter, uint16_t* packed);
+
+/* ---- routing ---- */
+/* logits[t][e] = sum_j x[t][j] * W_r[e][j] in fp64; x [T][d], W_r [E][d] bf16. */
+int oracle_router_logits(const uint16_t* x, int32_t T, const uint16_t* wr,
+                         int32_t d, int32_t E, double* logits);
+/* Per token: softmax over all E logits; the k experts with the largest logit
+ * (ties to the lower index); gates = their probabilities renormalised to 1.
+ * gap[t] = p_(k) - p_(k+1) of the full softmax (k-th minus (k+1)-th largest),
+ * or +inf when k == E. */
+int oracle_topk(const double* logits, int32_t T, int32_t E, int32_t k,
+                int32_t* ids, double* gates, double* gap);
+
+/* ---- experts ---- */
+/* Dense SwiGLU FFN of one expert: y = W_d (silu(W_g x) * (W_u x)).
+ * mats = {gate [I][d], up [I][d], down [d][I]}. */
+int oracle_expert_ffn(const oracle_matrix* mats, int32_t d, int32_t inter,
+                      const double* x, double* y);
+
+/* Whole layer. mats: (E+S)*3 matrices (unused experts may be NULL-pointered).
+ * out = sum_j gate_j * FFN_{id_j}(x) + sum_s FFN_{E+s}(x) (+ residual), fp64.
+ * ids_override (nullable) forces the routed ids (gates then come from those
+ * experts' probabilities, renormalised). ids/gates/gap/logits outputs nullable.
+ * n_threads >= 1 spreads the independent (token, expert) FFNs over threads;
+ * the arithmetic and its order do not depend on it. */
+int oracle_moe_forward(int32_t T, int32_t d, int32_t inter, int32_t E, int32_t k,
+                       int32_t S, const uint16_t* x, const uint16_t* wr,
+                       const oracle_matrix* mats, const uint16_t* residual,
+                       const int32_t* ids_override, int32_t n_threads,
+                       int32_t* ids_out, double* gates_out, double* gap_out,
+                       double* logits_out, double* out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
