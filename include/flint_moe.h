@@ -1,0 +1,227 @@
+/*
+ * flint_moe.h -- C ABI of libflint_moe.so: one Flint MoE layer's decode step on
+ * B200 (sm_100a), with NVFP4 weight-only (W4A16) experts.
+ *
+ * What the layer computes (sources, by page title and section):
+ *  - Routing: every MoE layer has 256 routed experts, picks 6 per token, and
+ *    adds one always-on shared expert ("Recursive Flint: 40B Local Coding
+ *    Model, Benchmarks", architecture table, row "Experts"; "Run the Flint
+ *    coding model on a CPU VPS", section "What Flint is, from the model card").
+ *  - A fused top-k router and expert-indexed GEMVs for small-batch decode, and a
+ *    grouped-GEMM path for larger batches ("[Model] Add Flint
+ *    (RecursiveSI/flint)", section "What happened", third paragraph).
+ *  - Weight-only NVFP4 serving, W4A16 ("[Model] Add Flint (RecursiveSI/flint)",
+ *    section "What happened", first paragraph).
+ *  - The pages fix no gating function, FFN type, shapes or bit layout; the layer
+ *    contract this library implements fixes them:
+ *      logits = x . W_r; softmax over the E logits; the top_k largest (ties to
+ *      the lower expert index); gates = their probabilities renormalised to 1;
+ *      each selected expert and each shared expert (weight 1) is a SwiGLU FFN
+ *        FFN(x) = W_down (silu(W_gate x) * (W_up x)),  silu(g) = g / (1 + e^-g);
+ *      out = sum_j gate_j FFN_{id_j}(x) + sum_s FFN_shared_s(x) (+ residual).
+ *    NVFP4 weights: E2M1 codes, one E4M3 scale per 16 consecutive elements
+ *    along K, one FP32 scale per (expert, matrix):
+ *        w = e2m1(q) * e4m3(sb) * s_t.
+ *
+ * Conventions for every entry point:
+ *  - Returns flint_status (0 = FLINT_OK). Nothing throws across the ABI.
+ *    flint_last_error() gives a message for the calling thread's last failure.
+ *  - Host-side validation happens before any launch; on a validation error no
+ *    work is enqueued.
+ *  - Device pointers are cudaMalloc'd (or equivalent) memory on the current
+ *    device, owned by the caller; the library never allocates or frees device
+ *    memory and never synchronises, except flint_moe_get_status (which reads
+ *    the device status word) and flint_debug_* helpers.
+ *  - All work is enqueued on `stream` (a cudaStream_t passed as void*; NULL =
+ *    the legacy default stream).
+ *  - bf16 tensors are raw 16-bit patterns (uint16_t); 16-byte alignment is
+ *    required for every device pointer (FLINT_ERR_MISALIGNED otherwise).
+ *
+ * Packed HBM layout of the expert weights (flint_pack_nvfp4 writes it):
+ *  Experts are stored expert-major: routed experts 0..E-1, then the shared
+ *  expert(s). Within an expert, the gate and up projections are row-interleaved
+ *  ("units"): unit u = [gate row u | up row u], u = 0..I-1, followed by the d
+ *  rows of the down projection.
+ *    packed (codes):  per expert 3*I*d/2 bytes. Unit u at byte u*d: gate row u
+ *                     (d/2 bytes) then up row u (d/2 bytes). Down row n at byte
+ *                     I*d + n*I/2. Within a row, byte j holds element 2j in its
+ *                     low nibble and element 2j+1 in its high nibble.
+ *    block_scales:    per expert 3*I*d/16 bytes, same rows in the same order:
+ *                     unit u at byte u*d/8 (gate row's d/16 scales, then up
+ *                     row's); down row n at byte I*d/8 + n*I/16. Scale byte b of
+ *                     a row covers elements 16b..16b+15.
+ *    tensor_scales:   float [E+S][3] = {gate, up, down} per expert.
+ *  So every row is a whole number of 16-byte vectors (d, I multiples of 32),
+ *  and any run of consecutive units or down rows is one contiguous span in
+ *  each of the two arrays.
+ *  BF16 weights (wdtype FLINT_W_BF16) use the same row order with bf16
+ *  elements in `packed` (per expert 3*I*d*2 bytes); block_scales and
+ *  tensor_scales are then ignored (NULL allowed).
+ *
+ * Supported shapes: d one of {512, 1024, 2048, 4096}; inter one of
+ * {128, 256, 512, 1024}; 1 <= n_experts <= 512; 1 <= top_k <= 8, top_k <=
+ * n_experts; n_shared 0 or 1. Others return FLINT_ERR_UNSUPPORTED_SHAPE.
+ */
+#ifndef FLINT_MOE_H
+#define FLINT_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum flint_status {
+  FLINT_OK = 0,
+  FLINT_ERR_INVALID_ARG = -1,       /* null pointer, negative size, bad enum */
+  FLINT_ERR_UNSUPPORTED_SHAPE = -2, /* shape outside the supported set */
+  FLINT_ERR_MISALIGNED = -3,        /* a device pointer not 16-byte aligned */
+  FLINT_ERR_WORKSPACE = -4,         /* workspace NULL or smaller than required */
+  FLINT_ERR_CUDA = -5,              /* a CUDA runtime call failed (message kept) */
+  FLINT_ERR_DEVICE_CHECK = -6,      /* a kernel recorded a failed check */
+  FLINT_ERR_TIMEOUT = -7            /* a bounded device-side wait ran out */
+} flint_status;
+
+typedef enum flint_wdtype { FLINT_W_NVFP4 = 0, FLINT_W_BF16 = 1 } flint_wdtype;
+
+typedef struct flint_moe_shape {
+  int32_t d;         /* hidden size */
+  int32_t inter;     /* expert intermediate width I */
+  int32_t n_experts; /* routed experts E */
+  int32_t top_k;     /* experts selected per token */
+  int32_t n_shared;  /* always-on shared experts (0 or 1), gate weight 1 */
+  int32_t wdtype;    /* flint_wdtype of the expert weights */
+} flint_moe_shape;
+
+typedef struct flint_moe_weights {
+  const void* packed;          /* device; NVFP4 codes or bf16 weights, layout above */
+  const uint8_t* block_scales; /* device; E4M3 block scales (NVFP4 only) */
+  const float* tensor_scales;  /* device; float [E+S][3] (NVFP4 only) */
+} flint_moe_weights;
+
+/* Device-side check codes recorded in the workspace status word. */
+enum {
+  FLINT_DEVCHECK_EXPERT_ID = 1,   /* an expert id outside [0, E) reached a kernel */
+  FLINT_DEVCHECK_NONFINITE = 2,   /* a non-finite weight reached the packer */
+  FLINT_DEVCHECK_WAIT = 4,        /* a bounded wait gave up (FLINT_ERR_TIMEOUT) */
+  FLINT_DEVCHECK_MMA = 8          /* the tensor-core path rejected a tile */
+};
+
+typedef enum flint_path {
+  FLINT_PATH_AUTO = 0, /* GEMV kernels below 32 tokens, tensor-core path from 32 */
+  FLINT_PATH_GEMV = 1, /* CUDA-core dequant-GEMV kernels at any token count */
+  FLINT_PATH_MMA = 2   /* TMA-staged dequant-to-smem + tcgen05 MMA at any count */
+} flint_path;
+
+typedef struct flint_moe_options {
+  int32_t path;          /* flint_path */
+  int32_t use_pdl;       /* 1 (default when options == NULL): chain the layer's
+                            kernels with programmatic dependent launch */
+  int32_t* topk_ids;     /* optional device int32 [T][top_k]: routed ids written here */
+  float* topk_weights;   /* optional device float [T][top_k]: their gates */
+  int32_t input_rmsnorm; /* 1: each token's x is divided by its RMS, sqrt(mean(x^2) + 1e-6)
+                            (no learned weight), before the router and the experts;
+                            the residual is added unnormalised. 0 (default): no norm */
+  void* profile_events;  /* optional cudaEvent_t[2], recorded on `stream` just before
+                            and just after the layer's gate/up kernel (the one that
+                            streams most of the weights); the record between kernels
+                            serialises them, so use it for per-kernel timing only */
+} flint_moe_options;
+
+/* Bytes of the packed codes / block scales / tensor scales for a shape. Return 0
+ * for an unsupported shape. For FLINT_W_BF16 the codes figure is the bf16 size
+ * and the other two are 0. */
+size_t flint_packed_bytes(const flint_moe_shape* shape);
+size_t flint_block_scale_bytes(const flint_moe_shape* shape);
+size_t flint_tensor_scale_bytes(const flint_moe_shape* shape);
+
+/* flint_pack_nvfp4 -- quantise and lay out all experts' weights.
+ *  w: device, [E+S][3][I*d] fp32 (w_is_bf16 = 0) or bf16 bits (w_is_bf16 = 1):
+ *     matrix 0 = gate [I][d], 1 = up [I][d], 2 = down [d][I], row-major.
+ *  Writes packed / block_scales / tensor_scales in the layout above, following
+ *  the recipe: s_t = amax/2688 (1 if amax = 0); per block of 16 along K
+ *  sb = E4M3_rne_satfinite((amax_b/6)/s_t); q = E2M1_rne_satfinite(w/(e4m3(sb)*s_t)),
+ *  q = 0 when e4m3(sb) = 0; all fp32 steps round to nearest, no fused
+ *  multiply-add. A non-finite weight sets FLINT_DEVCHECK_NONFINITE in the
+ *  status word of `workspace` (needs flint_moe_workspace_bytes(shape, 1) bytes)
+ *  and its tensor is left unspecified. shape->wdtype must be FLINT_W_NVFP4. */
+int flint_pack_nvfp4(const void* w, int32_t w_is_bf16, const flint_moe_shape* shape,
+                     void* packed, uint8_t* block_scales, float* tensor_scales,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/* flint_pack_bf16 -- lay out bf16 weights ([E+S][3][I*d] bf16 bits, device) in
+ * the same expert-major row order, for shape->wdtype == FLINT_W_BF16. */
+int flint_pack_bf16(const uint16_t* w, const flint_moe_shape* shape, uint16_t* packed,
+                    void* stream);
+
+/* Workspace bytes for calls of up to max_tokens tokens. The workspace holds the
+ * status word, router logits, routing, grouping and the FFN intermediates; it
+ * must not be shared by calls that may overlap on the GPU. */
+size_t flint_moe_workspace_bytes(const flint_moe_shape* shape, int32_t max_tokens);
+
+/* Clears the workspace's status word (its first 256 bytes). Call once after
+ * allocating a workspace, before its first use; kernels only ever set bits in
+ * it, and flint_moe_get_status reads and clears it. */
+int flint_moe_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/* flint_moe_route -- the router alone.
+ *  x: device bf16 [T][d]; router_w: device bf16 [E][d] (W_r transposed, row e
+ *  is expert e); topk_ids: device int32 [T][top_k] (descending logit, ties to
+ *  the lower index); topk_weights: device float [T][top_k], summing to 1 per
+ *  token. T = 0 is a no-op. */
+int flint_moe_route(const uint16_t* x, int32_t T, const uint16_t* router_w,
+                    const flint_moe_shape* shape, int32_t* topk_ids, float* topk_weights,
+                    void* workspace, size_t ws_bytes, void* stream);
+
+/* flint_moe_forward -- the whole layer: route, group tokens by expert, run the
+ * selected and shared experts' SwiGLU FFNs from the packed weights, combine.
+ *  x: device bf16 [T][d]; residual: device bf16 [T][d] or NULL (added to the
+ *  combined output before rounding); out: device bf16 [T][d], round to nearest
+ *  even. out may alias residual but not x. T = 0 is a no-op. */
+int flint_moe_forward(const uint16_t* x, int32_t T, const uint16_t* router_w,
+                      const flint_moe_weights* weights, const flint_moe_shape* shape,
+                      const uint16_t* residual, uint16_t* out, void* workspace,
+                      size_t ws_bytes, void* stream);
+
+/* As flint_moe_forward, with options (path choice, PDL, routing outputs).
+ * options == NULL behaves as flint_moe_forward. */
+int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
+                         const flint_moe_weights* weights, const flint_moe_shape* shape,
+                         const uint16_t* residual, uint16_t* out, void* workspace,
+                         size_t ws_bytes, const flint_moe_options* options, void* stream);
+
+/* Synchronises `stream`, reads the workspace status word into *device_flags
+ * (FLINT_DEVCHECK_* bits, may be NULL) and clears it. Returns FLINT_OK, or
+ * FLINT_ERR_TIMEOUT / FLINT_ERR_DEVICE_CHECK when a flag was set. */
+int flint_moe_get_status(void* workspace, int32_t* device_flags, void* stream);
+
+/* Message of the calling thread's last failed call ("" if none). */
+const char* flint_last_error(void);
+
+/* Debug helper: the exact products e2m1(q) * e4m3(sb) of consecutive rows of
+ * one expert's weights, decoded by the same device routines the FFN kernels
+ * use. matrix 0: `rows` gate/up units from unit row0, written as fp32
+ * [2*rows][d] (gate row, then up row, per unit); matrix 1: `rows` down rows
+ * from row0, fp32 [rows][I]. out is device memory. tensor_scale_out (host,
+ * nullable) receives {gate, up} scales for matrix 0, the down scale for 1.
+ * Synchronises the stream. */
+int flint_debug_dequant(const flint_moe_weights* weights, const flint_moe_shape* shape,
+                        int32_t expert, int32_t matrix, int32_t row0, int32_t rows,
+                        float* out, float* tensor_scale_out, void* stream);
+
+/* Failure-detection hook: launches one kernel whose bounded wait on a
+ * shared-memory barrier that nothing completes gives up after `cycles` SM clock
+ * cycles (clamped to [1, 2e9]) and records FLINT_DEVCHECK_WAIT in the
+ * workspace status word, the way every wait in the layer kernels does. It
+ * leaves no copy in flight and the context stays usable; read the result with
+ * flint_moe_get_status. */
+int flint_debug_wait_timeout(void* workspace, int64_t cycles, void* stream);
+
+/* Library version string. */
+const char* flint_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FLINT_MOE_H */

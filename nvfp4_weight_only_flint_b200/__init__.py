@@ -1,0 +1,210 @@
+"""Flint MoE layer decode on B200: Python binding of libflint_moe.so.
+
+Each function below has the name and arguments of the C entry point it wraps
+(see include/flint_moe.h); it only turns torch tensors into device pointers,
+passes the current CUDA stream, and raises FlintError on a non-zero status.
+Every step of the layer runs in the library's CUDA kernels: there is no CPU or
+PyTorch fallback, and importing this package on a machine without the built
+library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .build import SO as _SO_PATH
+
+__all__ = [
+    "FlintError", "Shape", "Weights", "Options", "lib",
+    "FLINT_W_NVFP4", "FLINT_W_BF16", "FLINT_PATH_AUTO", "FLINT_PATH_GEMV", "FLINT_PATH_MMA",
+    "flint_packed_bytes", "flint_block_scale_bytes", "flint_tensor_scale_bytes",
+    "flint_moe_workspace_bytes", "flint_moe_workspace_init", "flint_pack_nvfp4", "flint_pack_bf16", "flint_moe_route",
+    "flint_moe_forward", "flint_moe_forward_ex", "flint_moe_get_status", "flint_last_error",
+    "flint_debug_dequant", "flint_debug_wait_timeout", "flint_version",
+]
+
+FLINT_W_NVFP4, FLINT_W_BF16 = 0, 1
+FLINT_PATH_AUTO, FLINT_PATH_GEMV, FLINT_PATH_MMA = 0, 1, 2
+STATUS_NAMES = {0: "FLINT_OK", -1: "FLINT_ERR_INVALID_ARG", -2: "FLINT_ERR_UNSUPPORTED_SHAPE",
+                -3: "FLINT_ERR_MISALIGNED", -4: "FLINT_ERR_WORKSPACE", -5: "FLINT_ERR_CUDA",
+                -6: "FLINT_ERR_DEVICE_CHECK", -7: "FLINT_ERR_TIMEOUT"}
+
+
+class FlintError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("inter", ctypes.c_int32), ("n_experts", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("wdtype", ctypes.c_int32)]
+
+
+class Weights(ctypes.Structure):
+    _fields_ = [("packed", ctypes.c_void_p), ("block_scales", ctypes.c_void_p),
+                ("tensor_scales", ctypes.c_void_p)]
+
+
+class Options(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("use_pdl", ctypes.c_int32),
+                ("topk_ids", ctypes.c_void_p), ("topk_weights", ctypes.c_void_p),
+                ("input_rmsnorm", ctypes.c_int32), ("profile_events", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_SO_PATH):
+            raise FlintError(-5, f"{_SO_PATH} is missing: run nvfp4_weight_only_flint_b200.build.build()")
+        L = ctypes.CDLL(_SO_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        P = ctypes.POINTER
+        L.flint_packed_bytes.argtypes = [P(Shape)]
+        L.flint_packed_bytes.restype = sz
+        L.flint_block_scale_bytes.argtypes = [P(Shape)]
+        L.flint_block_scale_bytes.restype = sz
+        L.flint_tensor_scale_bytes.argtypes = [P(Shape)]
+        L.flint_tensor_scale_bytes.restype = sz
+        L.flint_moe_workspace_bytes.argtypes = [P(Shape), i32]
+        L.flint_moe_workspace_bytes.restype = sz
+        L.flint_pack_nvfp4.argtypes = [vp, i32, P(Shape), vp, vp, vp, vp, sz, vp]
+        L.flint_pack_nvfp4.restype = i32
+        L.flint_pack_bf16.argtypes = [vp, P(Shape), vp, vp]
+        L.flint_pack_bf16.restype = i32
+        L.flint_moe_route.argtypes = [vp, i32, vp, P(Shape), vp, vp, vp, sz, vp]
+        L.flint_moe_route.restype = i32
+        L.flint_moe_forward.argtypes = [vp, i32, vp, P(Weights), P(Shape), vp, vp, vp, sz, vp]
+        L.flint_moe_forward.restype = i32
+        L.flint_moe_forward_ex.argtypes = [vp, i32, vp, P(Weights), P(Shape), vp, vp, vp, sz,
+                                           P(Options), vp]
+        L.flint_moe_forward_ex.restype = i32
+        L.flint_moe_workspace_init.argtypes = [vp, sz, vp]
+        L.flint_moe_workspace_init.restype = i32
+        L.flint_moe_get_status.argtypes = [vp, P(i32), vp]
+        L.flint_moe_get_status.restype = i32
+        L.flint_last_error.argtypes = []
+        L.flint_last_error.restype = ctypes.c_char_p
+        L.flint_debug_dequant.argtypes = [P(Weights), P(Shape), i32, i32, i32, i32, vp, vp, vp]
+        L.flint_debug_dequant.restype = i32
+        L.flint_debug_wait_timeout.argtypes = [vp, ctypes.c_int64, vp]
+        L.flint_debug_wait_timeout.restype = i32
+        L.flint_version.argtypes = []
+        L.flint_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+# ------------------------------------------------------------------ marshalling helpers
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise FlintError(-1, "expected a CUDA tensor")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise FlintError(rc, lib().flint_last_error().decode())
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def flint_last_error() -> str:
+    return lib().flint_last_error().decode()
+
+
+def flint_version() -> str:
+    return lib().flint_version().decode()
+
+
+def flint_packed_bytes(shape: Shape) -> int:
+    return lib().flint_packed_bytes(ctypes.byref(shape))
+
+
+def flint_block_scale_bytes(shape: Shape) -> int:
+    return lib().flint_block_scale_bytes(ctypes.byref(shape))
+
+
+def flint_tensor_scale_bytes(shape: Shape) -> int:
+    return lib().flint_tensor_scale_bytes(ctypes.byref(shape))
+
+
+def flint_moe_workspace_bytes(shape: Shape, max_tokens: int) -> int:
+    return lib().flint_moe_workspace_bytes(ctypes.byref(shape), int(max_tokens))
+
+
+def flint_moe_workspace_init(workspace, stream=None) -> None:
+    _check(lib().flint_moe_workspace_init(_ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def flint_pack_nvfp4(w, w_is_bf16: int, shape: Shape, packed, block_scales, tensor_scales,
+                     workspace, stream=None) -> None:
+    _check(lib().flint_pack_nvfp4(_ptr(w), int(w_is_bf16), ctypes.byref(shape), _ptr(packed),
+                                  _ptr(block_scales), _ptr(tensor_scales), _ptr(workspace),
+                                  _nbytes(workspace), _stream(stream)))
+
+
+def flint_pack_bf16(w, shape: Shape, packed, stream=None) -> None:
+    _check(lib().flint_pack_bf16(_ptr(w), ctypes.byref(shape), _ptr(packed), _stream(stream)))
+
+
+def flint_moe_route(x, T: int, router_w, shape: Shape, topk_ids, topk_weights, workspace,
+                    stream=None) -> None:
+    _check(lib().flint_moe_route(_ptr(x), int(T), _ptr(router_w), ctypes.byref(shape),
+                                 _ptr(topk_ids), _ptr(topk_weights), _ptr(workspace),
+                                 _nbytes(workspace), _stream(stream)))
+
+
+def flint_moe_forward(x, T: int, router_w, weights: Weights, shape: Shape, residual, out,
+                      workspace, stream=None) -> None:
+    _check(lib().flint_moe_forward(_ptr(x), int(T), _ptr(router_w), ctypes.byref(weights),
+                                   ctypes.byref(shape), _ptr(residual), _ptr(out),
+                                   _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def flint_moe_forward_ex(x, T: int, router_w, weights: Weights, shape: Shape, residual, out,
+                         workspace, options: Options | None, stream=None) -> None:
+    _check(lib().flint_moe_forward_ex(_ptr(x), int(T), _ptr(router_w), ctypes.byref(weights),
+                                      ctypes.byref(shape), _ptr(residual), _ptr(out),
+                                      _ptr(workspace), _nbytes(workspace),
+                                      ctypes.byref(options) if options is not None else None,
+                                      _stream(stream)))
+
+
+def flint_moe_get_status(workspace, stream=None) -> tuple[int, int]:
+    """Returns (status, device_flags) without raising."""
+    flags = ctypes.c_int32(0)
+    rc = lib().flint_moe_get_status(_ptr(workspace), ctypes.byref(flags), _stream(stream))
+    return rc, flags.value
+
+
+def flint_debug_dequant(weights: Weights, shape: Shape, expert: int, matrix: int, row0: int,
+                        rows: int, out, stream=None) -> tuple[float, ...]:
+    ts = (ctypes.c_float * 2)()
+    _check(lib().flint_debug_dequant(ctypes.byref(weights), ctypes.byref(shape), int(expert),
+                                     int(matrix), int(row0), int(rows), _ptr(out), ts,
+                                     _stream(stream)))
+    return (ts[0], ts[1]) if matrix == 0 else (ts[0],)
+
+
+def flint_debug_wait_timeout(workspace, cycles: int, stream=None) -> None:
+    _check(lib().flint_debug_wait_timeout(_ptr(workspace), int(cycles), _stream(stream)))

@@ -1,0 +1,714 @@
+// flint_moe.cu -- packer, debug kernels and the C ABI of libflint_moe.so (see
+// include/flint_moe.h). The layer kernels are in layer_kernels.cuh: per layer
+// k_route -> k_gateup -> k_down, chained with programmatic dependent launch on
+// the caller's stream. The packer quantises and lays out weights (fp32 recipe,
+// bit-exact against the CPU oracle).
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "layer_kernels.cuh"
+
+namespace flint {
+
+// ======================================================================= kernels
+// ----------------------------------------------------------------- packer
+// Per-matrix amax (as uint bits of non-negative floats) and non-finite check.
+template <bool BF16IN>
+__global__ void k_pack_amax(const void* w, long long per_mat, unsigned* amax_bits, int* status) {
+  const int mat = blockIdx.y;
+  float m = 0.f;
+  bool bad = false;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < per_mat;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long gi = static_cast<long long>(mat) * per_mat + i;
+    const float v = BF16IN ? bf16_bits_to_f32(static_cast<const uint16_t*>(w)[gi])
+                           : static_cast<const float*>(w)[gi];
+    if (!isfinite(v)) bad = true;
+    else m = fmaxf(m, fabsf(v));
+  }
+  if (bad) atomicOr(status, FLINT_DEVCHECK_NONFINITE);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(&amax_bits[mat], __float_as_uint(m));
+}
+
+__device__ __forceinline__ uint32_t f32_to_e4m3(float v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.f), "f"(v));
+  return r & 0xFFu;
+}
+// Two values -> one byte of E2M1 codes, `lo` in the low nibble.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n .reg .b8 b;\n cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n cvt.u32.u8 %0, b;\n}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r & 0xFFu;
+}
+
+// One thread per 16-element block: the recipe's fp32 steps, then the layout.
+template <bool BF16IN>
+__global__ void k_pack_quant(const void* w, int d, int I, long long n_blocks, long long cpe, long long spe,
+                             const unsigned* amax_bits, uint8_t* codes, uint8_t* scales, float* ts) {
+  const long long gb = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  if (gb >= n_blocks) return;
+  const long long per_mat = static_cast<long long>(I) * d;
+  const long long blocks_per_mat = per_mat / 16;
+  const int mat = static_cast<int>(gb / blocks_per_mat);
+  const long long bi = gb % blocks_per_mat;
+  const int e = mat / 3, m = mat % 3;
+  const int cols = (m < 2) ? d : I;
+  const int r = static_cast<int>(bi / (cols / 16)), b = static_cast<int>(bi % (cols / 16));
+  float v[16];
+  const long long base = static_cast<long long>(mat) * per_mat + static_cast<long long>(r) * cols + 16LL * b;
+  if (BF16IN) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(w) + base);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint4 u = src[q];
+      const uint32_t ww[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[8 * q + 2 * i] = bf16_bits_to_f32(ww[i] & 0xFFFFu);
+        v[8 * q + 2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u);
+      }
+    }
+  } else {
+    const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(w) + base);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 f = src[q];
+      v[4 * q] = f.x;
+      v[4 * q + 1] = f.y;
+      v[4 * q + 2] = f.z;
+      v[4 * q + 3] = f.w;
+    }
+  }
+  const float amax = __uint_as_float(amax_bits[mat]);
+  const float s_t = (amax > 0.f) ? __fdiv_rn(amax, 2688.f) : 1.f;
+  float amax_b = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
+  const uint32_t sb = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax_b, 6.f), s_t));
+  const float dec = e4m3x2_to_f32x2(sb).x;
+  const float denom = __fmul_rn(dec, s_t);
+  uint32_t lo = 0, hi = 0;
+  if (denom != 0.f) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      lo |= f32x2_to_e2m1x2(__fdiv_rn(v[2 * i], denom), __fdiv_rn(v[2 * i + 1], denom)) << (8 * i);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      hi |= f32x2_to_e2m1x2(__fdiv_rn(v[8 + 2 * i], denom), __fdiv_rn(v[8 + 2 * i + 1], denom)) << (8 * i);
+  }
+  long long co, so;
+  if (m == 0) {
+    co = static_cast<long long>(r) * d + 8LL * b;
+    so = static_cast<long long>(r) * (d / 8) + b;
+  } else if (m == 1) {
+    co = static_cast<long long>(r) * d + d / 2 + 8LL * b;
+    so = static_cast<long long>(r) * (d / 8) + d / 16 + b;
+  } else {
+    co = static_cast<long long>(I) * d + static_cast<long long>(r) * (I / 2) + 8LL * b;
+    so = static_cast<long long>(I) * d / 8 + static_cast<long long>(r) * (I / 16) + b;
+  }
+  *reinterpret_cast<uint2*>(codes + e * cpe + co) = make_uint2(lo, hi);
+  scales[e * spe + so] = static_cast<uint8_t>(sb);
+  if (r == 0 && b == 0) ts[mat] = s_t;
+}
+
+// bf16 weights in the same expert-major row order (16-byte vectors).
+__global__ void k_pack_bf16(const uint16_t* w, int d, int I, long long n_vec, uint16_t* out) {
+  const long long gv = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  if (gv >= n_vec) return;
+  const long long per_mat = static_cast<long long>(I) * d;
+  const long long vec_per_mat = per_mat / 8;
+  const int mat = static_cast<int>(gv / vec_per_mat);
+  const long long vi = gv % vec_per_mat;
+  const int e = mat / 3, m = mat % 3;
+  const int cols = (m < 2) ? d : I;
+  const int r = static_cast<int>(vi / (cols / 8)), c8 = static_cast<int>(vi % (cols / 8));
+  const uint4 val = reinterpret_cast<const uint4*>(w + static_cast<long long>(mat) * per_mat)[vi];
+  long long o = static_cast<long long>(e) * 3 * per_mat;
+  if (m == 0) o += static_cast<long long>(r) * 2 * d + 8LL * c8;
+  else if (m == 1) o += static_cast<long long>(r) * 2 * d + d + 8LL * c8;
+  else o += 2LL * I * d + static_cast<long long>(r) * I + 8LL * c8;
+  *reinterpret_cast<uint4*>(out + o) = val;
+}
+
+// Decoded e2m1*e4m3 products of rows of one expert matrix, through the same
+// decode routines the layer kernels use. One thread per 32-element vector.
+__global__ void k_debug_dequant(const uint8_t* codes, const uint8_t* scales, int K, long long rows,
+                                float* out) {
+  const long long gv = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  const int vpr = K / 32;
+  if (gv >= rows * vpr) return;
+  const long long r = gv / vpr;
+  const int v = static_cast<int>(gv % vpr);
+  const uint4 c = *reinterpret_cast<const uint4*>(codes + r * (K / 2) + v * 16);
+  const uint32_t s2 = *reinterpret_cast<const uint16_t*>(scales + r * (K / 16) + v * 2);
+  const float2 s = e4m3x2_to_f32x2(s2);
+  const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int wi = 0; wi < 4; ++wi) {
+    uint32_t q[4];
+    e2m1x8_to_f16x2(words[wi], q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&q[i]));
+      const float sc = (wi < 2) ? s.x : s.y;
+      out[r * K + v * 32 + wi * 8 + 2 * i] = f.x * sc;
+      out[r * K + v * 32 + wi * 8 + 2 * i + 1] = f.y * sc;
+    }
+  }
+}
+
+// A wait on a barrier that no thread or copy ever completes: the bounded loop
+// gives up after `cycles` and records FLINT_DEVCHECK_WAIT.
+__global__ void k_debug_wait(int* status, long long cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(&bar, 0)) {
+      if (clock64() - t0 > cycles) {
+        atomicOr(status, FLINT_DEVCHECK_WAIT);
+        break;
+      }
+    }
+  }
+}
+
+// ======================================================================= host side
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(FLINT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+struct Dims {
+  int d, I, E, k, S, wd;
+};
+
+int check_shape(const flint_moe_shape* s, Dims* out) {
+  if (s == nullptr) return fail(FLINT_ERR_INVALID_ARG, "shape is NULL");
+  const int d = s->d, I = s->inter, E = s->n_experts, k = s->top_k, S = s->n_shared;
+  if (s->wdtype != FLINT_W_NVFP4 && s->wdtype != FLINT_W_BF16)
+    return fail(FLINT_ERR_INVALID_ARG, "wdtype %d is not a flint_wdtype", s->wdtype);
+  if (!(d == 512 || d == 1024 || d == 2048 || d == 4096))
+    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "d=%d: supported 512, 1024, 2048, 4096", d);
+  if (!(I == 128 || I == 256 || I == 512 || I == 1024))
+    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "inter=%d: supported 128, 256, 512, 1024", I);
+  if (E < 1 || E > kMaxExperts) return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "n_experts=%d: supported 1..%d", E, kMaxExperts);
+  if (k < 1 || k > kMaxTopK || k > E) return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "top_k=%d: supported 1..min(8, E)", k);
+  if (S < 0 || S > 1) return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "n_shared=%d: supported 0 or 1", S);
+  *out = Dims{d, I, E, k, S, s->wdtype};
+  return FLINT_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct WsLayout {
+  size_t status, counter, amax, desc, logits, ids, gates, h, total;
+};
+
+size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace carve-up for calls of up to maxT tokens. The first 256 bytes hold
+// the status word (byte 0) and the router's arrival counter (byte 4); both
+// start at zero (flint_moe_workspace_init) and are left at zero by every call.
+WsLayout ws_layout(const Dims& s, int maxT) {
+  WsLayout w{};
+  size_t o = 0;
+  w.status = 0;
+  w.counter = 4;
+  o += 256;
+  w.amax = o;
+  o += al256(sizeof(float) * (s.E + s.S) * 3);
+  w.desc = o;
+  o += al256(sizeof(RouteDesc));
+  w.logits = o;
+  o += al256(sizeof(float) * static_cast<size_t>(maxT) * s.E);
+  w.ids = o;
+  o += al256(sizeof(int) * static_cast<size_t>(maxT) * s.k);
+  w.gates = o;
+  o += al256(sizeof(float) * static_cast<size_t>(maxT) * s.k);
+  w.h = o;
+  o += al256(sizeof(float) * static_cast<size_t>(maxT) * (s.k + s.S) * s.I);
+  w.total = o;
+  return w;
+}
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+// Raise a kernel's dynamic shared-memory limit to the device's opt-in maximum,
+// once per (kernel, device). The limit only bounds what a launch may request.
+cudaError_t ensure_smem(const void* kern) {
+  static std::mutex mu;
+  static const void* done_kern[256];
+  static int done_dev[256];
+  static int n_done = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done_kern[i] == kern && done_dev[i] == dev) return cudaSuccess;
+  int optin = 0;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           optin - static_cast<int>(fa.sharedSizeBytes));
+  if (e == cudaSuccess && n_done < 256) {
+    done_kern[n_done] = kern;
+    done_dev[n_done] = dev;
+    ++n_done;
+  }
+  return e;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                   Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// Shared-memory budget of one CTA of the streaming kernels (rings + staged
+// activations), below the 227 KB opt-in limit with room for static arrays.
+constexpr int kSmemBudget = 200 * 1024;
+
+void fill_common(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, int T) {
+  p.T = T;
+  p.d = s.d;
+  p.I = s.I;
+  p.E = s.E;
+  p.k = s.k;
+  p.S = s.S;
+  p.cpe = 3LL * s.I * s.d / 2;
+  p.spe = 3LL * s.I * s.d / 16;
+  p.status = reinterpret_cast<int*>(ws + w.status);
+  p.counter = reinterpret_cast<unsigned*>(ws + w.counter);
+  p.desc = reinterpret_cast<RouteDesc*>(ws + w.desc);
+  p.logits = reinterpret_cast<float*>(ws + w.logits);
+  p.ids = reinterpret_cast<int*>(ws + w.ids);
+  p.gates = reinterpret_cast<float*>(ws + w.gates);
+  p.h = reinterpret_cast<float*>(ws + w.h);
+}
+
+int gateup_stage_bytes(int d) {
+  const int cu = (d <= 1024) ? 4 : (d == 2048 ? 2 : 1);
+  return cu * (d + d / 8);
+}
+
+// Ring depths, row blocking of the down kernel and activation staging for a call.
+void configure(LayerParams& p, const Dims& s, int T) {
+  const int sms = num_sms();
+  const int desc = static_cast<int>(sizeof(RouteDesc));
+  // gate/up: stage x in shared memory when two stages per warp still fit
+  p.stage_gateup = gateup_stage_bytes(s.d);
+  const int ring2 = kGemvWarps * 2 * p.stage_gateup;
+  const int xbytes = T * s.d * 2;
+  p.x_in_smem = (desc + xbytes + ring2 <= kSmemBudget) ? 1 : 0;
+  const int room_g = kSmemBudget - desc - (p.x_in_smem ? xbytes : 0);
+  p.ns_gateup = room_g / (kGemvWarps * p.stage_gateup);
+  if (p.ns_gateup > 4) p.ns_gateup = 4;
+  if (p.ns_gateup < 2) p.ns_gateup = 2;
+  // down: rows per CTA ~ d / #SMs in whole warp steps; items of up to four steps
+  const int rps = 32 / (s.I / 32);
+  int nb = (s.d + sms - 1) / sms;
+  nb = ((nb + rps - 1) / rps) * rps;
+  if (nb % 2) nb += rps;
+  p.down_nb = nb;
+  p.down_rb = (4 * rps < nb) ? 4 * rps : nb;
+  p.stage_down = ((p.down_rb * (s.I / 2 + s.I / 16)) + 15) & ~15;
+  const int ybytes = ((4 * T * (s.k + s.S) * nb) + 127) & ~127;
+  const int hbytes = T * (s.k + s.S) * s.I * 4;
+  const int ring2d = kGemvWarps * 2 * p.stage_down;
+  p.h_in_smem = (desc + hbytes + ybytes + ring2d <= kSmemBudget) ? 1 : 0;
+  const int room_d = kSmemBudget - desc - ybytes - (p.h_in_smem ? hbytes : 0);
+  p.ns_down = room_d / (kGemvWarps * p.stage_down);
+  if (p.ns_down > 4) p.ns_down = 4;
+  if (p.ns_down < 2) p.ns_down = 2;
+}
+
+size_t gateup_smem(const LayerParams& p) {
+  return sizeof(RouteDesc) + (p.x_in_smem ? static_cast<size_t>(p.T) * p.d * 2 : 0) +
+         static_cast<size_t>(kGemvWarps) * p.ns_gateup * p.stage_gateup;
+}
+size_t down_smem(const LayerParams& p) {
+  const size_t ybytes = ((sizeof(float) * static_cast<size_t>(p.T) * (p.k + p.S) * p.down_nb) + 127) & ~static_cast<size_t>(127);
+  return sizeof(RouteDesc) + (p.h_in_smem ? static_cast<size_t>(p.T) * (p.k + p.S) * p.I * 4 : 0) + ybytes +
+         static_cast<size_t>(kGemvWarps) * p.ns_down * p.stage_down;
+}
+
+template <typename K>
+cudaError_t launch_smem(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                        const LayerParams& p) {
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern));
+  if (e != cudaSuccess) return e;
+  return launch(kern, grid, block, smem, st, pdl, p);
+}
+
+cudaError_t launch_route_fwd(const LayerParams& p, cudaStream_t st, bool pdl) {
+  const int tasks = p.E + p.S * p.I;
+  const dim3 grid((tasks + kRouteWarps - 1) / kRouteWarps), block(kRouteWarps * 32);
+  const size_t smem = static_cast<size_t>(p.T) * p.d * 2;
+  switch (p.d) {
+    case 512: return launch_smem(k_route<512>, grid, block, smem, st, pdl, p);
+    case 1024: return launch_smem(k_route<1024>, grid, block, smem, st, pdl, p);
+    case 2048: return launch_smem(k_route<2048>, grid, block, smem, st, pdl, p);
+    default: return launch_smem(k_route<4096>, grid, block, smem, st, pdl, p);
+  }
+}
+
+cudaError_t launch_router_only(const LayerParams& p, cudaStream_t st) {
+  const dim3 grid((p.E + 7) / 8), block(256);
+  switch (p.d) {
+    case 512: return launch(k_router_only<512>, grid, block, 0, st, false, p);
+    case 1024: return launch(k_router_only<1024>, grid, block, 0, st, false, p);
+    case 2048: return launch(k_router_only<2048>, grid, block, 0, st, false, p);
+    default: return launch(k_router_only<4096>, grid, block, 0, st, false, p);
+  }
+}
+
+cudaError_t launch_gateup(const LayerParams& p, cudaStream_t st, bool pdl) {
+  const dim3 grid(num_sms()), block(kGemvWarps * 32);
+  const size_t smem = gateup_smem(p);
+  switch (p.d) {
+    case 512: return launch_smem(k_gateup<512>, grid, block, smem, st, pdl, p);
+    case 1024: return launch_smem(k_gateup<1024>, grid, block, smem, st, pdl, p);
+    case 2048: return launch_smem(k_gateup<2048>, grid, block, smem, st, pdl, p);
+    default: return launch_smem(k_gateup<4096>, grid, block, smem, st, pdl, p);
+  }
+}
+
+cudaError_t launch_down(const LayerParams& p, cudaStream_t st, bool pdl) {
+  const dim3 grid((p.d + p.down_nb - 1) / p.down_nb), block(kGemvWarps * 32);
+  const size_t smem = down_smem(p);
+  switch (p.I) {
+    case 128: return launch_smem(k_down<128>, grid, block, smem, st, pdl, p);
+    case 256: return launch_smem(k_down<256>, grid, block, smem, st, pdl, p);
+    case 512: return launch_smem(k_down<512>, grid, block, smem, st, pdl, p);
+    default: return launch_smem(k_down<1024>, grid, block, smem, st, pdl, p);
+  }
+}
+
+}  // namespace
+}  // namespace flint
+
+using namespace flint;
+
+// ======================================================================= C ABI
+extern "C" {
+
+const char* flint_last_error(void) { return g_last_error.c_str(); }
+
+const char* flint_version(void) { return "flint_moe 0.1 (sm_100a)"; }
+
+size_t flint_packed_bytes(const flint_moe_shape* shape) {
+  Dims s;
+  if (check_shape(shape, &s) != FLINT_OK) return 0;
+  const size_t n = static_cast<size_t>(s.E + s.S) * 3 * s.I * s.d;
+  return s.wd == FLINT_W_BF16 ? n * 2 : n / 2;
+}
+
+size_t flint_block_scale_bytes(const flint_moe_shape* shape) {
+  Dims s;
+  if (check_shape(shape, &s) != FLINT_OK || s.wd == FLINT_W_BF16) return 0;
+  return static_cast<size_t>(s.E + s.S) * 3 * s.I * s.d / 16;
+}
+
+size_t flint_tensor_scale_bytes(const flint_moe_shape* shape) {
+  Dims s;
+  if (check_shape(shape, &s) != FLINT_OK || s.wd == FLINT_W_BF16) return 0;
+  return static_cast<size_t>(s.E + s.S) * 3 * sizeof(float);
+}
+
+size_t flint_moe_workspace_bytes(const flint_moe_shape* shape, int32_t max_tokens) {
+  Dims s;
+  if (check_shape(shape, &s) != FLINT_OK || max_tokens < 0) return 0;
+  return ws_layout(s, max_tokens < 1 ? 1 : max_tokens).total;
+}
+
+int flint_pack_nvfp4(const void* w, int32_t w_is_bf16, const flint_moe_shape* shape, void* packed,
+                     uint8_t* block_scales, float* tensor_scales, void* workspace, size_t ws_bytes,
+                     void* stream) {
+  Dims s;
+  int rc = check_shape(shape, &s);
+  if (rc != FLINT_OK) return rc;
+  if (s.wd != FLINT_W_NVFP4) return fail(FLINT_ERR_INVALID_ARG, "flint_pack_nvfp4 needs wdtype FLINT_W_NVFP4");
+  if (!w || !packed || !block_scales || !tensor_scales || !workspace)
+    return fail(FLINT_ERR_INVALID_ARG, "flint_pack_nvfp4: NULL pointer");
+  if (!aligned16(w) || !aligned16(packed) || !aligned16(block_scales) || !aligned16(tensor_scales) ||
+      !aligned16(workspace))
+    return fail(FLINT_ERR_MISALIGNED, "flint_pack_nvfp4: pointers must be 16-byte aligned");
+  const WsLayout lay = ws_layout(s, 1);
+  if (ws_bytes < lay.total) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, lay.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int n_mats = (s.E + s.S) * 3;
+  const long long per_mat = static_cast<long long>(s.I) * s.d;
+  unsigned* amax = reinterpret_cast<unsigned*>(ws + lay.amax);
+  int* status = reinterpret_cast<int*>(ws + lay.status);
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned) * n_mats, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  const dim3 ga(32, n_mats);
+  if (w_is_bf16)
+    k_pack_amax<true><<<ga, 256, 0, st>>>(w, per_mat, amax, status);
+  else
+    k_pack_amax<false><<<ga, 256, 0, st>>>(w, per_mat, amax, status);
+  const long long n_blocks = static_cast<long long>(n_mats) * per_mat / 16;
+  const unsigned gq = static_cast<unsigned>((n_blocks + 255) / 256);
+  const long long cpe = 3LL * s.I * s.d / 2, spe = 3LL * s.I * s.d / 16;
+  if (w_is_bf16)
+    k_pack_quant<true><<<gq, 256, 0, st>>>(w, s.d, s.I, n_blocks, cpe, spe, amax,
+                                           static_cast<uint8_t*>(packed), block_scales, tensor_scales);
+  else
+    k_pack_quant<false><<<gq, 256, 0, st>>>(w, s.d, s.I, n_blocks, cpe, spe, amax,
+                                            static_cast<uint8_t*>(packed), block_scales, tensor_scales);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "flint_pack_nvfp4 launch");
+  return FLINT_OK;
+}
+
+int flint_pack_bf16(const uint16_t* w, const flint_moe_shape* shape, uint16_t* packed, void* stream) {
+  Dims s;
+  int rc = check_shape(shape, &s);
+  if (rc != FLINT_OK) return rc;
+  if (s.wd != FLINT_W_BF16) return fail(FLINT_ERR_INVALID_ARG, "flint_pack_bf16 needs wdtype FLINT_W_BF16");
+  if (!w || !packed) return fail(FLINT_ERR_INVALID_ARG, "flint_pack_bf16: NULL pointer");
+  if (!aligned16(w) || !aligned16(packed)) return fail(FLINT_ERR_MISALIGNED, "flint_pack_bf16: unaligned pointer");
+  const long long n_vec = static_cast<long long>(s.E + s.S) * 3 * s.I * s.d / 8;
+  k_pack_bf16<<<static_cast<unsigned>((n_vec + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      w, s.d, s.I, n_vec, packed);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "flint_pack_bf16 launch");
+  return FLINT_OK;
+}
+
+int flint_moe_route(const uint16_t* x, int32_t T, const uint16_t* router_w, const flint_moe_shape* shape,
+                    int32_t* topk_ids, float* topk_weights, void* workspace, size_t ws_bytes, void* stream) {
+  Dims s;
+  int rc = check_shape(shape, &s);
+  if (rc != FLINT_OK) return rc;
+  if (T < 0) return fail(FLINT_ERR_INVALID_ARG, "T=%d", T);
+  if (T == 0) return FLINT_OK;
+  if (!x || !router_w || !topk_ids || !topk_weights || !workspace)
+    return fail(FLINT_ERR_INVALID_ARG, "flint_moe_route: NULL pointer");
+  if (!aligned16(x) || !aligned16(router_w) || !aligned16(topk_ids) || !aligned16(topk_weights) ||
+      !aligned16(workspace))
+    return fail(FLINT_ERR_MISALIGNED, "flint_moe_route: pointers must be 16-byte aligned");
+  const WsLayout lay = ws_layout(s, T);
+  if (ws_bytes < lay.total) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, lay.total);
+  LayerParams p{};
+  fill_common(p, s, lay, static_cast<uint8_t*>(workspace), T);
+  p.x = x;
+  p.wr = router_w;
+  p.ids = topk_ids;
+  p.gates = topk_weights;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_router_only(p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "k_router_only launch");
+  e = launch(k_topk, dim3((T + 7) / 8), dim3(256), 0, st, true, p);
+  if (e != cudaSuccess) return cuda_fail(e, "k_topk launch");
+  return FLINT_OK;
+}
+
+int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
+                         const flint_moe_weights* weights, const flint_moe_shape* shape,
+                         const uint16_t* residual, uint16_t* out, void* workspace, size_t ws_bytes,
+                         const flint_moe_options* options, void* stream) {
+  Dims s;
+  int rc = check_shape(shape, &s);
+  if (rc != FLINT_OK) return rc;
+  if (T < 0) return fail(FLINT_ERR_INVALID_ARG, "T=%d", T);
+  if (T == 0) return FLINT_OK;
+  if (!x || !router_w || !weights || !weights->packed || !out || !workspace)
+    return fail(FLINT_ERR_INVALID_ARG, "flint_moe_forward: NULL pointer");
+  if (s.wd == FLINT_W_NVFP4 && (!weights->block_scales || !weights->tensor_scales))
+    return fail(FLINT_ERR_INVALID_ARG, "flint_moe_forward: NVFP4 weights need block and tensor scales");
+  if (!aligned16(x) || !aligned16(router_w) || !aligned16(weights->packed) || !aligned16(out) ||
+      !aligned16(workspace) || (residual && !aligned16(residual)) ||
+      (weights->block_scales && !aligned16(weights->block_scales)) ||
+      (weights->tensor_scales && !aligned16(weights->tensor_scales)))
+    return fail(FLINT_ERR_MISALIGNED, "flint_moe_forward: pointers must be 16-byte aligned");
+  const int path = options ? options->path : FLINT_PATH_AUTO;
+  const bool pdl = options ? options->use_pdl != 0 : true;
+  if (path < FLINT_PATH_AUTO || path > FLINT_PATH_MMA) return fail(FLINT_ERR_INVALID_ARG, "path %d", path);
+  if (options && ((options->topk_ids == nullptr) != (options->topk_weights == nullptr)))
+    return fail(FLINT_ERR_INVALID_ARG, "topk_ids and topk_weights go together");
+  const bool use_gemv = (path == FLINT_PATH_GEMV) || (path == FLINT_PATH_AUTO && T < kMaxGemvTokens);
+  if (!use_gemv || s.wd != FLINT_W_NVFP4)
+    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "tensor-core path not available in this build (T=%d)", T);
+  const int gemv_max_t = (s.d == 4096) ? kMaxGemvTokens / 2 : kMaxGemvTokens;
+  if (T > gemv_max_t)
+    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "GEMV path takes at most %d tokens at d=%d", gemv_max_t, s.d);
+  const WsLayout lay = ws_layout(s, T);
+  if (ws_bytes < lay.total) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, lay.total);
+
+  LayerParams p{};
+  fill_common(p, s, lay, static_cast<uint8_t*>(workspace), T);
+  p.x = x;
+  p.wr = router_w;
+  p.codes = static_cast<const uint8_t*>(weights->packed);
+  p.scales = weights->block_scales;
+  p.tscale = weights->tensor_scales;
+  p.residual = residual;
+  p.out = out;
+  if (options && options->topk_ids) {
+    p.ids_out = options->topk_ids;
+    p.gates_out = options->topk_weights;
+  }
+  p.input_norm = (options && options->input_rmsnorm) ? 1 : 0;
+  configure(p, s, T);
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaEvent_t* ev = options ? static_cast<cudaEvent_t*>(options->profile_events) : nullptr;
+  cudaError_t e = launch_route_fwd(p, st, pdl);
+  if (e != cudaSuccess) return cuda_fail(e, "k_route launch");
+  if (ev) {
+    e = cudaEventRecord(ev[0], st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  }
+  e = launch_gateup(p, st, pdl && !ev);
+  if (e != cudaSuccess) return cuda_fail(e, "k_gateup launch");
+  if (ev) {
+    e = cudaEventRecord(ev[1], st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  }
+  e = launch_down(p, st, pdl && !ev);
+  if (e != cudaSuccess) return cuda_fail(e, "k_down launch");
+  return FLINT_OK;
+}
+
+int flint_moe_forward(const uint16_t* x, int32_t T, const uint16_t* router_w, const flint_moe_weights* weights,
+                      const flint_moe_shape* shape, const uint16_t* residual, uint16_t* out, void* workspace,
+                      size_t ws_bytes, void* stream) {
+  return flint_moe_forward_ex(x, T, router_w, weights, shape, residual, out, workspace, ws_bytes, nullptr,
+                              stream);
+}
+
+int flint_moe_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
+  if (!workspace) return fail(FLINT_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned16(workspace)) return fail(FLINT_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  if (ws_bytes < 256) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < 256 bytes", ws_bytes);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 256, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  return FLINT_OK;
+}
+
+int flint_moe_get_status(void* workspace, int32_t* device_flags, void* stream) {
+  if (!workspace) return fail(FLINT_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t flags = 0;
+  cudaError_t e = cudaMemcpyAsync(&flags, workspace, sizeof flags, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof flags, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "flint_moe_get_status");
+  if (device_flags) *device_flags = flags;
+  if (flags & FLINT_DEVCHECK_WAIT) return fail(FLINT_ERR_TIMEOUT, "a bounded device wait ran out");
+  if (flags) return fail(FLINT_ERR_DEVICE_CHECK, "device check flags 0x%x", flags);
+  return FLINT_OK;
+}
+
+int flint_debug_dequant(const flint_moe_weights* weights, const flint_moe_shape* shape, int32_t expert,
+                        int32_t matrix, int32_t row0, int32_t rows, float* out, float* tensor_scale_out,
+                        void* stream) {
+  Dims s;
+  int rc = check_shape(shape, &s);
+  if (rc != FLINT_OK) return rc;
+  if (s.wd != FLINT_W_NVFP4 || !weights || !weights->packed || !weights->block_scales ||
+      !weights->tensor_scales || !out)
+    return fail(FLINT_ERR_INVALID_ARG, "flint_debug_dequant: NVFP4 weights and output needed");
+  if (expert < 0 || expert >= s.E + s.S || (matrix != 0 && matrix != 1) || row0 < 0 || rows < 0)
+    return fail(FLINT_ERR_INVALID_ARG, "flint_debug_dequant: bad expert/matrix/rows");
+  const int max_rows = matrix == 0 ? s.I : s.d;
+  if (row0 + rows > max_rows) return fail(FLINT_ERR_INVALID_ARG, "flint_debug_dequant: rows out of range");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long cpe = 3LL * s.I * s.d / 2, spe = 3LL * s.I * s.d / 16;
+  const uint8_t* codes = static_cast<const uint8_t*>(weights->packed) + expert * cpe;
+  const uint8_t* scales = weights->block_scales + expert * spe;
+  int K;
+  long long nrows;
+  if (matrix == 0) {  // units: gate row, up row
+    codes += static_cast<long long>(row0) * s.d;
+    scales += static_cast<long long>(row0) * s.d / 8;
+    K = s.d;
+    nrows = 2LL * rows;
+  } else {
+    codes += static_cast<long long>(s.I) * s.d + static_cast<long long>(row0) * s.I / 2;
+    scales += static_cast<long long>(s.I) * s.d / 8 + static_cast<long long>(row0) * s.I / 16;
+    K = s.I;
+    nrows = rows;
+  }
+  const long long nv = nrows * (K / 32);
+  if (nv > 0)
+    k_debug_dequant<<<static_cast<unsigned>((nv + 255) / 256), 256, 0, st>>>(codes, scales, K, nrows, out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "k_debug_dequant launch");
+  if (tensor_scale_out) {
+    e = cudaMemcpyAsync(tensor_scale_out, weights->tensor_scales + 3 * expert + (matrix == 0 ? 0 : 2),
+                        (matrix == 0 ? 2 : 1) * sizeof(float), cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync");
+  }
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  return FLINT_OK;
+}
+
+int flint_debug_wait_timeout(void* workspace, int64_t cycles, void* stream) {
+  if (!workspace) return fail(FLINT_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned16(workspace)) return fail(FLINT_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  long long c = cycles < 1 ? 1 : cycles;
+  if (c > kWaitCycles) c = kWaitCycles;
+  k_debug_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<int*>(workspace), c);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "k_debug_wait launch");
+  return FLINT_OK;
+}
+
+}  // extern "C"

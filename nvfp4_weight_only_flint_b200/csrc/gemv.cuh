@@ -1,0 +1,376 @@
+// gemv.cuh -- shared pieces of the small-batch layer path: parameters, the
+// routing descriptor, top-k by warp shuffles, token grouping, lane maps of the
+// gate/up and down GEMVs, and warp reductions.
+#pragma once
+
+#include "common.cuh"
+
+namespace flint {
+
+constexpr int kMaxGemvTokens = 32;   // tokens per call on this path
+constexpr int kMaxExperts = 512;
+constexpr int kMaxTopK = 8;
+constexpr int kMaxPairs = kMaxGemvTokens * kMaxTopK;
+constexpr int kMaxStages = 8;
+constexpr float kRmsEps = 1e-6f;
+
+// Routing result published once per call by the router kernel's last CTA:
+// active experts (routed in ascending id order, then the shared expert), the
+// (token << 8 | slot) pairs of each in ascending token order, and per-token
+// activation scales.
+struct alignas(16) RouteDesc {
+  int n_routed;                                     // routed experts in use
+  int n_active;                                     // + shared experts
+  int act[kMaxExperts + 1];                         // expert id per active slot
+  int off[kMaxExperts + 2];                         // pair offsets per active slot
+  unsigned short pair[kMaxPairs + kMaxGemvTokens];  // (token << 8) | slot
+  float sigma[kMaxGemvTokens];                      // power-of-two f16 staging scale
+  float irms[kMaxGemvTokens];                       // 1/rms(x) with input norm, else 1
+};
+
+// Everything a layer kernel needs; passed by value.
+struct LayerParams {
+  const uint16_t* x;         // [T][d] bf16
+  const uint16_t* wr;        // [E][d] bf16
+  const uint8_t* codes;      // packed E2M1 codes
+  const uint8_t* scales;     // packed E4M3 block scales
+  const float* tscale;       // [E+S][3]
+  const uint16_t* residual;  // [T][d] bf16 or null
+  uint16_t* out;             // [T][d] bf16
+  int* status;               // workspace status word
+  unsigned* counter;         // router arrival counter (workspace, self-resetting)
+  RouteDesc* desc;           // routing descriptor (workspace)
+  float* logits;             // [T][E]
+  int* ids;                  // [T][k]
+  float* gates;              // [T][k]
+  float* h;                  // [T*(k+S)][I] fp32 SwiGLU intermediates
+  int* ids_out;              // optional public copy
+  float* gates_out;          // optional public copy
+  long long cpe;             // code bytes per expert (3*I*d/2)
+  long long spe;             // scale bytes per expert (3*I*d/16)
+  int T, d, I, E, k, S;
+  int input_norm;            // 1: x / rms(x) feeds the router and the experts
+  int x_in_smem;             // gate/up kernel stages x in shared memory
+  int down_nb;               // output rows per down-kernel CTA
+  int down_rb;               // rows per down work item
+  int h_in_smem;             // down kernel stages every h row in shared memory
+  int ns_gateup, ns_down;    // ring depths (stages per warp)
+  int stage_gateup, stage_down;  // stage bytes
+};
+
+// ----------------------------------------------------------------- reductions
+// Transposed butterfly reduction over aligned segments of SEG lanes. Each lane
+// holds V partial values (V a power of two, V <= SEG); afterwards every lane
+// holds the segment total of value index (lane_in_segment >> (log2 SEG - log2 V)).
+// Costs V-1 + log2(SEG/V) shuffles instead of V*log2(SEG).
+template <int O, int N>
+struct XReduce {
+  __device__ static __forceinline__ void run(float* v, int lane) {
+    if constexpr (O == 0) {
+      return;
+    } else if constexpr (N > 1) {
+      const bool up = (lane & O) != 0;
+#pragma unroll
+      for (int i = 0; i < N / 2; ++i) {
+        const float send = up ? v[i] : v[i + N / 2];
+        const float keep = up ? v[i + N / 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+      }
+      XReduce<O / 2, N / 2>::run(v, lane);
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+      XReduce<O / 2, 1>::run(v, lane);
+    }
+  }
+};
+
+template <int SEG, int V>
+__device__ __forceinline__ float xreduce(float* v, int lane) {
+  static_assert(V >= 1 && V <= SEG && (V & (V - 1)) == 0, "V must be a power of two <= SEG");
+  XReduce<SEG / 2, V>::run(v, lane);
+  return v[0];
+}
+
+__host__ __device__ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v / 2); }
+
+// ----------------------------------------------------------------- routing
+// Order-preserving 64-bit key: larger logit first, then lower expert index.
+__device__ __forceinline__ unsigned long long route_key(float v, int e) {
+  if (v == 0.f) v = 0.f;  // -0 and +0 compare equal: one key
+  const uint32_t u = __float_as_uint(v);
+  const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<unsigned long long>(ord) << 32) | static_cast<uint32_t>(0xFFFFFFFFu - e);
+}
+__device__ __forceinline__ float route_key_value(unsigned long long key) {
+  const uint32_t ord = static_cast<uint32_t>(key >> 32);
+  const uint32_t u = (ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord;
+  return __uint_as_float(u);
+}
+__device__ __forceinline__ int route_key_expert(unsigned long long key) {
+  return static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
+}
+
+// One warp: top-k of one token's logits by repeated warp-wide argmax, then the
+// renormalised softmax gates exp(l_j - l_max) / sum_sel exp(l_i - l_max).
+// Results land in ids[0..k) / gates[0..k) (written by lane 0).
+__device__ __forceinline__ void topk_warp(const float* lg, int E, int k, int* ids, float* gates,
+                                          int lane) {
+  constexpr int NE = kMaxExperts / 32;
+  unsigned long long key[NE];
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = (e < E) ? route_key(__ldcg(lg + e), e) : 0ull;
+  }
+  float vals[kMaxTopK];
+  int sel[kMaxTopK];
+#pragma unroll
+  for (int r = 0; r < kMaxTopK; ++r) {
+    vals[r] = 0.f;
+    sel[r] = 0;
+    if (r < k) {
+      unsigned long long best = 0ull;
+#pragma unroll
+      for (int i = 0; i < NE; ++i) best = key[i] > best ? key[i] : best;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+        best = other > best ? other : best;
+      }
+#pragma unroll
+      for (int i = 0; i < NE; ++i)
+        if (key[i] == best) key[i] = 0ull;
+      vals[r] = route_key_value(best);
+      sel[r] = route_key_expert(best);
+    }
+  }
+  float ex[kMaxTopK];
+  float sum = 0.f;
+#pragma unroll
+  for (int r = 0; r < kMaxTopK; ++r) {
+    ex[r] = (r < k) ? expf(vals[r] - vals[0]) : 0.f;
+    sum += ex[r];
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int r = 0; r < kMaxTopK; ++r)
+      if (r < k) {
+        ids[r] = sel[r];
+        gates[r] = ex[r] / sum;
+      }
+  }
+}
+
+// Token grouping built by a whole CTA from ids [T][k] (T <= 32): active
+// experts in ascending id order (then the shared experts, with every token in
+// slot k+s), and for each its (token, slot) pairs in ascending token order.
+struct Grouping {
+  int n_active;
+  int n_routed;
+  int act[kMaxExperts + 1];
+  int off[kMaxExperts + 2];
+  unsigned short pair[kMaxPairs + kMaxGemvTokens];
+  int ecount[kMaxExperts];   // scratch: per-expert count, then offset
+  unsigned emask[kMaxExperts];  // scratch: per-expert token bitmask
+};
+
+__device__ void build_grouping(Grouping& g, const int* ids, int T, int k, int E, int S, int* status) {
+  const int tid = threadIdx.x;
+  for (int e = tid; e < E; e += blockDim.x) {
+    g.ecount[e] = 0;
+    g.emask[e] = 0u;
+  }
+  __syncthreads();
+  for (int i = tid; i < T * k; i += blockDim.x) {
+    const int e = ids[i];
+    if (e < 0 || e >= E) {
+      atomicOr(status, FLINT_DEVCHECK_EXPERT_ID);
+      continue;
+    }
+    atomicAdd(&g.ecount[e], 1);
+    atomicOr(&g.emask[e], 1u << (i / k));
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const int per = (E + 31) / 32;
+    const int e0 = tid * per;
+    int cnt = 0, act = 0;
+    for (int i = 0; i < per; ++i) {
+      const int e = e0 + i;
+      if (e < E) {
+        cnt += g.ecount[e];
+        act += g.ecount[e] > 0;
+      }
+    }
+    int cnt_ex = cnt, act_ex = act;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, cnt_ex, o);
+      const int b = __shfl_up_sync(0xffffffffu, act_ex, o);
+      if (tid >= o) {
+        cnt_ex += a;
+        act_ex += b;
+      }
+    }
+    cnt_ex -= cnt;
+    act_ex -= act;
+    for (int i = 0; i < per; ++i) {
+      const int e = e0 + i;
+      if (e < E) {
+        const int c = g.ecount[e];
+        if (c > 0) {
+          g.act[act_ex] = e;
+          g.off[act_ex] = cnt_ex;
+          ++act_ex;
+        }
+        g.ecount[e] = cnt_ex;
+        cnt_ex += c;
+      }
+    }
+    if (tid == 31) {
+      g.n_routed = act_ex;
+      int na = act_ex, total = cnt_ex;
+      for (int s = 0; s < S; ++s) {
+        g.act[na] = E + s;
+        g.off[na] = total;
+        total += T;
+        ++na;
+      }
+      g.off[na] = total;
+      g.n_active = na;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < T * k; i += blockDim.x) {
+    const int e = ids[i];
+    if (e < 0 || e >= E) continue;
+    const int t = i / k, j = i % k;
+    const int pos = g.ecount[e] + __popc(g.emask[e] & ((1u << t) - 1u));
+    g.pair[pos] = static_cast<unsigned short>((t << 8) | j);
+  }
+  for (int i = tid; i < S * T; i += blockDim.x) {
+    const int s = i / T, t = i % T;
+    g.pair[g.off[g.n_routed + s] + t] = static_cast<unsigned short>((t << 8) | (k + s));
+  }
+  __syncthreads();
+}
+
+// Warp-synchronous token grouping for T*k <= 64 pairs: a bitonic sort of the
+// keys (expert << 16 | token << 8 | slot), two per lane, then run boundaries
+// by ballot. Writes the same descriptor fields as build_grouping.
+__device__ void warp_grouping(const int* ids, int T, int k, int E, int S, RouteDesc* d, int lane,
+                              int* status) {
+  const int n = T * k;
+  uint32_t key[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = 2 * lane + h;
+    uint32_t kv = 0xFFFFFFFFu;
+    if (i < n) {
+      int e = ids[i];
+      if (e < 0 || e >= E) {  // cannot come from top-k; keep indexing in bounds
+        atomicOr(status, FLINT_DEVCHECK_EXPERT_ID);
+        e = 0;
+      }
+      kv = (static_cast<uint32_t>(e) << 16) | (static_cast<uint32_t>(i / k) << 8) | static_cast<uint32_t>(i % k);
+    }
+    key[h] = kv;
+  }
+  // bitonic sort of 64 keys; element index i = 2*lane + h
+#pragma unroll
+  for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+    for (int stride = size / 2; stride > 0; stride >>= 1) {
+      if (stride == 1) {
+        const bool asc = ((2 * lane) & size) == 0;
+        const uint32_t lo = min(key[0], key[1]), hi = max(key[0], key[1]);
+        key[0] = asc ? lo : hi;
+        key[1] = asc ? hi : lo;
+      } else {
+        const int lstride = stride / 2;  // partner lane distance
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int i = 2 * lane + h;
+          const uint32_t other = __shfl_xor_sync(0xffffffffu, key[h], lstride);
+          const bool asc = (i & size) == 0;
+          const bool lower = (i & stride) == 0;
+          key[h] = (asc == lower) ? min(key[h], other) : max(key[h], other);
+        }
+      }
+    }
+  }
+  // run boundaries (new expert) and their ranks
+  const uint32_t prev_b = __shfl_up_sync(0xffffffffu, key[1], 1);
+  const bool valid0 = (2 * lane) < n, valid1 = (2 * lane + 1) < n;
+  const bool b0 = valid0 && (lane == 0 || (key[0] >> 16) != (prev_b >> 16));
+  const bool b1 = valid1 && ((key[1] >> 16) != (key[0] >> 16));
+  const uint32_t m0 = __ballot_sync(0xffffffffu, b0), m1 = __ballot_sync(0xffffffffu, b1);
+  const uint32_t below = (1u << lane) - 1u;
+  const int r0 = __popc(m0 & below) + __popc(m1 & below);  // boundaries before element 2*lane
+  const int r1 = r0 + (b0 ? 1 : 0);
+  const int U = __popc(m0) + __popc(m1);
+  if (b0) {
+    d->act[r0] = static_cast<int>(key[0] >> 16);
+    d->off[r0] = 2 * lane;
+  }
+  if (b1) {
+    d->act[r1] = static_cast<int>(key[1] >> 16);
+    d->off[r1] = 2 * lane + 1;
+  }
+  if (valid0) d->pair[2 * lane] = static_cast<unsigned short>(key[0] & 0xFFFFu);
+  if (valid1) d->pair[2 * lane + 1] = static_cast<unsigned short>(key[1] & 0xFFFFu);
+  for (int i = lane; i < S * T; i += 32) {
+    const int s = i / T, t = i % T;
+    d->pair[n + i] = static_cast<unsigned short>((t << 8) | (k + s));
+  }
+  if (lane == 0) {
+    for (int s = 0; s < S; ++s) {
+      d->act[U + s] = E + s;
+      d->off[U + s] = n + s * T;
+    }
+    d->off[U + S] = n + S * T;
+    d->n_routed = U;
+    d->n_active = U + S;
+  }
+}
+
+// ----------------------------------------------------------------- gate/up lane map
+// A unit is [gate row u | up row u] (D columns each). Lane's j-th 16-byte code
+// vector covers columns 32*cb .. 32*cb+31 of row r, with x column block xi.
+template <int D>
+struct GateUpMap {
+  static constexpr int VR = D / 32;                    // 16-byte code vectors per row
+  static constexpr int NVU = D / 512;                  // vectors per lane per unit
+  static constexpr int XV = (VR >= 32) ? VR / 32 : 1;  // x column blocks per lane
+  static constexpr int XS = XV * 16;                   // f16x2 registers per token
+  static constexpr int TGMAX = (D == 4096) ? 1 : 2;     // tokens per pass
+  static constexpr int CU = (D <= 1024) ? 4 : (D == 2048 ? 2 : 1);  // units per chunk
+  static constexpr int UNIT_CODE = D;
+  static constexpr int UNIT_SCALE = D / 8;
+  static constexpr int UNIT_BYTES = UNIT_CODE + UNIT_SCALE;
+  __device__ static __forceinline__ int xblock(int lane, int xi) {
+    return (VR >= 32) ? lane + 32 * xi : (lane & 15);
+  }
+  __device__ static __forceinline__ void vec(int lane, int j, int& code_off, int& scale_off, int& row,
+                                             int& xi) {
+    int cb;
+    if constexpr (VR >= 32) {
+      row = j / XV;
+      xi = j % XV;
+      cb = lane + 32 * xi;
+    } else {
+      row = lane >> 4;
+      xi = 0;
+      cb = lane & 15;
+    }
+    code_off = row * (D / 2) + cb * 16;
+    scale_off = row * (D / 16) + cb * 2;
+  }
+};
+
+// bf16 words -> f16x2 scaled by sg (element 2i in the low half).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t w, float sg) {
+  return pack_f16x2(bf16_bits_to_f32(w & 0xFFFFu) * sg, __uint_as_float(w & 0xFFFF0000u) * sg);
+}
+
+}  // namespace flint

@@ -82,7 +82,7 @@ def lib():
         L.oracle_expert_ffn.argtypes = [ctypes.POINTER(OracleMatrix), i32, i32, vp, vp]
         L.oracle_expert_ffn.restype = i32
         L.oracle_moe_forward.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp,
-                                         ctypes.POINTER(OracleMatrix), vp, vp, i32,
+                                         ctypes.POINTER(OracleMatrix), vp, vp, i32, i32,
                                          vp, vp, vp, vp, vp]
         L.oracle_moe_forward.restype = i32
         _lib = L
@@ -241,7 +241,7 @@ def expert_ffn(trip, x: np.ndarray) -> np.ndarray:
 
 
 def moe_forward(x_bits, wr_bits, experts, *, d, inter, E, k, S, residual_bits=None,
-                ids_override=None, n_threads=1):
+                ids_override=None, input_norm=False, n_threads=1):
     """experts: list of length E+S; entry e is a (gate, up, down) triple or None (unused)."""
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
     wr_bits = np.ascontiguousarray(wr_bits, dtype=np.uint16)
@@ -258,7 +258,8 @@ def moe_forward(x_bits, wr_bits, experts, *, d, inter, E, k, S, residual_bits=No
     gap = np.zeros(T, dtype=np.float64)
     logits = np.zeros((T, E), dtype=np.float64)
     rc = lib().oracle_moe_forward(T, d, inter, E, k, S, _ptr(x_bits), _ptr(wr_bits), arr,
-                                  _ptr(res), _ptr(ovr), int(n_threads), _ptr(ids), _ptr(gates),
+                                  _ptr(res), _ptr(ovr), int(bool(input_norm)), int(n_threads),
+                                  _ptr(ids), _ptr(gates),
                                   _ptr(gap), _ptr(logits), _ptr(out))
     if rc != 0:
         raise ValueError("oracle_moe_forward failed")

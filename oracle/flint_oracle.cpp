@@ -344,14 +344,33 @@ int oracle_expert_ffn(const oracle_matrix* mats, int32_t d, int32_t inter, const
 
 int oracle_moe_forward(int32_t T, int32_t d, int32_t inter, int32_t E, int32_t k, int32_t S,
                        const uint16_t* x, const uint16_t* wr, const oracle_matrix* mats,
-                       const uint16_t* residual, const int32_t* ids_override, int32_t n_threads,
+                       const uint16_t* residual, const int32_t* ids_override, int32_t input_norm,
+                       int32_t n_threads,
                        int32_t* ids_out, double* gates_out, double* gap_out, double* logits_out,
                        double* out) {
   if (T < 0 || d <= 0 || inter <= 0 || E <= 0 || k < 1 || k > E || S < 0) return -1;
   if (T == 0) return 0;
+  // 0. layer input: x, or x / rms(x) with input_norm
+  std::vector<double> xd(static_cast<size_t>(T) * d);
+  for (size_t i = 0; i < xd.size(); ++i) xd[i] = bf16_bits_to_double(x[i]);
+  if (input_norm) {
+    for (int t = 0; t < T; ++t) {
+      double ms = 0.0;
+      for (int j = 0; j < d; ++j) ms += xd[static_cast<size_t>(t) * d + j] * xd[static_cast<size_t>(t) * d + j];
+      const double r = std::sqrt(ms / d + 1e-6);
+      for (int j = 0; j < d; ++j) xd[static_cast<size_t>(t) * d + j] /= r;
+    }
+  }
   // 1. router logits and top-k gating
   std::vector<double> logits(static_cast<size_t>(T) * E);
-  oracle_router_logits(x, T, wr, d, E, logits.data());
+  std::vector<double> wrd(static_cast<size_t>(E) * d);
+  for (size_t i = 0; i < wrd.size(); ++i) wrd[i] = bf16_bits_to_double(wr[i]);
+  for (int t = 0; t < T; ++t)
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int j = 0; j < d; ++j) acc += xd[static_cast<size_t>(t) * d + j] * wrd[static_cast<size_t>(e) * d + j];
+      logits[static_cast<size_t>(t) * E + e] = acc;
+    }
   std::vector<int32_t> ids(static_cast<size_t>(T) * k);
   std::vector<double> gates(static_cast<size_t>(T) * k), gap(T);
   if (oracle_topk(logits.data(), T, E, k, ids.data(), gates.data(), gap.data())) return -1;
@@ -376,8 +395,6 @@ int oracle_moe_forward(int32_t T, int32_t d, int32_t inter, int32_t E, int32_t k
   }
   // 2. every (token, slot) pair: slots 0..k-1 are the routed experts, k..k+S-1 the shared ones
   const int slots = k + S;
-  std::vector<double> xd(static_cast<size_t>(T) * d);
-  for (size_t i = 0; i < xd.size(); ++i) xd[i] = bf16_bits_to_double(x[i]);
   std::vector<double> y(static_cast<size_t>(T) * slots * d, 0.0);
   // one job per expert in use: decode it once, run it for each token that selected it
   std::vector<std::vector<std::pair<int, int>>> users(E + S);

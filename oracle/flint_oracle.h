@@ -108,7 +108,9 @@ int oracle_expert_ffn(const oracle_matrix* mats, int32_t d, int32_t inter,
                       const double* x, double* y);
 
 /* Whole layer. mats: (E+S)*3 matrices (unused experts may be NULL-pointered).
- * out = sum_j gate_j * FFN_{id_j}(x) + sum_s FFN_{E+s}(x) (+ residual), fp64.
+ * out = sum_j gate_j * FFN_{id_j}(xn) + sum_s FFN_{E+s}(xn) (+ residual), fp64,
+ * where xn = x, or with input_norm = 1 the weightless RMS normalisation
+ * xn = x / sqrt(mean(x^2) + 1e-6) that also feeds the router.
  * ids_override (nullable) forces the routed ids (gates then come from those
  * experts' probabilities, renormalised). ids/gates/gap/logits outputs nullable.
  * n_threads >= 1 spreads the independent (token, expert) FFNs over threads;
@@ -116,7 +118,7 @@ int oracle_expert_ffn(const oracle_matrix* mats, int32_t d, int32_t inter,
 int oracle_moe_forward(int32_t T, int32_t d, int32_t inter, int32_t E, int32_t k,
                        int32_t S, const uint16_t* x, const uint16_t* wr,
                        const oracle_matrix* mats, const uint16_t* residual,
-                       const int32_t* ids_override, int32_t n_threads,
+                       const int32_t* ids_override, int32_t input_norm, int32_t n_threads,
                        int32_t* ids_out, double* gates_out, double* gap_out,
                        double* logits_out, double* out);
 

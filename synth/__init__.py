@@ -121,10 +121,7 @@ def _shape_router(w: np.ndarray, x: np.ndarray, bias: np.ndarray) -> np.ndarray:
     return w + coef.T @ x                           # [E][d]
 
 
-def overlap_targets(seed: int, T: int, E: int, k: int, p_reuse: float):
-    """Per token a set of k target experts; each slot reuses, with probability
-    p_reuse, an expert already picked by another token, else draws a fresh one."""
-    g = rng(seed, "targets", T, E, k)
+def _draw_targets(g, T, E, k, p_reuse):
     sets = []
     used = []
     for t in range(T):
@@ -139,6 +136,20 @@ def overlap_targets(seed: int, T: int, E: int, k: int, p_reuse: float):
             s.append(e)
         sets.append(s)
         used.extend(e for e in s if e not in used)
+    return sets
+
+
+def overlap_targets(seed: int, T: int, E: int, k: int, p_reuse: float, target: float = 0.4,
+                    tol: float = 0.05):
+    """Per token a set of k target experts; each slot reuses, with probability
+    p_reuse, an expert already picked by another token, else draws a fresh one.
+    Draws are repeated (deterministically, by sub-stream) until the fraction of
+    selections shared with another token is within tol of target."""
+    sets = None
+    for attempt in range(1000):
+        sets = _draw_targets(rng(seed, "targets", T, E, k, attempt), T, E, k, p_reuse)
+        if T < 2 or abs(overlap_fraction(np.array(sets)) - target) <= tol:
+            break
     return sets
 
 

@@ -1,0 +1,111 @@
+"""The C ABI library loads, exports every entry point include/*.h declares, and
+rejects bad arguments on the host before touching the GPU (no compute calls)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import nvfp4_weight_only_flint_b200 as fm
+from nvfp4_weight_only_flint_b200 import build as fbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(flint_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def L():
+    fbuild.build()
+    return fm.lib()
+
+
+def test_header_declares_the_layer_calls():
+    names = _declared_functions()
+    for required in ("flint_pack_nvfp4", "flint_moe_route", "flint_moe_forward"):
+        assert required in names
+    assert len(names) >= 12
+
+
+def test_every_declared_symbol_is_exported(L):
+    missing = [n for n in _declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def _shape(d=2048, inter=512, E=256, k=6, S=1, wd=0):
+    return fm.Shape(d, inter, E, k, S, wd)
+
+
+def test_sizes(L):
+    s = _shape()
+    assert fm.flint_packed_bytes(s) == 257 * 3 * 512 * 2048 // 2
+    assert fm.flint_block_scale_bytes(s) == 257 * 3 * 512 * 2048 // 16
+    assert fm.flint_tensor_scale_bytes(s) == 257 * 3 * 4
+    sb = _shape(wd=1)
+    assert fm.flint_packed_bytes(sb) == 257 * 3 * 512 * 2048 * 2
+    assert fm.flint_block_scale_bytes(sb) == 0
+    assert fm.flint_moe_workspace_bytes(s, 8) > fm.flint_moe_workspace_bytes(s, 1) > 0
+
+
+@pytest.mark.parametrize("bad", [dict(d=1000), dict(d=8192), dict(inter=96), dict(E=0), dict(E=513),
+                                 dict(k=0), dict(k=9), dict(E=4, k=5), dict(S=2), dict(wd=7)])
+def test_unsupported_shapes(L, bad):
+    s = _shape(**bad)
+    assert fm.flint_packed_bytes(s) == 0
+    rc = L.flint_moe_forward(None, 1, None, None, ctypes.byref(s), None, None, None, 0, None)
+    assert rc in (-1, -2)
+    assert fm.flint_last_error()
+
+
+def _weights(p=0x10000, b=0x20000, t=0x30000):
+    return fm.Weights(p, b, t)
+
+
+def test_host_validation_errors(L):
+    s = _shape()
+    ws_need = fm.flint_moe_workspace_bytes(s, 4)
+    w = _weights()
+    # NULL pointers
+    assert L.flint_moe_forward(None, 4, 0x40000, ctypes.byref(w), ctypes.byref(s), None, 0x50000,
+                               0x60000, ws_need, None) == -1
+    # misaligned activations
+    assert L.flint_moe_forward(0x40008, 4, 0x40000, ctypes.byref(w), ctypes.byref(s), None, 0x50000,
+                               0x60000, ws_need, None) == -3
+    # workspace too small
+    assert L.flint_moe_forward(0x40000, 4, 0x40000, ctypes.byref(w), ctypes.byref(s), None, 0x50000,
+                               0x60000, ws_need - 1, None) == -4
+    assert "workspace" in fm.flint_last_error()
+    # negative token count; zero tokens is a no-op
+    assert L.flint_moe_forward(0x40000, -1, 0x40000, ctypes.byref(w), ctypes.byref(s), None, 0x50000,
+                               0x60000, ws_need, None) == -1
+    assert L.flint_moe_forward(0x40000, 0, 0x40000, ctypes.byref(w), ctypes.byref(s), None, 0x50000,
+                               0x60000, ws_need, None) == 0
+    # bad path option
+    opt = fm.Options(9, 1, None, None)
+    assert L.flint_moe_forward_ex(0x40000, 4, 0x40000, ctypes.byref(w), ctypes.byref(s), None, 0x50000,
+                                  0x60000, ws_need, ctypes.byref(opt), None) == -1
+    # NVFP4 weights without scales
+    w2 = fm.Weights(0x10000, None, None)
+    assert L.flint_moe_forward(0x40000, 4, 0x40000, ctypes.byref(w2), ctypes.byref(s), None, 0x50000,
+                               0x60000, ws_need, None) == -1
+    # route: NULL outputs
+    assert L.flint_moe_route(0x40000, 4, 0x40000, ctypes.byref(s), None, None, 0x60000, ws_need, None) == -1
+    # packer: wrong weight type
+    sb = _shape(wd=1)
+    assert L.flint_pack_nvfp4(0x40000, 0, ctypes.byref(sb), 0x10000, 0x20000, 0x30000, 0x60000,
+                              ws_need, None) == -1
+    # status without workspace
+    assert L.flint_moe_get_status(None, None, None) == -1
+
+
+def test_version(L):
+    assert "sm_100a" in fm.flint_version()

@@ -146,3 +146,29 @@ def test_packed_layout_offsets():
             assert codes[e * cpe + inter * d + n * inter // 2 + 15] == dn.codes[n, 15]
             assert scales[e * spe + inter * d // 8 + n * inter // 16 + 1] == dn.scales[n, 1]
         assert ts[3 * e: 3 * e + 3].tolist() == [1.0 + e, 1.25 + e, 1.5 + e]
+
+
+def test_input_norm_single_expert_equals_dense_on_normalised_x():
+    # weightless RMS normalisation of the layer input: xn = x / sqrt(mean(x^2) + 1e-6)
+    d, inter = 64, 32
+    ex = _experts(1, d, inter, seed=9)
+    x = synth.x_bits(9, 3, d)
+    res = synth.x_bits(10, 3, d)
+    wr = synth.to_bf16_bits(np.random.default_rng(9).standard_normal((1, d)) * 0.02)
+    r = oracle.moe_forward(x, wr, ex, d=d, inter=inter, E=1, k=1, S=0, residual_bits=res, input_norm=True)
+    xf = synth.bf16_bits_to_f64(x)
+    for t in range(3):
+        xn = xf[t] / np.sqrt(np.mean(xf[t] ** 2) + 1e-6)
+        want = _dense_swiglu(ex[0], xn) + synth.bf16_bits_to_f64(res)[t]
+        np.testing.assert_allclose(r["out"][t], want, rtol=1e-12, atol=1e-13)
+
+
+def test_input_norm_router_sees_normalised_x():
+    d, E = 64, 8
+    x = synth.x_bits(11, 2, d)
+    wr = synth.to_bf16_bits(np.random.default_rng(11).standard_normal((E, d)) * 0.3)
+    ex = _experts(E, d, 32, seed=11)
+    r = oracle.moe_forward(x, wr, ex, d=d, inter=32, E=E, k=2, S=0, input_norm=True)
+    xf = synth.bf16_bits_to_f64(x)
+    rms = np.sqrt(np.mean(xf ** 2, axis=1, keepdims=True) + 1e-6)
+    np.testing.assert_allclose(r["logits"], (xf / rms) @ synth.bf16_bits_to_f64(wr).T, rtol=1e-12)
