@@ -191,6 +191,32 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
                          const uint16_t* residual, uint16_t* out, void* workspace,
                          size_t ws_bytes, const flint_moe_options* options, void* stream);
 
+/* flint_moe_forward_noalloc -- the same layer forward as flint_moe_forward,
+ * for callers that cannot allocate device memory when they call it: runtimes
+ * that hand all device memory to their own pool up front, plug-ins hosted by
+ * an application that forbids allocations on its serving path, or latency-
+ * critical paths that cannot afford an allocation. (This entry point has no
+ * counterpart in the pages; it is a packaging convenience.)
+ *  Instead of a caller workspace it uses a scratch array of 1 MiB compiled into
+ *  the library as a device global: every GPU that loads the library holds those
+ *  1 MiB until the process exits. It allocates nothing: no cudaMalloc, no
+ *  cudaFree, no allocating library routine.
+ *  Arguments as for flint_moe_forward. A call whose scratch would exceed 1 MiB
+ *  (flint_moe_workspace_bytes(shape, T) > 1048576) returns FLINT_ERR_WORKSPACE
+ *  with a message, before any launch.
+ *  The first call on each device looks up the array's device address
+ *  (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *  first call before any stream capture. Each call clears the status word and
+ *  the router counter at the start of the array (an asynchronous memset on
+ *  `stream`), so device check flags are not kept between calls.
+ *  All calls share the one array, which keeps the previous call's contents:
+ *  calls that may run at the same time on the GPU (different streams, or
+ *  different host threads) race on it and corrupt each other's results;
+ *  serialise them on one stream. */
+int flint_moe_forward_noalloc(const uint16_t* x, int32_t T, const uint16_t* router_w,
+                              const flint_moe_weights* weights, const flint_moe_shape* shape,
+                              const uint16_t* residual, uint16_t* out, void* stream);
+
 /* Synchronises `stream`, reads the workspace status word into *device_flags
  * (FLINT_DEVCHECK_* bits, may be NULL) and clears it. Returns FLINT_OK, or
  * FLINT_ERR_TIMEOUT / FLINT_ERR_DEVICE_CHECK when a flag was set. */

@@ -19,7 +19,7 @@ __all__ = [
     "FLINT_W_NVFP4", "FLINT_W_BF16", "FLINT_PATH_AUTO", "FLINT_PATH_GEMV", "FLINT_PATH_MMA",
     "flint_packed_bytes", "flint_block_scale_bytes", "flint_tensor_scale_bytes",
     "flint_moe_workspace_bytes", "flint_moe_workspace_init", "flint_pack_nvfp4", "flint_pack_bf16", "flint_moe_route",
-    "flint_moe_forward", "flint_moe_forward_ex", "flint_moe_get_status", "flint_last_error",
+    "flint_moe_forward", "flint_moe_forward_ex", "flint_moe_forward_noalloc", "flint_moe_get_status", "flint_last_error",
     "flint_debug_dequant", "flint_debug_wait_timeout", "flint_version",
 ]
 
@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.flint_moe_forward_ex.argtypes = [vp, i32, vp, P(Weights), P(Shape), vp, vp, vp, sz,
                                            P(Options), vp]
         L.flint_moe_forward_ex.restype = i32
+        L.flint_moe_forward_noalloc.argtypes = [vp, i32, vp, P(Weights), P(Shape), vp, vp, vp]
+        L.flint_moe_forward_noalloc.restype = i32
         L.flint_moe_workspace_init.argtypes = [vp, sz, vp]
         L.flint_moe_workspace_init.restype = i32
         L.flint_moe_get_status.argtypes = [vp, P(i32), vp]
@@ -188,6 +190,13 @@ def flint_moe_forward_ex(x, T: int, router_w, weights: Weights, shape: Shape, re
                                       _ptr(workspace), _nbytes(workspace),
                                       ctypes.byref(options) if options is not None else None,
                                       _stream(stream)))
+
+
+def flint_moe_forward_noalloc(x, T: int, router_w, weights: Weights, shape: Shape, residual, out,
+                              stream=None) -> None:
+    _check(lib().flint_moe_forward_noalloc(_ptr(x), int(T), _ptr(router_w), ctypes.byref(weights),
+                                           ctypes.byref(shape), _ptr(residual), _ptr(out),
+                                           _stream(stream)))
 
 
 def flint_moe_get_status(workspace, stream=None) -> tuple[int, int]:

@@ -700,6 +700,62 @@ int flint_debug_dequant(const flint_moe_weights* weights, const flint_moe_shape*
   return FLINT_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Layer forward for callers that cannot allocate device memory: the scratch
+// lives in a fixed, file-scope device array instead of a caller workspace.
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace flint {
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB, held by every device that loads the library
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {nullptr};
+}  // namespace
+}  // namespace flint
+
+extern "C" {
+
+int flint_moe_forward_noalloc(const uint16_t* x, int32_t T, const uint16_t* router_w,
+                              const flint_moe_weights* weights, const flint_moe_shape* shape,
+                              const uint16_t* residual, uint16_t* out, void* stream) {
+  Dims s;
+  int rc = check_shape(shape, &s);
+  if (rc != FLINT_OK) return rc;
+  if (T < 0) return fail(FLINT_ERR_INVALID_ARG, "T=%d", T);
+  if (T == 0) return FLINT_OK;
+  const size_t need = ws_layout(s, T).total;
+  if (need > kNoAllocScratchBytes)
+    return fail(FLINT_ERR_WORKSPACE,
+                "flint_moe_forward_noalloc: this call needs %zu bytes of scratch; the built-in scratch holds %zu "
+                "(use flint_moe_forward with a caller workspace)",
+                need, kNoAllocScratchBytes);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(FLINT_ERR_INVALID_ARG, "device ordinal %d out of range", dev);
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+      // Host code cannot use the array's name as a device address: look the
+      // address up once per device, with that device current.
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+      g_noalloc_addr[dev] = p;
+    }
+    scratch = g_noalloc_addr[dev];
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The status word and the router's arrival counter must start at zero.
+  e = cudaMemsetAsync(scratch, 0, 256, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  return flint_moe_forward_ex(x, T, router_w, weights, shape, residual, out, scratch, kNoAllocScratchBytes,
+                              nullptr, stream);
+}
+
 int flint_debug_wait_timeout(void* workspace, int64_t cycles, void* stream) {
   if (!workspace) return fail(FLINT_ERR_INVALID_ARG, "workspace is NULL");
   if (!aligned16(workspace)) return fail(FLINT_ERR_MISALIGNED, "workspace must be 16-byte aligned");
