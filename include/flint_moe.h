@@ -120,13 +120,16 @@ typedef struct flint_moe_options {
                             kernels with programmatic dependent launch */
   int32_t* topk_ids;     /* optional device int32 [T][top_k]: routed ids written here */
   float* topk_weights;   /* optional device float [T][top_k]: their gates */
+  int32_t split_kernels; /* 1: run batch <= 8 as three kernels chained with programmatic
+                            dependent launch instead of one persistent kernel */
   int32_t input_rmsnorm; /* 1: each token's x is divided by its RMS, sqrt(mean(x^2) + 1e-6)
                             (no learned weight), before the router and the experts;
                             the residual is added unnormalised. 0 (default): no norm */
   void* profile_events;  /* optional cudaEvent_t[2], recorded on `stream` just before
-                            and just after the layer's gate/up kernel (the one that
-                            streams most of the weights); the record between kernels
-                            serialises them, so use it for per-kernel timing only */
+                            and just after the kernel that streams the expert weights
+                            (the persistent layer kernel, or the gate/up kernel of the
+                            three-kernel path, whose records then serialise the chain);
+                            for per-kernel timing */
 } flint_moe_options;
 
 /* Bytes of the packed codes / block scales / tensor scales for a shape. Return 0
@@ -160,9 +163,12 @@ int flint_pack_bf16(const uint16_t* w, const flint_moe_shape* shape, uint16_t* p
  * must not be shared by calls that may overlap on the GPU. */
 size_t flint_moe_workspace_bytes(const flint_moe_shape* shape, int32_t max_tokens);
 
-/* Clears the workspace's status word (its first 256 bytes). Call once after
- * allocating a workspace, before its first use; kernels only ever set bits in
- * it, and flint_moe_get_status reads and clears it. */
+/* Clears the workspace's control block (its first 1024 bytes: the status word,
+ * the router's arrival counter and the persistent kernel's grid-barrier epoch
+ * flags). Call once after allocating a workspace, before its first use, and
+ * again after a call reported FLINT_DEVCHECK_WAIT (a CTA that gave up a wait
+ * leaves the epochs unequal). Kernels only ever set bits in the status word,
+ * and flint_moe_get_status reads and clears it. */
 int flint_moe_workspace_init(void* workspace, size_t ws_bytes, void* stream);
 
 /* flint_moe_route -- the router alone.

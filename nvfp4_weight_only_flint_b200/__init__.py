@@ -49,7 +49,8 @@ class Weights(ctypes.Structure):
 class Options(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("use_pdl", ctypes.c_int32),
                 ("topk_ids", ctypes.c_void_p), ("topk_weights", ctypes.c_void_p),
-                ("input_rmsnorm", ctypes.c_int32), ("profile_events", ctypes.c_void_p)]
+                ("split_kernels", ctypes.c_int32), ("input_rmsnorm", ctypes.c_int32),
+                ("profile_events", ctypes.c_void_p)]
 
 
 _lib = None

@@ -7,10 +7,11 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <string>
 
-#include "layer_kernels.cuh"
+#include "fused_layer.cuh"
 
 namespace flint {
 
@@ -233,16 +234,19 @@ struct WsLayout {
 };
 
 size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+constexpr size_t kCtrlBytes = 64 + 4 * kMaxGridFlags;
 
-// Workspace carve-up for calls of up to maxT tokens. The first 256 bytes hold
-// the status word (byte 0) and the router's arrival counter (byte 4); both
-// start at zero (flint_moe_workspace_init) and are left at zero by every call.
+// Workspace carve-up for calls of up to maxT tokens. The first kCtrlBytes hold
+// the control block: the status word (byte 0), the router's arrival counter
+// (byte 4, left at zero by every call) and, from byte 64, one grid-barrier
+// epoch flag per CTA of the persistent layer kernel (each call advances them
+// by 2). All start at zero (flint_moe_workspace_init).
 WsLayout ws_layout(const Dims& s, int maxT) {
   WsLayout w{};
   size_t o = 0;
   w.status = 0;
   w.counter = 4;
-  o += 256;
+  o += kCtrlBytes;
   w.amax = o;
   o += al256(sizeof(float) * (s.E + s.S) * 3);
   w.desc = o;
@@ -382,6 +386,77 @@ size_t down_smem(const LayerParams& p) {
   const size_t ybytes = ((sizeof(float) * static_cast<size_t>(p.T) * (p.k + p.S) * p.down_nb) + 127) & ~static_cast<size_t>(127);
   return sizeof(RouteDesc) + (p.h_in_smem ? static_cast<size_t>(p.T) * (p.k + p.S) * p.I * 4 : 0) + ybytes +
          static_cast<size_t>(kGemvWarps) * p.ns_down * p.stage_down;
+}
+
+// Configuration of the persistent single-kernel layer (T <= 8): returns the
+// dynamic shared-memory bytes, or 0 if the call does not fit it.
+size_t configure_fused(LayerParams& p, const Dims& s, int T) {
+  const int sms = num_sms();
+  if (sms > kMaxGridFlags) return 0;
+  p.stage_gateup = gateup_stage_bytes(s.d);
+  p.ns_gateup = 2;
+  const int rps = 32 / (s.I / 32);
+  int nb = (s.d + sms - 1) / sms;
+  nb = ((nb + rps - 1) / rps) * rps;
+  if (nb % 2) nb += rps;
+  p.down_nb = nb;
+  p.down_rb = (4 * rps < nb) ? 4 * rps : nb;
+  p.stage_down = ((p.down_rb * (s.I / 2 + s.I / 16)) + 15) & ~15;
+  p.ns_down = 2;
+  const size_t a128 = 127;
+  const size_t head = sizeof(RouteDesc) + ((static_cast<size_t>(T) * s.d * 2 + a128) & ~a128) +
+                      static_cast<size_t>((s.E + sms - 1) / sms) * s.d * 2;
+  const size_t ybytes = ((4 * static_cast<size_t>(T) * (s.k + s.S) * nb) + a128) & ~a128;
+  const size_t hbytes = static_cast<size_t>(T) * (s.k + s.S) * s.I * 4;
+  const size_t ring_d = static_cast<size_t>(kFusedWarps) * p.ns_down * p.stage_down;
+  const size_t budget = 210 * 1024;
+  // deeper gate/up rings while they fit (the down ring takes the next 2 of
+  // each warp's kMaxStages barriers)
+  while (p.ns_gateup < kMaxStages - 2 && p.ns_gateup < 4 &&
+         head + static_cast<size_t>(kFusedWarps) * (p.ns_gateup + 1) * p.stage_gateup <= budget)
+    ++p.ns_gateup;
+  const size_t ring_g = static_cast<size_t>(kFusedWarps) * p.ns_gateup * p.stage_gateup;
+  p.h_in_smem = (head + std::max(ring_g, hbytes + ybytes + ring_d) <= budget) ? 1 : 0;
+  const size_t work = std::max(ring_g, (p.h_in_smem ? hbytes : 0) + ybytes + ring_d);
+  if (head + work > budget) return 0;
+  return head + work;
+}
+
+template <int D, int I>
+cudaError_t launch_fused_di(const LayerParams& p, size_t smem, cudaStream_t st) {
+  auto kern = k_layer<D, I>;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms());
+  cfg.blockDim = dim3(kFusedWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+template <int D>
+cudaError_t launch_fused_d(const LayerParams& p, size_t smem, cudaStream_t st) {
+  switch (p.I) {
+    case 128: return launch_fused_di<D, 128>(p, smem, st);
+    case 256: return launch_fused_di<D, 256>(p, smem, st);
+    case 512: return launch_fused_di<D, 512>(p, smem, st);
+    default: return launch_fused_di<D, 1024>(p, smem, st);
+  }
+}
+
+cudaError_t launch_fused(const LayerParams& p, size_t smem, cudaStream_t st) {
+  switch (p.d) {
+    case 512: return launch_fused_d<512>(p, smem, st);
+    case 1024: return launch_fused_d<1024>(p, smem, st);
+    case 2048: return launch_fused_d<2048>(p, smem, st);
+    default: return launch_fused_d<4096>(p, smem, st);
+  }
 }
 
 template <typename K>
@@ -603,10 +678,26 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
     p.gates_out = options->topk_weights;
   }
   p.input_norm = (options && options->input_rmsnorm) ? 1 : 0;
-  configure(p, s, T);
-
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaEvent_t* ev = options ? static_cast<cudaEvent_t*>(options->profile_events) : nullptr;
+  const bool split = options && options->split_kernels;
+  if (T <= kFusedMaxTokens && !split) {
+    const size_t smem = configure_fused(p, s, T);
+    if (smem > 0) {
+      if (ev) {
+        cudaError_t e = cudaEventRecord(ev[0], st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+      }
+      cudaError_t e = launch_fused(p, smem, st);
+      if (e != cudaSuccess) return cuda_fail(e, "k_layer launch");
+      if (ev) {
+        e = cudaEventRecord(ev[1], st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+      }
+      return FLINT_OK;
+    }
+  }
+  configure(p, s, T);
   cudaError_t e = launch_route_fwd(p, st, pdl);
   if (e != cudaSuccess) return cuda_fail(e, "k_route launch");
   if (ev) {
@@ -634,8 +725,8 @@ int flint_moe_forward(const uint16_t* x, int32_t T, const uint16_t* router_w, co
 int flint_moe_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
   if (!workspace) return fail(FLINT_ERR_INVALID_ARG, "workspace is NULL");
   if (!aligned16(workspace)) return fail(FLINT_ERR_MISALIGNED, "workspace must be 16-byte aligned");
-  if (ws_bytes < 256) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < 256 bytes", ws_bytes);
-  cudaError_t e = cudaMemsetAsync(workspace, 0, 256, static_cast<cudaStream_t>(stream));
+  if (ws_bytes < kCtrlBytes) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kCtrlBytes);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kCtrlBytes, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   return FLINT_OK;
 }
@@ -749,8 +840,8 @@ int flint_moe_forward_noalloc(const uint16_t* x, int32_t T, const uint16_t* rout
     scratch = g_noalloc_addr[dev];
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // The status word and the router's arrival counter must start at zero.
-  e = cudaMemsetAsync(scratch, 0, 256, st);
+  // The control block (status word, router counter, barrier flags) must start at zero.
+  e = cudaMemsetAsync(scratch, 0, kCtrlBytes, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   return flint_moe_forward_ex(x, T, router_w, weights, shape, residual, out, scratch, kNoAllocScratchBytes,
                               nullptr, stream);

@@ -94,33 +94,30 @@ __device__ __forceinline__ float xreduce(float* v, int lane) {
 __host__ __device__ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v / 2); }
 
 // ----------------------------------------------------------------- routing
-// Order-preserving 64-bit key: larger logit first, then lower expert index.
-__device__ __forceinline__ unsigned long long route_key(float v, int e) {
-  if (v == 0.f) v = 0.f;  // -0 and +0 compare equal: one key
+// One warp, one token: top-k (k <= 8) of E <= 32*NE logits by k rounds of a
+// warp-wide argmax. Each lane keeps its NE order-preserving 32-bit logit codes
+// (larger logit = larger code, -0 == +0) and its current best; a round takes
+// the warp maximum of the codes with redux.sync, then among the lanes holding
+// that code the lowest expert index (a second redux over 0xFFFFFFFF - e), and
+// the lane that owns the winner drops it. Gates are the renormalised softmax
+// exp(l_j - l_max) / sum_sel exp(l_i - l_max). Lanes 0..k-1 write ids/gates.
+__device__ __forceinline__ uint32_t route_code(float v) {
+  if (v == 0.f) v = 0.f;
   const uint32_t u = __float_as_uint(v);
-  const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  return (static_cast<unsigned long long>(ord) << 32) | static_cast<uint32_t>(0xFFFFFFFFu - e);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-__device__ __forceinline__ float route_key_value(unsigned long long key) {
-  const uint32_t ord = static_cast<uint32_t>(key >> 32);
-  const uint32_t u = (ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord;
-  return __uint_as_float(u);
-}
-__device__ __forceinline__ int route_key_expert(unsigned long long key) {
-  return static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
+__device__ __forceinline__ float route_code_value(uint32_t ord) {
+  return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
 }
 
-// One warp: top-k of one token's logits by repeated warp-wide argmax, then the
-// renormalised softmax gates exp(l_j - l_max) / sum_sel exp(l_i - l_max).
-// Results land in ids[0..k) / gates[0..k) (written by lane 0).
-__device__ __forceinline__ void topk_warp(const float* lg, int E, int k, int* ids, float* gates,
-                                          int lane) {
-  constexpr int NE = kMaxExperts / 32;
-  unsigned long long key[NE];
+template <int NE>
+__device__ __forceinline__ void topk_warp(const float* lg, int E, int k, int* ids, float* gates, int lane) {
+  uint32_t code[NE];
 #pragma unroll
   for (int i = 0; i < NE; ++i) {
     const int e = lane + 32 * i;
-    key[i] = (e < E) ? route_key(__ldcg(lg + e), e) : 0ull;
+    // code 0 marks "absent"; a finite logit's code is never 0
+    code[i] = (e < E) ? max(route_code(__ldcg(lg + e)), 1u) : 0u;
   }
   float vals[kMaxTopK];
   int sel[kMaxTopK];
@@ -129,36 +126,53 @@ __device__ __forceinline__ void topk_warp(const float* lg, int E, int k, int* id
     vals[r] = 0.f;
     sel[r] = 0;
     if (r < k) {
-      unsigned long long best = 0ull;
+      uint32_t best = code[0];
+      int bi = 0;
 #pragma unroll
-      for (int i = 0; i < NE; ++i) best = key[i] > best ? key[i] : best;
+      for (int i = 1; i < NE; ++i)
+        if (code[i] > best) {  // strict: equal codes keep the lower index
+          best = code[i];
+          bi = i;
+        }
+      const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+      const uint32_t w = __reduce_max_sync(0xffffffffu, best == m ? 0xFFFFFFFFu - (lane + 32 * bi) : 0u);
+      const int e = static_cast<int>(0xFFFFFFFFu - w);
+      if ((e & 31) == lane) {
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-        best = other > best ? other : best;
+        for (int i = 0; i < NE; ++i)
+          if (i == (e >> 5)) code[i] = 0u;
       }
-#pragma unroll
-      for (int i = 0; i < NE; ++i)
-        if (key[i] == best) key[i] = 0ull;
-      vals[r] = route_key_value(best);
-      sel[r] = route_key_expert(best);
+      vals[r] = route_code_value(m);
+      sel[r] = e;
     }
   }
   float ex[kMaxTopK];
   float sum = 0.f;
 #pragma unroll
   for (int r = 0; r < kMaxTopK; ++r) {
-    ex[r] = (r < k) ? expf(vals[r] - vals[0]) : 0.f;
+    ex[r] = (r < k) ? __expf(vals[r] - vals[0]) : 0.f;
     sum += ex[r];
   }
-  if (lane == 0) {
+  const float inv = 1.f / sum;
+  if (lane < k) {
+    int id = 0;
+    float gt = 0.f;
 #pragma unroll
     for (int r = 0; r < kMaxTopK; ++r)
-      if (r < k) {
-        ids[r] = sel[r];
-        gates[r] = ex[r] / sum;
+      if (r == lane) {
+        id = sel[r];
+        gt = ex[r] * inv;
       }
+    ids[lane] = id;
+    gates[lane] = gt;
   }
+}
+
+__device__ __forceinline__ void topk_token(const float* lg, int E, int k, int* ids, float* gates, int lane) {
+  if (E <= 256)
+    topk_warp<8>(lg, E, k, ids, gates, lane);
+  else
+    topk_warp<kMaxExperts / 32>(lg, E, k, ids, gates, lane);
 }
 
 // Token grouping built by a whole CTA from ids [T][k] (T <= 32): active

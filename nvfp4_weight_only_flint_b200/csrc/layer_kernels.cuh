@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(256) k_topk(LayerParams p) {
   pdl_trigger();
   const int t = blockIdx.x * 8 + warp;
   if (t >= p.T) return;
-  topk_warp(p.logits + static_cast<size_t>(t) * p.E, p.E, p.k, p.ids + static_cast<size_t>(t) * p.k,
+  topk_token(p.logits + static_cast<size_t>(t) * p.E, p.E, p.k, p.ids + static_cast<size_t>(t) * p.k,
             p.gates + static_cast<size_t>(t) * p.k, lane);
 }
 
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32, 1) k_route(LayerParams p) {
   if (!s_last) return;
   __threadfence();
   for (int t = warp; t < T; t += kRouteWarps)
-    topk_warp(p.logits + static_cast<size_t>(t) * E, E, k, &s_ids[t * k], &s_gates[t * k], lane);
+    topk_token(p.logits + static_cast<size_t>(t) * E, E, k, &s_ids[t * k], &s_gates[t * k], lane);
   __syncthreads();
   for (int i = tid; i < T * k; i += blockDim.x) {
     p.ids[i] = s_ids[i];

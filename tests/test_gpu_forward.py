@@ -25,10 +25,10 @@ def _layer(name, seed=0, **kw):
     return _LAYERS[key]
 
 
-def _run_and_check(layer, x_bits, wr_bits, residual_bits=None, path=fm.FLINT_PATH_AUTO, what=""):
+def _run_and_check(layer, x_bits, wr_bits, residual_bits=None, path=fm.FLINT_PATH_AUTO, what="", split=False):
     x, wr = bits_to_cuda(x_bits), bits_to_cuda(wr_bits)
     res = bits_to_cuda(residual_bits) if residual_bits is not None else None
-    out, ids, gates = layer.forward(x, wr, residual=res, path=path)
+    out, ids, gates = layer.forward(x, wr, residual=res, path=path, split=split)
     torch.cuda.synchronize()
     ids_np, gates_np = ids.cpu().numpy(), gates.cpu().numpy()
     near = check_routing(ids_np, gates_np, oracle.router_logits(x_bits, wr_bits), layer.w.k)
@@ -62,6 +62,19 @@ def test_forward_cfg2_batch8_overlap():
     _, ids, _, _ = _run_and_check(layer, x, wr, what="cfg2")
     assert 0.3 <= synth.overlap_fraction(ids) <= 0.5
     assert len(set(ids.ravel().tolist())) < w.T * w.k
+
+
+@pytest.mark.parametrize("name,T", [("cfg1", 1), ("cfg2", 8), ("cfg0", 4)])
+def test_forward_split_kernel_path(name, T):
+    # batch <= 8 runs as one persistent kernel by default; the three-kernel
+    # path must give the same results within the tolerance
+    w = synth.CONFIGS[name]
+    layer = _layer("cfg0" if name == "cfg0" else "cfg1", max_tokens=32)
+    x = synth.x_bits(40 + T, T, w.d)
+    wr = synth.make_router(w, 40, x)
+    a, ids_a, _, _ = _run_and_check(layer, x, wr, what=f"{name} fused")
+    b, ids_b, _, _ = _run_and_check(layer, x, wr, what=f"{name} split", split=True)
+    assert np.array_equal(ids_a, ids_b)
 
 
 @pytest.mark.parametrize("T", [2, 3, 5, 9, 13, 31])
