@@ -50,6 +50,22 @@ def _peaks():
         return 6650.0, "fallback"
 
 
+def _tensor_peak(wdtype: str):
+    """Dense tensor peak (TFLOP/s) of the MMA's operand type: the measured bf16
+    figure (f16 runs at the same rate on tcgen05 kind::f16)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), "measured (bf16 burst; f16 operands run at the bf16 rate)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+# DRAM bytes (read + write) of one k_layer launch at batch 1, from the ncu
+# capture summarised in profiles/; None until a capture of the current kernel.
+TRAFFIC_K_LAYER_T1 = None
+
+
 def _host_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -111,31 +127,45 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- flint arm
 class Stack:
-    """`n` independently drawn layers of one shape, packed NVFP4, resident on the GPU."""
+    """`n` independently drawn layers of one shape, packed NVFP4 (or laid out in
+    bf16), resident on the GPU."""
 
-    def __init__(self, w: synth.Workload, n: int, seed: int, max_tokens: int):
+    def __init__(self, w: synth.Workload, n: int, seed: int, max_tokens: int, wdtype: str = "nvfp4"):
         import torch
         import nvfp4_weight_only_flint_b200 as fm
-        self.fm, self.w = fm, w
-        self.shape = fm.Shape(w.d, w.inter, w.E, w.k, w.S, fm.FLINT_W_NVFP4)
+        self.fm, self.w, self.wdtype = fm, w, wdtype
+        self.shape = fm.Shape(w.d, w.inter, w.E, w.k, w.S, fm.FLINT_W_NVFP4 if wdtype == "nvfp4" else fm.FLINT_W_BF16)
         self.ws = torch.empty(fm.flint_moe_workspace_bytes(self.shape, max_tokens), dtype=torch.uint8, device="cuda")
         fm.flint_moe_workspace_init(self.ws)
         self.layers = []
         for l in range(n):
             wf = synth.layer_weights_torch(seed, l, w.E + w.S, w.d, w.inter, w.std, device="cuda")
-            packed = torch.empty(fm.flint_packed_bytes(self.shape), dtype=torch.uint8, device="cuda")
-            scales = torch.empty(fm.flint_block_scale_bytes(self.shape), dtype=torch.uint8, device="cuda")
-            ts = torch.empty((w.E + w.S) * 3, dtype=torch.float32, device="cuda")
-            fm.flint_pack_nvfp4(wf, 0, self.shape, packed, scales, ts, self.ws)
+            if wdtype == "nvfp4":
+                packed = torch.empty(fm.flint_packed_bytes(self.shape), dtype=torch.uint8, device="cuda")
+                scales = torch.empty(fm.flint_block_scale_bytes(self.shape), dtype=torch.uint8, device="cuda")
+                ts = torch.empty((w.E + w.S) * 3, dtype=torch.float32, device="cuda")
+                fm.flint_pack_nvfp4(wf, 0, self.shape, packed, scales, ts, self.ws)
+                wts = fm.Weights(packed.data_ptr(), scales.data_ptr(), ts.data_ptr())
+            else:
+                wb = wf.to(torch.bfloat16)
+                packed = torch.empty(fm.flint_packed_bytes(self.shape) // 2, dtype=torch.int16, device="cuda")
+                fm.flint_pack_bf16(wb.view(torch.int16), self.shape, packed)
+                torch.cuda.synchronize()
+                del wb
+                scales = ts = None
+                wts = fm.Weights(packed.data_ptr(), None, None)
             del wf
-            self.layers.append((packed, scales, ts, fm.Weights(packed.data_ptr(), scales.data_ptr(), ts.data_ptr())))
+            self.layers.append((packed, scales, ts, wts))
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
 
     def expert_bytes(self):
+        """(gate+up, down) bytes of one expert: codes and block scales, or bf16."""
         w = self.w
-        gu = w.inter * w.d // 2 * 2 + w.inter * w.d // 16 * 2     # gate+up codes and scales
-        dn = w.inter * w.d // 2 + w.inter * w.d // 16             # down codes and scales
+        if self.wdtype == "bf16":
+            return 2 * w.inter * w.d * 2, w.inter * w.d * 2
+        gu = w.inter * w.d // 2 * 2 + w.inter * w.d // 16 * 2
+        dn = w.inter * w.d // 2 + w.inter * w.d // 16
         return gu, dn
 
 
@@ -213,9 +243,11 @@ def run_chain(stack: Stack, routers, T: int, K: int, W: int, sampler=None, resid
     return ms, clocks
 
 
-def gateup_kernel_timing(stack: Stack, routers, T: int, n_calls: int, fixed_inputs=None, norm: int = 0):
-    """Per-launch duration of the gate/up kernel (CUDA events on the launching
-    stream around each launch) and its algorithmic bytes per launch."""
+def kernel_timing(stack: Stack, routers, T: int, n_calls: int, fixed_inputs=None, norm: int = 0):
+    """Per-launch duration of the kernel that streams the expert weights (CUDA
+    events the library records on the launching stream around it: the
+    persistent layer kernel at T <= 8, the gate/up tensor-core kernel from 32)
+    and its algorithmic bytes and flops per launch."""
     import torch
     fm = stack.fm
     L = len(stack.layers)
@@ -245,23 +277,32 @@ def gateup_kernel_timing(stack: Stack, routers, T: int, n_calls: int, fixed_inpu
     torch.cuda.synchronize()
     ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(n_calls)]
     ids_np = ids.cpu().numpy()
-    byt = []
+    byt, flops = [], []
+    P = T * (w.k + w.S)
     for i in range(n_calls):
         U = len(np.unique(ids_np[i]))
-        # routed gate/up streamed by the kernel + the down rows of every active
-        # expert it prefetches into L2 + activations in (x) and out (h, fp32)
-        byt.append(U * gu + (U + w.S) * dn + T * w.d * 2 + T * (w.k + w.S) * w.inter * 4)
+        if T <= 8:
+            # the whole layer: union of the selected experts + the shared one, x in, out
+            byt.append(step_bytes(w, ids_np[i], stack.wdtype))
+            flops.append(2.0 * P * 3 * w.inter * w.d)
+        else:
+            # gate/up on the tensor cores: the union's gate/up weights, the
+            # gathered activation rows (16-bit) in, h (fp32) out
+            byt.append((U + w.S) * gu + P * w.d * 2 + P * w.inter * 4)
+            flops.append(2.0 * P * 2 * w.inter * w.d)
     skip = min(n_calls // 4, L)  # first launches warm the code paths
-    return float(np.mean(ms[skip:])), float(np.mean(byt[skip:])), ids_np
+    return float(np.mean(ms[skip:])), float(np.mean(byt[skip:])), float(np.mean(flops[skip:])), ids_np
 
 
-def step_bytes(w: synth.Workload, ids_np):
-    """North-star byte count of one step: union of selected experts' weights and
+def step_bytes(w: synth.Workload, ids_np, wdtype: str = "nvfp4"):
+    """Byte count of one step: union of the selected experts' weights and
     scales plus the shared expert's, plus x in and out (bf16)."""
-    gu = w.inter * w.d // 2 * 2 + w.inter * w.d // 16 * 2
-    dn = w.inter * w.d // 2 + w.inter * w.d // 16
+    if wdtype == "bf16":
+        per = 3 * w.inter * w.d * 2
+    else:
+        per = 3 * (w.inter * w.d // 2 + w.inter * w.d // 16)
     U = len(np.unique(ids_np))
-    return (U + w.S) * (gu + dn) + 2 * ids_np.shape[0] * w.d * 2
+    return (U + w.S) * per + 2 * ids_np.shape[0] * w.d * 2
 
 
 def run_e2e(stack: Stack, routers, T: int, K: int, norm: int = 0):
@@ -387,7 +428,7 @@ def main():
     ms_step = ms / K
 
     # per-kernel timing of the dominant kernel and byte counts
-    gk_ms, gk_bytes, ids_np = gateup_kernel_timing(stack, routers1, 1, 4 * N_LAYERS, norm=1)
+    gk_ms, gk_bytes, _, ids_np = kernel_timing(stack, routers1, 1, 4 * N_LAYERS, norm=1)
     peak, peak_kind = _peaks()
     sb = np.mean([step_bytes(w1, ids_np[i]) for i in range(ids_np.shape[0])])
     step_gbs = sb / (ms_step / 1e3) / 1e9
@@ -405,7 +446,7 @@ def main():
         K8 = 2 * N_LAYERS * 40
         ms8, _ = run_chain(stack, r8, w2.T, K8, 2 * N_LAYERS, fixed_inputs=fx8)
         ms8 = _max_over_ranks(ms8)
-        g8_ms, g8_bytes, ids8 = gateup_kernel_timing(stack, r8, w2.T, 2 * N_LAYERS, fixed_inputs=fx8)
+        g8_ms, g8_bytes, _, ids8 = kernel_timing(stack, r8, w2.T, 2 * N_LAYERS, fixed_inputs=fx8)
         sb8 = np.mean([step_bytes(w2, ids8[i]) for i in range(ids8.shape[0])])
         unions = [len(np.unique(ids8[i])) for i in range(ids8.shape[0])]
         ov = [synth.overlap_fraction(ids8[i]) for i in range(ids8.shape[0])]
@@ -416,13 +457,45 @@ def main():
                             "frac_of_8tbs": sb8 / (ms8 / K8 / 1e3) / 1e9 / NOMINAL_HBM_GBS,
                             "frac_of_peak": sb8 / (ms8 / K8 / 1e3) / 1e9 / peak,
                             "union_experts_mean": float(np.mean(unions)), "overlap_mean": float(np.mean(ov)),
-                            "gateup_kernel": {"us": g8_ms * 1e3, "bytes": g8_bytes,
-                                              "gbs": g8_bytes / (g8_ms / 1e3) / 1e9}}
+                            "layer_kernel": {"name": "k_layer", "us": g8_ms * 1e3, "bytes": g8_bytes,
+                                             "gbs": g8_bytes / (g8_ms / 1e3) / 1e9,
+                                             "frac_of_peak": g8_bytes / (g8_ms / 1e3) / 1e9 / peak}}
         # 47-layer stack at batch 4 (residual chain)
         w4 = synth.CONFIGS["cfg3_t4"]
         K4 = 2 * N_LAYERS * 40
         ms4, _ = run_chain(stack, routers1, w4.T, K4, 2 * N_LAYERS, norm=1)
         ms4 = _max_over_ranks(ms4)
+        # batch 64 on the tensor cores (config 4: Zipf-skewed routing), NVFP4
+        # and bf16 weights; 8 resident layers used in turn (inputs > L2)
+        w4n = synth.CONFIGS["cfg4_nvfp4"]
+        extras["batch64"] = {}
+        del stack
+        torch.cuda.empty_cache()
+        for wd in ("nvfp4", "bf16"):
+            st64 = Stack(w4n, 8, args.seed, max_tokens=64, wdtype=wd)
+            xs64 = [synth.x_bits(args.seed + 2000 + l, w4n.T, w4n.d) for l in range(8)]
+            r64 = [_bits_to_cuda(synth.make_router(w4n, args.seed, xs64[l], layer=l)) for l in range(8)]
+            fx64 = [_bits_to_cuda(x) for x in xs64]
+            K64 = 8 * 25
+            ms64, _ = run_chain(st64, r64, w4n.T, K64, 16, fixed_inputs=fx64)
+            ms64 = _max_over_ranks(ms64)
+            k_ms, k_bytes, k_flops, ids64 = kernel_timing(st64, r64, w4n.T, 16, fixed_inputs=fx64)
+            sb64 = np.mean([step_bytes(w4n, ids64[i], wd) for i in range(ids64.shape[0])])
+            tf_peak, tf_kind = _tensor_peak(wd)
+            extras["batch64"][wd] = {
+                "workload": f"cfg4: 64 tokens, Zipf(1.1)-skewed routing, {wd} weights, tensor-core path",
+                "tokens_per_s": world * w4n.T * K64 / (ms64 / 1e3), "us_per_layer": ms64 / K64 * 1e3,
+                "step_bytes": sb64, "achieved_gbs": sb64 / (ms64 / K64 / 1e3) / 1e9,
+                "frac_of_peak": sb64 / (ms64 / K64 / 1e3) / 1e9 / peak,
+                "union_experts_mean": float(np.mean([len(np.unique(ids64[i])) for i in range(ids64.shape[0])])),
+                "gateup_kernel": {"name": "k_mma_ffn<gate/up>", "us": k_ms * 1e3, "bytes": k_bytes,
+                                  "gbs": k_bytes / (k_ms / 1e3) / 1e9,
+                                  "frac_of_hbm_peak": k_bytes / (k_ms / 1e3) / 1e9 / peak,
+                                  "tflops": k_flops / (k_ms / 1e3) / 1e12,
+                                  "frac_of_tensor_peak": k_flops / (k_ms / 1e3) / 1e12 / tf_peak,
+                                  "tensor_peak_tflops": tf_peak, "tensor_peak_kind": tf_kind}}
+            del st64, fx64, r64
+            torch.cuda.empty_cache()
         extras["stack47"] = {
             "workload": "cfg3: 47 resident layers (21.4 GB NVFP4), residual chain, no attention",
             "batch1_tokens_per_s": tok_s / N_LAYERS, "batch1_us_per_layer": ms_step * 1e3,
@@ -443,16 +516,16 @@ def main():
                        "l2": "inputs larger than L2: 47 resident layer weight sets (21.4 GB) used in turn, "
                              "each step's output feeding the next (residual chain, input RMS-normalised "
                              "inside the layer so the chain stays finite)",
-                       "launch": "CUDA graph of 94 layer calls, 3 kernels per call chained with PDL",
+                       "launch": "CUDA graph of 94 layer calls, one persistent cooperative kernel per call",
                        "weights": "nvfp4", "activations": "bf16", "accumulate": "f32"},
             "hbm": {"step_bytes": sb, "achieved_gbs": step_gbs, "frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS,
                     "frac_of_peak": step_gbs / peak, "peak_gbs": peak, "peak_kind": peak_kind,
                     "router_bytes_excluded": w1.E * w1.d * 2},
-            "roofline": {"bound": "hbm", "kernel": "k_gateup", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+            "roofline": {"bound": "hbm", "kernel": "k_layer", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": TRAFFIC_K_LAYER_T1, "peak_kind": peak_kind,
                          "kernel_us": gk_ms * 1e3, "algorithmic_bytes": gk_bytes},
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 3 * K,
+            "gpu_launches": K,
             "clocks": clocks,
         }
         line.update(extras)

@@ -109,9 +109,12 @@ enum {
 };
 
 typedef enum flint_path {
-  FLINT_PATH_AUTO = 0, /* GEMV kernels below 32 tokens, tensor-core path from 32 */
+  FLINT_PATH_AUTO = 0, /* NVFP4: GEMV kernels below 32 tokens, tensor-core path from
+                          32; bf16 weights: tensor-core path */
   FLINT_PATH_GEMV = 1, /* CUDA-core dequant-GEMV kernels at any token count */
-  FLINT_PATH_MMA = 2   /* TMA-staged dequant-to-smem + tcgen05 MMA at any count */
+  FLINT_PATH_MMA = 2   /* TMA-staged dequant-to-smem + tcgen05 MMA at any count up
+                          to 128 tokens; NVFP4 weights need inter >= 256; no
+                          input_rmsnorm */
 } flint_path;
 
 typedef struct flint_moe_options {
@@ -163,12 +166,11 @@ int flint_pack_bf16(const uint16_t* w, const flint_moe_shape* shape, uint16_t* p
  * must not be shared by calls that may overlap on the GPU. */
 size_t flint_moe_workspace_bytes(const flint_moe_shape* shape, int32_t max_tokens);
 
-/* Clears the workspace's control block (its first 1024 bytes: the status word,
- * the router's arrival counter and the persistent kernel's grid-barrier epoch
- * flags). Call once after allocating a workspace, before its first use, and
- * again after a call reported FLINT_DEVCHECK_WAIT (a CTA that gave up a wait
- * leaves the epochs unequal). Kernels only ever set bits in the status word,
- * and flint_moe_get_status reads and clears it. */
+/* Zeroes the whole workspace (ws_bytes bytes): the control block at its head
+ * (status word, router arrival counter, the single-kernel path's launch
+ * generation and grid-barrier counters) and the tagged router logits. Call
+ * once after allocating a workspace, before its first use. Kernels only ever
+ * set bits in the status word, and flint_moe_get_status reads and clears it. */
 int flint_moe_workspace_init(void* workspace, size_t ws_bytes, void* stream);
 
 /* flint_moe_route -- the router alone.
@@ -191,7 +193,15 @@ int flint_moe_forward(const uint16_t* x, int32_t T, const uint16_t* router_w,
                       size_t ws_bytes, void* stream);
 
 /* As flint_moe_forward, with options (path choice, PDL, routing outputs).
- * options == NULL behaves as flint_moe_forward. */
+ * options == NULL behaves as flint_moe_forward.
+ * The tensor-core path (FLINT_PATH_MMA, or AUTO from 32 tokens) multiplies on
+ * tcgen05 (kind::f16, fp32 accumulators in tensor memory): NVFP4 weights are
+ * dequantised in shared memory to f16, exactly (an e2m1 code times an e4m3
+ * scale has at most 6 significant bits), against x scaled per token by a power
+ * of two into f16; bf16 weights multiply bf16 x directly. SwiGLU intermediates
+ * are kept in fp32 and fed to the down projection as f16 (NVFP4, power-of-two
+ * row scale) or bf16 (bf16 weights). Its profile events bracket the gate/up
+ * kernel. */
 int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
                          const flint_moe_weights* weights, const flint_moe_shape* shape,
                          const uint16_t* residual, uint16_t* out, void* workspace,
@@ -212,10 +222,10 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
  *  with a message, before any launch.
  *  The first call on each device looks up the array's device address
  *  (cudaGetSymbolAddress, with that device current) and caches it; make that
- *  first call before any stream capture. Each call clears the status word and
- *  the router counter at the start of the array (an asynchronous memset on
- *  `stream`), so device check flags are not kept between calls.
- *  All calls share the one array, which keeps the previous call's contents:
+ *  first call before any stream capture. Each call first zeroes the part of
+ *  the array it uses (an asynchronous memset on `stream`), so device check
+ *  flags are not kept between calls.
+ *  All calls share the one array:
  *  calls that may run at the same time on the GPU (different streams, or
  *  different host threads) race on it and corrupt each other's results;
  *  serialise them on one stream. */

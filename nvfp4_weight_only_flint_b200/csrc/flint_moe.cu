@@ -12,6 +12,9 @@
 #include <string>
 
 #include "fused_layer.cuh"
+#include "mma_path.cuh"
+
+#include <cudaTypedefs.h>
 
 namespace flint {
 
@@ -230,17 +233,20 @@ int check_shape(const flint_moe_shape* s, Dims* out) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct WsLayout {
-  size_t status, counter, amax, desc, logits, ids, gates, h, total;
+  size_t status, counter, amax, desc, logits, tlogits, ids, gates, h;
+  size_t mma_n, mma_act, mma_off, mma_pair, xinv, hinv, xrows, hrows, y;  // tensor-core path
+  size_t total;
 };
 
 size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-constexpr size_t kCtrlBytes = 64 + 4 * kMaxGridFlags;
+constexpr size_t kCtrlBytes = 1024;
 
 // Workspace carve-up for calls of up to maxT tokens. The first kCtrlBytes hold
 // the control block: the status word (byte 0), the router's arrival counter
-// (byte 4, left at zero by every call) and, from byte 64, one grid-barrier
-// epoch flag per CTA of the persistent layer kernel (each call advances them
-// by 2). All start at zero (flint_moe_workspace_init).
+// (byte 4, left at zero by every call), the persistent layer kernel's launch
+// generation (byte 8) and its four grid-barrier counters (bytes 132, 260, 388,
+// 516; one 128-byte line each). The tagged logits start with a tag of 0, which
+// no launch uses. flint_moe_workspace_init zeroes the whole workspace.
 WsLayout ws_layout(const Dims& s, int maxT) {
   WsLayout w{};
   size_t o = 0;
@@ -253,12 +259,33 @@ WsLayout ws_layout(const Dims& s, int maxT) {
   o += al256(sizeof(RouteDesc));
   w.logits = o;
   o += al256(sizeof(float) * static_cast<size_t>(maxT) * s.E);
+  w.tlogits = o;
+  o += al256(sizeof(unsigned long long) * static_cast<size_t>(maxT) * s.E);
   w.ids = o;
   o += al256(sizeof(int) * static_cast<size_t>(maxT) * s.k);
   w.gates = o;
   o += al256(sizeof(float) * static_cast<size_t>(maxT) * s.k);
   w.h = o;
-  o += al256(sizeof(float) * static_cast<size_t>(maxT) * (s.k + s.S) * s.I);
+  const size_t P = static_cast<size_t>(maxT) * (s.k + s.S);
+  o += al256(sizeof(float) * P * s.I);
+  w.mma_n = o;
+  o += 256;
+  w.mma_act = o;
+  o += al256(sizeof(int) * (s.E + s.S));
+  w.mma_off = o;
+  o += al256(sizeof(int) * (s.E + s.S + 1));
+  w.mma_pair = o;
+  o += al256(sizeof(int) * P);
+  w.xinv = o;
+  o += al256(sizeof(float) * P);
+  w.hinv = o;
+  o += al256(sizeof(float) * P);
+  w.xrows = o;
+  o += al256(2 * P * s.d);
+  w.hrows = o;
+  o += al256(2 * P * s.I);
+  w.y = o;
+  o += al256(sizeof(float) * P * s.d);
   w.total = o;
   return w;
 }
@@ -337,6 +364,7 @@ void fill_common(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, 
   p.counter = reinterpret_cast<unsigned*>(ws + w.counter);
   p.desc = reinterpret_cast<RouteDesc*>(ws + w.desc);
   p.logits = reinterpret_cast<float*>(ws + w.logits);
+  p.tlogits = reinterpret_cast<unsigned long long*>(ws + w.tlogits);
   p.ids = reinterpret_cast<int*>(ws + w.ids);
   p.gates = reinterpret_cast<float*>(ws + w.gates);
   p.h = reinterpret_cast<float*>(ws + w.h);
@@ -392,7 +420,6 @@ size_t down_smem(const LayerParams& p) {
 // dynamic shared-memory bytes, or 0 if the call does not fit it.
 size_t configure_fused(LayerParams& p, const Dims& s, int T) {
   const int sms = num_sms();
-  if (sms > kMaxGridFlags) return 0;
   p.stage_gateup = gateup_stage_bytes(s.d);
   p.ns_gateup = 2;
   const int rps = 32 / (s.I / 32);
@@ -403,12 +430,14 @@ size_t configure_fused(LayerParams& p, const Dims& s, int T) {
   p.down_rb = (4 * rps < nb) ? 4 * rps : nb;
   p.stage_down = ((p.down_rb * (s.I / 2 + s.I / 16)) + 15) & ~15;
   p.ns_down = 2;
+  p.h_in_smem = 1;
   const size_t a128 = 127;
+  const int R = T * (s.k + s.S);
   const size_t head = sizeof(RouteDesc) + ((static_cast<size_t>(T) * s.d * 2 + a128) & ~a128) +
                       static_cast<size_t>((s.E + sms - 1) / sms) * s.d * 2;
-  const size_t ybytes = ((4 * static_cast<size_t>(T) * (s.k + s.S) * nb) + a128) & ~a128;
-  const size_t hbytes = static_cast<size_t>(T) * (s.k + s.S) * s.I * 4;
+  const size_t ybytes = ((4 * static_cast<size_t>(R) * nb) + a128) & ~a128;
   const size_t ring_d = static_cast<size_t>(kFusedWarps) * p.ns_down * p.stage_down;
+  const size_t down = fused_h16_bytes(R, s.I) + ybytes + ring_d;
   const size_t budget = 210 * 1024;
   // deeper gate/up rings while they fit (the down ring takes the next 2 of
   // each warp's kMaxStages barriers)
@@ -416,8 +445,7 @@ size_t configure_fused(LayerParams& p, const Dims& s, int T) {
          head + static_cast<size_t>(kFusedWarps) * (p.ns_gateup + 1) * p.stage_gateup <= budget)
     ++p.ns_gateup;
   const size_t ring_g = static_cast<size_t>(kFusedWarps) * p.ns_gateup * p.stage_gateup;
-  p.h_in_smem = (head + std::max(ring_g, hbytes + ybytes + ring_d) <= budget) ? 1 : 0;
-  const size_t work = std::max(ring_g, (p.h_in_smem ? hbytes : 0) + ybytes + ring_d);
+  const size_t work = std::max(ring_g, down);
   if (head + work > budget) return 0;
   return head + work;
 }
@@ -509,6 +537,144 @@ cudaError_t launch_down(const LayerParams& p, cudaStream_t st, bool pdl) {
     case 512: return launch_smem(k_down<512>, grid, block, smem, st, pdl, p);
     default: return launch_smem(k_down<1024>, grid, block, smem, st, pdl, p);
   }
+}
+
+// ----------------------------------------------------------------- tensor-core path (host)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// Row-major tensor of `rank` dims (dim 0 innermost, in elements), strides of
+// dims 1.. in bytes, box in elements.
+int encode_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
+               const cuuint64_t* strides, const cuuint32_t* box, bool swizzle128) {
+  auto fn = tensor_map_encoder();
+  if (fn == nullptr) return fail(FLINT_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FLINT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return FLINT_OK;
+}
+
+// Tensor maps of one projection. gate/up: rows 2I, K = d, starting at the
+// expert base; down: rows d, K = I, starting I*d (NVFP4 bytes) after it.
+int mma_maps(MmaMaps* mp, const Dims& s, const flint_moe_weights* wts, bool gateup, const uint16_t* brows, int P) {
+  const int K = gateup ? s.d : s.I, rows = gateup ? 2 * s.I : s.d;
+  const cuuint64_t ne = static_cast<cuuint64_t>(s.E + s.S);
+  int rc;
+  if (s.wd == FLINT_W_NVFP4) {
+    const uint8_t* codes = static_cast<const uint8_t*>(wts->packed) + (gateup ? 0 : static_cast<size_t>(s.I) * s.d);
+    const uint8_t* scales = wts->block_scales + (gateup ? 0 : static_cast<size_t>(s.I) * s.d / 8);
+    const cuuint64_t cdims[3] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows), ne};
+    const cuuint64_t cstr[2] = {static_cast<cuuint64_t>(K / 2), 3ull * s.I * s.d / 2};
+    const cuuint32_t cbox[3] = {128, 128, 1};
+    if ((rc = encode_map(&mp->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, codes, cdims, cstr, cbox, true)) != FLINT_OK)
+      return rc;
+    const cuuint64_t sdims[3] = {static_cast<cuuint64_t>(K / 16), static_cast<cuuint64_t>(rows), ne};
+    const cuuint64_t sstr[2] = {static_cast<cuuint64_t>(K / 16), 3ull * s.I * s.d / 16};
+    const cuuint32_t sbox[3] = {16, 128, 1};
+    if ((rc = encode_map(&mp->scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, scales, sdims, sstr, sbox, false)) != FLINT_OK)
+      return rc;
+  } else {
+    const uint16_t* w = static_cast<const uint16_t*>(wts->packed) + (gateup ? 0 : 2 * static_cast<size_t>(s.I) * s.d);
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows), ne};
+    const cuuint64_t str[2] = {static_cast<cuuint64_t>(K) * 2, 3ull * s.I * s.d * 2};
+    const cuuint32_t box[3] = {64, 128, 1};
+    if ((rc = encode_map(&mp->codes, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w, dims, str, box, true)) != FLINT_OK)
+      return rc;
+    mp->scales = mp->codes;
+  }
+  const cuuint64_t bdims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(P)};
+  const cuuint64_t bstr[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t bbox[2] = {64, 16};
+  return encode_map(&mp->brows, s.wd == FLINT_W_NVFP4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    2, brows, bdims, bstr, bbox, true);
+}
+
+size_t mma_smem(bool nvfp4) {
+  return 1024 + (nvfp4 ? kMmaRawStages * kMmaRawBytes : 0) + kMmaAStages * kMmaABytes + kMmaBStages * kMmaBBytes;
+}
+
+// The tensor-core layer: router, top-k, grouping, B rows, gate/up, h rows,
+// down, combine.
+int run_mma_path(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, const flint_moe_weights* wts,
+                 cudaEvent_t* ev, bool pdl, cudaStream_t st) {
+  const int T = p.T, P = T * (s.k + s.S);
+  MmaParams m{};
+  m.x = p.x;
+  m.tscale = (s.wd == FLINT_W_NVFP4) ? wts->tensor_scales : nullptr;
+  m.residual = p.residual;
+  m.out = p.out;
+  m.status = p.status;
+  m.ids = p.ids;
+  m.gates = p.gates;
+  m.ids_out = p.ids_out;
+  m.gates_out = p.gates_out;
+  m.rt.n_active = reinterpret_cast<int*>(ws + w.mma_n);
+  m.rt.act = reinterpret_cast<int*>(ws + w.mma_act);
+  m.rt.off = reinterpret_cast<int*>(ws + w.mma_off);
+  m.rt.pair = reinterpret_cast<int*>(ws + w.mma_pair);
+  m.xrows = reinterpret_cast<uint16_t*>(ws + w.xrows);
+  m.xinv = reinterpret_cast<float*>(ws + w.xinv);
+  m.h = p.h;
+  m.hrows = reinterpret_cast<uint16_t*>(ws + w.hrows);
+  m.hinv = reinterpret_cast<float*>(ws + w.hinv);
+  m.y = reinterpret_cast<float*>(ws + w.y);
+  m.T = T;
+  m.d = s.d;
+  m.I = s.I;
+  m.E = s.E;
+  m.k = s.k;
+  m.S = s.S;
+  m.nvfp4 = (s.wd == FLINT_W_NVFP4) ? 1 : 0;
+  MmaMaps gu{}, dn{};
+  int rc = mma_maps(&gu, s, wts, true, m.xrows, P);
+  if (rc != FLINT_OK) return rc;
+  rc = mma_maps(&dn, s, wts, false, m.hrows, P);
+  if (rc != FLINT_OK) return rc;
+
+  cudaError_t e = launch_router_only(p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "k_router_only launch");
+  e = launch(k_topk, dim3((T + 7) / 8), dim3(256), 0, st, pdl, p);
+  if (e != cudaSuccess) return cuda_fail(e, "k_topk launch");
+  e = launch(k_mma_group, dim3(1), dim3(512), 0, st, pdl, m);
+  if (e != cudaSuccess) return cuda_fail(e, "k_mma_group launch");
+  e = launch(k_mma_prep, dim3((P + 7) / 8), dim3(256), 0, st, pdl, m);
+  if (e != cudaSuccess) return cuda_fail(e, "k_mma_prep launch");
+  const size_t smem = mma_smem(m.nvfp4 != 0);
+  const int ncols = 2 * kMmaMaxTokens;
+  const dim3 grid(num_sms()), block(kMmaWarps * 32);
+  e = ensure_smem(reinterpret_cast<const void*>(k_mma_ffn<kEpiGateUp>));
+  if (e == cudaSuccess) e = ensure_smem(reinterpret_cast<const void*>(k_mma_ffn<kEpiDown>));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  if (ev) {
+    e = cudaEventRecord(ev[0], st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  }
+  e = launch(k_mma_ffn<kEpiGateUp>, grid, block, smem, st, pdl && !ev, m, gu, ncols);
+  if (e != cudaSuccess) return cuda_fail(e, "k_mma_ffn (gate/up) launch");
+  if (ev) {
+    e = cudaEventRecord(ev[1], st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  }
+  e = launch(k_mma_hconv, dim3((P + 7) / 8), dim3(256), 0, st, pdl && !ev, m);
+  if (e != cudaSuccess) return cuda_fail(e, "k_mma_hconv launch");
+  e = launch(k_mma_ffn<kEpiDown>, grid, block, smem, st, pdl, m, dn, ncols);
+  if (e != cudaSuccess) return cuda_fail(e, "k_mma_ffn (down) launch");
+  e = launch(k_mma_combine, dim3((T * (s.d / 8) + 255) / 256), dim3(256), 0, st, pdl, m);
+  if (e != cudaSuccess) return cuda_fail(e, "k_mma_combine launch");
+  return FLINT_OK;
 }
 
 }  // namespace
@@ -655,12 +821,22 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
   if (path < FLINT_PATH_AUTO || path > FLINT_PATH_MMA) return fail(FLINT_ERR_INVALID_ARG, "path %d", path);
   if (options && ((options->topk_ids == nullptr) != (options->topk_weights == nullptr)))
     return fail(FLINT_ERR_INVALID_ARG, "topk_ids and topk_weights go together");
-  const bool use_gemv = (path == FLINT_PATH_GEMV) || (path == FLINT_PATH_AUTO && T < kMaxGemvTokens);
-  if (!use_gemv || s.wd != FLINT_W_NVFP4)
-    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "tensor-core path not available in this build (T=%d)", T);
-  const int gemv_max_t = (s.d == 4096) ? kMaxGemvTokens / 2 : kMaxGemvTokens;
-  if (T > gemv_max_t)
-    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "GEMV path takes at most %d tokens at d=%d", gemv_max_t, s.d);
+  const bool use_gemv = (path == FLINT_PATH_GEMV) ||
+                        (path == FLINT_PATH_AUTO && T < kMaxGemvTokens && s.wd == FLINT_W_NVFP4);
+  if (use_gemv) {
+    if (s.wd != FLINT_W_NVFP4)
+      return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "the GEMV path takes NVFP4 weights; bf16 weights use the tensor-core path");
+    const int gemv_max_t = (s.d == 4096) ? kMaxGemvTokens / 2 : kMaxGemvTokens;
+    if (T > gemv_max_t)
+      return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "GEMV path takes at most %d tokens at d=%d", gemv_max_t, s.d);
+  } else {
+    if (T > kMmaMaxTokens)
+      return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "tensor-core path takes at most %d tokens (T=%d)", kMmaMaxTokens, T);
+    if (s.wd == FLINT_W_NVFP4 && s.I < 256)
+      return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "tensor-core path with NVFP4 weights needs inter >= 256 (inter=%d)", s.I);
+    if (options && options->input_rmsnorm)
+      return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "input_rmsnorm is a GEMV-path option");
+  }
   const WsLayout lay = ws_layout(s, T);
   if (ws_bytes < lay.total) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, lay.total);
 
@@ -680,6 +856,7 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
   p.input_norm = (options && options->input_rmsnorm) ? 1 : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaEvent_t* ev = options ? static_cast<cudaEvent_t*>(options->profile_events) : nullptr;
+  if (!use_gemv) return run_mma_path(p, s, lay, static_cast<uint8_t*>(workspace), weights, ev, pdl, st);
   const bool split = options && options->split_kernels;
   if (T <= kFusedMaxTokens && !split) {
     const size_t smem = configure_fused(p, s, T);
@@ -726,7 +903,7 @@ int flint_moe_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
   if (!workspace) return fail(FLINT_ERR_INVALID_ARG, "workspace is NULL");
   if (!aligned16(workspace)) return fail(FLINT_ERR_MISALIGNED, "workspace must be 16-byte aligned");
   if (ws_bytes < kCtrlBytes) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kCtrlBytes);
-  cudaError_t e = cudaMemsetAsync(workspace, 0, kCtrlBytes, static_cast<cudaStream_t>(stream));
+  cudaError_t e = cudaMemsetAsync(workspace, 0, ws_bytes, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   return FLINT_OK;
 }
@@ -840,8 +1017,9 @@ int flint_moe_forward_noalloc(const uint16_t* x, int32_t T, const uint16_t* rout
     scratch = g_noalloc_addr[dev];
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // The control block (status word, router counter, barrier flags) must start at zero.
-  e = cudaMemsetAsync(scratch, 0, kCtrlBytes, st);
+  // Every call starts from a zeroed scratch (the control block and the tagged
+  // logits must; the rest is rewritten before it is read).
+  e = cudaMemsetAsync(scratch, 0, need, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   return flint_moe_forward_ex(x, T, router_w, weights, shape, residual, out, scratch, kNoAllocScratchBytes,
                               nullptr, stream);

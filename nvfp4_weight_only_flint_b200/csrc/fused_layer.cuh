@@ -1,22 +1,28 @@
 // fused_layer.cuh -- the whole layer in one persistent kernel (batch <= 8).
 //
 // One CTA per SM (8 warps), every SM busy in every phase:
-//   P0  bulk copies of x and of this CTA's router rows; L2 prefetch of this
-//       CTA's slice of the shared expert (gate/up units and down rows)
-//   P1  router logits ((row, token) tasks over the warps) and per-token scales
-//   --  grid barrier 1 (all logits written)
-//   P2  every CTA: top-k of every token (sorted-list butterfly merge, warp per
-//       token) and the token grouping (one warp), kept in shared memory
-//   P3  gate/up of the routed experts and the shared expert through per-warp
-//       bulk-copy rings, work split by compute cost; L2 prefetch of this CTA's
-//       block of down rows of every routed active expert
-//   --  grid barrier 2 (all h written)
-//   P4  down: h staged in shared memory (or read from L2), down rows streamed
-//       through per-warp rings, fixed-order gated combine (+ residual)
-// The grid barrier is a flag per CTA in the workspace: a CTA publishes its epoch
-// with a release store and polls every flag with relaxed loads (one round trip
-// per poll, no atomics), then fences. Waits are bounded (FLINT_DEVCHECK_WAIT).
-// The launch is cooperative, so every CTA is resident.
+//   P0  bulk copies of x, of this CTA's router rows and of each warp's slice
+//       of the shared expert's gate/up units; L2 prefetch of this CTA's block
+//       of the shared expert's down rows
+//   P1  router logits ((row, token) tasks over the warps), stored as tagged
+//       64-bit words (launch tag | logit), and per-token scales; then each
+//       warp's slice of the shared expert's gate/up units (they need no
+//       routing; their bulk copies were issued at the start)
+//   P2  every CTA: top-k of every token (a warp per token waits until all E
+//       logits carry this launch's tag, then selects) and the token grouping,
+//       kept in shared memory; L2 prefetch of this CTA's block of down rows of
+//       every routed active expert
+//   P3  gate/up of the routed experts through per-warp bulk-copy rings, work
+//       split by compute cost
+//   --  grid barrier (all h written)
+//   P4  h converted once per CTA to f16 (power-of-two scale per row) in shared
+//       memory, down rows streamed through per-warp rings, fixed-order gated
+//       combine (+ residual)
+// The launch tag and the barrier targets come from a generation word in the
+// workspace control block that CTA 0 advances after the barrier. The barrier
+// spreads arrivals over four counters in separate lines (fewer same-address
+// atomics in series). Every wait is bounded (FLINT_DEVCHECK_WAIT). The launch
+// is cooperative, so every CTA is resident.
 #pragma once
 
 #include "layer_kernels.cuh"
@@ -25,7 +31,8 @@ namespace flint {
 
 constexpr int kFusedMaxTokens = 8;
 constexpr int kFusedWarps = 8;
-constexpr int kMaxGridFlags = 240;  // CTAs of the persistent kernel (flags in the control block)
+constexpr int kFusedDownTokens = 4;   // tokens per pass in the down phase
+constexpr int kBarrierCounters = 4;   // control-block words 32, 64, 96, 128
 
 __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
   unsigned v;
@@ -33,19 +40,24 @@ __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
   return v;
 }
 
-// Grid barrier: this CTA stores `target` in its flag, then waits until every
-// CTA's flag has reached `target` (wrap-safe comparison).
-__device__ __forceinline__ bool flag_barrier(unsigned* flags, unsigned target, int* status, int* s_ok) {
+// Grid barrier over monotonically increasing counters: CTA c adds 1 to counter
+// c % 4 (release); a call's barrier is complete when counter i holds
+// n_i * (gen + 1), n_i the number of CTAs with c % 4 == i.
+__device__ __forceinline__ bool grid_barrier(unsigned* ctrl, unsigned gen, int* status, int* s_ok) {
   __syncthreads();
   if (threadIdx.x < 32) {
-    if (threadIdx.x == 0)
-      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flags + blockIdx.x), "r"(target) : "memory");
+    const int lane = threadIdx.x, G = gridDim.x;
+    if (lane == 0)
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctrl + 32 * (1 + blockIdx.x % kBarrierCounters))
+                   : "memory");
+    const unsigned n_i =
+        lane < kBarrierCounters ? static_cast<unsigned>((G - lane + kBarrierCounters - 1) / kBarrierCounters) : 0u;
+    const unsigned target = n_i * (gen + 1u);
     const long long t0 = clock64();
     bool ok = true;
     for (;;) {
-      bool mine = true;
-      for (int i = threadIdx.x; i < static_cast<int>(gridDim.x); i += 32)
-        mine &= static_cast<int>(ld_relaxed_u32(flags + i) - target) >= 0;
+      const bool mine =
+          lane >= kBarrierCounters || static_cast<int>(ld_relaxed_u32(ctrl + 32 * (1 + lane)) - target) >= 0;
       if (__all_sync(0xffffffffu, mine)) break;
       if (clock64() - t0 > kWaitCycles) {
         ok = false;
@@ -53,7 +65,7 @@ __device__ __forceinline__ bool flag_barrier(unsigned* flags, unsigned target, i
       }
     }
     asm volatile("fence.acq_rel.gpu;" ::: "memory");
-    if (threadIdx.x == 0) {
+    if (lane == 0) {
       *s_ok = ok ? 1 : 0;
       if (!ok) atomicOr(status, FLINT_DEVCHECK_WAIT);
     }
@@ -88,25 +100,32 @@ __device__ __forceinline__ void cost_prefix(const RouteDesc* dsc, int n_active, 
   if (lane == 31) cost[n_active] = ex;
 }
 
+// Shared-memory bytes of the down phase's h copy: R rows of I f16.
+__host__ __device__ constexpr size_t fused_h16_bytes(int R, int I) {
+  return ((static_cast<size_t>(R) * I * 2) + 127) & ~static_cast<size_t>(127);
+}
+
 template <int D, int I>
 __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   using M = GateUpMap<D>;
   constexpr int NVR = D / 256;   // router: 8-element bf16 vectors per lane
-  constexpr int VRD = I / 32;    // down: 16-byte vectors per row
+  constexpr int VRD = I / 32;    // down: 16-byte vectors per row (lanes per row)
   constexpr int RPS = 32 / VRD;  // down: rows per warp step
-  constexpr int TGD = kDownTokens;
+  constexpr int TGD = kFusedDownTokens;
   constexpr int ROWC = I / 2, ROWS = I / 16;
+  constexpr int MAXR = kFusedMaxTokens * (kMaxTopK + 1);
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_ids[kFusedMaxTokens * kMaxTopK];
   __shared__ float s_gates[kFusedMaxTokens * kMaxTopK];
   __shared__ float s_sigma[kFusedMaxTokens], s_f[kFusedMaxTokens];
   __shared__ int s_cost[kFusedWarps][kFusedMaxTokens * kMaxTopK + 2];  // per-warp cost prefix over <= T*k+1 experts
-  __shared__ unsigned s_base;
-  __shared__ int s_ok;
-  __shared__ __align__(8) uint64_t s_bar[kFusedWarps * kMaxStages + 3];
+  __shared__ float s_hinv[MAXR];
+  __shared__ unsigned s_gen;
+  __shared__ int s_ok, s_fail;
+  __shared__ __align__(8) uint64_t s_bar[kFusedWarps * kMaxStages + 2];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int T = p.T, E = p.E, k = p.k, S = p.S, KS = k + S, G = gridDim.x, c = blockIdx.x;
-  unsigned* flags = p.counter + 15;  // control block bytes 64.. : one flag per CTA
+  const int R = T * KS;
 
   // ---- shared-memory carve-up: [desc][x][router rows][work]
   RouteDesc* dsc = reinterpret_cast<RouteDesc*>(smem);
@@ -115,31 +134,26 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   uint8_t* rsm = xsm + ((xbytes + 127) & ~static_cast<size_t>(127));
   const int rpc = (E + G - 1) / G;  // router rows per CTA
   uint8_t* work = rsm + static_cast<size_t>(rpc) * D * 2;
-  uint64_t* ring_bars = s_bar;                          // [warp][kMaxStages]
-  uint64_t* xbar = s_bar + kFusedWarps * kMaxStages;    // x
-  uint64_t* rbar = xbar + 1;                            // router rows
-  uint64_t* hbar = xbar + 2;                            // h staged for the down phase
+  uint64_t* ring_bars = s_bar;                        // [warp][kMaxStages]
+  uint64_t* xbar = s_bar + kFusedWarps * kMaxStages;  // x
+  uint64_t* rbar = xbar + 1;                          // router rows
   const int ns_g = p.ns_gateup, ns_d = p.ns_down;
   const int nb = p.down_nb, n0 = c * nb, nrows = max(0, min(nb, p.d - n0));
   const int r_begin = min(E, c * rpc), r_end = min(E, (c + 1) * rpc);
 
   // ---- P0: start the copies before anything else
   if (tid == 0) {
-    for (int i = 0; i < kFusedWarps * kMaxStages + 3; ++i) mbar_init(&s_bar[i], 1);
+    for (int i = 0; i < kFusedWarps * kMaxStages + 2; ++i) mbar_init(&s_bar[i], 1);
     fence_barrier_init();
     mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(xbytes));
     bulk_g2s(xsm, p.x, static_cast<uint32_t>(xbytes), xbar);
     const uint32_t rbytes = static_cast<uint32_t>(r_end - r_begin) * D * 2;
     mbar_arrive_expect_tx(rbar, rbytes);
     if (rbytes) bulk_g2s(rsm, p.wr + static_cast<size_t>(r_begin) * D, rbytes, rbar);
-    s_base = ld_relaxed_u32(flags + c);
+    s_gen = ld_relaxed_u32(p.counter + 1);
+    s_fail = 0;
   } else if (tid == 32 && S > 0) {
     const long long e = E;
-    const int u0 = c * I / G, u1 = (c + 1) * I / G;
-    if (u1 > u0) {
-      prefetch_l2(p.codes + e * p.cpe + static_cast<long long>(u0) * D, (u1 - u0) * D);
-      prefetch_l2(p.scales + e * p.spe + static_cast<long long>(u0) * (D / 8), (u1 - u0) * (D / 8));
-    }
     if (nrows > 0) {
       prefetch_l2(p.codes + e * p.cpe + static_cast<long long>(I) * p.d + static_cast<long long>(n0) * ROWC, nrows * ROWC);
       prefetch_l2(p.scales + e * p.spe + static_cast<long long>(I) * p.d / 8 + static_cast<long long>(n0) * ROWS,
@@ -147,12 +161,36 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     }
   }
   __syncthreads();
-  const unsigned base = s_base;
+  const unsigned gen = s_gen, tag = gen + 1u;
+
+  // ---- the warp's bulk-copy ring: first the shared expert's units (they do
+  // not depend on the routing, so they are fetched now and computed after the
+  // router tasks), then a range of the routed experts' units (after P2)
+  uint8_t* ring = work + static_cast<size_t>(warp) * ns_g * p.stage_gateup;
+  uint64_t* bars = ring_bars + warp * kMaxStages;
+  int issued = 0, consumed = 0;
+  auto issue_units = [&](int e, int uu, int cu, int slot) {
+    uint8_t* st = ring + slot * p.stage_gateup;
+    mbar_arrive_expect_tx(&bars[slot], cu * M::UNIT_BYTES);
+    bulk_g2s(st, p.codes + e * p.cpe + static_cast<long long>(uu) * D, cu * M::UNIT_CODE, &bars[slot]);
+    bulk_g2s(st + M::CU * M::UNIT_CODE, p.scales + e * p.spe + static_cast<long long>(uu) * (D / 8),
+             cu * M::UNIT_SCALE, &bars[slot]);
+  };
+  const long long NW = static_cast<long long>(G) * kFusedWarps;
+  const long long gw = static_cast<long long>(c) * kFusedWarps + warp;
+  const int sh_begin = S > 0 ? static_cast<int>(gw * I / NW) : 0;
+  const int sh_end = S > 0 ? static_cast<int>((gw + 1) * I / NW) : 0;
+  int sh_issue = sh_begin;
+  while (issued < ns_g && sh_issue < sh_end) {
+    const int cu = min(M::CU, sh_end - sh_issue);
+    if (lane == 0) issue_units(E, sh_issue, cu, issued % ns_g);
+    sh_issue += cu;
+    ++issued;
+  }
 
   // ---- P1: token statistics, router logits
   bool ok = mbar_wait(xbar, 0, p.status);
   const uint16_t* xs = reinterpret_cast<const uint16_t*>(xsm);
-  float irms_t = 1.f;
   if (warp < T && ok) {
     const int t = warp;
     float amax = 0.f, ss = 0.f;
@@ -171,11 +209,11 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     ss = warp_sum(ss);
-    irms_t = p.input_norm ? 1.f / sqrtf(ss / static_cast<float>(D) + kRmsEps) : 1.f;
+    const float irms = p.input_norm ? 1.f / sqrtf(ss / static_cast<float>(D) + kRmsEps) : 1.f;
     if (lane == 0) {
       const float sg = pow2_scale_for(amax);
       s_sigma[t] = sg;
-      s_f[t] = irms_t / sg;
+      s_f[t] = irms / sg;
     }
   }
   __syncthreads();
@@ -183,7 +221,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   for (int task = warp; task < (r_end - r_begin) * T && ok; task += kFusedWarps) {
     const int r = task / T, t = task % T;
     const uint16_t* wrow = reinterpret_cast<const uint16_t*>(rsm) + static_cast<size_t>(r) * D;
-    float acc[NVR];
+    float sum = 0.f;
 #pragma unroll
     for (int i = 0; i < NVR; ++i) {
       const uint4 wv = lds128(wrow + 8 * (lane + 32 * i));
@@ -196,20 +234,106 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
         a = fmaf(bf16_bits_to_f32(ww[q] & 0xFFFFu), bf16_bits_to_f32(xx[q] & 0xFFFFu), a);
         a = fmaf(__uint_as_float(ww[q] & 0xFFFF0000u), __uint_as_float(xx[q] & 0xFFFF0000u), a);
       }
-      acc[i] = a;
+      sum += a;
     }
-    float sum = 0.f;
-#pragma unroll
-    for (int i = 0; i < NVR; ++i) sum += acc[i];
     sum = warp_sum(sum);
-    if (lane == 0) p.logits[static_cast<size_t>(t) * E + r_begin + r] = sum * s_f[t] * s_sigma[t];
+    if (lane == 0) st_tagged(p.tlogits + static_cast<size_t>(t) * E + r_begin + r, tag, sum * s_f[t] * s_sigma[t]);
   }
-  if (!flag_barrier(flags, base + 1u, p.status, &s_ok)) ok = false;
 
-  // ---- P2: top-k and grouping, in every CTA
-  if (warp < T && ok)
-    topk_token(p.logits + static_cast<size_t>(warp) * E, E, k, &s_ids[warp * k], &s_gates[warp * k], lane);
+  // gate/up of one staged chunk of `cu` units from unit uu, for the tokens
+  // pair(i), i < nt (pair = token << 8 | slot); x is restaged in registers
+  // only when the expert key or the token pass changes
+  uint32_t xh[M::TGMAX * M::XS];
+  int cur_key = -1, cur_g0 = -1;
+  // pairs == nullptr: every token, slot kslot (the shared expert)
+  auto compute_chunk = [&](const uint8_t* st, int cu, int uu, float sg, float su, int key, int nt,
+                           const unsigned short* pairs, int kslot) {
+    auto pair_of = [&](int i) { return pairs != nullptr ? static_cast<int>(pairs[i]) : ((i << 8) | kslot); };
+    for (int g0 = 0; g0 < nt; g0 += M::TGMAX) {
+      const int n = min(M::TGMAX, nt - g0);
+      int hrow[M::TGMAX];
+      float fg[M::TGMAX], fu[M::TGMAX];
+#pragma unroll
+      for (int t = 0; t < M::TGMAX; ++t) {
+        const int pr = (t < n) ? pair_of(g0 + t) : 0;
+        const int tok = pr >> 8;
+        hrow[t] = tok * KS + (pr & 0xFF);
+        fg[t] = (t < n) ? s_f[tok] * sg : 0.f;
+        fu[t] = (t < n) ? s_f[tok] * su : 0.f;
+      }
+      if (key != cur_key || g0 != cur_g0) {
+#pragma unroll
+        for (int t = 0; t < M::TGMAX; ++t) {
+          const int tok = pair_of(g0 + min(t, n - 1)) >> 8;
+          const float sgm = (t < n) ? s_sigma[tok] : 0.f;
+#pragma unroll
+          for (int xi = 0; xi < M::XV; ++xi) {
+            const uint16_t* src = xs + static_cast<size_t>(tok) * D + 32 * M::xblock(lane, xi);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 v = lds128(src + 8 * q);
+              xh[t * M::XS + xi * 16 + 4 * q + 0] = bf16x2_to_f16x2_scaled(v.x, sgm);
+              xh[t * M::XS + xi * 16 + 4 * q + 1] = bf16x2_to_f16x2_scaled(v.y, sgm);
+              xh[t * M::XS + xi * 16 + 4 * q + 2] = bf16x2_to_f16x2_scaled(v.z, sgm);
+              xh[t * M::XS + xi * 16 + 4 * q + 3] = bf16x2_to_f16x2_scaled(v.w, sgm);
+            }
+          }
+        }
+        cur_key = key;
+        cur_g0 = g0;
+      }
+      if (n == 1 && M::TGMAX > 1)
+        gateup_chunk<D, 1>(st, cu, xh, lane, n, fg, fu, hrow, p.h, I, uu);
+      else
+        gateup_chunk<D, M::TGMAX>(st, cu, xh, lane, n, fg, fu, hrow, p.h, I, uu);
+    }
+  };
+
+  // ---- P1b: the shared expert's units of this warp, for every token
+  if (sh_end > sh_begin) {
+    const float sg = __ldg(p.tscale + 3 * E + 0), su = __ldg(p.tscale + 3 * E + 1);
+    for (int u = sh_begin; u < sh_end && ok;) {
+      const int cu = min(M::CU, sh_end - u);
+      const int slot = consumed % ns_g;
+      if (!mbar_wait(&bars[slot], (consumed / ns_g) & 1, p.status)) {
+        ok = false;
+        break;
+      }
+      compute_chunk(ring + slot * p.stage_gateup, cu, u, sg, su, 1 << 20, T, nullptr, k);
+      __syncwarp();
+      ++consumed;
+      u += cu;
+      if (sh_issue < sh_end) {
+        const int cn = min(M::CU, sh_end - sh_issue);
+        if (lane == 0) {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          issue_units(E, sh_issue, cn, issued % ns_g);
+        }
+        sh_issue += cn;
+        ++issued;
+      }
+    }
+    if (!ok) {
+      drain_ring(bars, ns_g, consumed, issued, p.status);
+      consumed = issued;
+    }
+  }
+
+  // ---- P2: top-k (waits for every CTA's logits) and grouping, in every CTA
+  if (warp < T) {
+    bool okt = false;
+    if (ok) {
+      if (E <= 256)
+        okt = topk_warp_tagged<8>(p.tlogits + static_cast<size_t>(warp) * E, E, k, tag, &s_ids[warp * k],
+                                  &s_gates[warp * k], lane, p.status);
+      else
+        okt = topk_warp_tagged<kMaxExperts / 32>(p.tlogits + static_cast<size_t>(warp) * E, E, k, tag,
+                                                 &s_ids[warp * k], &s_gates[warp * k], lane, p.status);
+    }
+    if (!okt && lane == 0) s_fail = 1;
+  }
   __syncthreads();
+  if (s_fail) ok = false;
   if (warp == 0 && ok) warp_grouping(s_ids, T, k, E, S, dsc, lane, p.status);
   __syncthreads();
   if (c == 0 && ok) {
@@ -224,24 +348,24 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   }
   const int n_active = ok ? dsc->n_active : 0;
   // L2 prefetch of this CTA's block of down rows of every routed active expert
-  if (tid < dsc->n_routed && nrows > 0 && ok) {
+  if (ok && tid < dsc->n_routed && nrows > 0) {
     const long long e = dsc->act[tid];
     prefetch_l2(p.codes + e * p.cpe + static_cast<long long>(I) * p.d + static_cast<long long>(n0) * ROWC, nrows * ROWC);
     prefetch_l2(p.scales + e * p.spe + static_cast<long long>(I) * p.d / 8 + static_cast<long long>(n0) * ROWS,
                 nrows * ROWS);
   }
 
-  // ---- P3: gate/up. This warp's range of the cost space, mapped to units.
+  // ---- P3: gate/up of the routed experts. This warp's range of the cost
+  // space (units x token passes), mapped to units.
   {
+    const int n_routed = ok ? dsc->n_routed : 0;
     int* cost = s_cost[warp];
-    cost_prefix(dsc, n_active, I, M::TGMAX, cost, lane);
+    cost_prefix(dsc, n_routed, I, M::TGMAX, cost, lane);
     __syncwarp();
-    const long long C = n_active > 0 ? cost[n_active] : 0;
-    const long long NW = static_cast<long long>(G) * kFusedWarps;
-    const long long gw = static_cast<long long>(c) * kFusedWarps + warp;
+    const long long C = n_routed > 0 ? cost[n_routed] : 0;
     const long long c_begin = gw * C / NW, c_end = (gw + 1) * C / NW;
     auto to_unit = [&](long long cc, int& a, int& u) {
-      int lo = 0, hi = n_active - 1;
+      int lo = 0, hi = n_routed - 1;
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (cost[mid] <= cc) lo = mid;
@@ -264,86 +388,40 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
         if (pa == a0 && pu == u0) ++g_begin;
       }
     }
-    uint8_t* ring = work + static_cast<size_t>(warp) * ns_g * p.stage_gateup;
-    uint64_t* bars = ring_bars + warp * kMaxStages;
     auto chunk_len = [&](int g) { return min(M::CU, min(I - g % I, g_end - g)); };
-    auto issue = [&](int g, int slot) {
-      const int a = g / I, uu = g % I, cu = chunk_len(g);
-      const long long e = dsc->act[a];
-      uint8_t* st = ring + slot * p.stage_gateup;
-      mbar_arrive_expect_tx(&bars[slot], cu * M::UNIT_BYTES);
-      bulk_g2s(st, p.codes + e * p.cpe + static_cast<long long>(uu) * D, cu * M::UNIT_CODE, &bars[slot]);
-      bulk_g2s(st + M::CU * M::UNIT_CODE, p.scales + e * p.spe + static_cast<long long>(uu) * (D / 8),
-               cu * M::UNIT_SCALE, &bars[slot]);
-    };
-    int issue_g = g_begin, issued = 0, consumed = 0;
-    while (issued < ns_g && issue_g < g_end) {
-      if (lane == 0) issue(issue_g, issued % ns_g);
+    int issue_g = g_begin;
+    while (issued - consumed < ns_g && issue_g < g_end) {
+      if (lane == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue_units(dsc->act[issue_g / I], issue_g % I, chunk_len(issue_g), issued % ns_g);
+      }
       issue_g += chunk_len(issue_g);
       ++issued;
     }
-    uint32_t xh[M::TGMAX * M::XS];
-    int cur_a = -1, cur_g0 = -1;
+    int cur_a = -1;
     float sg = 0.f, su = 0.f;
-    for (int g = g_begin; g < g_end;) {
+    for (int g = g_begin; g < g_end && ok;) {
       const int a = g / I, uu = g % I, cu = chunk_len(g);
       if (a != cur_a) {  // tensor scales of the expert, fetched before the stage wait
         const int e = dsc->act[a];
         sg = __ldg(p.tscale + 3 * e + 0);
         su = __ldg(p.tscale + 3 * e + 1);
+        cur_a = a;
       }
       const int slot = consumed % ns_g;
       if (!mbar_wait(&bars[slot], (consumed / ns_g) & 1, p.status)) {
         ok = false;
         break;
       }
-      const uint8_t* st = ring + slot * p.stage_gateup;
       const int pb = dsc->off[a], nt = dsc->off[a + 1] - pb;
-      for (int g0 = 0; g0 < nt; g0 += M::TGMAX) {
-        const int n = min(M::TGMAX, nt - g0);
-        int hrow[M::TGMAX];
-        float fg[M::TGMAX], fu[M::TGMAX];
-#pragma unroll
-        for (int t = 0; t < M::TGMAX; ++t) {
-          const int pr = (t < n) ? dsc->pair[pb + g0 + t] : 0;
-          const int tok = pr >> 8;
-          hrow[t] = tok * KS + (pr & 0xFF);
-          fg[t] = (t < n) ? s_f[tok] * sg : 0.f;
-          fu[t] = (t < n) ? s_f[tok] * su : 0.f;
-        }
-        if (a != cur_a || g0 != cur_g0) {
-#pragma unroll
-          for (int t = 0; t < M::TGMAX; ++t) {
-            const int tok = dsc->pair[pb + g0 + min(t, n - 1)] >> 8;
-            const float sgm = (t < n) ? s_sigma[tok] : 0.f;
-#pragma unroll
-            for (int xi = 0; xi < M::XV; ++xi) {
-              const uint16_t* src = xs + static_cast<size_t>(tok) * D + 32 * M::xblock(lane, xi);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const uint4 v = lds128(src + 8 * q);
-                xh[t * M::XS + xi * 16 + 4 * q + 0] = bf16x2_to_f16x2_scaled(v.x, sgm);
-                xh[t * M::XS + xi * 16 + 4 * q + 1] = bf16x2_to_f16x2_scaled(v.y, sgm);
-                xh[t * M::XS + xi * 16 + 4 * q + 2] = bf16x2_to_f16x2_scaled(v.z, sgm);
-                xh[t * M::XS + xi * 16 + 4 * q + 3] = bf16x2_to_f16x2_scaled(v.w, sgm);
-              }
-            }
-          }
-          cur_g0 = g0;
-        }
-        cur_a = a;
-        if (n == 1 && M::TGMAX > 1)
-          gateup_chunk<D, 1>(st, cu, xh, lane, n, fg, fu, hrow, p.h, I, uu);
-        else
-          gateup_chunk<D, M::TGMAX>(st, cu, xh, lane, n, fg, fu, hrow, p.h, I, uu);
-      }
+      compute_chunk(ring + slot * p.stage_gateup, cu, uu, sg, su, a, nt, dsc->pair + pb, 0);
       __syncwarp();
       ++consumed;
       g += cu;
       if (issue_g < g_end) {
         if (lane == 0) {
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          issue(issue_g, issued % ns_g);
+          issue_units(dsc->act[issue_g / I], issue_g % I, chunk_len(issue_g), issued % ns_g);
         }
         issue_g += chunk_len(issue_g);
         ++issued;
@@ -351,27 +429,21 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     }
     if (!ok) drain_ring(bars, ns_g, consumed, issued, p.status);
   }
-  if (!flag_barrier(flags, base + 2u, p.status, &s_ok)) ok = false;
+  if (!grid_barrier(p.counter, gen, p.status, &s_ok)) ok = false;
+  if (c == 0 && tid == 0) asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p.counter + 1), "r"(gen + 1u) : "memory");
 
   // ---- P4: down rows of this CTA's block of outputs, for every active expert
-  const size_t hbytes = p.h_in_smem ? static_cast<size_t>(T) * KS * I * 4 : 0;
-  float* hsm = reinterpret_cast<float*>(work);
-  float* s_y = reinterpret_cast<float*>(work + hbytes);
-  const size_t ybytes = ((sizeof(float) * static_cast<size_t>(T) * KS * nb) + 127) & ~static_cast<size_t>(127);
-  uint8_t* dring = work + hbytes + ybytes + static_cast<size_t>(warp) * ns_d * p.stage_down;
+  // work area: [h16 R x I f16, lane-interleaved][s_y R x nb fp32][rings]
+  uint16_t* h16 = reinterpret_cast<uint16_t*>(work);
+  float* s_y = reinterpret_cast<float*>(work + fused_h16_bytes(R, I));
+  const size_t ybytes = ((sizeof(float) * static_cast<size_t>(R) * nb) + 127) & ~static_cast<size_t>(127);
+  uint8_t* dring = work + fused_h16_bytes(R, I) + ybytes + static_cast<size_t>(warp) * ns_d * p.stage_down;
   // the down ring uses this warp's barriers the gate/up ring left unused
   // (slots ns_g.. of its kMaxStages), so their phases start from zero
   uint64_t* bars_d = ring_bars + warp * kMaxStages + ns_g;
   const int RB = p.down_rb;
   const int nsub = (nrows + RB - 1) / RB;
   const int roff = RB * ROWC;
-  // the work area was last read through the generic proxy (gate/up stages);
-  // order those reads before the bulk copies that overwrite it
-  if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  if (tid == 0 && hbytes && ok) {
-    mbar_arrive_expect_tx(hbar, static_cast<uint32_t>(hbytes));
-    bulk_g2s(hsm, p.h, static_cast<uint32_t>(hbytes), hbar);
-  }
   const int n_items = (ok && nrows > 0) ? n_active * nsub : 0;
   int consumed_d = 0, issued_d = 0, next_issue = warp;
   auto issue_d = [&](int it, int slot) {
@@ -385,12 +457,43 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     bulk_g2s(st + roff, p.scales + e * p.spe + static_cast<long long>(I) * p.d / 8 + static_cast<long long>(n0 + r0) * ROWS,
              rows * ROWS, &bars_d[slot]);
   };
+  // the rings overwrite smem last read through the generic proxy (gate/up
+  // stages): order those reads before the bulk copies
+  if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   while (issued_d < ns_d && next_issue < n_items) {
     if (lane == 0) issue_d(next_issue, issued_d % ns_d);
     next_issue += kFusedWarps;
     ++issued_d;
   }
-  if (hbytes && ok) ok = mbar_wait(hbar, 0, p.status);
+  // h (fp32, written by every CTA) -> f16 rows with a power-of-two scale each.
+  // Element i of row P sits at P*I + ((i%32)/8 * VRD + i/32) * 8 + i%8, so the
+  // 16-byte vectors the lanes of a down step read are contiguous.
+  if (ok) {
+    constexpr int F4 = I / 128;  // float4 per lane per row
+    for (int P = warp; P < R; P += kFusedWarps) {
+      float4 v[F4];
+#pragma unroll
+      for (int m = 0; m < F4; ++m) v[m] = ldg_cg4(p.h + static_cast<size_t>(P) * I + 4 * (lane + 32 * m));
+      float amax = 0.f;
+#pragma unroll
+      for (int m = 0; m < F4; ++m)
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[m].x), fabsf(v[m].y)), fmaxf(fabsf(v[m].z), fabsf(v[m].w))));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float sig = pow2_scale_for(amax);
+      if (lane == 0) s_hinv[P] = 1.f / sig;
+#pragma unroll
+      for (int m = 0; m < F4; ++m) {
+        const int i0 = 4 * (lane + 32 * m);
+        const int pos = (((i0 & 31) >> 3) * VRD + (i0 >> 5)) * 8 + (i0 & 7);
+        uint2 w;
+        w.x = pack_f16x2(v[m].x * sig, v[m].y * sig);
+        w.y = pack_f16x2(v[m].z * sig, v[m].w * sig);
+        *reinterpret_cast<uint2*>(h16 + static_cast<size_t>(P) * I + pos) = w;
+      }
+    }
+  }
+  __syncthreads();
   const int rs = lane / VRD, cbk = lane % VRD;
   for (int it = warp; it < n_items && ok; it += kFusedWarps) {
     const int a = it / nsub, sb = it % nsub;
@@ -410,32 +513,17 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
       int P[TGD];
 #pragma unroll
       for (int t = 0; t < TGD; ++t) {
-        P[t] = 0;
-        yscale[t] = 0.f;
-        if (t < n) {
-          const int pr = dsc->pair[pb + g0 + t];
-          P[t] = (pr >> 8) * KS + (pr & 0xFF);
-          float v[32];
+        const int pr = dsc->pair[pb + g0 + min(t, n - 1)];
+        P[t] = (pr >> 8) * KS + (pr & 0xFF);
+        yscale[t] = sd * s_hinv[P[t]];
+        const uint16_t* hp = h16 + static_cast<size_t>(P[t]) * I + cbk * 8;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 f = hbytes ? *reinterpret_cast<const float4*>(hsm + static_cast<size_t>(P[t]) * I + cbk * 32 + 4 * q)
-                                    : ldg_cg4(p.h + static_cast<size_t>(P[t]) * I + cbk * 32 + 4 * q);
-            v[4 * q] = f.x;
-            v[4 * q + 1] = f.y;
-            v[4 * q + 2] = f.z;
-            v[4 * q + 3] = f.w;
-          }
-          float m = 0.f;
-#pragma unroll
-          for (int q = 0; q < 32; ++q) m = fmaxf(m, fabsf(v[q]));
-          m = segment_max<VRD>(m);
-          const float sig = pow2_scale_for(m);
-          yscale[t] = sd / sig;
-#pragma unroll
-          for (int q = 0; q < 16; ++q) hh[t * 16 + q] = pack_f16x2(v[2 * q] * sig, v[2 * q + 1] * sig);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 16; ++q) hh[t * 16 + q] = 0u;
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = (t < n) ? lds128(hp + q * VRD * 8) : make_uint4(0u, 0u, 0u, 0u);
+          hh[t * 16 + 4 * q + 0] = v.x;
+          hh[t * 16 + 4 * q + 1] = v.y;
+          hh[t * 16 + 4 * q + 2] = v.z;
+          hh[t * 16 + 4 * q + 3] = v.w;
         }
       }
       for (int rr = 0; rr < rows; rr += RPS) {

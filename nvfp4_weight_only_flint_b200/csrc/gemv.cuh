@@ -38,9 +38,12 @@ struct LayerParams {
   const uint16_t* residual;  // [T][d] bf16 or null
   uint16_t* out;             // [T][d] bf16
   int* status;               // workspace status word
-  unsigned* counter;         // router arrival counter (workspace, self-resetting)
+  unsigned* counter;         // control block word 1: router arrival counter (self-resetting);
+                             // word 2: launch generation of the persistent kernel;
+                             // words 32*(i+1), i < 4: its grid-barrier arrival counters
   RouteDesc* desc;           // routing descriptor (workspace)
   float* logits;             // [T][E]
+  unsigned long long* tlogits;  // [T][E] tagged logits of the persistent kernel
   int* ids;                  // [T][k]
   float* gates;              // [T][k]
   float* h;                  // [T*(k+S)][I] fp32 SwiGLU intermediates
@@ -110,15 +113,9 @@ __device__ __forceinline__ float route_code_value(uint32_t ord) {
   return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
 }
 
+// Selection on codes already loaded (code 0 = absent).
 template <int NE>
-__device__ __forceinline__ void topk_warp(const float* lg, int E, int k, int* ids, float* gates, int lane) {
-  uint32_t code[NE];
-#pragma unroll
-  for (int i = 0; i < NE; ++i) {
-    const int e = lane + 32 * i;
-    // code 0 marks "absent"; a finite logit's code is never 0
-    code[i] = (e < E) ? max(route_code(__ldcg(lg + e)), 1u) : 0u;
-  }
+__device__ __forceinline__ void topk_select(uint32_t (&code)[NE], int k, int* ids, float* gates, int lane) {
   float vals[kMaxTopK];
   int sel[kMaxTopK];
 #pragma unroll
@@ -168,11 +165,78 @@ __device__ __forceinline__ void topk_warp(const float* lg, int E, int k, int* id
   }
 }
 
+template <int NE>
+__device__ __forceinline__ void topk_warp(const float* lg, int E, int k, int* ids, float* gates, int lane) {
+  uint32_t code[NE];
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const int e = lane + 32 * i;
+    // code 0 marks "absent"; a finite logit's code is never 0
+    code[i] = (e < E) ? max(route_code(__ldcg(lg + e)), 1u) : 0u;
+  }
+  topk_select<NE>(code, k, ids, gates, lane);
+}
+
 __device__ __forceinline__ void topk_token(const float* lg, int E, int k, int* ids, float* gates, int lane) {
   if (E <= 256)
     topk_warp<8>(lg, E, k, ids, gates, lane);
   else
     topk_warp<kMaxExperts / 32>(lg, E, k, ids, gates, lane);
+}
+
+// Tagged logits: each is one 64-bit word (tag << 32 | float bits), stored with a
+// single relaxed 64-bit store, so a reader that sees the current tag also sees
+// that logit. Reading every logit of a token with the current tag is the
+// producer/consumer handshake: no fence or counter is needed.
+__device__ __forceinline__ void st_tagged(unsigned long long* p, uint32_t tag, float v) {
+  const unsigned long long w = (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_tagged(const unsigned long long* p) {
+  unsigned long long w;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return w;
+}
+
+// One warp, one token: waits (bounded) until all E logits carry `tag`, then
+// selects as topk_warp. Returns false (and records FLINT_DEVCHECK_WAIT) if the
+// wait gave up.
+template <int NE>
+__device__ __forceinline__ bool topk_warp_tagged(const unsigned long long* lg, int E, int k, uint32_t tag, int* ids,
+                                                 float* gates, int lane, int* status) {
+  uint32_t code[NE];
+  unsigned pending = 0;
+#pragma unroll
+  for (int i = 0; i < NE; ++i)
+    if (lane + 32 * i < E) pending |= 1u << i;
+  const long long t0 = clock64();
+  bool ok = true;
+  for (;;) {
+    unsigned long long w[NE];  // all loads issued before any is inspected
+#pragma unroll
+    for (int i = 0; i < NE; ++i) w[i] = (pending & (1u << i)) ? ld_tagged(lg + lane + 32 * i) : 0ull;
+#pragma unroll
+    for (int i = 0; i < NE; ++i) {
+      if ((pending & (1u << i)) && static_cast<uint32_t>(w[i] >> 32) == tag) {
+        pending &= ~(1u << i);
+        code[i] = max(route_code(__uint_as_float(static_cast<uint32_t>(w[i]))), 1u);
+      }
+    }
+    if (__all_sync(0xffffffffu, pending == 0)) break;
+    if (clock64() - t0 > kWaitCycles) {
+      ok = false;
+      break;
+    }
+  }
+  if (!ok) {
+    if (lane == 0) atomicOr(status, FLINT_DEVCHECK_WAIT);
+    return false;
+  }
+#pragma unroll
+  for (int i = 0; i < NE; ++i)
+    if (lane + 32 * i >= E) code[i] = 0u;
+  topk_select<NE>(code, k, ids, gates, lane);
+  return true;
 }
 
 // Token grouping built by a whole CTA from ids [T][k] (T <= 32): active

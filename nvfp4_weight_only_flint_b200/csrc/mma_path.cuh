@@ -1,0 +1,613 @@
+// mma_path.cuh -- the batch >= 32 layer path on the 5th-generation tensor cores.
+//
+// Kernels, chained with programmatic dependent launch:
+//   k_router_only / k_topk  router logits, top-k and gates (layer_kernels.cuh)
+//   k_mma_group     one CTA: expert histogram and token permutation -- the
+//                   active experts in ascending id order (shared expert last)
+//                   and, per expert, its (token, slot) pairs in token order
+//   k_mma_prep      the gathered activation rows in pair order, the MMA's B
+//                   operand: NVFP4 weights -> f16 rows x*sigma_t (sigma_t a
+//                   power of two per token, |x*sigma_t| <= 2^15); bf16 weights
+//                   -> the bf16 rows as they are
+//   k_mma_ffn<GATEUP>  persistent: work item (active expert, 64 units = 128
+//                   interleaved gate/up rows). Weights reach shared memory by
+//                   TMA; NVFP4 codes and scales are dequantised there to f16
+//                   (e2m1 * e4m3 is exact in f16) in the 128-byte-swizzled
+//                   K-major operand layout; tcgen05.mma (kind::f16, M=128,
+//                   N = the expert's tokens rounded up to 16, fp32 accumulators
+//                   in tensor memory, double-buffered) and an epilogue warpgroup
+//                   that applies the tensor scales, 1/sigma_t and SiLU*mul and
+//                   writes h (fp32) in pair order
+//   k_mma_hconv     h rows -> the down projection's B operand (f16 with a
+//                   power-of-two scale per row for NVFP4 weights, bf16 else)
+//   k_mma_ffn<DOWN> persistent: work item (active expert, 128 output rows),
+//                   K = I; the epilogue writes y_pair = s_d * W_d h per (token,
+//                   slot) in fp32
+//   k_mma_combine   out_t = sum_j gate_tj y_(t,j) + y_(t,shared) (+ residual),
+//                   fixed order, bf16
+// Roles in the persistent kernels (16 warps): warp 0 issues the TMA loads,
+// warp 1 owns the tensor memory and issues the MMAs (one thread), warps 4-7
+// are the epilogue warpgroup (warp 4+i reads accumulator lanes 32i..32i+31),
+// warps 8-15 dequantise. Every wait is bounded; a wait that gives up records
+// FLINT_DEVCHECK_WAIT, raises a CTA-wide abort flag, and every role then drains
+// what it started (copies in flight, MMAs committed) before the tensor memory
+// is released.
+#pragma once
+
+#include <cuda.h>
+
+#include "layer_kernels.cuh"
+
+namespace flint {
+
+constexpr int kMmaMaxTokens = 128;  // N of one MMA <= 128 (tokens of one expert)
+constexpr int kMmaWarps = 16;
+constexpr int kMmaRawStages = 3;    // NVFP4 codes+scales, 256 elements of K per stage
+constexpr int kMmaAStages = 4;      // A operand buffers (128 rows x 64 elements)
+constexpr int kMmaBStages = 4;      // B operand buffers (N rows x 64 elements)
+constexpr int kMmaRawBytes = 128 * 128 + 128 * 16;  // 18 KiB: codes (swizzled) + scales
+constexpr int kMmaABytes = 128 * 128;               // 16 KiB
+constexpr int kMmaBBytes = kMmaMaxTokens * 128;     // 16 KiB
+
+enum MmaEpi { kEpiGateUp = 0, kEpiDown = 1 };
+
+// Routing of the tensor-core path, in the workspace.
+struct MmaRoute {
+  int* n_active;  // [1]
+  int* act;       // [E+S] active experts (routed ascending, then shared)
+  int* off;       // [E+S+1] first pair of each active expert
+  int* pair;      // [T*(k+S)] token << 8 | slot, grouped by expert, token order
+};
+
+struct MmaParams {
+  const uint16_t* x;        // [T][d] bf16
+  const float* tscale;      // [E+S][3] (NVFP4) or null (bf16 weights: scale 1)
+  const uint16_t* residual; // [T][d] or null
+  uint16_t* out;            // [T][d]
+  int* status;
+  const int* ids;           // [T][k] from k_topk
+  const float* gates;       // [T][k]
+  int* ids_out;             // optional public copies
+  float* gates_out;
+  MmaRoute rt;
+  uint16_t* xrows;          // [P][d] B operand of gate/up (pair order)
+  float* xinv;              // [P] 1/sigma of each row (1 for bf16)
+  float* h;                 // [P][I] fp32, pair order
+  uint16_t* hrows;          // [P][I] B operand of down
+  float* hinv;              // [P]
+  float* y;                 // [T*(k+S)][d] fp32, row t*(k+S)+slot
+  int T, d, I, E, k, S;
+  int nvfp4;                // 1: NVFP4 weights, f16 operands; 0: bf16 weights, bf16 operands
+};
+
+// ----------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16, cta_group::1.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// Arrives on `bar` once every tcgen05 operation this thread issued so far is done.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+// 16 consecutive fp32 columns of this thread's accumulator lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory operand descriptor: K-major, 128-byte swizzle, 8-row groups of
+// 1024 bytes (stride dimension offset), version 1 (tcgen05).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t dsc = 0;
+  dsc |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  dsc |= static_cast<uint64_t>(16 >> 4) << 16;
+  dsc |= static_cast<uint64_t>(1024 >> 4) << 32;
+  dsc |= static_cast<uint64_t>(1) << 46;
+  dsc |= static_cast<uint64_t>(2) << 61;
+  return dsc;
+}
+// Instruction descriptor of kind::f16: fp32 accumulate, A and B both f16 or
+// both bf16, both K-major, M x N.
+__host__ __device__ constexpr uint32_t mma_idesc(int M, int N, bool bf16) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Bounded wait that also gives up when another role of the CTA aborted.
+__device__ __forceinline__ bool mma_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort_flag = 1;
+      atomicOr(status, FLINT_DEVCHECK_WAIT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// ----------------------------------------------------------------- grouping
+// One CTA of 512 threads, thread e counts expert e (E <= 512).
+__global__ void __launch_bounds__(512) k_mma_group(MmaParams p) {
+  __shared__ int s_ids[kMmaMaxTokens * kMaxTopK];
+  __shared__ int s_scan[512];
+  __shared__ int s_act[512];
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x, T = p.T, k = p.k, E = p.E, S = p.S, TK = T * k;
+  for (int i = tid; i < TK; i += blockDim.x) {
+    int e = p.ids[i];
+    if (e < 0 || e >= E) {
+      atomicOr(p.status, FLINT_DEVCHECK_EXPERT_ID);
+      e = -1;
+    }
+    s_ids[i] = e;
+    if (p.ids_out != nullptr) {
+      p.ids_out[i] = p.ids[i];
+      p.gates_out[i] = p.gates[i];
+    }
+  }
+  __syncthreads();
+  int cnt = 0;
+  if (tid < E)
+    for (int i = 0; i < TK; ++i) cnt += (s_ids[i] == tid) ? 1 : 0;
+  // block-wide exclusive scans of the counts and of the active flags
+  s_scan[tid] = cnt;
+  s_act[tid] = cnt > 0 ? 1 : 0;
+  __syncthreads();
+  for (int o = 1; o < 512; o <<= 1) {
+    const int a = tid >= o ? s_scan[tid - o] : 0, b = tid >= o ? s_act[tid - o] : 0;
+    __syncthreads();
+    s_scan[tid] += a;
+    s_act[tid] += b;
+    __syncthreads();
+  }
+  const int off = s_scan[tid] - cnt, pos = s_act[tid] - (cnt > 0 ? 1 : 0);
+  const int n_routed = s_act[511], routed_pairs = s_scan[511];
+  if (tid < E && cnt > 0) {
+    p.rt.act[pos] = tid;
+    p.rt.off[pos] = off;
+    int j = 0;
+    for (int i = 0; i < TK; ++i)
+      if (s_ids[i] == tid) p.rt.pair[off + j++] = ((i / k) << 8) | (i % k);
+  }
+  for (int s = 0; s < S; ++s) {
+    if (tid == 0) {
+      p.rt.act[n_routed + s] = E + s;
+      p.rt.off[n_routed + s] = routed_pairs + s * T;
+    }
+    for (int t = tid; t < T; t += blockDim.x) p.rt.pair[routed_pairs + s * T + t] = (t << 8) | (k + s);
+  }
+  if (tid == 0) {
+    p.rt.off[n_routed + S] = routed_pairs + S * T;
+    p.rt.n_active[0] = n_routed + S;
+  }
+}
+
+// ----------------------------------------------------------------- B rows of gate/up
+// Warp per pair row: x[token] (bf16) -> f16 * sigma_t (NVFP4) or bf16 copy.
+__global__ void __launch_bounds__(256) k_mma_prep(MmaParams p) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int P = p.T * (p.k + p.S), d = p.d;
+  for (int q = blockIdx.x * 8 + (threadIdx.x >> 5); q < P; q += gridDim.x * 8) {
+    const int tok = p.rt.pair[q] >> 8;
+    const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(tok) * d);
+    uint4* dst = reinterpret_cast<uint4*>(p.xrows + static_cast<size_t>(q) * d);
+    if (!p.nvfp4) {
+      for (int i = lane; i < d / 8; i += 32) dst[i] = __ldg(src + i);
+      if (lane == 0) p.xinv[q] = 1.f;
+      continue;
+    }
+    float amax = 0.f;
+    for (int i = lane; i < d / 8; i += 32) {
+      const uint4 v = __ldg(src + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu)), fabsf(__uint_as_float(w[j] & 0xFFFF0000u))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sg = pow2_scale_for(amax);
+    for (int i = lane; i < d / 8; i += 32) {
+      const uint4 v = __ldg(src + i);
+      uint4 o;
+      o.x = bf16x2_to_f16x2_scaled(v.x, sg);
+      o.y = bf16x2_to_f16x2_scaled(v.y, sg);
+      o.z = bf16x2_to_f16x2_scaled(v.z, sg);
+      o.w = bf16x2_to_f16x2_scaled(v.w, sg);
+      dst[i] = o;
+    }
+    if (lane == 0) p.xinv[q] = 1.f / sg;
+  }
+}
+
+// ----------------------------------------------------------------- B rows of down
+// Warp per pair row: h (fp32) -> f16 * sigma_row (NVFP4) or bf16.
+__global__ void __launch_bounds__(256) k_mma_hconv(MmaParams p) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int P = p.T * (p.k + p.S), I = p.I;
+  for (int q = blockIdx.x * 8 + (threadIdx.x >> 5); q < P; q += gridDim.x * 8) {
+    const float4* src = reinterpret_cast<const float4*>(p.h + static_cast<size_t>(q) * I);
+    uint2* dst = reinterpret_cast<uint2*>(p.hrows + static_cast<size_t>(q) * I);
+    float sg = 1.f;
+    if (p.nvfp4) {
+      float amax = 0.f;
+      for (int i = lane; i < I / 4; i += 32) {
+        const float4 v = __ldcg(src + i);
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      sg = pow2_scale_for(amax);
+    }
+    for (int i = lane; i < I / 4; i += 32) {
+      const float4 v = __ldcg(src + i);
+      uint2 o;
+      if (p.nvfp4) {
+        o.x = pack_f16x2(v.x * sg, v.y * sg);
+        o.y = pack_f16x2(v.z * sg, v.w * sg);
+      } else {
+        const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+        o.x = *reinterpret_cast<const uint32_t*>(&a);
+        o.y = *reinterpret_cast<const uint32_t*>(&b);
+      }
+      dst[i] = o;
+    }
+    if (lane == 0) p.hinv[q] = 1.f / sg;
+  }
+}
+
+// ----------------------------------------------------------------- combine
+// Thread per 8 outputs: fixed slot order 0..k-1, then the shared expert.
+__global__ void __launch_bounds__(256) k_mma_combine(MmaParams p) {
+  pdl_wait();
+  pdl_trigger();
+  const int KS = p.k + p.S, d8 = p.d / 8;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= p.T * d8) return;
+  const int t = idx / d8, c = idx % d8;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int j = 0; j < KS; ++j) {
+    const float g = (j < p.k) ? p.gates[t * p.k + j] : 1.f;
+    const float4* yr = reinterpret_cast<const float4*>(p.y + static_cast<size_t>(t * KS + j) * p.d + 8 * c);
+    const float4 a = __ldcg(yr), b = __ldcg(yr + 1);
+    acc[0] = fmaf(g, a.x, acc[0]);
+    acc[1] = fmaf(g, a.y, acc[1]);
+    acc[2] = fmaf(g, a.z, acc[2]);
+    acc[3] = fmaf(g, a.w, acc[3]);
+    acc[4] = fmaf(g, b.x, acc[4]);
+    acc[5] = fmaf(g, b.y, acc[5]);
+    acc[6] = fmaf(g, b.z, acc[6]);
+    acc[7] = fmaf(g, b.w, acc[7]);
+  }
+  const size_t o = static_cast<size_t>(t) * p.d + 8 * c;
+  if (p.residual != nullptr) {
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(p.residual + o));
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      acc[2 * j] += bf16_bits_to_f32(w[j] & 0xFFFFu);
+      acc[2 * j + 1] += __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  }
+  uint4 ov;
+  uint32_t* ow = reinterpret_cast<uint32_t*>(&ov);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * j], acc[2 * j + 1]);
+    ow[j] = *reinterpret_cast<const uint32_t*>(&b);
+  }
+  *reinterpret_cast<uint4*>(p.out + o) = ov;
+}
+
+// ----------------------------------------------------------------- the tensor-core FFN kernel
+// Tensor maps of one call. Raw NVFP4: codes [experts][rows][K/2] bytes, box
+// (128 B, 128 rows, 1), 128-byte swizzle; scales [experts][rows][K/16], box
+// (16 B, 128, 1). bf16 weights: [experts][rows][K] bf16, box (64, 128, 1),
+// 128-byte swizzle. B rows: [P][K] 16-bit, box (64, 16), 128-byte swizzle.
+struct MmaMaps {
+  CUtensorMap codes;
+  CUtensorMap scales;
+  CUtensorMap brows;
+};
+
+// Dequantise one 64-element slice of K of the 128-row A tile (256 threads):
+// thread (row r, half h) turns 32 codes and their 2 scales into 32 f16 values
+// written to the swizzled operand (16-byte chunk c of row r at c ^ (r % 8)).
+__device__ __forceinline__ void dequant_slice(const uint8_t* raw, int sub, uint8_t* a16, int dt) {
+  const int w = dt >> 5, l = dt & 31;
+  const int half = (l >> 3) & 1;
+  const int r = 16 * w + 8 * (l >> 4) + (l & 7);
+  const int chunk = 2 * sub + half;  // 16-byte code chunk of the 128-byte raw row
+  const uint4 cv = lds128(raw + r * 128 + ((chunk ^ (r & 7)) << 4));
+  const uint32_t s2 = *reinterpret_cast<const uint16_t*>(raw + 128 * 128 + r * 16 + 4 * sub + 2 * half);
+  uint32_t sh;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(sh) : "h"(static_cast<uint16_t>(s2)));
+  const __half2 hs = *reinterpret_cast<const __half2*>(&sh);
+  const __half2 sc[2] = {__low2half2(hs), __high2half2(hs)};
+  const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+  uint8_t* row = a16 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {  // 8 elements per q; words 0,1 -> block 0, words 2,3 -> block 1
+    uint32_t f[4];
+    e2m1x8_to_f16x2(cw[q], *reinterpret_cast<uint32_t(*)[4]>(&f[0]));
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&f[j]), sc[q >> 1]);
+      ow[j] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    const int c8 = 4 * half + q;  // 16-byte chunk of the 128-byte f16 row
+    *reinterpret_cast<uint4*>(row + ((c8 ^ (r & 7)) << 4)) = o;
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kMmaWarps * 32, 1)
+    k_mma_ffn(MmaParams p, const __grid_constant__ MmaMaps maps, int ncols) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t raw_full[kMmaRawStages], raw_empty[kMmaRawStages];
+  __shared__ __align__(8) uint64_t a_full[kMmaAStages], a_empty[kMmaAStages];
+  __shared__ __align__(8) uint64_t b_full[kMmaBStages], b_empty[kMmaBStages];
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ int s_nact;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool fp4 = p.nvfp4 != 0;
+  // 1024-aligned carve-up: [raw stages (NVFP4 only)][A stages][B stages]
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* raw = base;
+  uint8_t* abuf = raw + (fp4 ? kMmaRawStages * kMmaRawBytes : 0);
+  uint8_t* bbuf = abuf + kMmaAStages * kMmaABytes;
+  const int K = EPI == kEpiGateUp ? p.d : p.I;
+  const int tiles = EPI == kEpiGateUp ? p.I / 64 : p.d / 128;
+  const int n_sub = K / 64;
+  const int KS = p.k + p.S;
+
+  if (tid == 0) {
+    for (int i = 0; i < kMmaRawStages; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], 8);
+    }
+    for (int i = 0; i < kMmaAStages; ++i) {
+      mbar_init(&a_full[i], fp4 ? 8 : 1);
+      mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < kMmaBStages; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    mbar_init(&mma_done, 1);
+    fence_barrier_init();
+    s_abort = 0;
+  }
+  if (warp == 1) tmem_alloc(&s_tmem, static_cast<uint32_t>(ncols));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();
+  if (tid == 0) s_nact = p.rt.n_active[0];
+  __syncthreads();
+  pdl_trigger();
+  const uint32_t tmem = s_tmem;
+  const int n_items = s_nact * tiles;
+  volatile int* abort_flag = &s_abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int rc = 0, bc = 0, ac = 0;  // stages issued: raw, B, A (bf16 weights)
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const int a = it / tiles, t = it % tiles;
+        const int e = p.rt.act[a];
+        const int off = p.rt.off[a], nt = p.rt.off[a + 1] - off;
+        const int npad = (nt + 15) & ~15;
+        for (int s = 0; s < n_sub && ok; ++s) {
+          if (fp4 && (s & 3) == 0) {
+            const int slot = rc % kMmaRawStages;
+            if (!(ok = mma_wait(&raw_empty[slot], ((rc / kMmaRawStages) & 1) ^ 1, abort_flag, p.status))) break;
+            uint8_t* st = raw + slot * kMmaRawBytes;
+            mbar_arrive_expect_tx(&raw_full[slot], kMmaRawBytes);
+            tma_load_3d(st, &maps.codes, (s / 4) * 128, t * 128, e, &raw_full[slot]);
+            tma_load_3d(st + 128 * 128, &maps.scales, (s / 4) * 16, t * 128, e, &raw_full[slot]);
+            ++rc;
+          }
+          if (!fp4) {
+            const int slot = ac % kMmaAStages;
+            if (!(ok = mma_wait(&a_empty[slot], ((ac / kMmaAStages) & 1) ^ 1, abort_flag, p.status))) break;
+            mbar_arrive_expect_tx(&a_full[slot], kMmaABytes);
+            tma_load_3d(abuf + slot * kMmaABytes, &maps.codes, s * 64, t * 128, e, &a_full[slot]);
+            ++ac;
+          }
+          const int slot = bc % kMmaBStages;
+          if (!(ok = mma_wait(&b_empty[slot], ((bc / kMmaBStages) & 1) ^ 1, abort_flag, p.status))) break;
+          mbar_arrive_expect_tx(&b_full[slot], npad * 128);
+          for (int j = 0; j < npad / 16; ++j)
+            tma_load_2d(bbuf + slot * kMmaBBytes + j * 2048, &maps.brows, s * 64, off + 16 * j, &b_full[slot]);
+          ++bc;
+        }
+      }
+      // on abort: wait (bounded) for every copy this thread started; stages
+      // older than the ring depth were consumed, so they have landed
+      if (!ok) {
+        auto drain = [&](uint64_t* full, int ns, int n) {
+          for (int i = max(0, n - ns); i < n; ++i) mbar_wait(&full[i % ns], (i / ns) & 1, p.status);
+        };
+        drain(raw_full, kMmaRawStages, rc);
+        drain(a_full, kMmaAStages, ac);
+        drain(b_full, kMmaBStages, bc);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int sc = 0, bcount = 0, icount = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++icount) {
+        const int a = it / tiles;
+        const int nt = p.rt.off[a + 1] - p.rt.off[a];
+        const int npad = (nt + 15) & ~15;
+        const uint32_t idesc = mma_idesc(128, npad, !fp4);
+        const int ab = icount & 1;
+        if (!(ok = mma_wait(&acc_empty[ab], ((icount >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * kMmaMaxTokens);
+        for (int s = 0; s < n_sub; ++s) {
+          const int as = sc % kMmaAStages, bs = bcount % kMmaBStages;
+          if (!(ok = mma_wait(&a_full[as], (sc / kMmaAStages) & 1, abort_flag, p.status))) break;
+          if (!(ok = mma_wait(&b_full[bs], (bcount / kMmaBStages) & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          const uint32_t aaddr = smem_addr(abuf + as * kMmaABytes), baddr = smem_addr(bbuf + bs * kMmaBBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(d_tmem, sw128_desc(aaddr + 32 * kk), sw128_desc(baddr + 32 * kk), idesc, (s | kk) ? 1u : 0u);
+          mma_commit(&a_empty[as]);
+          mma_commit(&b_empty[bs]);
+          ++sc;
+          ++bcount;
+        }
+        if (ok) mma_commit(&acc_full[ab]);
+      }
+      // every MMA this thread issued completes before tensor memory is freed
+      mma_commit(&mma_done);
+      mbar_wait(&mma_done, 0, p.status);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------ epilogue warpgroup
+    const int ew = warp - 4, m = 32 * ew + lane;  // accumulator lane = A tile row
+    int icount = 0;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++icount) {
+      const int a = it / tiles, t = it % tiles;
+      const int e = p.rt.act[a];
+      const int off = p.rt.off[a], nt = p.rt.off[a + 1] - off;
+      const int ab = icount & 1;
+      if (!mma_wait(&acc_full[ab], (icount >> 1) & 1, abort_flag, p.status)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * ew) << 16) + static_cast<uint32_t>(ab * kMmaMaxTokens);
+      if (EPI == kEpiGateUp) {
+        const float sgt = fp4 ? __ldg(p.tscale + 3 * e + 0) : 1.f, sut = fp4 ? __ldg(p.tscale + 3 * e + 1) : 1.f;
+        const int unit = t * 64 + (m >> 1);
+        for (int c0 = 0; c0 < nt; c0 += 16) {
+          float v[16];
+          tmem_ld16(taddr + c0, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
+            const int n = c0 + j;
+            if ((m & 1) == 0 && n < nt) {
+              const float xi = p.xinv[off + n];
+              p.h[static_cast<size_t>(off + n) * p.I + unit] = swiglu(v[j] * sgt * xi, other * sut * xi);
+            }
+          }
+        }
+      } else {
+        const float sdt = fp4 ? __ldg(p.tscale + 3 * e + 2) : 1.f;
+        const int row = t * 128 + m;
+        for (int c0 = 0; c0 < nt; c0 += 16) {
+          float v[16];
+          tmem_ld16(taddr + c0, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + j;
+            if (n < nt) {
+              const int pr = p.rt.pair[off + n];
+              const int yrow = (pr >> 8) * KS + (pr & 0xFF);
+              p.y[static_cast<size_t>(yrow) * p.d + row] = v[j] * sdt * p.hinv[off + n];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+    }
+  } else if (warp >= 8 && fp4) {
+    // ------------------------------------------------ dequantisers (NVFP4)
+    const int dt = tid - 8 * 32;
+    int rc = 0, sc = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      for (int s = 0; s < n_sub; ++s) {
+        const int rs = rc % kMmaRawStages, as = sc % kMmaAStages;
+        if (!(ok = mma_wait(&raw_full[rs], (rc / kMmaRawStages) & 1, abort_flag, p.status))) break;
+        if (!(ok = mma_wait(&a_empty[as], ((sc / kMmaAStages) & 1) ^ 1, abort_flag, p.status))) break;
+        dequant_slice(raw + rs * kMmaRawBytes, s & 3, abuf + as * kMmaABytes, dt);
+        // generic-proxy writes of the operand -> visible to the tensor cores
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[as]);
+        ++sc;
+        if ((s & 3) == 3) {
+          if (lane == 0) mbar_arrive(&raw_empty[rs]);
+          ++rc;
+        }
+      }
+    }
+  }
+  // ------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, static_cast<uint32_t>(ncols));
+  }
+}
+
+}  // namespace flint
