@@ -391,8 +391,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=47 * 2 * 3)
     ap.add_argument("--impl", choices=["flint", "reference"], default="flint")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--no-extras", action="store_true", help="skip the batch-8 / batch-4 lines")
+    ap.add_argument("--no-extras", action="store_true", help="skip the batch-8 / batch-4 / batch-64 lines")
+    ap.add_argument("--profile", choices=["t1", "t8", "t64_nvfp4", "t64_bf16"], default=None,
+                    help="profiling case: one layer, --steps eager layer calls, no timing output")
     args = ap.parse_args()
+    if args.profile:
+        return run_profile_case(args)
     if args.warmup < 3:
         args.warmup = 3
 
@@ -535,6 +539,29 @@ def main():
     if _DIST["on"]:
         import torch.distributed as dist
         dist.destroy_process_group()
+    return 0
+
+
+def run_profile_case(args):
+    """A small, self-contained case for ncu: one Flint-shaped layer (0.46 GB
+    NVFP4 or 1.6 GB bf16 on the device) and `--steps` eager layer calls."""
+    import torch
+    import nvfp4_weight_only_flint_b200 as fm
+    fm.lib()
+    name = {"t1": "cfg1", "t8": "cfg2", "t64_nvfp4": "cfg4_nvfp4", "t64_bf16": "cfg4_bf16"}[args.profile]
+    w = synth.CONFIGS[name]
+    st = Stack(synth.CONFIGS["cfg1"], 1, args.seed, max_tokens=w.T, wdtype=w.wdtype)
+    xb = synth.x_bits(args.seed + 3000, w.T, w.d)
+    x = _bits_to_cuda(xb)
+    wr = _bits_to_cuda(synth.make_router(w, args.seed, xb))
+    out = torch.empty_like(x)
+    opt = fm.Options(path=fm.FLINT_PATH_AUTO, use_pdl=1)
+    for _ in range(max(1, args.steps)):
+        fm.flint_moe_forward_ex(x, w.T, wr, st.layers[0][3], st.shape, None, out, st.ws, opt)
+    torch.cuda.synchronize()
+    rc, flags = fm.flint_moe_get_status(st.ws)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} flags {flags}")
     return 0
 
 

@@ -289,136 +289,103 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     }
   };
 
-  // ---- P1b: the shared expert's units of this warp, for every token
-  if (sh_end > sh_begin) {
-    const float sg = __ldg(p.tscale + 3 * E + 0), su = __ldg(p.tscale + 3 * E + 1);
-    for (int u = sh_begin; u < sh_end && ok;) {
-      const int cu = min(M::CU, sh_end - u);
-      const int slot = consumed % ns_g;
-      if (!mbar_wait(&bars[slot], (consumed / ns_g) & 1, p.status)) {
-        ok = false;
-        break;
-      }
-      compute_chunk(ring + slot * p.stage_gateup, cu, u, sg, su, 1 << 20, T, nullptr, k);
-      __syncwarp();
-      ++consumed;
-      u += cu;
-      if (sh_issue < sh_end) {
-        const int cn = min(M::CU, sh_end - sh_issue);
-        if (lane == 0) {
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          issue_units(E, sh_issue, cn, issued % ns_g);
-        }
-        sh_issue += cn;
-        ++issued;
-      }
-    }
-    if (!ok) {
-      drain_ring(bars, ns_g, consumed, issued, p.status);
-      consumed = issued;
-    }
-  }
-
   // ---- P2: top-k (waits for every CTA's logits) and grouping, in every CTA
-  if (warp < T) {
-    bool okt = false;
-    if (ok) {
-      if (E <= 256)
-        okt = topk_warp_tagged<8>(p.tlogits + static_cast<size_t>(warp) * E, E, k, tag, &s_ids[warp * k],
-                                  &s_gates[warp * k], lane, p.status);
-      else
-        okt = topk_warp_tagged<kMaxExperts / 32>(p.tlogits + static_cast<size_t>(warp) * E, E, k, tag,
-                                                 &s_ids[warp * k], &s_gates[warp * k], lane, p.status);
+  // (called once by every warp, from inside the chunk loop below)
+  auto routing_step = [&]() {
+    if (!ok && lane == 0) s_fail = 1;  // a wait of this warp gave up: the CTA stops together
+    if (warp < T) {
+      bool okt = false;
+      if (ok) {
+        if (E <= 256)
+          okt = topk_warp_tagged<8>(p.tlogits + static_cast<size_t>(warp) * E, E, k, tag, &s_ids[warp * k],
+                                    &s_gates[warp * k], lane, p.status);
+        else
+          okt = topk_warp_tagged<kMaxExperts / 32>(p.tlogits + static_cast<size_t>(warp) * E, E, k, tag,
+                                                   &s_ids[warp * k], &s_gates[warp * k], lane, p.status);
+      }
+      if (!okt && lane == 0) s_fail = 1;
     }
-    if (!okt && lane == 0) s_fail = 1;
-  }
-  __syncthreads();
-  if (s_fail) ok = false;
-  if (warp == 0 && ok) warp_grouping(s_ids, T, k, E, S, dsc, lane, p.status);
-  __syncthreads();
-  if (c == 0 && ok) {
-    for (int i = tid; i < T * k; i += blockDim.x) {
-      p.ids[i] = s_ids[i];
-      p.gates[i] = s_gates[i];
-      if (p.ids_out != nullptr) {
-        p.ids_out[i] = s_ids[i];
-        p.gates_out[i] = s_gates[i];
+    __syncthreads();
+    if (s_fail) ok = false;
+    // the ring area is idle here (every warp has drained its shared-expert
+    // chunks), so it serves as the grouping's scratch
+    if (ok) cta_grouping(s_ids, T, k, E, S, dsc, work, p.status);
+    if (c == 0 && ok) {
+      for (int i = tid; i < T * k; i += blockDim.x) {
+        p.ids[i] = s_ids[i];
+        p.gates[i] = s_gates[i];
+        if (p.ids_out != nullptr) {
+          p.ids_out[i] = s_ids[i];
+          p.gates_out[i] = s_gates[i];
+        }
       }
     }
-  }
-  const int n_active = ok ? dsc->n_active : 0;
-  // L2 prefetch of this CTA's block of down rows of every routed active expert
-  if (ok && tid < dsc->n_routed && nrows > 0) {
-    const long long e = dsc->act[tid];
-    prefetch_l2(p.codes + e * p.cpe + static_cast<long long>(I) * p.d + static_cast<long long>(n0) * ROWC, nrows * ROWC);
-    prefetch_l2(p.scales + e * p.spe + static_cast<long long>(I) * p.d / 8 + static_cast<long long>(n0) * ROWS,
-                nrows * ROWS);
-  }
+    // L2 prefetch of this CTA's block of down rows of every routed active expert
+    if (ok && tid < dsc->n_routed && nrows > 0) {
+      const long long e = dsc->act[tid];
+      prefetch_l2(p.codes + e * p.cpe + static_cast<long long>(I) * p.d + static_cast<long long>(n0) * ROWC,
+                  nrows * ROWC);
+      prefetch_l2(p.scales + e * p.spe + static_cast<long long>(I) * p.d / 8 + static_cast<long long>(n0) * ROWS,
+                  nrows * ROWS);
+    }
+  };
 
-  // ---- P3: gate/up of the routed experts. This warp's range of the cost
-  // space (units x token passes), mapped to units.
-  {
-    const int n_routed = ok ? dsc->n_routed : 0;
-    int* cost = s_cost[warp];
-    cost_prefix(dsc, n_routed, I, M::TGMAX, cost, lane);
-    __syncwarp();
-    const long long C = n_routed > 0 ? cost[n_routed] : 0;
-    const long long c_begin = gw * C / NW, c_end = (gw + 1) * C / NW;
-    auto to_unit = [&](long long cc, int& a, int& u) {
-      int lo = 0, hi = n_routed - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (cost[mid] <= cc) lo = mid;
-        else hi = mid - 1;
+  // ---- P1b + P3: one stream of chunks per warp. Phase 0: this warp's slice
+  // of the shared expert's units (index = unit), for every token. Then the
+  // routing step, then phase 1: this warp's range of the routed experts' cost
+  // space (units x token passes), index = active expert * I + unit. One loop,
+  // so the chunk code exists once.
+  int phase = 0;
+  int g = sh_begin, g_end = sh_end, issue_g = sh_issue;
+  int cur_a = -1;
+  float sg = S > 0 ? __ldg(p.tscale + 3 * E + 0) : 0.f, su = S > 0 ? __ldg(p.tscale + 3 * E + 1) : 0.f;
+  auto chunk_len = [&](int gg) {
+    return phase == 0 ? min(M::CU, g_end - gg) : min(M::CU, min(I - gg % I, g_end - gg));
+  };
+  for (;;) {
+    if (g >= g_end || !ok) {
+      if (phase == 1) break;
+      if (!ok) {
+        drain_ring(bars, ns_g, consumed, issued, p.status);
+        consumed = issued;
       }
-      a = lo;
-      const int passes = (dsc->off[a + 1] - dsc->off[a] + M::TGMAX - 1) / M::TGMAX;
-      u = static_cast<int>((cc - cost[a]) / passes);
-    };
-    int g_begin = 0, g_end = 0;
-    if (c_end > c_begin) {
-      int a0, u0, a1, u1;
-      to_unit(c_begin, a0, u0);
-      to_unit(c_end - 1, a1, u1);
-      g_begin = a0 * I + u0;
-      g_end = a1 * I + u1 + 1;
-      if (c_begin > 0) {  // a unit already started by the previous warp's range is left to it
-        int pa, pu;
-        to_unit(c_begin - 1, pa, pu);
-        if (pa == a0 && pu == u0) ++g_begin;
-      }
-    }
-    auto chunk_len = [&](int g) { return min(M::CU, min(I - g % I, g_end - g)); };
-    int issue_g = g_begin;
-    while (issued - consumed < ns_g && issue_g < g_end) {
-      if (lane == 0) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue_units(dsc->act[issue_g / I], issue_g % I, chunk_len(issue_g), issued % ns_g);
-      }
-      issue_g += chunk_len(issue_g);
-      ++issued;
-    }
-    int cur_a = -1;
-    float sg = 0.f, su = 0.f;
-    for (int g = g_begin; g < g_end && ok;) {
-      const int a = g / I, uu = g % I, cu = chunk_len(g);
-      if (a != cur_a) {  // tensor scales of the expert, fetched before the stage wait
-        const int e = dsc->act[a];
-        sg = __ldg(p.tscale + 3 * e + 0);
-        su = __ldg(p.tscale + 3 * e + 1);
-        cur_a = a;
-      }
-      const int slot = consumed % ns_g;
-      if (!mbar_wait(&bars[slot], (consumed / ns_g) & 1, p.status)) {
-        ok = false;
-        break;
-      }
-      const int pb = dsc->off[a], nt = dsc->off[a + 1] - pb;
-      compute_chunk(ring + slot * p.stage_gateup, cu, uu, sg, su, a, nt, dsc->pair + pb, 0);
+      routing_step();
+      // this warp's range of the routed cost space, mapped to units
+      const int n_routed = ok ? dsc->n_routed : 0;
+      int* cost = s_cost[warp];
+      cost_prefix(dsc, n_routed, I, M::TGMAX, cost, lane);
       __syncwarp();
-      ++consumed;
-      g += cu;
-      if (issue_g < g_end) {
+      const long long C = n_routed > 0 ? cost[n_routed] : 0;
+      const long long c_begin = gw * C / NW, c_end = (gw + 1) * C / NW;
+      auto to_unit = [&](long long cc, int& a, int& u) {
+        int lo = 0, hi = n_routed - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (cost[mid] <= cc) lo = mid;
+          else hi = mid - 1;
+        }
+        a = lo;
+        const int passes = (dsc->off[a + 1] - dsc->off[a] + M::TGMAX - 1) / M::TGMAX;
+        u = static_cast<int>((cc - cost[a]) / passes);
+      };
+      int g_begin = 0;
+      g_end = 0;
+      if (c_end > c_begin) {
+        int a0, u0, a1, u1;
+        to_unit(c_begin, a0, u0);
+        to_unit(c_end - 1, a1, u1);
+        g_begin = a0 * I + u0;
+        g_end = a1 * I + u1 + 1;
+        if (c_begin > 0) {  // a unit already started by the previous warp's range is left to it
+          int pa, pu;
+          to_unit(c_begin - 1, pa, pu);
+          if (pa == a0 && pu == u0) ++g_begin;
+        }
+      }
+      phase = 1;
+      g = g_begin;
+      issue_g = g_begin;
+      while (issued - consumed < ns_g && issue_g < g_end) {
         if (lane == 0) {
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           issue_units(dsc->act[issue_g / I], issue_g % I, chunk_len(issue_g), issued % ns_g);
@@ -426,9 +393,53 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
         issue_g += chunk_len(issue_g);
         ++issued;
       }
+      continue;
     }
-    if (!ok) drain_ring(bars, ns_g, consumed, issued, p.status);
+    const int cu = chunk_len(g);
+    int key, nt, uu, kslot;
+    const unsigned short* pairs;
+    if (phase == 0) {
+      key = -2;
+      nt = T;
+      uu = g;
+      pairs = nullptr;
+      kslot = k;
+    } else {
+      const int a = g / I;
+      if (a != cur_a) {  // tensor scales of the expert, fetched before the stage wait
+        const int e = dsc->act[a];
+        sg = __ldg(p.tscale + 3 * e + 0);
+        su = __ldg(p.tscale + 3 * e + 1);
+        cur_a = a;
+      }
+      key = a;
+      uu = g % I;
+      const int pb = dsc->off[a];
+      nt = dsc->off[a + 1] - pb;
+      pairs = dsc->pair + pb;
+      kslot = 0;
+    }
+    const int slot = consumed % ns_g;
+    if (!mbar_wait(&bars[slot], (consumed / ns_g) & 1, p.status)) {
+      ok = false;
+      continue;
+    }
+    compute_chunk(ring + slot * p.stage_gateup, cu, uu, sg, su, key, nt, pairs, kslot);
+    __syncwarp();
+    ++consumed;
+    g += cu;
+    if (issue_g < g_end) {
+      const int cn = chunk_len(issue_g);
+      if (lane == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue_units(phase == 0 ? E : dsc->act[issue_g / I], phase == 0 ? issue_g : issue_g % I, cn, issued % ns_g);
+      }
+      issue_g += cn;
+      ++issued;
+    }
   }
+  const int n_active = ok ? dsc->n_active : 0;
+  if (!ok) drain_ring(bars, ns_g, consumed, issued, p.status);
   if (!grid_barrier(p.counter, gen, p.status, &s_ok)) ok = false;
   if (c == 0 && tid == 0) asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p.counter + 1), "r"(gen + 1u) : "memory");
 

@@ -113,55 +113,43 @@ __device__ __forceinline__ float route_code_value(uint32_t ord) {
   return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
 }
 
-// Selection on codes already loaded (code 0 = absent).
+// Selection on codes already loaded (code 0 = absent). Round r's winner is
+// kept by lane r, so the rounds need no per-lane arrays (a rolled loop: this
+// code runs once per token and launch, so its size matters more than its ILP).
 template <int NE>
 __device__ __forceinline__ void topk_select(uint32_t (&code)[NE], int k, int* ids, float* gates, int lane) {
-  float vals[kMaxTopK];
-  int sel[kMaxTopK];
+  float my_val = 0.f, v0 = 0.f;
+  int my_sel = 0;
+#pragma unroll 1
+  for (int r = 0; r < k; ++r) {
+    uint32_t best = code[0];
+    int bi = 0;
 #pragma unroll
-  for (int r = 0; r < kMaxTopK; ++r) {
-    vals[r] = 0.f;
-    sel[r] = 0;
-    if (r < k) {
-      uint32_t best = code[0];
-      int bi = 0;
-#pragma unroll
-      for (int i = 1; i < NE; ++i)
-        if (code[i] > best) {  // strict: equal codes keep the lower index
-          best = code[i];
-          bi = i;
-        }
-      const uint32_t m = __reduce_max_sync(0xffffffffu, best);
-      const uint32_t w = __reduce_max_sync(0xffffffffu, best == m ? 0xFFFFFFFFu - (lane + 32 * bi) : 0u);
-      const int e = static_cast<int>(0xFFFFFFFFu - w);
-      if ((e & 31) == lane) {
-#pragma unroll
-        for (int i = 0; i < NE; ++i)
-          if (i == (e >> 5)) code[i] = 0u;
+    for (int i = 1; i < NE; ++i)
+      if (code[i] > best) {  // strict: equal codes keep the lower index
+        best = code[i];
+        bi = i;
       }
-      vals[r] = route_code_value(m);
-      sel[r] = e;
+    const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+    const uint32_t w = __reduce_max_sync(0xffffffffu, best == m ? 0xFFFFFFFFu - (lane + 32 * bi) : 0u);
+    const int e = static_cast<int>(0xFFFFFFFFu - w);
+    if ((e & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i < NE; ++i)
+        if (i == (e >> 5)) code[i] = 0u;
+    }
+    const float v = route_code_value(m);
+    if (r == 0) v0 = v;
+    if (lane == r) {
+      my_val = v;
+      my_sel = e;
     }
   }
-  float ex[kMaxTopK];
-  float sum = 0.f;
-#pragma unroll
-  for (int r = 0; r < kMaxTopK; ++r) {
-    ex[r] = (r < k) ? __expf(vals[r] - vals[0]) : 0.f;
-    sum += ex[r];
-  }
-  const float inv = 1.f / sum;
+  const float ex = (lane < k) ? __expf(my_val - v0) : 0.f;
+  const float sum = warp_sum(ex);
   if (lane < k) {
-    int id = 0;
-    float gt = 0.f;
-#pragma unroll
-    for (int r = 0; r < kMaxTopK; ++r)
-      if (r == lane) {
-        id = sel[r];
-        gt = ex[r] * inv;
-      }
-    ids[lane] = id;
-    gates[lane] = gt;
+    ids[lane] = my_sel;
+    gates[lane] = ex * (1.f / sum);
   }
 }
 
@@ -410,6 +398,100 @@ __device__ void warp_grouping(const int* ids, int T, int k, int E, int S, RouteD
     d->n_routed = U;
     d->n_active = U + S;
   }
+}
+
+// Token grouping by a whole CTA (blockDim.x >= E/2, blockDim.x a multiple of
+// 32) for T*k <= 64 pairs, through a 64-bit pair mask per expert: pair i =
+// t*k + j sets bit i of its expert's mask, so a pair's place among its
+// expert's pairs (token order) is the popcount of the lower bits; exclusive
+// scans over the experts give the active list (ascending id) and the offsets.
+// Shared experts follow, with every token in slot k+s. `scratch`: 12*E bytes
+// of shared memory, 8-byte aligned. Writes the same fields as warp_grouping.
+__device__ void cta_grouping(const int* ids, int T, int k, int E, int S, RouteDesc* d, uint8_t* scratch,
+                             int* status) {
+  __shared__ int s_tot[2][32];
+  unsigned long long* emask = reinterpret_cast<unsigned long long*>(scratch);
+  int* eoff = reinterpret_cast<int*>(scratch + 8 * static_cast<size_t>(E));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5, n = T * k;
+  for (int e = tid; e < E; e += blockDim.x) emask[e] = 0ull;
+  __syncthreads();
+  for (int i = tid; i < n; i += blockDim.x) {
+    const int e = ids[i];
+    if (e < 0 || e >= E) {
+      atomicOr(status, FLINT_DEVCHECK_EXPERT_ID);
+      continue;
+    }
+    atomicOr(&emask[e], 1ull << i);
+  }
+  __syncthreads();
+  // thread owns experts 2*tid and 2*tid+1
+  const int e0 = 2 * tid, e1 = 2 * tid + 1;
+  const int c0 = e0 < E ? __popcll(emask[e0]) : 0, c1 = e1 < E ? __popcll(emask[e1]) : 0;
+  const int f0 = c0 > 0, f1 = c1 > 0;
+  int ic = c0 + c1, jf = f0 + f1;  // inclusive scans over the block
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int vc = __shfl_up_sync(0xffffffffu, ic, o), vf = __shfl_up_sync(0xffffffffu, jf, o);
+    if (lane >= o) {
+      ic += vc;
+      jf += vf;
+    }
+  }
+  if (lane == 31) {
+    s_tot[0][warp] = ic;
+    s_tot[1][warp] = jf;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int wc = lane < nw ? s_tot[0][lane] : 0, wf = lane < nw ? s_tot[1][lane] : 0;
+    const int xc = wc, xf = wf;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int vc = __shfl_up_sync(0xffffffffu, wc, o), vf = __shfl_up_sync(0xffffffffu, wf, o);
+      if (lane >= o) {
+        wc += vc;
+        wf += vf;
+      }
+    }
+    __syncwarp();
+    if (lane < nw) {
+      s_tot[0][lane] = wc - xc;  // exclusive prefix of the warp totals
+      s_tot[1][lane] = wf - xf;
+    }
+    if (lane == nw - 1) {
+      d->n_routed = wf;
+      d->n_active = wf + S;
+      for (int s = 0; s < S; ++s) {
+        d->act[wf + s] = E + s;
+        d->off[wf + s] = wc + s * T;
+      }
+      d->off[wf + S] = wc + S * T;
+    }
+  }
+  __syncthreads();
+  const int base_c = ic - (c0 + c1) + s_tot[0][warp], base_f = jf - (f0 + f1) + s_tot[1][warp];
+  if (f0) {
+    d->act[base_f] = e0;
+    d->off[base_f] = base_c;
+    eoff[e0] = base_c;
+  }
+  if (f1) {
+    d->act[base_f + f0] = e1;
+    d->off[base_f + f0] = base_c + c0;
+    eoff[e1] = base_c + c0;
+  }
+  __syncthreads();
+  for (int i = tid; i < n; i += blockDim.x) {
+    const int e = ids[i];
+    if (e < 0 || e >= E) continue;
+    const int pos = eoff[e] + __popcll(emask[e] & ((1ull << i) - 1ull));
+    d->pair[pos] = static_cast<unsigned short>(((i / k) << 8) | (i % k));
+  }
+  for (int i = tid; i < S * T; i += blockDim.x) {
+    const int s = i / T, t = i % T;
+    d->pair[n + i] = static_cast<unsigned short>((t << 8) | (k + s));
+  }
+  __syncthreads();
 }
 
 // ----------------------------------------------------------------- gate/up lane map

@@ -286,43 +286,43 @@ __device__ __forceinline__ void gateup_chunk(const uint8_t* st, int cu, const ui
                                              int n, const float* fscale_g, const float* fscale_u,
                                              const int* hrow, float* h, int I, int u0) {
   using M = GateUpMap<D>;
-  constexpr int V = M::CU * TG * 2;
+  constexpr int V = TG * 2;  // (token, gate|up) partial sums per unit
   constexpr int LV = ilog2(V);
-  float acc[V];
+  // one unit per iteration, reduced on its own: a rolled loop keeps the code
+  // this runs (once or twice per launch at decode batch) small
+#pragma unroll 1
+  for (int c = 0; c < cu; ++c) {
+    float acc[V];
 #pragma unroll
-  for (int i = 0; i < V; ++i) acc[i] = 0.f;
+    for (int i = 0; i < V; ++i) acc[i] = 0.f;
 #pragma unroll
-  for (int c = 0; c < M::CU; ++c) {
-    if (c < cu) {
+    for (int j = 0; j < M::NVU; ++j) {
+      int co, so, r, xi;
+      M::vec(lane, j, co, so, r, xi);
+      const uint4 cvec = lds128(st + c * M::UNIT_CODE + co);
+      const uint32_t s2 = *reinterpret_cast<const uint16_t*>(st + M::CU * M::UNIT_CODE + c * M::UNIT_SCALE + so);
+      float tmp[TG];
 #pragma unroll
-      for (int j = 0; j < M::NVU; ++j) {
-        int co, so, r, xi;
-        M::vec(lane, j, co, so, r, xi);
-        const uint4 cvec = lds128(st + c * M::UNIT_CODE + co);
-        const uint32_t s2 = *reinterpret_cast<const uint16_t*>(st + M::CU * M::UNIT_CODE + c * M::UNIT_SCALE + so);
-        float tmp[TG];
+      for (int t = 0; t < TG; ++t) tmp[t] = 0.f;
+      dot32_strided<TG, M::XS>(cvec, s2, xh + xi * 16, tmp);
 #pragma unroll
-        for (int t = 0; t < TG; ++t) tmp[t] = 0.f;
-        dot32_strided<TG, M::XS>(cvec, s2, xh + xi * 16, tmp);
-#pragma unroll
-        for (int t = 0; t < TG; ++t) {
-          if constexpr (M::VR >= 32) {
-            acc[((c * TG + t) << 1) | (j / M::XV)] += tmp[t];
-          } else {
-            acc[(c * TG + t) << 1] += r ? 0.f : tmp[t];
-            acc[((c * TG + t) << 1) | 1] += r ? tmp[t] : 0.f;
-          }
+      for (int t = 0; t < TG; ++t) {
+        if constexpr (M::VR >= 32) {
+          acc[(t << 1) | (j / M::XV)] += tmp[t];
+        } else {
+          acc[t << 1] += r ? 0.f : tmp[t];
+          acc[(t << 1) | 1] += r ? tmp[t] : 0.f;
         }
       }
     }
+    const float total = xreduce<32, V>(acc, lane);
+    const int rep = 5 - LV;  // lanes per value = 1 << rep
+    const float other = __shfl_xor_sync(0xffffffffu, total, 1 << rep);
+    const int idx = lane >> rep;
+    const int r = idx & 1, t = idx >> 1;
+    if (r == 0 && (lane & ((1 << rep) - 1)) == 0 && t < n)
+      h[static_cast<size_t>(hrow[t]) * I + u0 + c] = swiglu(total * fscale_g[t], other * fscale_u[t]);
   }
-  const float total = xreduce<32, V>(acc, lane);
-  const int rep = 5 - LV;  // lanes per value = 1 << rep
-  const float other = __shfl_xor_sync(0xffffffffu, total, 1 << rep);
-  const int idx = lane >> rep;
-  const int r = idx & 1, t = (idx >> 1) % TG, c = (idx >> 1) / TG;
-  if (r == 0 && (lane & ((1 << rep) - 1)) == 0 && c < cu && t < n)
-    h[static_cast<size_t>(hrow[t]) * I + u0 + c] = swiglu(total * fscale_g[t], other * fscale_u[t]);
 }
 
 template <int D>
