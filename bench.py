@@ -61,9 +61,11 @@ def _tensor_peak(wdtype: str):
         return 1590.0, "fallback"
 
 
-# DRAM bytes (read + write) of one k_layer launch at batch 1, from the ncu
-# capture summarised in profiles/; None until a capture of the current kernel.
-TRAFFIC_K_LAYER_T1 = None
+# DRAM bytes (read + write) of one k_layer launch at batch 1, from an ncu
+# capture of `bench.py --profile t1` (dram__bytes_read.sum 13,614,336 B,
+# dram__bytes_write.sum 0 B); set to None whenever the kernel changes until it
+# is captured again.
+TRAFFIC_K_LAYER_T1 = 13614336
 
 
 def _host_cores():
