@@ -138,13 +138,17 @@ __device__ __forceinline__ void dot32_strided(const uint4 c, uint32_t scale2, co
   const float2 s = e4m3x2_to_f32x2(scale2);
 #pragma unroll
   for (int t = 0; t < TG; ++t) {
-    float p0 = 0.f, p1 = 0.f;
+    // two partial sums per block: dependency chains of 8 fused multiply-adds
+    float p0a = 0.f, p0b = 0.f, p1a = 0.f, p1b = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) fma2_f16_f32(q[i], xh[t * XS + i], p0);
-#pragma unroll
-    for (int i = 8; i < 16; ++i) fma2_f16_f32(q[i], xh[t * XS + i], p1);
-    acc[t] = fmaf(p0, s.x, acc[t]);
-    acc[t] = fmaf(p1, s.y, acc[t]);
+    for (int i = 0; i < 8; i += 2) {
+      fma2_f16_f32(q[i], xh[t * XS + i], p0a);
+      fma2_f16_f32(q[i + 1], xh[t * XS + i + 1], p0b);
+      fma2_f16_f32(q[i + 8], xh[t * XS + i + 8], p1a);
+      fma2_f16_f32(q[i + 9], xh[t * XS + i + 9], p1b);
+    }
+    acc[t] = fmaf(p0a + p0b, s.x, acc[t]);
+    acc[t] = fmaf(p1a + p1b, s.y, acc[t]);
   }
 }
 

@@ -260,7 +260,7 @@ WsLayout ws_layout(const Dims& s, int maxT) {
   w.logits = o;
   o += al256(sizeof(float) * static_cast<size_t>(maxT) * s.E);
   w.tlogits = o;
-  o += al256(sizeof(unsigned long long) * static_cast<size_t>(maxT) * s.E);
+  o += al256(sizeof(unsigned long long) * kLogitReplicas * static_cast<size_t>(maxT) * s.E);
   w.ids = o;
   o += al256(sizeof(int) * static_cast<size_t>(maxT) * s.k);
   w.gates = o;
@@ -420,6 +420,7 @@ size_t down_smem(const LayerParams& p) {
 // dynamic shared-memory bytes, or 0 if the call does not fit it.
 size_t configure_fused(LayerParams& p, const Dims& s, int T) {
   const int sms = num_sms();
+  if (sms > 240) return 0;  // the kernel's work split uses 32-bit products of the CTA index
   p.stage_gateup = gateup_stage_bytes(s.d);
   p.ns_gateup = 2;
   const int rps = 32 / (s.I / 32);
@@ -433,8 +434,8 @@ size_t configure_fused(LayerParams& p, const Dims& s, int T) {
   p.h_in_smem = 1;
   const size_t a128 = 127;
   const int R = T * (s.k + s.S);
-  const size_t head = sizeof(RouteDesc) + ((static_cast<size_t>(T) * s.d * 2 + a128) & ~a128) +
-                      static_cast<size_t>((s.E + sms - 1) / sms) * s.d * 2;
+  const size_t head = sizeof(RouteDesc) + 2 * ((static_cast<size_t>(T) * s.d * 2 + a128) & ~a128) +
+                      fused_rows_bytes((s.E + sms - 1) / sms * s.d * 2, s.E);
   const size_t ybytes = ((4 * static_cast<size_t>(R) * nb) + a128) & ~a128;
   const size_t ring_d = static_cast<size_t>(kFusedWarps) * p.ns_down * p.stage_down;
   const size_t down = fused_h16_bytes(R, s.I) + ybytes + ring_d;
@@ -508,7 +509,7 @@ cudaError_t launch_route_fwd(const LayerParams& p, cudaStream_t st, bool pdl) {
 }
 
 cudaError_t launch_router_only(const LayerParams& p, cudaStream_t st) {
-  const dim3 grid((p.E + 7) / 8), block(256);
+  const dim3 grid((p.E + 7) / 8, (p.T + kRouterTokens - 1) / kRouterTokens), block(256);
   switch (p.d) {
     case 512: return launch(k_router_only<512>, grid, block, 0, st, false, p);
     case 1024: return launch(k_router_only<1024>, grid, block, 0, st, false, p);
@@ -602,8 +603,26 @@ int mma_maps(MmaMaps* mp, const Dims& s, const flint_moe_weights* wts, bool gate
                     2, brows, bdims, bstr, bbox, true);
 }
 
-size_t mma_smem(bool nvfp4) {
-  return 1024 + (nvfp4 ? kMmaRawStages * kMmaRawBytes : 0) + kMmaAStages * kMmaABytes + kMmaBStages * kMmaBBytes;
+// Ring depths of the tensor-core kernels for a call of T tokens: B stages hold
+// the largest expert's rows (T rounded up to 16), four of them; NVFP4 keeps
+// four A stages and as many raw-weight stages as fit; bf16 weights as many A
+// stages as fit. Returns the dynamic shared-memory bytes.
+size_t mma_configure(MmaParams& m, int T) {
+  constexpr size_t kBudget = 220 * 1024;
+  const int npad = std::min(kMmaMaxTokens, (T + 15) & ~15);
+  m.b_bytes = npad * 128;
+  m.n_b = 4;
+  size_t left = kBudget - 1024 - static_cast<size_t>(m.n_b) * m.b_bytes;
+  if (m.nvfp4) {
+    m.n_a = 4;
+    left -= static_cast<size_t>(m.n_a) * kMmaABytes;
+    m.n_raw = static_cast<int>(std::min<size_t>(kMmaMaxStages, left / kMmaRawBytes));
+  } else {
+    m.n_raw = 1;
+    m.n_a = static_cast<int>(std::min<size_t>(kMmaMaxStages, left / kMmaABytes));
+  }
+  return 1024 + (m.nvfp4 ? static_cast<size_t>(m.n_raw) * kMmaRawBytes : 0) +
+         static_cast<size_t>(m.n_a) * kMmaABytes + static_cast<size_t>(m.n_b) * m.b_bytes;
 }
 
 // The tensor-core layer: router, top-k, grouping, B rows, gate/up, h rows,
@@ -652,7 +671,7 @@ int run_mma_path(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, 
   if (e != cudaSuccess) return cuda_fail(e, "k_mma_group launch");
   e = launch(k_mma_prep, dim3((P + 7) / 8), dim3(256), 0, st, pdl, m);
   if (e != cudaSuccess) return cuda_fail(e, "k_mma_prep launch");
-  const size_t smem = mma_smem(m.nvfp4 != 0);
+  const size_t smem = mma_configure(m, T);
   const int ncols = 2 * kMmaMaxTokens;
   const dim3 grid(num_sms()), block(kMmaWarps * 32);
   e = ensure_smem(reinterpret_cast<const void*>(k_mma_ffn<kEpiGateUp>));

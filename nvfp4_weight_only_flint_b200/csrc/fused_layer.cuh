@@ -33,6 +33,9 @@ constexpr int kFusedMaxTokens = 8;
 constexpr int kFusedWarps = 8;
 constexpr int kFusedDownTokens = 4;   // tokens per pass in the down phase
 constexpr int kBarrierCounters = 4;   // control-block words 32, 64, 96, 128
+// Tagged logits are written to this many replicas; CTA c reads replica c % R,
+// so each line is polled by G/R CTAs instead of all of them.
+constexpr int kLogitReplicas = 8;
 
 __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
   unsigned v;
@@ -100,6 +103,46 @@ __device__ __forceinline__ void cost_prefix(const RouteDesc* dsc, int n_active, 
   if (lane == 31) cost[n_active] = ex;
 }
 
+// Down rows of one staged block (up to 4*RPS rows, RPS = rows per warp step)
+// against TG tokens' h (16 f16x2 registers each): each lane accumulates its
+// 32-column slice for all 4 steps x TG tokens, then one transposed butterfly
+// per row group (VRD lanes) reduces them. out[g] is the total of value index
+// g*VRD + (lane % VRD) (value index = step*TG + token) when 4*TG > VRD, else
+// out[0] is the total of index (lane % VRD) >> log2(VRD / (4*TG)).
+template <int I, int TG>
+__device__ __forceinline__ void down_block(const uint8_t* st, int roff, int rows, const uint32_t* hh, int lane,
+                                           float* out) {
+  constexpr int VRD = I / 32, RPS = 32 / VRD, ROWC = I / 2, ROWS = I / 16, V = 4 * TG;
+  const int rs = lane / VRD, cbk = lane % VRD;
+  float v[V];
+#pragma unroll
+  for (int step = 0; step < 4; ++step) {
+    const int row = step * RPS + rs;
+    float acc[TG];
+#pragma unroll
+    for (int t = 0; t < TG; ++t) acc[t] = 0.f;
+    if (row < rows) {
+      const uint4 cv = lds128(st + row * ROWC + cbk * 16);
+      const uint32_t s2 = *reinterpret_cast<const uint16_t*>(st + roff + row * ROWS + cbk * 2);
+      dot32_strided<TG, 16>(cv, s2, hh, acc);
+    }
+#pragma unroll
+    for (int t = 0; t < TG; ++t) v[step * TG + t] = acc[t];
+  }
+  if constexpr (V <= VRD) {
+    out[0] = xreduce<VRD, V>(v, lane);
+  } else {
+#pragma unroll
+    for (int g = 0; g < V / VRD; ++g) out[g] = xreduce<VRD, VRD>(v + g * VRD, lane);
+  }
+}
+
+// Shared-memory bytes of the router-rows region, which later serves as the
+// grouping's scratch (20 bytes per expert).
+__host__ __device__ constexpr size_t fused_rows_bytes(int row_bytes, int E) {
+  return ((static_cast<size_t>(row_bytes > 20 * E ? row_bytes : 20 * E)) + 127) & ~static_cast<size_t>(127);
+}
+
 // Shared-memory bytes of the down phase's h copy: R rows of I f16.
 __host__ __device__ constexpr size_t fused_h16_bytes(int R, int I) {
   return ((static_cast<size_t>(R) * I * 2) + 127) & ~static_cast<size_t>(127);
@@ -131,9 +174,14 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   RouteDesc* dsc = reinterpret_cast<RouteDesc*>(smem);
   uint8_t* xsm = smem + sizeof(RouteDesc);
   const size_t xbytes = static_cast<size_t>(T) * D * 2;
-  uint8_t* rsm = xsm + ((xbytes + 127) & ~static_cast<size_t>(127));
+  const size_t xpad = (xbytes + 127) & ~static_cast<size_t>(127);
+  // x * sigma_t as f16, lane-interleaved: element i of token t at
+  // t*D + (((i % 32) / 8) * (D / 32) + i / 32) * 8 + i % 8, so the 16-byte
+  // chunks the lanes of a gate/up step read are contiguous
+  uint16_t* x16 = reinterpret_cast<uint16_t*>(xsm + xpad);
+  uint8_t* rsm = xsm + 2 * xpad;
   const int rpc = (E + G - 1) / G;  // router rows per CTA
-  uint8_t* work = rsm + static_cast<size_t>(rpc) * D * 2;
+  uint8_t* work = rsm + fused_rows_bytes(rpc * D * 2, E);
   uint64_t* ring_bars = s_bar;                        // [warp][kMaxStages]
   uint64_t* xbar = s_bar + kFusedWarps * kMaxStages;  // x
   uint64_t* rbar = xbar + 1;                          // router rows
@@ -164,8 +212,8 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   const unsigned gen = s_gen, tag = gen + 1u;
 
   // ---- the warp's bulk-copy ring: first the shared expert's units (they do
-  // not depend on the routing, so they are fetched now and computed after the
-  // router tasks), then a range of the routed experts' units (after P2)
+  // not depend on the routing, so they are fetched now), then a range of the
+  // routed experts' units (after the routing step)
   uint8_t* ring = work + static_cast<size_t>(warp) * ns_g * p.stage_gateup;
   uint64_t* bars = ring_bars + warp * kMaxStages;
   int issued = 0, consumed = 0;
@@ -176,10 +224,9 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     bulk_g2s(st + M::CU * M::UNIT_CODE, p.scales + e * p.spe + static_cast<long long>(uu) * (D / 8),
              cu * M::UNIT_SCALE, &bars[slot]);
   };
-  const long long NW = static_cast<long long>(G) * kFusedWarps;
-  const long long gw = static_cast<long long>(c) * kFusedWarps + warp;
-  const int sh_begin = S > 0 ? static_cast<int>(gw * I / NW) : 0;
-  const int sh_end = S > 0 ? static_cast<int>((gw + 1) * I / NW) : 0;
+  const int NW = G * kFusedWarps, gw = c * kFusedWarps + warp;  // grid <= 240 CTAs (host check)
+  const int sh_begin = S > 0 ? gw * I / NW : 0;
+  const int sh_end = S > 0 ? (gw + 1) * I / NW : 0;
   int sh_issue = sh_begin;
   while (issued < ns_g && sh_issue < sh_end) {
     const int cu = min(M::CU, sh_end - sh_issue);
@@ -210,10 +257,21 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     ss = warp_sum(ss);
     const float irms = p.input_norm ? 1.f / sqrtf(ss / static_cast<float>(D) + kRmsEps) : 1.f;
+    const float sg = pow2_scale_for(amax);
     if (lane == 0) {
-      const float sg = pow2_scale_for(amax);
       s_sigma[t] = sg;
       s_f[t] = irms / sg;
+    }
+#pragma unroll
+    for (int i = 0; i < NVR; ++i) {
+      const int i0 = 8 * (lane + 32 * i);
+      const uint4 v = lds128(xs + static_cast<size_t>(t) * D + i0);
+      uint4 o;
+      o.x = bf16x2_to_f16x2_scaled(v.x, sg);
+      o.y = bf16x2_to_f16x2_scaled(v.y, sg);
+      o.z = bf16x2_to_f16x2_scaled(v.z, sg);
+      o.w = bf16x2_to_f16x2_scaled(v.w, sg);
+      *reinterpret_cast<uint4*>(x16 + static_cast<size_t>(t) * D + (((i0 & 31) >> 3) * (D / 32) + (i0 >> 5)) * 8) = o;
     }
   }
   __syncthreads();
@@ -237,7 +295,8 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
       sum += a;
     }
     sum = warp_sum(sum);
-    if (lane == 0) st_tagged(p.tlogits + static_cast<size_t>(t) * E + r_begin + r, tag, sum * s_f[t] * s_sigma[t]);
+    if (lane < kLogitReplicas)
+      st_tagged(p.tlogits + (static_cast<size_t>(lane) * T + t) * E + r_begin + r, tag, sum * s_f[t] * s_sigma[t]);
   }
 
   // gate/up of one staged chunk of `cu` units from unit uu, for the tokens
@@ -265,17 +324,17 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
 #pragma unroll
         for (int t = 0; t < M::TGMAX; ++t) {
           const int tok = pair_of(g0 + min(t, n - 1)) >> 8;
-          const float sgm = (t < n) ? s_sigma[tok] : 0.f;
+          const bool live = t < n;
 #pragma unroll
           for (int xi = 0; xi < M::XV; ++xi) {
-            const uint16_t* src = xs + static_cast<size_t>(tok) * D + 32 * M::xblock(lane, xi);
+            const uint16_t* src = x16 + static_cast<size_t>(tok) * D + M::xblock(lane, xi) * 8;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const uint4 v = lds128(src + 8 * q);
-              xh[t * M::XS + xi * 16 + 4 * q + 0] = bf16x2_to_f16x2_scaled(v.x, sgm);
-              xh[t * M::XS + xi * 16 + 4 * q + 1] = bf16x2_to_f16x2_scaled(v.y, sgm);
-              xh[t * M::XS + xi * 16 + 4 * q + 2] = bf16x2_to_f16x2_scaled(v.z, sgm);
-              xh[t * M::XS + xi * 16 + 4 * q + 3] = bf16x2_to_f16x2_scaled(v.w, sgm);
+              const uint4 v = lds128(src + q * D / 4);  // chunk q of the block: q * (D/32) * 8 elements on
+              xh[t * M::XS + xi * 16 + 4 * q + 0] = live ? v.x : 0u;
+              xh[t * M::XS + xi * 16 + 4 * q + 1] = live ? v.y : 0u;
+              xh[t * M::XS + xi * 16 + 4 * q + 2] = live ? v.z : 0u;
+              xh[t * M::XS + xi * 16 + 4 * q + 3] = live ? v.w : 0u;
             }
           }
         }
@@ -296,20 +355,21 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     if (warp < T) {
       bool okt = false;
       if (ok) {
+        const unsigned long long* lg = p.tlogits + (static_cast<size_t>(c % kLogitReplicas) * T + warp) * E;
         if (E <= 256)
-          okt = topk_warp_tagged<8>(p.tlogits + static_cast<size_t>(warp) * E, E, k, tag, &s_ids[warp * k],
-                                    &s_gates[warp * k], lane, p.status);
+          okt = topk_warp_tagged<8>(lg, E, k, tag, &s_ids[warp * k], &s_gates[warp * k], lane, p.status);
         else
-          okt = topk_warp_tagged<kMaxExperts / 32>(p.tlogits + static_cast<size_t>(warp) * E, E, k, tag,
-                                                   &s_ids[warp * k], &s_gates[warp * k], lane, p.status);
+          okt = topk_warp_tagged<kMaxExperts / 32>(lg, E, k, tag, &s_ids[warp * k], &s_gates[warp * k], lane,
+                                                   p.status);
       }
       if (!okt && lane == 0) s_fail = 1;
     }
     __syncthreads();
     if (s_fail) ok = false;
-    // the ring area is idle here (every warp has drained its shared-expert
-    // chunks), so it serves as the grouping's scratch
-    if (ok) cta_grouping(s_ids, T, k, E, S, dsc, work, p.status);
+    // the router rows are consumed by now (every warp's router tasks precede
+    // this point), so their region serves as the grouping's scratch
+    if (ok) cta_grouping(s_ids, T, k, E, S, dsc->act, dsc->off, dsc->pair, &dsc->n_routed, &dsc->n_active, rsm,
+                         p.status);
     if (c == 0 && ok) {
       for (int i = tid; i < T * k; i += blockDim.x) {
         p.ids[i] = s_ids[i];
@@ -320,122 +380,131 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
         }
       }
     }
-    // L2 prefetch of this CTA's block of down rows of every routed active expert
-    if (ok && tid < dsc->n_routed && nrows > 0) {
-      const long long e = dsc->act[tid];
-      prefetch_l2(p.codes + e * p.cpe + static_cast<long long>(I) * p.d + static_cast<long long>(n0) * ROWC,
-                  nrows * ROWC);
-      prefetch_l2(p.scales + e * p.spe + static_cast<long long>(I) * p.d / 8 + static_cast<long long>(n0) * ROWS,
-                  nrows * ROWS);
-    }
   };
 
-  // ---- P1b + P3: one stream of chunks per warp. Phase 0: this warp's slice
-  // of the shared expert's units (index = unit), for every token. Then the
-  // routing step, then phase 1: this warp's range of the routed experts' cost
-  // space (units x token passes), index = active expert * I + unit. One loop,
-  // so the chunk code exists once.
-  int phase = 0;
-  int g = sh_begin, g_end = sh_end, issue_g = sh_issue;
-  int cur_a = -1;
-  float sg = S > 0 ? __ldg(p.tscale + 3 * E + 0) : 0.f, su = S > 0 ? __ldg(p.tscale + 3 * E + 1) : 0.f;
-  auto chunk_len = [&](int gg) {
-    return phase == 0 ? min(M::CU, g_end - gg) : min(M::CU, min(I - gg % I, g_end - gg));
+  // ---- P2 right after the router: top-k and grouping
+  routing_step();
+  if (!ok) {
+    drain_ring(bars, ns_g, consumed, issued, p.status);
+    consumed = issued;
+  }
+
+  // ---- P3: one stream of chunks per warp, issued and consumed in the same
+  // order: phase 0 is this warp's slice of the shared expert's units (index =
+  // unit; fetched since the start), phase 1 its range of the routed experts'
+  // cost space (units x token passes; index = active expert * I + unit). One
+  // loop, so the chunk code exists once.
+  int u_begin = 0, u_end = 0;
+  {
+    const int n_routed = ok ? dsc->n_routed : 0;
+    int* cost = s_cost[warp];
+    cost_prefix(dsc, n_routed, I, M::TGMAX, cost, lane);
+    __syncwarp();
+    // 32-bit arithmetic: C <= 65 experts x 1024 units x 4 passes and
+    // gw < 240 * 8, so gw * C < 2^31
+    const int C = n_routed > 0 ? cost[n_routed] : 0;
+    const int c_begin = gw * C / NW, c_end = (gw + 1) * C / NW;
+    auto to_unit = [&](int cc, int& a, int& u) {
+      int lo = 0, hi = n_routed - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cost[mid] <= cc) lo = mid;
+        else hi = mid - 1;
+      }
+      a = lo;
+      const int passes = (dsc->off[a + 1] - dsc->off[a] + M::TGMAX - 1) / M::TGMAX;
+      u = (cc - cost[a]) / passes;
+    };
+    if (c_end > c_begin) {
+      int a0, u0, a1, u1;
+      to_unit(c_begin, a0, u0);
+      to_unit(c_end - 1, a1, u1);
+      u_begin = a0 * I + u0;
+      u_end = a1 * I + u1 + 1;
+      if (c_begin > 0) {  // a unit already started by the previous warp's range is left to it
+        int pa, pu;
+        to_unit(c_begin - 1, pa, pu);
+        if (pa == a0 && pu == u0) ++u_begin;
+      }
+    }
+  }
+  auto len_at = [&](int ph, int gg) {
+    return ph == 0 ? min(M::CU, sh_end - gg) : min(M::CU, min(I - gg % I, u_end - gg));
   };
-  for (;;) {
-    if (g >= g_end || !ok) {
-      if (phase == 1) break;
-      if (!ok) {
-        drain_ring(bars, ns_g, consumed, issued, p.status);
-        consumed = issued;
+  auto settle = [&](int& ph, int& gg) {  // phase 0 exhausted -> start of phase 1
+    if (ph == 0 && gg >= sh_end) {
+      ph = 1;
+      gg = u_begin;
+    }
+  };
+  auto issue_at = [&](int ph, int gg) {
+    if (lane == 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue_units(ph == 0 ? E : dsc->act[gg / I], ph == 0 ? gg : gg % I, len_at(ph, gg), issued % ns_g);
+    }
+  };
+  int iph = 0, ig = sh_issue;
+  settle(iph, ig);
+  while (ok && issued - consumed < ns_g && !(iph == 1 && ig >= u_end)) {
+    issue_at(iph, ig);
+    ig += len_at(iph, ig);
+    settle(iph, ig);
+    ++issued;
+  }
+  // then an L2 prefetch of this CTA's block of down rows of every routed
+  // active expert (queued behind the gate/up copies)
+  for (int a = warp * 32 + lane; ok && a < dsc->n_routed && nrows > 0; a += kFusedWarps * 32) {
+    const long long e = dsc->act[a];
+    prefetch_l2(p.codes + e * p.cpe + static_cast<long long>(I) * p.d + static_cast<long long>(n0) * ROWC,
+                nrows * ROWC);
+    prefetch_l2(p.scales + e * p.spe + static_cast<long long>(I) * p.d / 8 + static_cast<long long>(n0) * ROWS,
+                nrows * ROWS);
+  }
+  {
+    int cph = 0, cg = sh_begin, cur_a = -1;
+    settle(cph, cg);
+    float sg = S > 0 ? __ldg(p.tscale + 3 * E + 0) : 0.f, su = S > 0 ? __ldg(p.tscale + 3 * E + 1) : 0.f;
+    while (ok && !(cph == 1 && cg >= u_end)) {
+      const int cu = len_at(cph, cg);
+      int key, nt, uu, kslot;
+      const unsigned short* pairs;
+      if (cph == 0) {
+        key = -2;
+        nt = T;
+        uu = cg;
+        pairs = nullptr;
+        kslot = k;
+      } else {
+        const int a = cg / I;
+        if (a != cur_a) {  // tensor scales of the expert, fetched before the stage wait
+          const int e = dsc->act[a];
+          sg = __ldg(p.tscale + 3 * e + 0);
+          su = __ldg(p.tscale + 3 * e + 1);
+          cur_a = a;
+        }
+        key = a;
+        uu = cg % I;
+        const int pb = dsc->off[a];
+        nt = dsc->off[a + 1] - pb;
+        pairs = dsc->pair + pb;
+        kslot = 0;
       }
-      routing_step();
-      // this warp's range of the routed cost space, mapped to units
-      const int n_routed = ok ? dsc->n_routed : 0;
-      int* cost = s_cost[warp];
-      cost_prefix(dsc, n_routed, I, M::TGMAX, cost, lane);
+      const int slot = consumed % ns_g;
+      if (!mbar_wait(&bars[slot], (consumed / ns_g) & 1, p.status)) {
+        ok = false;
+        break;
+      }
+      compute_chunk(ring + slot * p.stage_gateup, cu, uu, sg, su, key, nt, pairs, kslot);
       __syncwarp();
-      const long long C = n_routed > 0 ? cost[n_routed] : 0;
-      const long long c_begin = gw * C / NW, c_end = (gw + 1) * C / NW;
-      auto to_unit = [&](long long cc, int& a, int& u) {
-        int lo = 0, hi = n_routed - 1;
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (cost[mid] <= cc) lo = mid;
-          else hi = mid - 1;
-        }
-        a = lo;
-        const int passes = (dsc->off[a + 1] - dsc->off[a] + M::TGMAX - 1) / M::TGMAX;
-        u = static_cast<int>((cc - cost[a]) / passes);
-      };
-      int g_begin = 0;
-      g_end = 0;
-      if (c_end > c_begin) {
-        int a0, u0, a1, u1;
-        to_unit(c_begin, a0, u0);
-        to_unit(c_end - 1, a1, u1);
-        g_begin = a0 * I + u0;
-        g_end = a1 * I + u1 + 1;
-        if (c_begin > 0) {  // a unit already started by the previous warp's range is left to it
-          int pa, pu;
-          to_unit(c_begin - 1, pa, pu);
-          if (pa == a0 && pu == u0) ++g_begin;
-        }
-      }
-      phase = 1;
-      g = g_begin;
-      issue_g = g_begin;
-      while (issued - consumed < ns_g && issue_g < g_end) {
-        if (lane == 0) {
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          issue_units(dsc->act[issue_g / I], issue_g % I, chunk_len(issue_g), issued % ns_g);
-        }
-        issue_g += chunk_len(issue_g);
+      ++consumed;
+      cg += cu;
+      settle(cph, cg);
+      if (!(iph == 1 && ig >= u_end)) {
+        issue_at(iph, ig);
+        ig += len_at(iph, ig);
+        settle(iph, ig);
         ++issued;
       }
-      continue;
-    }
-    const int cu = chunk_len(g);
-    int key, nt, uu, kslot;
-    const unsigned short* pairs;
-    if (phase == 0) {
-      key = -2;
-      nt = T;
-      uu = g;
-      pairs = nullptr;
-      kslot = k;
-    } else {
-      const int a = g / I;
-      if (a != cur_a) {  // tensor scales of the expert, fetched before the stage wait
-        const int e = dsc->act[a];
-        sg = __ldg(p.tscale + 3 * e + 0);
-        su = __ldg(p.tscale + 3 * e + 1);
-        cur_a = a;
-      }
-      key = a;
-      uu = g % I;
-      const int pb = dsc->off[a];
-      nt = dsc->off[a + 1] - pb;
-      pairs = dsc->pair + pb;
-      kslot = 0;
-    }
-    const int slot = consumed % ns_g;
-    if (!mbar_wait(&bars[slot], (consumed / ns_g) & 1, p.status)) {
-      ok = false;
-      continue;
-    }
-    compute_chunk(ring + slot * p.stage_gateup, cu, uu, sg, su, key, nt, pairs, kslot);
-    __syncwarp();
-    ++consumed;
-    g += cu;
-    if (issue_g < g_end) {
-      const int cn = chunk_len(issue_g);
-      if (lane == 0) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue_units(phase == 0 ? E : dsc->act[issue_g / I], phase == 0 ? issue_g : issue_g % I, cn, issued % ns_g);
-      }
-      issue_g += cn;
-      ++issued;
     }
   }
   const int n_active = ok ? dsc->n_active : 0;
@@ -537,22 +606,35 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
           hh[t * 16 + 4 * q + 3] = v.w;
         }
       }
-      for (int rr = 0; rr < rows; rr += RPS) {
-        const int row = rr + rs;
-        const uint4 cv = lds128(st + row * ROWC + cbk * 16);
-        const uint32_t s2 = *reinterpret_cast<const uint16_t*>(st + roff + row * ROWS + cbk * 2);
-        float acc[TGD];
+      // one pass: all rows of the block for these tokens, reduced once
+      if (n == 1) {
+        constexpr int V1 = 4;
+        float o[V1 > VRD ? V1 / VRD : 1];
+        down_block<I, 1>(st, roff, rows, hh, lane, o);
+        if constexpr (V1 <= VRD) {
+          const int rep = VRD / V1;  // lanes per value
+          const int idx = cbk / rep, row = idx * RPS + rs;
+          if (cbk % rep == 0 && row < rows) s_y[P[0] * nb + r0 + row] = o[0] * yscale[0];
+        } else {
 #pragma unroll
-        for (int t = 0; t < TGD; ++t) acc[t] = 0.f;
-        if (n == 1)
-          dot32_strided<1, 16>(cv, s2, hh, acc);
-        else
-          dot32_strided<TGD, 16>(cv, s2, hh, acc);
+          for (int g = 0; g < V1 / VRD; ++g) {
+            const int idx = g * VRD + cbk, row = idx * RPS + rs;
+            if (row < rows) s_y[P[0] * nb + r0 + row] = o[g] * yscale[0];
+          }
+        }
+      } else {
+        constexpr int VT = 4 * TGD;
+        float o[VT > VRD ? VT / VRD : 1];
+        down_block<I, TGD>(st, roff, rows, hh, lane, o);
+        if constexpr (VT <= VRD) {
+          const int rep = VRD / VT;
+          const int idx = cbk / rep, step = idx / TGD, t = idx % TGD, row = step * RPS + rs;
+          if (cbk % rep == 0 && t < n && row < rows) s_y[P[t] * nb + r0 + row] = o[0] * yscale[t];
+        } else {
 #pragma unroll
-        for (int t = 0; t < TGD; ++t) {
-          if (t < n) {
-            const float y = segment_sum<VRD>(acc[t]);
-            if (cbk == 0) s_y[P[t] * nb + r0 + row] = y * yscale[t];
+          for (int g = 0; g < VT / VRD; ++g) {
+            const int idx = g * VRD + cbk, step = idx / TGD, t = idx % TGD, row = step * RPS + rs;
+            if (t < n && row < rows) s_y[P[t] * nb + r0 + row] = o[g] * yscale[t];
           }
         }
       }

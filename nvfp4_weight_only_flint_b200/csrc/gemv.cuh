@@ -43,7 +43,7 @@ struct LayerParams {
                              // words 32*(i+1), i < 4: its grid-barrier arrival counters
   RouteDesc* desc;           // routing descriptor (workspace)
   float* logits;             // [T][E]
-  unsigned long long* tlogits;  // [T][E] tagged logits of the persistent kernel
+  unsigned long long* tlogits;  // [replicas][T][E] tagged logits of the persistent kernel
   int* ids;                  // [T][k]
   float* gates;              // [T][k]
   float* h;                  // [T*(k+S)][I] fp32 SwiGLU intermediates
@@ -113,30 +113,56 @@ __device__ __forceinline__ float route_code_value(uint32_t ord) {
   return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
 }
 
-// Selection on codes already loaded (code 0 = absent). Round r's winner is
-// kept by lane r, so the rounds need no per-lane arrays (a rolled loop: this
-// code runs once per token and launch, so its size matters more than its ILP).
+// Selection on codes already loaded (code 0 = absent). Each lane first sorts
+// its NE candidates (code descending, then expert index ascending) with a
+// bitonic network, so a round only compares the lanes' heads: redux.sync
+// takes the largest head code, a second one the lowest expert index among the
+// lanes holding it, and the winning lane shifts its list. Round r's winner is
+// kept by lane r; the rounds are a rolled loop (this runs once per token and
+// launch, so its code size matters more than its unrolled speed).
 template <int NE>
 __device__ __forceinline__ void topk_select(uint32_t (&code)[NE], int k, int* ids, float* gates, int lane) {
+  int slot[NE];
+#pragma unroll
+  for (int i = 0; i < NE; ++i) slot[i] = i;
+  // descending bitonic sort of (code, -slot)
+#pragma unroll
+  for (int size = 2; size <= NE; size <<= 1) {
+#pragma unroll
+    for (int stride = size / 2; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < NE; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool desc = (i & size) == 0;
+          // a "comes first" when its code is larger, or equal with a lower slot
+          const bool i_first = code[i] > code[j] || (code[i] == code[j] && slot[i] < slot[j]);
+          if (i_first != desc) {
+            const uint32_t tc = code[i];
+            code[i] = code[j];
+            code[j] = tc;
+            const int ts = slot[i];
+            slot[i] = slot[j];
+            slot[j] = ts;
+          }
+        }
+      }
+    }
+  }
   float my_val = 0.f, v0 = 0.f;
   int my_sel = 0;
 #pragma unroll 1
   for (int r = 0; r < k; ++r) {
-    uint32_t best = code[0];
-    int bi = 0;
-#pragma unroll
-    for (int i = 1; i < NE; ++i)
-      if (code[i] > best) {  // strict: equal codes keep the lower index
-        best = code[i];
-        bi = i;
-      }
-    const uint32_t m = __reduce_max_sync(0xffffffffu, best);
-    const uint32_t w = __reduce_max_sync(0xffffffffu, best == m ? 0xFFFFFFFFu - (lane + 32 * bi) : 0u);
+    const uint32_t m = __reduce_max_sync(0xffffffffu, code[0]);
+    const uint32_t w = __reduce_max_sync(0xffffffffu, code[0] == m ? 0xFFFFFFFFu - (lane + 32 * slot[0]) : 0u);
     const int e = static_cast<int>(0xFFFFFFFFu - w);
-    if ((e & 31) == lane) {
+    if ((e & 31) == lane) {  // the winner drops its head
 #pragma unroll
-      for (int i = 0; i < NE; ++i)
-        if (i == (e >> 5)) code[i] = 0u;
+      for (int i = 0; i + 1 < NE; ++i) {
+        code[i] = code[i + 1];
+        slot[i] = slot[i + 1];
+      }
+      code[NE - 1] = 0u;
     }
     const float v = route_code_value(m);
     if (r == 0) v0 = v;
@@ -400,33 +426,36 @@ __device__ void warp_grouping(const int* ids, int T, int k, int E, int S, RouteD
   }
 }
 
-// Token grouping by a whole CTA (blockDim.x >= E/2, blockDim.x a multiple of
-// 32) for T*k <= 64 pairs, through a 64-bit pair mask per expert: pair i =
-// t*k + j sets bit i of its expert's mask, so a pair's place among its
-// expert's pairs (token order) is the popcount of the lower bits; exclusive
-// scans over the experts give the active list (ascending id) and the offsets.
-// Shared experts follow, with every token in slot k+s. `scratch`: 12*E bytes
-// of shared memory, 8-byte aligned. Writes the same fields as warp_grouping.
-__device__ void cta_grouping(const int* ids, int T, int k, int E, int S, RouteDesc* d, uint8_t* scratch,
-                             int* status) {
+// Token grouping by a whole CTA (blockDim.x >= E/2, a multiple of 32) for
+// T <= 128 tokens, through a token mask per expert (two 64-bit words): pair
+// i = t*k + j sets bit t of its expert's mask (a token picks an expert at most
+// once), so a pair's place among its expert's pairs (token order) is the
+// popcount of the mask below bit t; exclusive scans over the experts give the
+// active list (ascending id) and the offsets. Shared experts follow, with
+// every token in slot k+s. `scratch`: 20*E bytes of shared memory, 8-byte
+// aligned. Writes act/off/pair and the two counts.
+template <typename PairT>
+__device__ void cta_grouping(const int* ids, int T, int k, int E, int S, int* act, int* off, PairT* pair,
+                             int* n_routed, int* n_active, uint8_t* scratch, int* status) {
   __shared__ int s_tot[2][32];
-  unsigned long long* emask = reinterpret_cast<unsigned long long*>(scratch);
-  int* eoff = reinterpret_cast<int*>(scratch + 8 * static_cast<size_t>(E));
+  unsigned long long* emask = reinterpret_cast<unsigned long long*>(scratch);  // [E][2]
+  int* eoff = reinterpret_cast<int*>(scratch + 16 * static_cast<size_t>(E));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5, n = T * k;
-  for (int e = tid; e < E; e += blockDim.x) emask[e] = 0ull;
+  for (int i = tid; i < 2 * E; i += blockDim.x) emask[i] = 0ull;
   __syncthreads();
   for (int i = tid; i < n; i += blockDim.x) {
-    const int e = ids[i];
+    const int e = ids[i], t = i / k;
     if (e < 0 || e >= E) {
       atomicOr(status, FLINT_DEVCHECK_EXPERT_ID);
       continue;
     }
-    atomicOr(&emask[e], 1ull << i);
+    atomicOr(&emask[2 * e + (t >> 6)], 1ull << (t & 63));
   }
   __syncthreads();
   // thread owns experts 2*tid and 2*tid+1
   const int e0 = 2 * tid, e1 = 2 * tid + 1;
-  const int c0 = e0 < E ? __popcll(emask[e0]) : 0, c1 = e1 < E ? __popcll(emask[e1]) : 0;
+  const int c0 = e0 < E ? __popcll(emask[2 * e0]) + __popcll(emask[2 * e0 + 1]) : 0;
+  const int c1 = e1 < E ? __popcll(emask[2 * e1]) + __popcll(emask[2 * e1 + 1]) : 0;
   const int f0 = c0 > 0, f1 = c1 > 0;
   int ic = c0 + c1, jf = f0 + f1;  // inclusive scans over the block
 #pragma unroll
@@ -459,37 +488,41 @@ __device__ void cta_grouping(const int* ids, int T, int k, int E, int S, RouteDe
       s_tot[1][lane] = wf - xf;
     }
     if (lane == nw - 1) {
-      d->n_routed = wf;
-      d->n_active = wf + S;
+      *n_routed = wf;
+      *n_active = wf + S;
       for (int s = 0; s < S; ++s) {
-        d->act[wf + s] = E + s;
-        d->off[wf + s] = wc + s * T;
+        act[wf + s] = E + s;
+        off[wf + s] = wc + s * T;
       }
-      d->off[wf + S] = wc + S * T;
+      off[wf + S] = wc + S * T;
     }
   }
   __syncthreads();
   const int base_c = ic - (c0 + c1) + s_tot[0][warp], base_f = jf - (f0 + f1) + s_tot[1][warp];
   if (f0) {
-    d->act[base_f] = e0;
-    d->off[base_f] = base_c;
+    act[base_f] = e0;
+    off[base_f] = base_c;
     eoff[e0] = base_c;
   }
   if (f1) {
-    d->act[base_f + f0] = e1;
-    d->off[base_f + f0] = base_c + c0;
+    act[base_f + f0] = e1;
+    off[base_f + f0] = base_c + c0;
     eoff[e1] = base_c + c0;
   }
   __syncthreads();
   for (int i = tid; i < n; i += blockDim.x) {
     const int e = ids[i];
     if (e < 0 || e >= E) continue;
-    const int pos = eoff[e] + __popcll(emask[e] & ((1ull << i) - 1ull));
-    d->pair[pos] = static_cast<unsigned short>(((i / k) << 8) | (i % k));
+    const int t = i / k;
+    const unsigned long long lo = emask[2 * e], hi = emask[2 * e + 1];
+    const int below = t < 64 ? __popcll(lo & ((1ull << t) - 1ull))
+                             : __popcll(lo) + __popcll(hi & ((1ull << (t - 64)) - 1ull));
+    pair[eoff[e] + below] = static_cast<PairT>((t << 8) | (i % k));
   }
+  const int nr = off[*n_routed];  // the shared experts' pairs follow the routed ones
   for (int i = tid; i < S * T; i += blockDim.x) {
     const int s = i / T, t = i % T;
-    d->pair[n + i] = static_cast<unsigned short>((t << 8) | (k + s));
+    pair[nr + i] = static_cast<PairT>((t << 8) | (k + s));
   }
   __syncthreads();
 }

@@ -41,7 +41,9 @@ __device__ __forceinline__ void drain_ring(uint64_t* bars, int ns, int consumed,
 }
 
 // ----------------------------------------------------------------- router only (any T)
-// Warp per expert row, tokens looped; x read through L1. Used by flint_moe_route.
+// Warp per expert row and block of kRouterTokens tokens (grid.y), x read
+// through L1. Used by flint_moe_route and the tensor-core path.
+constexpr int kRouterTokens = 8;
 template <int D>
 __global__ void __launch_bounds__(256) k_router_only(LayerParams p) {
   constexpr int NVR = D / 256;
@@ -52,7 +54,8 @@ __global__ void __launch_bounds__(256) k_router_only(LayerParams p) {
   const uint4* row = reinterpret_cast<const uint4*>(p.wr + static_cast<size_t>(e) * D);
 #pragma unroll
   for (int i = 0; i < NVR; ++i) wv[i] = __ldg(row + lane + 32 * i);
-  for (int t = 0; t < p.T; ++t) {
+  const int t_end = min(p.T, static_cast<int>(blockIdx.y + 1) * kRouterTokens);
+  for (int t = blockIdx.y * kRouterTokens; t < t_end; ++t) {
     const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t) * D);
     float acc = 0.f;
 #pragma unroll

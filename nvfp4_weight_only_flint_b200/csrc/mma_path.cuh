@@ -25,10 +25,11 @@
 //                   slot) in fp32
 //   k_mma_combine   out_t = sum_j gate_tj y_(t,j) + y_(t,shared) (+ residual),
 //                   fixed order, bf16
-// Roles in the persistent kernels (16 warps): warp 0 issues the TMA loads,
-// warp 1 owns the tensor memory and issues the MMAs (one thread), warps 4-7
-// are the epilogue warpgroup (warp 4+i reads accumulator lanes 32i..32i+31),
-// warps 8-15 dequantise. Every wait is bounded; a wait that gives up records
+// Roles in the persistent kernels (16 warps): warp 0 issues the weights' TMA
+// loads and warp 2 the activation rows' (two rings that run ahead of each
+// other independently), warp 1 owns the tensor memory and issues the MMAs
+// (one thread), warps 4-7 are the epilogue warpgroup (warp 4+i reads
+// accumulator lanes 32i..32i+31), warps 8-15 dequantise. Every wait is bounded; a wait that gives up records
 // FLINT_DEVCHECK_WAIT, raises a CTA-wide abort flag, and every role then drains
 // what it started (copies in flight, MMAs committed) before the tensor memory
 // is released.
@@ -42,12 +43,9 @@ namespace flint {
 
 constexpr int kMmaMaxTokens = 128;  // N of one MMA <= 128 (tokens of one expert)
 constexpr int kMmaWarps = 16;
-constexpr int kMmaRawStages = 3;    // NVFP4 codes+scales, 256 elements of K per stage
-constexpr int kMmaAStages = 4;      // A operand buffers (128 rows x 64 elements)
-constexpr int kMmaBStages = 4;      // B operand buffers (N rows x 64 elements)
-constexpr int kMmaRawBytes = 128 * 128 + 128 * 16;  // 18 KiB: codes (swizzled) + scales
-constexpr int kMmaABytes = 128 * 128;               // 16 KiB
-constexpr int kMmaBBytes = kMmaMaxTokens * 128;     // 16 KiB
+constexpr int kMmaMaxStages = 8;    // ring depths are chosen per call, up to this
+constexpr int kMmaRawBytes = 128 * 128 + 128 * 16;  // NVFP4 stage, 256 of K: codes (swizzled) + scales
+constexpr int kMmaABytes = 128 * 128;               // A operand stage: 128 rows x 64 of K, 16-bit
 
 enum MmaEpi { kEpiGateUp = 0, kEpiDown = 1 };
 
@@ -78,6 +76,8 @@ struct MmaParams {
   float* y;                 // [T*(k+S)][d] fp32, row t*(k+S)+slot
   int T, d, I, E, k, S;
   int nvfp4;                // 1: NVFP4 weights, f16 operands; 0: bf16 weights, bf16 operands
+  int n_raw, n_a, n_b;      // ring depths (raw NVFP4 stages, A stages, B stages)
+  int b_bytes;              // B stage: (tokens rounded up to 16, at most 128) x 128 bytes
 };
 
 // ----------------------------------------------------------------- PTX wrappers
@@ -170,61 +170,24 @@ __device__ __forceinline__ bool mma_wait(uint64_t* bar, uint32_t parity, volatil
 }
 
 // ----------------------------------------------------------------- grouping
-// One CTA of 512 threads, thread e counts expert e (E <= 512).
+// One CTA of 512 threads (E <= 1024, T <= 128).
 __global__ void __launch_bounds__(512) k_mma_group(MmaParams p) {
   __shared__ int s_ids[kMmaMaxTokens * kMaxTopK];
-  __shared__ int s_scan[512];
-  __shared__ int s_act[512];
+  __shared__ __align__(8) uint8_t s_scratch[20 * kMaxExperts];
   pdl_wait();
   pdl_trigger();
-  const int tid = threadIdx.x, T = p.T, k = p.k, E = p.E, S = p.S, TK = T * k;
+  const int tid = threadIdx.x, TK = p.T * p.k;
   for (int i = tid; i < TK; i += blockDim.x) {
-    int e = p.ids[i];
-    if (e < 0 || e >= E) {
-      atomicOr(p.status, FLINT_DEVCHECK_EXPERT_ID);
-      e = -1;
-    }
-    s_ids[i] = e;
+    s_ids[i] = p.ids[i];
     if (p.ids_out != nullptr) {
       p.ids_out[i] = p.ids[i];
       p.gates_out[i] = p.gates[i];
     }
   }
   __syncthreads();
-  int cnt = 0;
-  if (tid < E)
-    for (int i = 0; i < TK; ++i) cnt += (s_ids[i] == tid) ? 1 : 0;
-  // block-wide exclusive scans of the counts and of the active flags
-  s_scan[tid] = cnt;
-  s_act[tid] = cnt > 0 ? 1 : 0;
-  __syncthreads();
-  for (int o = 1; o < 512; o <<= 1) {
-    const int a = tid >= o ? s_scan[tid - o] : 0, b = tid >= o ? s_act[tid - o] : 0;
-    __syncthreads();
-    s_scan[tid] += a;
-    s_act[tid] += b;
-    __syncthreads();
-  }
-  const int off = s_scan[tid] - cnt, pos = s_act[tid] - (cnt > 0 ? 1 : 0);
-  const int n_routed = s_act[511], routed_pairs = s_scan[511];
-  if (tid < E && cnt > 0) {
-    p.rt.act[pos] = tid;
-    p.rt.off[pos] = off;
-    int j = 0;
-    for (int i = 0; i < TK; ++i)
-      if (s_ids[i] == tid) p.rt.pair[off + j++] = ((i / k) << 8) | (i % k);
-  }
-  for (int s = 0; s < S; ++s) {
-    if (tid == 0) {
-      p.rt.act[n_routed + s] = E + s;
-      p.rt.off[n_routed + s] = routed_pairs + s * T;
-    }
-    for (int t = tid; t < T; t += blockDim.x) p.rt.pair[routed_pairs + s * T + t] = (t << 8) | (k + s);
-  }
-  if (tid == 0) {
-    p.rt.off[n_routed + S] = routed_pairs + S * T;
-    p.rt.n_active[0] = n_routed + S;
-  }
+  __shared__ int s_nrouted;
+  cta_grouping(s_ids, p.T, p.k, p.E, p.S, p.rt.act, p.rt.off, p.rt.pair, &s_nrouted, p.rt.n_active, s_scratch,
+               p.status);
 }
 
 // ----------------------------------------------------------------- B rows of gate/up
@@ -397,35 +360,32 @@ template <int EPI>
 __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     k_mma_ffn(MmaParams p, const __grid_constant__ MmaMaps maps, int ncols) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t raw_full[kMmaRawStages], raw_empty[kMmaRawStages];
-  __shared__ __align__(8) uint64_t a_full[kMmaAStages], a_empty[kMmaAStages];
-  __shared__ __align__(8) uint64_t b_full[kMmaBStages], b_empty[kMmaBStages];
+  __shared__ __align__(8) uint64_t raw_full[kMmaMaxStages], raw_empty[kMmaMaxStages];
+  __shared__ __align__(8) uint64_t a_full[kMmaMaxStages], a_empty[kMmaMaxStages];
+  __shared__ __align__(8) uint64_t b_full[kMmaMaxStages], b_empty[kMmaMaxStages];
   __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_nact;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool fp4 = p.nvfp4 != 0;
+  const int NR = p.n_raw, NA = p.n_a, NB = p.n_b, BB = p.b_bytes;
   // 1024-aligned carve-up: [raw stages (NVFP4 only)][A stages][B stages]
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* raw = base;
-  uint8_t* abuf = raw + (fp4 ? kMmaRawStages * kMmaRawBytes : 0);
-  uint8_t* bbuf = abuf + kMmaAStages * kMmaABytes;
+  uint8_t* abuf = raw + (fp4 ? NR * kMmaRawBytes : 0);
+  uint8_t* bbuf = abuf + NA * kMmaABytes;
   const int K = EPI == kEpiGateUp ? p.d : p.I;
   const int tiles = EPI == kEpiGateUp ? p.I / 64 : p.d / 128;
   const int n_sub = K / 64;
   const int KS = p.k + p.S;
 
   if (tid == 0) {
-    for (int i = 0; i < kMmaRawStages; ++i) {
+    for (int i = 0; i < kMmaMaxStages; ++i) {
       mbar_init(&raw_full[i], 1);
       mbar_init(&raw_empty[i], 8);
-    }
-    for (int i = 0; i < kMmaAStages; ++i) {
       mbar_init(&a_full[i], fp4 ? 8 : 1);
       mbar_init(&a_empty[i], 1);
-    }
-    for (int i = 0; i < kMmaBStages; ++i) {
       mbar_init(&b_full[i], 1);
       mbar_init(&b_empty[i], 1);
     }
@@ -448,52 +408,63 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
   const uint32_t tmem = s_tmem;
   const int n_items = s_nact * tiles;
   volatile int* abort_flag = &s_abort;
+  // on abort: wait (bounded) for every copy a producer started; stages older
+  // than the ring depth were consumed, so they have landed
+  auto drain = [&](uint64_t* full, int ns, int n) {
+    for (int i = max(0, n - ns); i < n; ++i) mbar_wait(&full[i % ns], (i / ns) & 1, p.status);
+  };
 
   if (warp == 0) {
-    // ------------------------------------------------ TMA producer
+    // ------------------------------------------------ A producer: weights
     if (lane == 0) {
-      int rc = 0, bc = 0, ac = 0;  // stages issued: raw, B, A (bf16 weights)
+      int rc = 0, ac = 0;  // stages issued: raw NVFP4, A (bf16 weights)
       bool ok = true;
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
         const int a = it / tiles, t = it % tiles;
         const int e = p.rt.act[a];
-        const int off = p.rt.off[a], nt = p.rt.off[a + 1] - off;
-        const int npad = (nt + 15) & ~15;
         for (int s = 0; s < n_sub && ok; ++s) {
-          if (fp4 && (s & 3) == 0) {
-            const int slot = rc % kMmaRawStages;
-            if (!(ok = mma_wait(&raw_empty[slot], ((rc / kMmaRawStages) & 1) ^ 1, abort_flag, p.status))) break;
+          if (fp4) {
+            if ((s & 3) != 0) continue;
+            const int slot = rc % NR;
+            if (!(ok = mma_wait(&raw_empty[slot], ((rc / NR) & 1) ^ 1, abort_flag, p.status))) break;
             uint8_t* st = raw + slot * kMmaRawBytes;
             mbar_arrive_expect_tx(&raw_full[slot], kMmaRawBytes);
             tma_load_3d(st, &maps.codes, (s / 4) * 128, t * 128, e, &raw_full[slot]);
             tma_load_3d(st + 128 * 128, &maps.scales, (s / 4) * 16, t * 128, e, &raw_full[slot]);
             ++rc;
-          }
-          if (!fp4) {
-            const int slot = ac % kMmaAStages;
-            if (!(ok = mma_wait(&a_empty[slot], ((ac / kMmaAStages) & 1) ^ 1, abort_flag, p.status))) break;
+          } else {
+            const int slot = ac % NA;
+            if (!(ok = mma_wait(&a_empty[slot], ((ac / NA) & 1) ^ 1, abort_flag, p.status))) break;
             mbar_arrive_expect_tx(&a_full[slot], kMmaABytes);
             tma_load_3d(abuf + slot * kMmaABytes, &maps.codes, s * 64, t * 128, e, &a_full[slot]);
             ++ac;
           }
-          const int slot = bc % kMmaBStages;
-          if (!(ok = mma_wait(&b_empty[slot], ((bc / kMmaBStages) & 1) ^ 1, abort_flag, p.status))) break;
+        }
+      }
+      if (!ok) {
+        drain(raw_full, NR, rc);
+        drain(a_full, NA, ac);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------ B producer: activation rows
+    if (lane == 0) {
+      int bc = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const int a = it / tiles;
+        const int off = p.rt.off[a], nt = p.rt.off[a + 1] - off;
+        const int npad = (nt + 15) & ~15;
+        for (int s = 0; s < n_sub && ok; ++s) {
+          const int slot = bc % NB;
+          if (!(ok = mma_wait(&b_empty[slot], ((bc / NB) & 1) ^ 1, abort_flag, p.status))) break;
           mbar_arrive_expect_tx(&b_full[slot], npad * 128);
           for (int j = 0; j < npad / 16; ++j)
-            tma_load_2d(bbuf + slot * kMmaBBytes + j * 2048, &maps.brows, s * 64, off + 16 * j, &b_full[slot]);
+            tma_load_2d(bbuf + slot * BB + j * 2048, &maps.brows, s * 64, off + 16 * j, &b_full[slot]);
           ++bc;
         }
       }
-      // on abort: wait (bounded) for every copy this thread started; stages
-      // older than the ring depth were consumed, so they have landed
-      if (!ok) {
-        auto drain = [&](uint64_t* full, int ns, int n) {
-          for (int i = max(0, n - ns); i < n; ++i) mbar_wait(&full[i % ns], (i / ns) & 1, p.status);
-        };
-        drain(raw_full, kMmaRawStages, rc);
-        drain(a_full, kMmaAStages, ac);
-        drain(b_full, kMmaBStages, bc);
-      }
+      if (!ok) drain(b_full, NB, bc);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
@@ -510,11 +481,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * kMmaMaxTokens);
         for (int s = 0; s < n_sub; ++s) {
-          const int as = sc % kMmaAStages, bs = bcount % kMmaBStages;
-          if (!(ok = mma_wait(&a_full[as], (sc / kMmaAStages) & 1, abort_flag, p.status))) break;
-          if (!(ok = mma_wait(&b_full[bs], (bcount / kMmaBStages) & 1, abort_flag, p.status))) break;
+          const int as = sc % NA, bs = bcount % NB;
+          if (!(ok = mma_wait(&a_full[as], (sc / NA) & 1, abort_flag, p.status))) break;
+          if (!(ok = mma_wait(&b_full[bs], (bcount / NB) & 1, abort_flag, p.status))) break;
           tc_fence_after();
-          const uint32_t aaddr = smem_addr(abuf + as * kMmaABytes), baddr = smem_addr(bbuf + bs * kMmaBBytes);
+          const uint32_t aaddr = smem_addr(abuf + as * kMmaABytes), baddr = smem_addr(bbuf + bs * BB);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_f16(d_tmem, sw128_desc(aaddr + 32 * kk), sw128_desc(baddr + 32 * kk), idesc, (s | kk) ? 1u : 0u);
@@ -545,31 +516,36 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
         const float sgt = fp4 ? __ldg(p.tscale + 3 * e + 0) : 1.f, sut = fp4 ? __ldg(p.tscale + 3 * e + 1) : 1.f;
         const int unit = t * 64 + (m >> 1);
         for (int c0 = 0; c0 < nt; c0 += 16) {
+          // column scales: lane j (mod 16) loads column c0 + j, then broadcasts
+          const float xin = (c0 + (lane & 15) < nt) ? p.xinv[off + c0 + (lane & 15)] : 0.f;
           float v[16];
           tmem_ld16(taddr + c0, v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
+            const float xi = __shfl_sync(0xffffffffu, xin, j);
             const int n = c0 + j;
-            if ((m & 1) == 0 && n < nt) {
-              const float xi = p.xinv[off + n];
+            if ((m & 1) == 0 && n < nt)
               p.h[static_cast<size_t>(off + n) * p.I + unit] = swiglu(v[j] * sgt * xi, other * sut * xi);
-            }
           }
         }
       } else {
         const float sdt = fp4 ? __ldg(p.tscale + 3 * e + 2) : 1.f;
         const int row = t * 128 + m;
         for (int c0 = 0; c0 < nt; c0 += 16) {
+          const bool in = c0 + (lane & 15) < nt;
+          const float hin = in ? p.hinv[off + c0 + (lane & 15)] : 0.f;
+          const int prn = in ? p.rt.pair[off + c0 + (lane & 15)] : 0;
           float v[16];
           tmem_ld16(taddr + c0, v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int n = c0 + j;
+            const float hi = __shfl_sync(0xffffffffu, hin, j);
+            const int pr = __shfl_sync(0xffffffffu, prn, j);
             if (n < nt) {
-              const int pr = p.rt.pair[off + n];
               const int yrow = (pr >> 8) * KS + (pr & 0xFF);
-              p.y[static_cast<size_t>(yrow) * p.d + row] = v[j] * sdt * p.hinv[off + n];
+              p.y[static_cast<size_t>(yrow) * p.d + row] = v[j] * sdt * hi;
             }
           }
         }
@@ -585,9 +561,9 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     bool ok = true;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       for (int s = 0; s < n_sub; ++s) {
-        const int rs = rc % kMmaRawStages, as = sc % kMmaAStages;
-        if (!(ok = mma_wait(&raw_full[rs], (rc / kMmaRawStages) & 1, abort_flag, p.status))) break;
-        if (!(ok = mma_wait(&a_empty[as], ((sc / kMmaAStages) & 1) ^ 1, abort_flag, p.status))) break;
+        const int rs = rc % NR, as = sc % NA;
+        if (!(ok = mma_wait(&raw_full[rs], (rc / NR) & 1, abort_flag, p.status))) break;
+        if (!(ok = mma_wait(&a_empty[as], ((sc / NA) & 1) ^ 1, abort_flag, p.status))) break;
         dequant_slice(raw + rs * kMmaRawBytes, s & 3, abuf + as * kMmaABytes, dt);
         // generic-proxy writes of the operand -> visible to the tensor cores
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
