@@ -233,7 +233,7 @@ int check_shape(const flint_moe_shape* s, Dims* out) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct WsLayout {
-  size_t status, counter, amax, desc, logits, tlogits, ids, gates, h;
+  size_t status, counter, amax, desc, logits, tlogits, ids, gates, h, htag;
   size_t mma_n, mma_act, mma_off, mma_pair, xinv, hinv, xrows, hrows, y;  // tensor-core path
   size_t total;
 };
@@ -247,7 +247,9 @@ constexpr size_t kCtrlBytes = 1024;
 // generation (byte 8) and its four grid-barrier counters (bytes 132, 260, 388,
 // 516; one 128-byte line each). The tagged logits start with a tag of 0, which
 // no launch uses. flint_moe_workspace_init zeroes the whole workspace.
-WsLayout ws_layout(const Dims& s, int maxT) {
+// Regions of the tensor-core path are laid out only when `mma` (the call takes
+// that path; flint_moe_workspace_bytes reports the size with them).
+WsLayout ws_layout(const Dims& s, int maxT, bool mma) {
   WsLayout w{};
   size_t o = 0;
   w.status = 0;
@@ -268,6 +270,13 @@ WsLayout ws_layout(const Dims& s, int maxT) {
   w.h = o;
   const size_t P = static_cast<size_t>(maxT) * (s.k + s.S);
   o += al256(sizeof(float) * P * s.I);
+  w.htag = o;
+  o += al256(sizeof(unsigned long long) * std::min<size_t>(P, static_cast<size_t>(kFusedMaxTokens) * (s.k + s.S)) * s.I);
+  if (!mma) {
+    w.mma_n = w.mma_act = w.mma_off = w.mma_pair = w.xinv = w.hinv = w.xrows = w.hrows = w.y = 0;
+    w.total = o;
+    return w;
+  }
   w.mma_n = o;
   o += 256;
   w.mma_act = o;
@@ -365,6 +374,7 @@ void fill_common(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, 
   p.desc = reinterpret_cast<RouteDesc*>(ws + w.desc);
   p.logits = reinterpret_cast<float*>(ws + w.logits);
   p.tlogits = reinterpret_cast<unsigned long long*>(ws + w.tlogits);
+  p.htag = reinterpret_cast<unsigned long long*>(ws + w.htag);
   p.ids = reinterpret_cast<int*>(ws + w.ids);
   p.gates = reinterpret_cast<float*>(ws + w.gates);
   p.h = reinterpret_cast<float*>(ws + w.h);
@@ -730,7 +740,7 @@ size_t flint_tensor_scale_bytes(const flint_moe_shape* shape) {
 size_t flint_moe_workspace_bytes(const flint_moe_shape* shape, int32_t max_tokens) {
   Dims s;
   if (check_shape(shape, &s) != FLINT_OK || max_tokens < 0) return 0;
-  return ws_layout(s, max_tokens < 1 ? 1 : max_tokens).total;
+  return ws_layout(s, max_tokens < 1 ? 1 : max_tokens, true).total;
 }
 
 int flint_pack_nvfp4(const void* w, int32_t w_is_bf16, const flint_moe_shape* shape, void* packed,
@@ -745,7 +755,7 @@ int flint_pack_nvfp4(const void* w, int32_t w_is_bf16, const flint_moe_shape* sh
   if (!aligned16(w) || !aligned16(packed) || !aligned16(block_scales) || !aligned16(tensor_scales) ||
       !aligned16(workspace))
     return fail(FLINT_ERR_MISALIGNED, "flint_pack_nvfp4: pointers must be 16-byte aligned");
-  const WsLayout lay = ws_layout(s, 1);
+  const WsLayout lay = ws_layout(s, 1, false);
   if (ws_bytes < lay.total) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, lay.total);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -801,7 +811,7 @@ int flint_moe_route(const uint16_t* x, int32_t T, const uint16_t* router_w, cons
   if (!aligned16(x) || !aligned16(router_w) || !aligned16(topk_ids) || !aligned16(topk_weights) ||
       !aligned16(workspace))
     return fail(FLINT_ERR_MISALIGNED, "flint_moe_route: pointers must be 16-byte aligned");
-  const WsLayout lay = ws_layout(s, T);
+  const WsLayout lay = ws_layout(s, T, false);
   if (ws_bytes < lay.total) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, lay.total);
   LayerParams p{};
   fill_common(p, s, lay, static_cast<uint8_t*>(workspace), T);
@@ -856,7 +866,7 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
     if (options && options->input_rmsnorm)
       return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "input_rmsnorm is a GEMV-path option");
   }
-  const WsLayout lay = ws_layout(s, T);
+  const WsLayout lay = ws_layout(s, T, !use_gemv);
   if (ws_bytes < lay.total) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, lay.total);
 
   LayerParams p{};
@@ -1012,7 +1022,9 @@ int flint_moe_forward_noalloc(const uint16_t* x, int32_t T, const uint16_t* rout
   if (rc != FLINT_OK) return rc;
   if (T < 0) return fail(FLINT_ERR_INVALID_ARG, "T=%d", T);
   if (T == 0) return FLINT_OK;
-  const size_t need = ws_layout(s, T).total;
+  // the path flint_moe_forward takes for this call (options == NULL: automatic)
+  const bool mma = !(T < kMaxGemvTokens && s.wd == FLINT_W_NVFP4);
+  const size_t need = ws_layout(s, T, mma).total;
   if (need > kNoAllocScratchBytes)
     return fail(FLINT_ERR_WORKSPACE,
                 "flint_moe_forward_noalloc: this call needs %zu bytes of scratch; the built-in scratch holds %zu "

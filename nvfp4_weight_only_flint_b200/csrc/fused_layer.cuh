@@ -4,25 +4,26 @@
 //   P0  bulk copies of x, of this CTA's router rows and of each warp's slice
 //       of the shared expert's gate/up units; L2 prefetch of this CTA's block
 //       of the shared expert's down rows
-//   P1  router logits ((row, token) tasks over the warps), stored as tagged
-//       64-bit words (launch tag | logit), and per-token scales; then each
-//       warp's slice of the shared expert's gate/up units (they need no
-//       routing; their bulk copies were issued at the start)
+//   P1  per-token scales, x converted once to f16 (lane-interleaved), router
+//       logits ((row, token) tasks over the warps), stored as tagged 64-bit
+//       words (launch tag | logit) in 8 replicas
 //   P2  every CTA: top-k of every token (a warp per token waits until all E
 //       logits carry this launch's tag, then selects) and the token grouping,
-//       kept in shared memory; L2 prefetch of this CTA's block of down rows of
-//       every routed active expert
-//   P3  gate/up of the routed experts through per-warp bulk-copy rings, work
-//       split by compute cost
-//   --  grid barrier (all h written)
-//   P4  h converted once per CTA to f16 (power-of-two scale per row) in shared
-//       memory, down rows streamed through per-warp rings, fixed-order gated
-//       combine (+ residual)
-// The launch tag and the barrier targets come from a generation word in the
-// workspace control block that CTA 0 advances after the barrier. The barrier
-// spreads arrivals over four counters in separate lines (fewer same-address
-// atomics in series). Every wait is bounded (FLINT_DEVCHECK_WAIT). The launch
-// is cooperative, so every CTA is resident.
+//       kept in shared memory
+//   P3  gate/up through per-warp bulk-copy rings: first the warp's shared-
+//       expert units, then its range of the routed experts' units (split by
+//       compute cost); h written as tagged 64-bit words; L2 prefetch of this
+//       CTA's block of down rows of every routed expert
+//   P4  every h row polled until all its values carry this launch's tag, then
+//       converted once per CTA to f16 (power-of-two scale per row) in shared
+//       memory; down rows of this CTA's block streamed through per-warp rings,
+//       fixed-order gated combine (+ residual)
+// The launch tag comes from a generation word in the workspace control block
+// that CTA 0 advances once it has seen every h row (by then every CTA has read
+// the generation). There is no grid barrier: the two cross-CTA dependencies
+// (all logits before top-k, all h before the down phase) are the tagged
+// words themselves. Every wait is bounded (FLINT_DEVCHECK_WAIT). The launch is
+// cooperative, so every CTA is resident.
 #pragma once
 
 #include "layer_kernels.cuh"
@@ -32,7 +33,6 @@ namespace flint {
 constexpr int kFusedMaxTokens = 8;
 constexpr int kFusedWarps = 8;
 constexpr int kFusedDownTokens = 4;   // tokens per pass in the down phase
-constexpr int kBarrierCounters = 4;   // control-block words 32, 64, 96, 128
 // Tagged logits are written to this many replicas; CTA c reads replica c % R,
 // so each line is polled by G/R CTAs instead of all of them.
 constexpr int kLogitReplicas = 8;
@@ -41,40 +41,6 @@ __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
   unsigned v;
   asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
-}
-
-// Grid barrier over monotonically increasing counters: CTA c adds 1 to counter
-// c % 4 (release); a call's barrier is complete when counter i holds
-// n_i * (gen + 1), n_i the number of CTAs with c % 4 == i.
-__device__ __forceinline__ bool grid_barrier(unsigned* ctrl, unsigned gen, int* status, int* s_ok) {
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x, G = gridDim.x;
-    if (lane == 0)
-      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctrl + 32 * (1 + blockIdx.x % kBarrierCounters))
-                   : "memory");
-    const unsigned n_i =
-        lane < kBarrierCounters ? static_cast<unsigned>((G - lane + kBarrierCounters - 1) / kBarrierCounters) : 0u;
-    const unsigned target = n_i * (gen + 1u);
-    const long long t0 = clock64();
-    bool ok = true;
-    for (;;) {
-      const bool mine =
-          lane >= kBarrierCounters || static_cast<int>(ld_relaxed_u32(ctrl + 32 * (1 + lane)) - target) >= 0;
-      if (__all_sync(0xffffffffu, mine)) break;
-      if (clock64() - t0 > kWaitCycles) {
-        ok = false;
-        break;
-      }
-    }
-    asm volatile("fence.acq_rel.gpu;" ::: "memory");
-    if (lane == 0) {
-      *s_ok = ok ? 1 : 0;
-      if (!ok) atomicOr(status, FLINT_DEVCHECK_WAIT);
-    }
-  }
-  __syncthreads();
-  return *s_ok != 0;
 }
 
 // Exclusive prefix over the active experts of the gate/up cost of expert a,
@@ -164,7 +130,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   __shared__ int s_cost[kFusedWarps][kFusedMaxTokens * kMaxTopK + 2];  // per-warp cost prefix over <= T*k+1 experts
   __shared__ float s_hinv[MAXR];
   __shared__ unsigned s_gen;
-  __shared__ int s_ok, s_fail;
+  __shared__ int s_fail;
   __shared__ __align__(8) uint64_t s_bar[kFusedWarps * kMaxStages + 2];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int T = p.T, E = p.E, k = p.k, S = p.S, KS = k + S, G = gridDim.x, c = blockIdx.x;
@@ -342,9 +308,9 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
         cur_g0 = g0;
       }
       if (n == 1 && M::TGMAX > 1)
-        gateup_chunk<D, 1>(st, cu, xh, lane, n, fg, fu, hrow, p.h, I, uu);
+        gateup_chunk<D, 1>(st, cu, xh, lane, n, fg, fu, hrow, p.h, I, uu, p.htag, tag);
       else
-        gateup_chunk<D, M::TGMAX>(st, cu, xh, lane, n, fg, fu, hrow, p.h, I, uu);
+        gateup_chunk<D, M::TGMAX>(st, cu, xh, lane, n, fg, fu, hrow, p.h, I, uu, p.htag, tag);
     }
   };
 
@@ -403,7 +369,17 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     // 32-bit arithmetic: C <= 65 experts x 1024 units x 4 passes and
     // gw < 240 * 8, so gw * C < 2^31
     const int C = n_routed > 0 ? cost[n_routed] : 0;
-    const int c_begin = gw * C / NW, c_end = (gw + 1) * C / NW;
+    // balance routed + shared work: warp w's routed range starts where the
+    // combined cost w*(C + shared)/NW minus the shared cost of warps < w
+    // falls (the shared units were split by warp index before the routing)
+    const int ps = S > 0 ? (T + M::TGMAX - 1) / M::TGMAX : 0;  // passes of the shared expert
+    const int CT = C + I * ps;
+    auto rbound = [&](int w) { return min(C, max(0, w * CT / NW - (w * I / NW) * ps)); };
+    // the bounds never decrease when each warp's share of CT covers the most
+    // shared cost one warp can have
+    const bool balanced = CT / NW >= ps * ((I + NW - 1) / NW);
+    const int c_begin = balanced ? rbound(gw) : gw * C / NW;
+    const int c_end = balanced ? (gw + 1 == NW ? C : rbound(gw + 1)) : (gw + 1) * C / NW;
     auto to_unit = [&](int cc, int& a, int& u) {
       int lo = 0, hi = n_routed - 1;
       while (lo < hi) {
@@ -509,8 +485,9 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   }
   const int n_active = ok ? dsc->n_active : 0;
   if (!ok) drain_ring(bars, ns_g, consumed, issued, p.status);
-  if (!grid_barrier(p.counter, gen, p.status, &s_ok)) ok = false;
-  if (c == 0 && tid == 0) asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p.counter + 1), "r"(gen + 1u) : "memory");
+  // every warp of this CTA is past its gate/up stages before the down phase
+  // reuses their shared memory
+  __syncthreads();
 
   // ---- P4: down rows of this CTA's block of outputs, for every active expert
   // work area: [h16 R x I f16, lane-interleaved][s_y R x nb fp32][rings]
@@ -545,35 +522,57 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     next_issue += kFusedWarps;
     ++issued_d;
   }
-  // h (fp32, written by every CTA) -> f16 rows with a power-of-two scale each.
-  // Element i of row P sits at P*I + ((i%32)/8 * VRD + i/32) * 8 + i%8, so the
-  // 16-byte vectors the lanes of a down step read are contiguous.
+  // h rows (tagged, written by every CTA's gate/up) -> f16 rows with a
+  // power-of-two scale each, converted once a row's I values all carry this
+  // launch's tag: this wait is the layer's only cross-CTA dependency after the
+  // routing. Element i of row P sits at P*I + ((i%32)/8 * VRD + i/32) * 8 + i%8,
+  // so the 16-byte vectors the lanes of a down step read are contiguous.
   if (ok) {
-    constexpr int F4 = I / 128;  // float4 per lane per row
-    for (int P = warp; P < R; P += kFusedWarps) {
-      float4 v[F4];
+    constexpr int F = I / 32;  // values per lane per row, element lane + 32*m
+    for (int P = warp; P < R && ok; P += kFusedWarps) {
+      const unsigned long long* rowp = p.htag + static_cast<size_t>(P) * I;
+      float v[F];
+      unsigned pend = (F >= 32) ? 0xFFFFFFFFu : ((1u << F) - 1u);
+      const long long t0 = clock64();
+      for (;;) {
+        unsigned long long w[F];
 #pragma unroll
-      for (int m = 0; m < F4; ++m) v[m] = ldg_cg4(p.h + static_cast<size_t>(P) * I + 4 * (lane + 32 * m));
+        for (int m = 0; m < F; ++m) w[m] = (pend & (1u << m)) ? ld_tagged(rowp + lane + 32 * m) : 0ull;
+#pragma unroll
+        for (int m = 0; m < F; ++m)
+          if ((pend & (1u << m)) && static_cast<uint32_t>(w[m] >> 32) == tag) {
+            v[m] = __uint_as_float(static_cast<uint32_t>(w[m]));
+            pend &= ~(1u << m);
+          }
+        if (__all_sync(0xffffffffu, pend == 0)) break;
+        if (clock64() - t0 > kWaitCycles) {
+          ok = false;
+          if (lane == 0) atomicOr(p.status, FLINT_DEVCHECK_WAIT);
+          break;
+        }
+      }
+      if (!ok) break;
       float amax = 0.f;
 #pragma unroll
-      for (int m = 0; m < F4; ++m)
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[m].x), fabsf(v[m].y)), fmaxf(fabsf(v[m].z), fabsf(v[m].w))));
+      for (int m = 0; m < F; ++m) amax = fmaxf(amax, fabsf(v[m]));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
       const float sig = pow2_scale_for(amax);
       if (lane == 0) s_hinv[P] = 1.f / sig;
 #pragma unroll
-      for (int m = 0; m < F4; ++m) {
-        const int i0 = 4 * (lane + 32 * m);
-        const int pos = (((i0 & 31) >> 3) * VRD + (i0 >> 5)) * 8 + (i0 & 7);
-        uint2 w;
-        w.x = pack_f16x2(v[m].x * sig, v[m].y * sig);
-        w.y = pack_f16x2(v[m].z * sig, v[m].w * sig);
-        *reinterpret_cast<uint2*>(h16 + static_cast<size_t>(P) * I + pos) = w;
+      for (int m = 0; m < F; ++m) {
+        const __half hv = __float2half_rn(v[m] * sig);
+        h16[static_cast<size_t>(P) * I + (((lane >> 3) * VRD + m) << 3) + (lane & 7)] =
+            *reinterpret_cast<const uint16_t*>(&hv);
       }
     }
+    if (!ok && lane == 0) s_fail = 1;
   }
   __syncthreads();
+  if (s_fail) ok = false;
+  // every CTA read this launch's generation before it wrote any h row, so the
+  // generation can advance once all rows were seen
+  if (c == 0 && tid == 0) asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p.counter + 1), "r"(gen + 1u) : "memory");
   const int rs = lane / VRD, cbk = lane % VRD;
   for (int it = warp; it < n_items && ok; it += kFusedWarps) {
     const int a = it / nsub, sb = it % nsub;

@@ -47,6 +47,7 @@ struct LayerParams {
   int* ids;                  // [T][k]
   float* gates;              // [T][k]
   float* h;                  // [T*(k+S)][I] fp32 SwiGLU intermediates
+  unsigned long long* htag;  // [T*(k+S)][I] tagged h of the persistent kernel
   int* ids_out;              // optional public copy
   float* gates_out;          // optional public copy
   long long cpe;             // code bytes per expert (3*I*d/2)

@@ -284,10 +284,13 @@ __global__ void __launch_bounds__(kRouteWarps * 32, 1) k_route(LayerParams p) {
 // ----------------------------------------------------------------- k_gateup
 // One chunk (cu <= CU consecutive units of one expert, staged at `st`) against
 // TG tokens. Writes h for the chunk's (unit, token) pairs.
+// With htag != nullptr, h is written as tagged 64-bit words (tag << 32 | h
+// bits, one relaxed store each) instead of plain fp32.
 template <int D, int TG>
 __device__ __forceinline__ void gateup_chunk(const uint8_t* st, int cu, const uint32_t* xh, int lane,
                                              int n, const float* fscale_g, const float* fscale_u,
-                                             const int* hrow, float* h, int I, int u0) {
+                                             const int* hrow, float* h, int I, int u0,
+                                             unsigned long long* htag = nullptr, uint32_t tag = 0) {
   using M = GateUpMap<D>;
   constexpr int V = TG * 2;  // (token, gate|up) partial sums per unit
   constexpr int LV = ilog2(V);
@@ -323,8 +326,14 @@ __device__ __forceinline__ void gateup_chunk(const uint8_t* st, int cu, const ui
     const float other = __shfl_xor_sync(0xffffffffu, total, 1 << rep);
     const int idx = lane >> rep;
     const int r = idx & 1, t = idx >> 1;
-    if (r == 0 && (lane & ((1 << rep) - 1)) == 0 && t < n)
-      h[static_cast<size_t>(hrow[t]) * I + u0 + c] = swiglu(total * fscale_g[t], other * fscale_u[t]);
+    if (r == 0 && (lane & ((1 << rep) - 1)) == 0 && t < n) {
+      const float hv = swiglu(total * fscale_g[t], other * fscale_u[t]);
+      const size_t o = static_cast<size_t>(hrow[t]) * I + u0 + c;
+      if (htag != nullptr)
+        st_tagged(htag + o, tag, hv);
+      else
+        h[o] = hv;
+    }
   }
 }
 
