@@ -618,21 +618,27 @@ int mma_maps(MmaMaps* mp, const Dims& s, const flint_moe_weights* wts, bool gate
 // four A stages and as many raw-weight stages as fit; bf16 weights as many A
 // stages as fit. Returns the dynamic shared-memory bytes.
 size_t mma_configure(MmaParams& m, int T) {
-  constexpr size_t kBudget = 220 * 1024;
+  constexpr size_t kBudget = 220 * 1024 - 1024;
   const int npad = std::min(kMmaMaxTokens, (T + 15) & ~15);
   m.b_bytes = npad * 128;
-  m.n_b = 4;
-  size_t left = kBudget - 1024 - static_cast<size_t>(m.n_b) * m.b_bytes;
+  m.ksplit = (npad <= kMmaMaxTokens / 2) ? 2 : 1;
+  // A stages are recycled only after their MMAs complete, so the A ring must
+  // cover that round trip: NVFP4 keeps 8 stages in tensor memory (columns
+  // 256..511) fed by 4 raw stages; bf16 weights take the shared memory left
+  // after 6 activation-row stages
+  m.n_b = 6;
+  const size_t bbytes = static_cast<size_t>(m.n_b) * m.b_bytes;
+  size_t wbytes;
   if (m.nvfp4) {
-    m.n_a = 4;
-    left -= static_cast<size_t>(m.n_a) * kMmaABytes;
-    m.n_raw = static_cast<int>(std::min<size_t>(kMmaMaxStages, left / kMmaRawBytes));
+    m.n_a = 8;
+    m.n_raw = static_cast<int>(std::min<size_t>(8, (kBudget - bbytes) / kMmaRawBytes));
+    wbytes = static_cast<size_t>(m.n_raw) * kMmaRawBytes;
   } else {
     m.n_raw = 1;
-    m.n_a = static_cast<int>(std::min<size_t>(kMmaMaxStages, left / kMmaABytes));
+    m.n_a = static_cast<int>(std::min<size_t>(kMmaMaxStages, (kBudget - bbytes) / kMmaABytes));
+    wbytes = static_cast<size_t>(m.n_a) * kMmaABytes;
   }
-  return 1024 + (m.nvfp4 ? static_cast<size_t>(m.n_raw) * kMmaRawBytes : 0) +
-         static_cast<size_t>(m.n_a) * kMmaABytes + static_cast<size_t>(m.n_b) * m.b_bytes;
+  return 1024 + wbytes + bbytes;
 }
 
 // The tensor-core layer: router, top-k, grouping, B rows, gate/up, h rows,
@@ -682,7 +688,8 @@ int run_mma_path(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, 
   e = launch(k_mma_prep, dim3((P + 7) / 8), dim3(256), 0, st, pdl, m);
   if (e != cudaSuccess) return cuda_fail(e, "k_mma_prep launch");
   const size_t smem = mma_configure(m, T);
-  const int ncols = 2 * kMmaMaxTokens;
+  // tensor memory: two accumulators, plus the A stages for NVFP4 weights
+  const int ncols = m.nvfp4 ? 512 : 2 * kMmaMaxTokens;
   const dim3 grid(num_sms()), block(kMmaWarps * 32);
   e = ensure_smem(reinterpret_cast<const void*>(k_mma_ffn<kEpiGateUp>));
   if (e == cudaSuccess) e = ensure_smem(reinterpret_cast<const void*>(k_mma_ffn<kEpiDown>));

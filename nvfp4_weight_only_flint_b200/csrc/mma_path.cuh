@@ -43,7 +43,7 @@ namespace flint {
 
 constexpr int kMmaMaxTokens = 128;  // N of one MMA <= 128 (tokens of one expert)
 constexpr int kMmaWarps = 16;
-constexpr int kMmaMaxStages = 8;    // ring depths are chosen per call, up to this
+constexpr int kMmaMaxStages = 16;   // ring depths are chosen per call, up to this
 constexpr int kMmaRawBytes = 128 * 128 + 128 * 16;  // NVFP4 stage, 256 of K: codes (swizzled) + scales
 constexpr int kMmaABytes = 128 * 128;               // A operand stage: 128 rows x 64 of K, 16-bit
 
@@ -78,6 +78,7 @@ struct MmaParams {
   int nvfp4;                // 1: NVFP4 weights, f16 operands; 0: bf16 weights, bf16 operands
   int n_raw, n_a, n_b;      // ring depths (raw NVFP4 stages, A stages, B stages)
   int b_bytes;              // B stage: (tokens rounded up to 16, at most 128) x 128 bytes
+  int ksplit;               // accumulators per item (1 or 2), fed alternate K steps, summed in the epilogue
 };
 
 // ----------------------------------------------------------------- PTX wrappers
@@ -117,6 +118,27 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16, cta_group::1 (A: row i in lane
+// i, two 16-bit K elements per 32-bit column).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// 16 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // Arrives on `bar` once every tcgen05 operation this thread issued so far is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
@@ -356,6 +378,36 @@ __device__ __forceinline__ void dequant_slice(const uint8_t* raw, int sub, uint8
   }
 }
 
+// Dequantise one 64-element slice of K of the 128-row A tile straight into
+// tensor memory (NVFP4 weights): dequantiser warp w (8..15) owns the lanes of
+// its quarter (rows 32*(w%4)..+31) and half (w-8)/4 of the slice's K: 32 codes
+// and their 2 scales of its row -> 16 columns of two f16 values each. The
+// operand never passes through shared memory.
+__device__ __forceinline__ void dequant_slice_tmem(const uint8_t* raw, int sub, uint32_t a_tmem, int warp, int lane) {
+  const int qtr = warp & 3, half = (warp - 8) >> 2;
+  const int r = 32 * qtr + lane;
+  const int chunk = 2 * sub + half;  // 16-byte code chunk of the 128-byte raw row
+  const uint4 cv = lds128(raw + r * 128 + ((chunk ^ (r & 7)) << 4));
+  const uint32_t s2 = *reinterpret_cast<const uint16_t*>(raw + 128 * 128 + r * 16 + 4 * sub + 2 * half);
+  uint32_t sh;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(sh) : "h"(static_cast<uint16_t>(s2)));
+  const __half2 hs = *reinterpret_cast<const __half2*>(&sh);
+  const __half2 sc[2] = {__low2half2(hs), __high2half2(hs)};
+  const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+  uint32_t out[16];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {  // 8 elements per q; words 0,1 -> block 0, words 2,3 -> block 1
+    uint32_t f[4];
+    e2m1x8_to_f16x2(cw[q], *reinterpret_cast<uint32_t(*)[4]>(&f[0]));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&f[j]), sc[q >> 1]);
+      out[4 * q + j] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+  }
+  tmem_st16(a_tmem + (static_cast<uint32_t>(32 * qtr) << 16) + static_cast<uint32_t>(16 * half), out);
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     k_mma_ffn(MmaParams p, const __grid_constant__ MmaMaps maps, int ncols) {
@@ -373,8 +425,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
   // 1024-aligned carve-up: [raw stages (NVFP4 only)][A stages][B stages]
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* raw = base;
-  uint8_t* abuf = raw + (fp4 ? NR * kMmaRawBytes : 0);
-  uint8_t* bbuf = abuf + NA * kMmaABytes;
+  uint8_t* abuf = raw + (fp4 ? NR * kMmaRawBytes : 0);  // bf16 weights: A stages in shared memory
+  uint8_t* bbuf = abuf + (fp4 ? 0 : NA * kMmaABytes);
+  // tensor memory: two accumulators (columns 0..255), then the NVFP4 A stages
+  // (32 columns each: 128 rows x 64 of K in f16)
+  constexpr uint32_t kAccCols = 2 * kMmaMaxTokens;
   const int K = EPI == kEpiGateUp ? p.d : p.I;
   const int tiles = EPI == kEpiGateUp ? p.I / 64 : p.d / 128;
   const int n_sub = K / 64;
@@ -480,15 +535,29 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
         if (!(ok = mma_wait(&acc_empty[ab], ((icount >> 1) & 1) ^ 1, abort_flag, p.status))) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * kMmaMaxTokens);
+        // consecutive K steps alternate between `ksplit` accumulators of
+        // kMmaMaxTokens / ksplit columns: independent accumulation chains
+        const uint32_t dstep = static_cast<uint32_t>(kMmaMaxTokens / p.ksplit);
+        const int kmask = p.ksplit - 1;
         for (int s = 0; s < n_sub; ++s) {
           const int as = sc % NA, bs = bcount % NB;
           if (!(ok = mma_wait(&a_full[as], (sc / NA) & 1, abort_flag, p.status))) break;
           if (!(ok = mma_wait(&b_full[bs], (bcount / NB) & 1, abort_flag, p.status))) break;
           tc_fence_after();
-          const uint32_t aaddr = smem_addr(abuf + as * kMmaABytes), baddr = smem_addr(bbuf + bs * BB);
+          const uint32_t baddr = smem_addr(bbuf + bs * BB);
+          if (fp4) {
+            const uint32_t a_tmem = tmem + kAccCols + static_cast<uint32_t>(32 * as);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16(d_tmem, sw128_desc(aaddr + 32 * kk), sw128_desc(baddr + 32 * kk), idesc, (s | kk) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ts(d_tmem + dstep * (kk & kmask), a_tmem + 8 * kk, sw128_desc(baddr + 32 * kk), idesc,
+                         (s > 0 || kk > kmask) ? 1u : 0u);
+          } else {
+            const uint32_t aaddr = smem_addr(abuf + as * kMmaABytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16(d_tmem + dstep * (kk & kmask), sw128_desc(aaddr + 32 * kk), sw128_desc(baddr + 32 * kk), idesc,
+                      (s > 0 || kk > kmask) ? 1u : 0u);
+          }
           mma_commit(&a_empty[as]);
           mma_commit(&b_empty[bs]);
           ++sc;
@@ -520,6 +589,12 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
           const float xin = (c0 + (lane & 15) < nt) ? p.xinv[off + c0 + (lane & 15)] : 0.f;
           float v[16];
           tmem_ld16(taddr + c0, v);
+          if (p.ksplit > 1) {
+            float v2[16];
+            tmem_ld16(taddr + kMmaMaxTokens / 2 + c0, v2);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += v2[j];
+          }
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
@@ -538,6 +613,12 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
           const int prn = in ? p.rt.pair[off + c0 + (lane & 15)] : 0;
           float v[16];
           tmem_ld16(taddr + c0, v);
+          if (p.ksplit > 1) {
+            float v2[16];
+            tmem_ld16(taddr + kMmaMaxTokens / 2 + c0, v2);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += v2[j];
+          }
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int n = c0 + j;
@@ -556,7 +637,6 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     }
   } else if (warp >= 8 && fp4) {
     // ------------------------------------------------ dequantisers (NVFP4)
-    const int dt = tid - 8 * 32;
     int rc = 0, sc = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
@@ -564,9 +644,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
         const int rs = rc % NR, as = sc % NA;
         if (!(ok = mma_wait(&raw_full[rs], (rc / NR) & 1, abort_flag, p.status))) break;
         if (!(ok = mma_wait(&a_empty[as], ((sc / NA) & 1) ^ 1, abort_flag, p.status))) break;
-        dequant_slice(raw + rs * kMmaRawBytes, s & 3, abuf + as * kMmaABytes, dt);
-        // generic-proxy writes of the operand -> visible to the tensor cores
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_after();  // the stage's previous MMAs are done (a_empty) before it is rewritten
+        dequant_slice_tmem(raw + rs * kMmaRawBytes, s & 3, tmem + kAccCols + static_cast<uint32_t>(32 * as), warp,
+                           lane);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&a_full[as]);
         ++sc;
