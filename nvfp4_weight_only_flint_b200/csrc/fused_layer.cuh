@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
 
   // ---- P2: top-k (waits for every CTA's logits) and grouping, in every CTA
   // (called once by every warp, from inside the chunk loop below)
-  auto routing_step = [&]() {
+  auto routing_topk = [&]() {
     if (!ok && lane == 0) s_fail = 1;  // a wait of this warp gave up: the CTA stops together
     if (warp < T) {
       bool okt = false;
@@ -332,6 +332,8 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     }
     __syncthreads();
     if (s_fail) ok = false;
+  };
+  auto routing_group = [&]() {
     // the router rows are consumed by now (every warp's router tasks precede
     // this point), so their region serves as the grouping's scratch
     if (ok) cta_grouping(s_ids, T, k, E, S, dsc->act, dsc->off, dsc->pair, &dsc->n_routed, &dsc->n_active, rsm,
@@ -349,11 +351,28 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   };
 
   // ---- P2 right after the router: top-k and grouping
-  routing_step();
+  routing_topk();
   if (!ok) {
     drain_ring(bars, ns_g, consumed, issued, p.status);
     consumed = issued;
   }
+  // One token: its k experts are distinct and each costs I units x 1 pass, so
+  // the routed work split needs only their sorted ids, known right after the
+  // top-k: the routed copies are issued before the grouping runs. Lane r of
+  // every warp holds the r-th smallest id.
+  const bool early = (T == 1) && ok;
+  int my_act = 0;
+  if (early) {
+    const int v = lane < k ? s_ids[lane] : 0x7FFFFFFF;
+    int rank = 0;
+    for (int i = 0; i < k; ++i) rank += s_ids[i] < v ? 1 : 0;
+    for (int j = 0; j < k; ++j) {
+      const int vj = __shfl_sync(0xffffffffu, v, j), rj = __shfl_sync(0xffffffffu, rank, j);
+      if (rj == lane) my_act = vj;
+    }
+  }
+  auto act_of = [&](int a) { return early ? __shfl_sync(0xffffffffu, my_act, a) : static_cast<int>(dsc->act[a]); };
+  if (!early) routing_group();
 
   // ---- P3: one stream of chunks per warp, issued and consumed in the same
   // order: phase 0 is this warp's slice of the shared expert's units (index =
@@ -362,13 +381,15 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   // loop, so the chunk code exists once.
   int u_begin = 0, u_end = 0;
   {
-    const int n_routed = ok ? dsc->n_routed : 0;
+    const int n_routed = early ? k : (ok ? dsc->n_routed : 0);
     int* cost = s_cost[warp];
-    cost_prefix(dsc, n_routed, I, M::TGMAX, cost, lane);
-    __syncwarp();
+    if (!early) {
+      cost_prefix(dsc, n_routed, I, M::TGMAX, cost, lane);
+      __syncwarp();
+    }
     // 32-bit arithmetic: C <= 65 experts x 1024 units x 4 passes and
     // gw < 240 * 8, so gw * C < 2^31
-    const int C = n_routed > 0 ? cost[n_routed] : 0;
+    const int C = early ? k * I : (n_routed > 0 ? cost[n_routed] : 0);
     // balance routed + shared work: warp w's routed range starts where the
     // combined cost w*(C + shared)/NW minus the shared cost of warps < w
     // falls (the shared units were split by warp index before the routing)
@@ -391,7 +412,10 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
       const int passes = (dsc->off[a + 1] - dsc->off[a] + M::TGMAX - 1) / M::TGMAX;
       u = (cc - cost[a]) / passes;
     };
-    if (c_end > c_begin) {
+    if (early) {  // cost index == unit index (one pass per unit)
+      u_begin = c_begin;
+      u_end = c_end;
+    } else if (c_end > c_begin) {
       int a0, u0, a1, u1;
       to_unit(c_begin, a0, u0);
       to_unit(c_end - 1, a1, u1);
@@ -414,9 +438,10 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     }
   };
   auto issue_at = [&](int ph, int gg) {
+    const int e = ph == 0 ? E : act_of(gg / I);  // every lane (act_of may shuffle)
     if (lane == 0) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue_units(ph == 0 ? E : dsc->act[gg / I], ph == 0 ? gg : gg % I, len_at(ph, gg), issued % ns_g);
+      issue_units(e, ph == 0 ? gg : gg % I, len_at(ph, gg), issued % ns_g);
     }
   };
   int iph = 0, ig = sh_issue;
@@ -427,6 +452,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     settle(iph, ig);
     ++issued;
   }
+  if (early) routing_group();
   // then an L2 prefetch of this CTA's block of down rows of every routed
   // active expert (queued behind the gate/up copies)
   for (int a = warp * 32 + lane; ok && a < dsc->n_routed && nrows > 0; a += kFusedWarps * 32) {
