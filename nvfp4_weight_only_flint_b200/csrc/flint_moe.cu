@@ -444,7 +444,7 @@ size_t configure_fused(LayerParams& p, const Dims& s, int T) {
   p.h_in_smem = 1;
   const size_t a128 = 127;
   const int R = T * (s.k + s.S);
-  const size_t head = sizeof(RouteDesc) + 2 * ((static_cast<size_t>(T) * s.d * 2 + a128) & ~a128) +
+  const size_t head = sizeof(RouteDesc) + ((static_cast<size_t>(T) * s.d * 2 + a128) & ~a128) +
                       fused_rows_bytes((s.E + sms - 1) / sms * s.d * 2, s.E);
   const size_t ybytes = ((4 * static_cast<size_t>(R) * nb) + a128) & ~a128;
   const size_t ring_d = static_cast<size_t>(kFusedWarps) * p.ns_down * p.stage_down;

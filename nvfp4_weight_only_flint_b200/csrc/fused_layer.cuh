@@ -1,9 +1,9 @@
 // fused_layer.cuh -- the whole layer in one persistent kernel (batch <= 8).
 //
-// One CTA per SM (8 warps), every SM busy in every phase:
-//   P0  bulk copies of x, of this CTA's router rows and of each warp's slice
-//       of the shared expert's gate/up units; L2 prefetch of this CTA's block
-//       of the shared expert's down rows
+// One CTA per SM (16 warps), every SM busy in every phase:
+//   P0  bulk copies of this CTA's router rows and of each warp's slice of
+//       the shared expert's gate/up units; L2 prefetch of this CTA's block of
+//       the shared expert's down rows
 //   P1  per-token scales, x converted once to f16 (lane-interleaved), router
 //       logits ((row, token) tasks over the warps), stored as tagged 64-bit
 //       words (launch tag | logit) in 8 replicas
@@ -31,7 +31,7 @@
 namespace flint {
 
 constexpr int kFusedMaxTokens = 8;
-constexpr int kFusedWarps = 8;
+constexpr int kFusedWarps = 16;
 constexpr int kFusedDownTokens = 4;   // tokens per pass in the down phase
 // Tagged logits are written to this many replicas; CTA c reads replica c % R,
 // so each line is polled by G/R CTAs instead of all of them.
@@ -138,19 +138,17 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
 
   // ---- shared-memory carve-up: [desc][x][router rows][work]
   RouteDesc* dsc = reinterpret_cast<RouteDesc*>(smem);
-  uint8_t* xsm = smem + sizeof(RouteDesc);
   const size_t xbytes = static_cast<size_t>(T) * D * 2;
   const size_t xpad = (xbytes + 127) & ~static_cast<size_t>(127);
   // x * sigma_t as f16, lane-interleaved: element i of token t at
   // t*D + (((i % 32) / 8) * (D / 32) + i / 32) * 8 + i % 8, so the 16-byte
   // chunks the lanes of a gate/up step read are contiguous
-  uint16_t* x16 = reinterpret_cast<uint16_t*>(xsm + xpad);
-  uint8_t* rsm = xsm + 2 * xpad;
+  uint16_t* x16 = reinterpret_cast<uint16_t*>(smem + sizeof(RouteDesc));
+  uint8_t* rsm = smem + sizeof(RouteDesc) + xpad;
   const int rpc = (E + G - 1) / G;  // router rows per CTA
   uint8_t* work = rsm + fused_rows_bytes(rpc * D * 2, E);
   uint64_t* ring_bars = s_bar;                        // [warp][kMaxStages]
-  uint64_t* xbar = s_bar + kFusedWarps * kMaxStages;  // x
-  uint64_t* rbar = xbar + 1;                          // router rows
+  uint64_t* rbar = s_bar + kFusedWarps * kMaxStages;  // router rows
   const int ns_g = p.ns_gateup, ns_d = p.ns_down;
   const int nb = p.down_nb, n0 = c * nb, nrows = max(0, min(nb, p.d - n0));
   const int r_begin = min(E, c * rpc), r_end = min(E, (c + 1) * rpc);
@@ -159,8 +157,6 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   if (tid == 0) {
     for (int i = 0; i < kFusedWarps * kMaxStages + 2; ++i) mbar_init(&s_bar[i], 1);
     fence_barrier_init();
-    mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(xbytes));
-    bulk_g2s(xsm, p.x, static_cast<uint32_t>(xbytes), xbar);
     const uint32_t rbytes = static_cast<uint32_t>(r_end - r_begin) * D * 2;
     mbar_arrive_expect_tx(rbar, rbytes);
     if (rbytes) bulk_g2s(rsm, p.wr + static_cast<size_t>(r_begin) * D, rbytes, rbar);
@@ -202,14 +198,15 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   }
 
   // ---- P1: token statistics, router logits
-  bool ok = mbar_wait(xbar, 0, p.status);
-  const uint16_t* xs = reinterpret_cast<const uint16_t*>(xsm);
+  bool ok = true;
+  // x (bf16, read-only for the whole launch) is read through the L1 cache
+  const uint4* xg = reinterpret_cast<const uint4*>(p.x);
   if (warp < T && ok) {
     const int t = warp;
     float amax = 0.f, ss = 0.f;
 #pragma unroll
     for (int i = 0; i < NVR; ++i) {
-      const uint4 v = lds128(xs + static_cast<size_t>(t) * D + 8 * (lane + 32 * i));
+      const uint4 v = __ldg(xg + (static_cast<size_t>(t) * D + 8 * (lane + 32 * i)) / 8);
       const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -231,7 +228,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
 #pragma unroll
     for (int i = 0; i < NVR; ++i) {
       const int i0 = 8 * (lane + 32 * i);
-      const uint4 v = lds128(xs + static_cast<size_t>(t) * D + i0);
+      const uint4 v = __ldg(xg + (static_cast<size_t>(t) * D + i0) / 8);
       uint4 o;
       o.x = bf16x2_to_f16x2_scaled(v.x, sg);
       o.y = bf16x2_to_f16x2_scaled(v.y, sg);
@@ -249,7 +246,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
 #pragma unroll
     for (int i = 0; i < NVR; ++i) {
       const uint4 wv = lds128(wrow + 8 * (lane + 32 * i));
-      const uint4 xv = lds128(xs + static_cast<size_t>(t) * D + 8 * (lane + 32 * i));
+      const uint4 xv = __ldg(xg + (static_cast<size_t>(t) * D + 8 * (lane + 32 * i)) / 8);
       const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
       const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
       float a = 0.f;
@@ -388,7 +385,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
       __syncwarp();
     }
     // 32-bit arithmetic: C <= 65 experts x 1024 units x 4 passes and
-    // gw < 240 * 8, so gw * C < 2^31
+    // gw < 240 * 16, so gw * C < 2^31
     const int C = early ? k * I : (n_routed > 0 ? cost[n_routed] : 0);
     // balance routed + shared work: warp w's routed range starts where the
     // combined cost w*(C + shared)/NW minus the shared cost of warps < w
