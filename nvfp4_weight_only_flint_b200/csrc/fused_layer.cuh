@@ -197,12 +197,46 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     ++issued;
   }
 
-  // ---- P1: token statistics, router logits
+  // ---- P1: router logits first (the top-k waits for them), then token
+  // statistics and the f16 copy of x the gate/up phase reads after the routing
   bool ok = true;
   // x (bf16, read-only for the whole launch) is read through the L1 cache
   const uint4* xg = reinterpret_cast<const uint4*>(p.x);
-  if (warp < T && ok) {
-    const int t = warp;
+  const int n_tasks = (r_end - r_begin) * T;
+  if (warp < n_tasks && ok) ok = mbar_wait(rbar, 0, p.status);
+  for (int task = warp; task < n_tasks && ok; task += kFusedWarps) {
+    const int r = task / T, t = task % T;
+    const uint16_t* wrow = reinterpret_cast<const uint16_t*>(rsm) + static_cast<size_t>(r) * D;
+    // the token's sum of squares in the same order as the statistics below,
+    // so the input-norm factor is the same value
+    float sum = 0.f, ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < NVR; ++i) {
+      const uint4 wv = lds128(wrow + 8 * (lane + 32 * i));
+      const uint4 xv = __ldg(xg + (static_cast<size_t>(t) * D + 8 * (lane + 32 * i)) / 8);
+      const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+      const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
+      float a = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float xa = bf16_bits_to_f32(xx[q] & 0xFFFFu), xb = __uint_as_float(xx[q] & 0xFFFF0000u);
+        a = fmaf(bf16_bits_to_f32(ww[q] & 0xFFFFu), xa, a);
+        a = fmaf(__uint_as_float(ww[q] & 0xFFFF0000u), xb, a);
+        ss = fmaf(xa, xa, ss);
+        ss = fmaf(xb, xb, ss);
+      }
+      sum += a;
+    }
+    sum = warp_sum(sum);
+    ss = warp_sum(ss);
+    const float irms = p.input_norm ? 1.f / sqrtf(ss / static_cast<float>(D) + kRmsEps) : 1.f;
+    if (lane < kLogitReplicas)
+      st_tagged(p.tlogits + (static_cast<size_t>(lane) * T + t) * E + r_begin + r, tag, sum * irms);
+  }
+  // statistics of token t on warp kFusedWarps-1-t (idle during the router at
+  // one token)
+  if (kFusedWarps - 1 - warp < T && ok) {
+    const int t = kFusedWarps - 1 - warp;
     float amax = 0.f, ss = 0.f;
 #pragma unroll
     for (int i = 0; i < NVR; ++i) {
@@ -236,30 +270,6 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
       o.w = bf16x2_to_f16x2_scaled(v.w, sg);
       *reinterpret_cast<uint4*>(x16 + static_cast<size_t>(t) * D + (((i0 & 31) >> 3) * (D / 32) + (i0 >> 5)) * 8) = o;
     }
-  }
-  __syncthreads();
-  if (r_end > r_begin && ok) ok = mbar_wait(rbar, 0, p.status);
-  for (int task = warp; task < (r_end - r_begin) * T && ok; task += kFusedWarps) {
-    const int r = task / T, t = task % T;
-    const uint16_t* wrow = reinterpret_cast<const uint16_t*>(rsm) + static_cast<size_t>(r) * D;
-    float sum = 0.f;
-#pragma unroll
-    for (int i = 0; i < NVR; ++i) {
-      const uint4 wv = lds128(wrow + 8 * (lane + 32 * i));
-      const uint4 xv = __ldg(xg + (static_cast<size_t>(t) * D + 8 * (lane + 32 * i)) / 8);
-      const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-      const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
-      float a = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        a = fmaf(bf16_bits_to_f32(ww[q] & 0xFFFFu), bf16_bits_to_f32(xx[q] & 0xFFFFu), a);
-        a = fmaf(__uint_as_float(ww[q] & 0xFFFF0000u), __uint_as_float(xx[q] & 0xFFFF0000u), a);
-      }
-      sum += a;
-    }
-    sum = warp_sum(sum);
-    if (lane < kLogitReplicas)
-      st_tagged(p.tlogits + (static_cast<size_t>(lane) * T + t) * E + r_begin + r, tag, sum * s_f[t] * s_sigma[t]);
   }
 
   // gate/up of one staged chunk of `cu` units from unit uu, for the tokens
@@ -358,14 +368,43 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
   // top-k: the routed copies are issued before the grouping runs. Lane r of
   // every warp holds the r-th smallest id.
   const bool early = (T == 1) && ok;
-  int my_act = 0;
+  int my_act = 0, my_slot = 0;
   if (early) {
     const int v = lane < k ? s_ids[lane] : 0x7FFFFFFF;
     int rank = 0;
     for (int i = 0; i < k; ++i) rank += s_ids[i] < v ? 1 : 0;
     for (int j = 0; j < k; ++j) {
       const int vj = __shfl_sync(0xffffffffu, v, j), rj = __shfl_sync(0xffffffffu, rank, j);
-      if (rj == lane) my_act = vj;
+      if (rj == lane) {
+        my_act = vj;
+        my_slot = j;
+      }
+    }
+    // the grouping of one token: active slot a < k is the a-th smallest id,
+    // serving the token once (pair = slot of that id in the top-k list); the
+    // shared experts follow. Nothing reads the descriptor before the barrier
+    // that ends the gate/up phase.
+    if (warp == 0) {
+      if (lane < k) {
+        dsc->act[lane] = my_act;
+        dsc->pair[lane] = static_cast<unsigned short>(my_slot);
+      } else if (lane < k + S) {
+        dsc->act[lane] = E + (lane - k);
+        dsc->pair[lane] = static_cast<unsigned short>(lane);
+      }
+      if (lane <= k + S) dsc->off[lane] = lane;
+      if (lane == 0) {
+        dsc->n_routed = k;
+        dsc->n_active = k + S;
+      }
+      if (c == 0 && lane < k) {
+        p.ids[lane] = s_ids[lane];
+        p.gates[lane] = s_gates[lane];
+        if (p.ids_out != nullptr) {
+          p.ids_out[lane] = s_ids[lane];
+          p.gates_out[lane] = s_gates[lane];
+        }
+      }
     }
   }
   auto act_of = [&](int a) { return early ? __shfl_sync(0xffffffffu, my_act, a) : static_cast<int>(dsc->act[a]); };
@@ -449,11 +488,11 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
     settle(iph, ig);
     ++issued;
   }
-  if (early) routing_group();
   // then an L2 prefetch of this CTA's block of down rows of every routed
   // active expert (queued behind the gate/up copies)
-  for (int a = warp * 32 + lane; ok && a < dsc->n_routed && nrows > 0; a += kFusedWarps * 32) {
-    const long long e = dsc->act[a];
+  const int n_pf = early ? k : (ok ? dsc->n_routed : 0);
+  for (int a = warp * 32 + lane; ok && a < n_pf && nrows > 0; a += kFusedWarps * 32) {
+    const long long e = early ? my_act : dsc->act[a];  // early: a == lane
     prefetch_l2(p.codes + e * p.cpe + static_cast<long long>(I) * p.d + static_cast<long long>(n0) * ROWC,
                 nrows * ROWC);
     prefetch_l2(p.scales + e * p.spe + static_cast<long long>(I) * p.d / 8 + static_cast<long long>(n0) * ROWS,
@@ -476,17 +515,23 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
       } else {
         const int a = cg / I;
         if (a != cur_a) {  // tensor scales of the expert, fetched before the stage wait
-          const int e = dsc->act[a];
+          const int e = act_of(a);
           sg = __ldg(p.tscale + 3 * e + 0);
           su = __ldg(p.tscale + 3 * e + 1);
           cur_a = a;
         }
         key = a;
         uu = cg % I;
-        const int pb = dsc->off[a];
-        nt = dsc->off[a + 1] - pb;
-        pairs = dsc->pair + pb;
-        kslot = 0;
+        if (early) {  // one token, in the slot the lane-held ids give
+          nt = 1;
+          pairs = nullptr;
+          kslot = __shfl_sync(0xffffffffu, my_slot, a);
+        } else {
+          const int pb = dsc->off[a];
+          nt = dsc->off[a + 1] - pb;
+          pairs = dsc->pair + pb;
+          kslot = 0;
+        }
       }
       const int slot = consumed % ns_g;
       if (!mbar_wait(&bars[slot], (consumed / ns_g) & 1, p.status)) {
@@ -506,11 +551,11 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p) {
       }
     }
   }
-  const int n_active = ok ? dsc->n_active : 0;
   if (!ok) drain_ring(bars, ns_g, consumed, issued, p.status);
   // every warp of this CTA is past its gate/up stages before the down phase
   // reuses their shared memory
   __syncthreads();
+  const int n_active = ok ? dsc->n_active : 0;
 
   // ---- P4: down rows of this CTA's block of outputs, for every active expert
   // work area: [h16 R x I f16, lane-interleaved][s_y R x nb fp32][rings]
