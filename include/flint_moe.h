@@ -117,6 +117,12 @@ typedef enum flint_path {
                           input_rmsnorm */
 } flint_path;
 
+typedef enum flint_layer_variant {
+  FLINT_LAYER_AUTO = 0, /* tensor-core inner loops from 2 tokens, CUDA-core at 1 */
+  FLINT_LAYER_FMA = 1,  /* CUDA-core dot products (fma.rn.f32.f16) */
+  FLINT_LAYER_MMA = 2   /* register-fragment mma.sync m16n8k16 */
+} flint_layer_variant;
+
 typedef struct flint_moe_options {
   int32_t path;          /* flint_path */
   int32_t use_pdl;       /* 1 (default when options == NULL): chain the layer's
@@ -133,6 +139,11 @@ typedef struct flint_moe_options {
                             (the persistent layer kernel, or the gate/up kernel of the
                             three-kernel path, whose records then serialise the chain);
                             for per-kernel timing */
+  int32_t layer_variant; /* flint_layer_variant: inner loops of the persistent
+                            single-kernel path (batch <= 8). FLINT_LAYER_MMA
+                            multiplies the in-register decoded NVFP4 weights (exact
+                            in f16) with the f16-staged activations, f32
+                            accumulate; other values FLINT_ERR_INVALID_ARG */
 } flint_moe_options;
 
 /* Bytes of the packed codes / block scales / tensor scales for a shape. Return 0

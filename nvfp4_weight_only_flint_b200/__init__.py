@@ -25,6 +25,7 @@ __all__ = [
 
 FLINT_W_NVFP4, FLINT_W_BF16 = 0, 1
 FLINT_PATH_AUTO, FLINT_PATH_GEMV, FLINT_PATH_MMA = 0, 1, 2
+FLINT_LAYER_AUTO, FLINT_LAYER_FMA, FLINT_LAYER_MMA = 0, 1, 2
 STATUS_NAMES = {0: "FLINT_OK", -1: "FLINT_ERR_INVALID_ARG", -2: "FLINT_ERR_UNSUPPORTED_SHAPE",
                 -3: "FLINT_ERR_MISALIGNED", -4: "FLINT_ERR_WORKSPACE", -5: "FLINT_ERR_CUDA",
                 -6: "FLINT_ERR_DEVICE_CHECK", -7: "FLINT_ERR_TIMEOUT"}
@@ -50,7 +51,7 @@ class Options(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("use_pdl", ctypes.c_int32),
                 ("topk_ids", ctypes.c_void_p), ("topk_weights", ctypes.c_void_p),
                 ("split_kernels", ctypes.c_int32), ("input_rmsnorm", ctypes.c_int32),
-                ("profile_events", ctypes.c_void_p)]
+                ("profile_events", ctypes.c_void_p), ("layer_variant", ctypes.c_int32)]
 
 
 _lib = None

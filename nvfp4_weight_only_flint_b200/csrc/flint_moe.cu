@@ -426,11 +426,50 @@ size_t down_smem(const LayerParams& p) {
          static_cast<size_t>(kGemvWarps) * p.ns_down * p.stage_down;
 }
 
+// Configuration of the tensor-core variant of the persistent layer kernel:
+// gate/up rings of 16-row x 512-column stages (two 2 KiB swizzled code boxes
+// + 512 B of scales, 1 KiB-aligned), K-part sum slots for the most tiles one
+// CTA can get, down stages of 16 rows; the down phase's buffers lie over
+// everything after the routing descriptor. Returns the dynamic shared-memory
+// bytes, or 0 if the call does not fit.
+size_t configure_fused_tc(LayerParams& p, const Dims& s, int T, int sms) {
+  const size_t a128 = 127;
+  auto al = [&](size_t v) { return (v + a128) & ~a128; };
+  const int rps = 32 / (s.I / 32);
+  int nb = (s.d + sms - 1) / sms;
+  nb = ((nb + rps - 1) / rps) * rps;
+  if (nb % 2) nb += rps;
+  p.down_nb = nb;
+  p.down_rb = 16;
+  p.stage_down = 16 * (s.I / 2 + s.I / 16);
+  p.ns_gateup = 2;
+  p.stage_gateup = kTcStageCodes + kTcStageScales;
+  p.h_in_smem = 1;
+  const long long nt_max = static_cast<long long>(std::min(s.E, T * s.k) + s.S) * (s.I / kTcUnits);
+  p.tc_lt = static_cast<int>((nt_max + sms - 1) / sms) + 2;
+  const int R = T * (s.k + s.S);
+  const size_t head = sizeof(RouteDesc) + al(static_cast<size_t>(T) * tc_b_stride(s.d)) +
+                      fused_rows_bytes((s.E + sms - 1) / sms * s.d * 2, s.E) + 1024;
+  const size_t p3 = static_cast<size_t>(kFusedWarps) * p.ns_gateup * (kTcStageCodes + kTcStageScales) +
+                    al(static_cast<size_t>(p.tc_lt) * 129 * 4);
+  const size_t budget = 218 * 1024;
+  size_t p4 = 0;
+  for (p.ns_down = 2; p.ns_down >= 1; --p.ns_down) {  // one down stage per warp when two do not fit (inter 1024)
+    p4 = al(sizeof(RouteDesc)) + al(static_cast<size_t>(R) * tc_b_stride(s.I)) + al(4 * static_cast<size_t>(R) * nb) +
+         static_cast<size_t>(kFusedWarps) * p.ns_down * p.stage_down;
+    if (p4 <= budget) break;
+  }
+  const size_t need = std::max(head + p3, p4);
+  return (p.ns_down >= 1 && need <= budget) ? need : 0;
+}
+
 // Configuration of the persistent single-kernel layer (T <= 8): returns the
 // dynamic shared-memory bytes, or 0 if the call does not fit it.
-size_t configure_fused(LayerParams& p, const Dims& s, int T) {
+size_t configure_fused(LayerParams& p, const Dims& s, int T, bool tc) {
   const int sms = num_sms();
   if (sms > 240) return 0;  // the kernel's work split uses 32-bit products of the CTA index
+  p.tc_lt = 0;
+  if (tc) return configure_fused_tc(p, s, T, sms);
   p.stage_gateup = gateup_stage_bytes(s.d);
   p.ns_gateup = 2;
   const int rps = 32 / (s.I / 32);
@@ -461,9 +500,9 @@ size_t configure_fused(LayerParams& p, const Dims& s, int T) {
   return head + work;
 }
 
-template <int D, int I>
-cudaError_t launch_fused_di(const LayerParams& p, size_t smem, cudaStream_t st) {
-  auto kern = k_layer<D, I>;
+template <int D, int I, bool TC>
+cudaError_t launch_fused_di(const LayerParams& p, const FusedMaps& maps, size_t smem, cudaStream_t st) {
+  auto kern = k_layer<D, I, TC>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -476,26 +515,34 @@ cudaError_t launch_fused_di(const LayerParams& p, size_t smem, cudaStream_t st) 
   at[0].val.cooperative = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  return cudaLaunchKernelEx(&cfg, kern, p, maps);
 }
 
-template <int D>
-cudaError_t launch_fused_d(const LayerParams& p, size_t smem, cudaStream_t st) {
+template <int D, bool TC>
+cudaError_t launch_fused_d(const LayerParams& p, const FusedMaps& maps, size_t smem, cudaStream_t st) {
   switch (p.I) {
-    case 128: return launch_fused_di<D, 128>(p, smem, st);
-    case 256: return launch_fused_di<D, 256>(p, smem, st);
-    case 512: return launch_fused_di<D, 512>(p, smem, st);
-    default: return launch_fused_di<D, 1024>(p, smem, st);
+    case 128: return launch_fused_di<D, 128, TC>(p, maps, smem, st);
+    case 256: return launch_fused_di<D, 256, TC>(p, maps, smem, st);
+    case 512: return launch_fused_di<D, 512, TC>(p, maps, smem, st);
+    default: return launch_fused_di<D, 1024, TC>(p, maps, smem, st);
   }
 }
 
-cudaError_t launch_fused(const LayerParams& p, size_t smem, cudaStream_t st) {
+template <bool TC>
+cudaError_t launch_fused_t(const LayerParams& p, const FusedMaps& maps, size_t smem, cudaStream_t st) {
   switch (p.d) {
-    case 512: return launch_fused_d<512>(p, smem, st);
-    case 1024: return launch_fused_d<1024>(p, smem, st);
-    case 2048: return launch_fused_d<2048>(p, smem, st);
-    default: return launch_fused_d<4096>(p, smem, st);
+    case 512: return launch_fused_d<512, TC>(p, maps, smem, st);
+    case 1024: return launch_fused_d<1024, TC>(p, maps, smem, st);
+    case 2048: return launch_fused_d<2048, TC>(p, maps, smem, st);
+    default: return launch_fused_d<4096, TC>(p, maps, smem, st);
   }
+}
+
+cudaError_t launch_fused(const LayerParams& p, const FusedMaps* maps, size_t smem, cudaStream_t st) {
+  if (maps != nullptr) return launch_fused_t<true>(p, *maps, smem, st);
+  FusedMaps none;
+  std::memset(&none, 0, sizeof(none));
+  return launch_fused_t<false>(p, none, smem, st);
 }
 
 template <typename K>
@@ -611,6 +658,22 @@ int mma_maps(MmaMaps* mp, const Dims& s, const flint_moe_weights* wts, bool gate
   const cuuint32_t bbox[2] = {64, 16};
   return encode_map(&mp->brows, s.wd == FLINT_W_NVFP4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                     2, brows, bdims, bstr, bbox, true);
+}
+
+// Tensor maps of the tensor-core variant of the layer kernel over the gate/up
+// rows of every expert: codes [E+S][2*inter][d/2] bytes, box 128 x 16 with the
+// 128-byte swizzle; block scales [E+S][2*inter][d/16] bytes, box 32 x 16.
+int fused_maps(FusedMaps* m, const Dims& s, const flint_moe_weights* wts) {
+  const cuuint64_t ne = static_cast<cuuint64_t>(s.E + s.S);
+  const cuuint64_t cdims[3] = {static_cast<cuuint64_t>(s.d / 2), static_cast<cuuint64_t>(2 * s.I), ne};
+  const cuuint64_t cstr[2] = {static_cast<cuuint64_t>(s.d / 2), 3ull * s.I * s.d / 2};
+  const cuuint32_t cbox[3] = {128, 16, 1};
+  int rc = encode_map(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, wts->packed, cdims, cstr, cbox, true);
+  if (rc != FLINT_OK) return rc;
+  const cuuint64_t sdims[3] = {static_cast<cuuint64_t>(s.d / 16), static_cast<cuuint64_t>(2 * s.I), ne};
+  const cuuint64_t sstr[2] = {static_cast<cuuint64_t>(s.d / 16), 3ull * s.I * s.d / 16};
+  const cuuint32_t sbox[3] = {32, 16, 1};
+  return encode_map(&m->scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, wts->block_scales, sdims, sstr, sbox, false);
 }
 
 // Ring depths of the tensor-core kernels for a call of T tokens: B stages hold
@@ -857,6 +920,8 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
   if (path < FLINT_PATH_AUTO || path > FLINT_PATH_MMA) return fail(FLINT_ERR_INVALID_ARG, "path %d", path);
   if (options && ((options->topk_ids == nullptr) != (options->topk_weights == nullptr)))
     return fail(FLINT_ERR_INVALID_ARG, "topk_ids and topk_weights go together");
+  const int variant = options ? options->layer_variant : FLINT_LAYER_AUTO;
+  if (variant < FLINT_LAYER_AUTO || variant > FLINT_LAYER_MMA) return fail(FLINT_ERR_INVALID_ARG, "layer_variant %d", variant);
   const bool use_gemv = (path == FLINT_PATH_GEMV) ||
                         (path == FLINT_PATH_AUTO && T < kMaxGemvTokens && s.wd == FLINT_W_NVFP4);
   if (use_gemv) {
@@ -895,13 +960,23 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
   if (!use_gemv) return run_mma_path(p, s, lay, static_cast<uint8_t*>(workspace), weights, ev, pdl, st);
   const bool split = options && options->split_kernels;
   if (T <= kFusedMaxTokens && !split) {
-    const size_t smem = configure_fused(p, s, T);
+    bool tc = variant == FLINT_LAYER_MMA || (variant == FLINT_LAYER_AUTO && T >= kTcMinTokens);
+    size_t smem = configure_fused(p, s, T, tc);
+    if (smem == 0 && tc && variant == FLINT_LAYER_AUTO) {
+      tc = false;
+      smem = configure_fused(p, s, T, false);
+    }
+    FusedMaps maps;
+    if (smem > 0 && tc) {
+      const int rc = fused_maps(&maps, s, weights);
+      if (rc != FLINT_OK) return rc;
+    }
     if (smem > 0) {
       if (ev) {
         cudaError_t e = cudaEventRecord(ev[0], st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
       }
-      cudaError_t e = launch_fused(p, smem, st);
+      cudaError_t e = launch_fused(p, tc ? &maps : nullptr, smem, st);
       if (e != cudaSuccess) return cuda_fail(e, "k_layer launch");
       if (ev) {
         e = cudaEventRecord(ev[1], st);

@@ -59,6 +59,7 @@ struct LayerParams {
   int down_rb;               // rows per down work item
   int h_in_smem;             // down kernel stages every h row in shared memory
   int ns_gateup, ns_down;    // ring depths (stages per warp)
+  int tc_lt;                 // tensor-core variant of the layer kernel: K-part sum slots per CTA
   int stage_gateup, stage_down;  // stage bytes
 };
 

@@ -90,14 +90,14 @@ class GpuLayer:
 
     # ------------------------------------------------------------- GPU side
     def forward(self, x: torch.Tensor, wr: torch.Tensor, residual=None, path=fm.FLINT_PATH_AUTO, pdl=True,
-                out=None, input_norm=False, split=False):
+                out=None, input_norm=False, split=False, variant=fm.FLINT_LAYER_AUTO):
         T = x.shape[0]
         out = torch.empty_like(x) if out is None else out
         ids = torch.empty((T, self.w.k), dtype=torch.int32, device="cuda")
         gates = torch.empty((T, self.w.k), dtype=torch.float32, device="cuda")
         opt = fm.Options(path=path, use_pdl=1 if pdl else 0, topk_ids=ids.data_ptr(),
                          topk_weights=gates.data_ptr(), input_rmsnorm=1 if input_norm else 0,
-                         split_kernels=1 if split else 0)
+                         split_kernels=1 if split else 0, layer_variant=variant)
         fm.flint_moe_forward_ex(x, T, wr, self.weights, self.shape, residual, out, self.ws, opt)
         return out, ids, gates
 

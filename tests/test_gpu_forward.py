@@ -25,10 +25,11 @@ def _layer(name, seed=0, **kw):
     return _LAYERS[key]
 
 
-def _run_and_check(layer, x_bits, wr_bits, residual_bits=None, path=fm.FLINT_PATH_AUTO, what="", split=False):
+def _run_and_check(layer, x_bits, wr_bits, residual_bits=None, path=fm.FLINT_PATH_AUTO, what="", split=False,
+                   variant=fm.FLINT_LAYER_AUTO):
     x, wr = bits_to_cuda(x_bits), bits_to_cuda(wr_bits)
     res = bits_to_cuda(residual_bits) if residual_bits is not None else None
-    out, ids, gates = layer.forward(x, wr, residual=res, path=path, split=split)
+    out, ids, gates = layer.forward(x, wr, residual=res, path=path, split=split, variant=variant)
     torch.cuda.synchronize()
     ids_np, gates_np = ids.cpu().numpy(), gates.cpu().numpy()
     near = check_routing(ids_np, gates_np, oracle.router_logits(x_bits, wr_bits), layer.w.k)
@@ -75,6 +76,30 @@ def test_forward_split_kernel_path(name, T):
     a, ids_a, _, _ = _run_and_check(layer, x, wr, what=f"{name} fused")
     b, ids_b, _, _ = _run_and_check(layer, x, wr, what=f"{name} split", split=True)
     assert np.array_equal(ids_a, ids_b)
+
+
+@pytest.mark.parametrize("variant", [fm.FLINT_LAYER_FMA, fm.FLINT_LAYER_MMA])
+@pytest.mark.parametrize("T", [1, 2, 5, 8])
+def test_forward_single_kernel_variants(T, variant):
+    # the persistent kernel's two inner-loop variants (CUDA-core dot products,
+    # register-fragment tensor-core MMA) at batch 1..8, including batches
+    # whose experts serve one token (7 of the 8 MMA columns unused)
+    w = synth.CONFIGS["cfg1"]
+    layer = _layer("cfg1", max_tokens=32)
+    x = synth.x_bits(60 + T, T, w.d)
+    _run_and_check(layer, x, synth.make_router(w, 60 + T, x), what=f"T={T} variant {variant}", variant=variant)
+
+
+def test_forward_single_kernel_variants_agree():
+    w = synth.CONFIGS["cfg2"]
+    layer = _layer("cfg1", max_tokens=32)
+    x = synth.x_bits(70, w.T, w.d)
+    wr = synth.make_router(w, 70, x)
+    a, ids_a, _, _ = _run_and_check(layer, x, wr, what="fma", variant=fm.FLINT_LAYER_FMA)
+    b, ids_b, _, _ = _run_and_check(layer, x, wr, what="mma", variant=fm.FLINT_LAYER_MMA)
+    assert np.array_equal(ids_a, ids_b)
+    da, db = synth.bf16_bits_to_f64(cuda_to_bits(a)), synth.bf16_bits_to_f64(cuda_to_bits(b))
+    assert np.linalg.norm(da - db) <= 5e-3 * np.linalg.norm(db)
 
 
 @pytest.mark.parametrize("T", [2, 3, 5, 9, 13, 31])
@@ -124,15 +149,16 @@ def test_forward_deterministic_and_pdl_invariant():
     assert torch.equal(a.view(torch.int16), c.view(torch.int16))
 
 
+@pytest.mark.parametrize("variant", [fm.FLINT_LAYER_FMA, fm.FLINT_LAYER_MMA])
 @pytest.mark.parametrize("d,inter,E,k,S,T", [(512, 128, 1, 1, 0, 3), (512, 128, 8, 8, 1, 5),
                                              (1024, 256, 64, 4, 1, 6), (4096, 1024, 12, 2, 1, 3),
                                              (2048, 128, 40, 6, 0, 4), (1024, 1024, 16, 3, 1, 2)])
-def test_forward_shape_variants(d, inter, E, k, S, T):
+def test_forward_shape_variants(d, inter, E, k, S, T, variant):
     w = synth.Workload("var", d=d, inter=inter, E=E, k=k, S=S, T=T)
     layer = GpuLayer(w, seed=d + inter + E, max_tokens=T)
     x = synth.x_bits(E, T, d)
     wr = synth.to_bf16_bits(np.random.default_rng(E).standard_normal((E, d)) * 0.02)
-    _run_and_check(layer, x, wr, what=f"shape {d},{inter},{E},{k},{S}")
+    _run_and_check(layer, x, wr, what=f"shape {d},{inter},{E},{k},{S} variant {variant}", variant=variant)
 
 
 @pytest.mark.parametrize("T", [1, 4])
