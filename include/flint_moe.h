@@ -174,12 +174,16 @@ int flint_pack_bf16(const uint16_t* w, const flint_moe_shape* shape, uint16_t* p
 
 /* Workspace bytes for calls of up to max_tokens tokens. The workspace holds the
  * status word, router logits, routing, grouping and the FFN intermediates; it
- * must not be shared by calls that may overlap on the GPU. */
+ * must not be shared by calls that may overlap on the GPU. Calls of any token
+ * count up to max_tokens may alternate on one workspace; a workspace serves
+ * one shape (after a shape change, flint_moe_workspace_init it again). */
 size_t flint_moe_workspace_bytes(const flint_moe_shape* shape, int32_t max_tokens);
 
 /* Zeroes the whole workspace (ws_bytes bytes): the control block at its head
  * (status word, router arrival counter, the single-kernel path's launch
- * generation and grid-barrier counters) and the tagged router logits. Call
+ * generation and grid-barrier counters) and the single-kernel path's tagged
+ * router logits and SwiGLU values, which follow it at offsets that depend on
+ * the shape only. Call
  * once after allocating a workspace, before its first use. Kernels only ever
  * set bits in the status word, and flint_moe_get_status reads and clears it. */
 int flint_moe_workspace_init(void* workspace, size_t ws_bytes, void* stream);

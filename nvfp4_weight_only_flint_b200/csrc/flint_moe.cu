@@ -255,14 +255,19 @@ WsLayout ws_layout(const Dims& s, int maxT, bool mma) {
   w.status = 0;
   w.counter = 4;
   o += kCtrlBytes;
+  // the persistent kernel's tagged regions sit at offsets that do not depend
+  // on the call's token count, so they only ever hold zeros or tagged words
+  // of earlier launches on this workspace (older tags)
+  w.tlogits = o;
+  o += al256(sizeof(unsigned long long) * kLogitReplicas * static_cast<size_t>(kFusedMaxTokens) * s.E);
+  w.htag = o;
+  o += al256(sizeof(unsigned long long) * static_cast<size_t>(kFusedMaxTokens) * (s.k + s.S) * s.I);
   w.amax = o;
   o += al256(sizeof(float) * (s.E + s.S) * 3);
   w.desc = o;
   o += al256(sizeof(RouteDesc));
   w.logits = o;
   o += al256(sizeof(float) * static_cast<size_t>(maxT) * s.E);
-  w.tlogits = o;
-  o += al256(sizeof(unsigned long long) * kLogitReplicas * static_cast<size_t>(maxT) * s.E);
   w.ids = o;
   o += al256(sizeof(int) * static_cast<size_t>(maxT) * s.k);
   w.gates = o;
@@ -270,8 +275,6 @@ WsLayout ws_layout(const Dims& s, int maxT, bool mma) {
   w.h = o;
   const size_t P = static_cast<size_t>(maxT) * (s.k + s.S);
   o += al256(sizeof(float) * P * s.I);
-  w.htag = o;
-  o += al256(sizeof(unsigned long long) * std::min<size_t>(P, static_cast<size_t>(kFusedMaxTokens) * (s.k + s.S)) * s.I);
   if (!mma) {
     w.mma_n = w.mma_act = w.mma_off = w.mma_pair = w.xinv = w.hinv = w.xrows = w.hrows = w.y = 0;
     w.total = o;

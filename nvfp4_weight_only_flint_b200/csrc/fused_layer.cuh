@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p, co
     ss = warp_sum(ss);
     const float irms = p.input_norm ? 1.f / sqrtf(ss / static_cast<float>(D) + kRmsEps) : 1.f;
     if (lane < kLogitReplicas)
-      st_tagged(p.tlogits + (static_cast<size_t>(lane) * T + t) * E + r_begin + r, tag, sum * irms);
+      st_tagged(p.tlogits + (static_cast<size_t>(t) * kLogitReplicas + lane) * E + r_begin + r, tag, sum * irms);
   }
   // statistics of token t on warp kFusedWarps-1-t (idle during the router at
   // one token)
@@ -412,7 +412,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) k_layer(LayerParams p, co
     if (warp < T) {
       bool okt = false;
       if (ok) {
-        const unsigned long long* lg = p.tlogits + (static_cast<size_t>(c % kLogitReplicas) * T + warp) * E;
+        const unsigned long long* lg = p.tlogits + (static_cast<size_t>(warp) * kLogitReplicas + c % kLogitReplicas) * E;
         if (E <= 256)
           okt = topk_warp_tagged<8>(lg, E, k, tag, &s_ids[warp * k], &s_gates[warp * k], lane, p.status);
         else

@@ -43,11 +43,11 @@ struct LayerParams {
                              // words 32*(i+1), i < 4: its grid-barrier arrival counters
   RouteDesc* desc;           // routing descriptor (workspace)
   float* logits;             // [T][E]
-  unsigned long long* tlogits;  // [replicas][T][E] tagged logits of the persistent kernel
+  unsigned long long* tlogits;  // [8 tokens][replicas][E] tagged logits of the persistent kernel
   int* ids;                  // [T][k]
   float* gates;              // [T][k]
   float* h;                  // [T*(k+S)][I] fp32 SwiGLU intermediates
-  unsigned long long* htag;  // [T*(k+S)][I] tagged h of the persistent kernel
+  unsigned long long* htag;  // [8*(k+S)][I] tagged h of the persistent kernel
   int* ids_out;              // optional public copy
   float* gates_out;          // optional public copy
   long long cpe;             // code bytes per expert (3*I*d/2)

@@ -102,6 +102,36 @@ def test_forward_single_kernel_variants_agree():
     assert np.linalg.norm(da - db) <= 5e-3 * np.linalg.norm(db)
 
 
+def test_forward_mixed_batches_one_workspace():
+    # batch sizes change from call to call on one workspace: the persistent
+    # kernel's tagged logits and h sit at offsets that do not move with T
+    w = synth.CONFIGS["cfg1"]
+    layer = _layer("cfg1", max_tokens=32)
+    for i, T in enumerate([1, 8, 3, 8, 1, 6, 2, 8]):
+        x = synth.x_bits(90 + i, T, w.d)
+        _run_and_check(layer, x, synth.make_router(w, 90 + i, x), what=f"call {i}, T={T}")
+
+
+def test_forward_batch8_after_many_batch1():
+    # the SwiGLU values travel between CTAs under a launch tag: a batch-8 call
+    # after 4095 batch-1 calls (whose launches leave rows 7.. of the tagged h
+    # untouched) must see only its own values
+    w1, w8 = synth.CONFIGS["cfg1"], synth.CONFIGS["cfg2"]
+    layer = _layer("cfg1", max_tokens=32)
+    x = synth.x_bits(95, 8, w8.d)
+    _run_and_check(layer, x, synth.make_router(w8, 95, x), what="batch 8, first")
+    x1 = bits_to_cuda(synth.x_bits(96, 1, w1.d))
+    wr1 = bits_to_cuda(synth.make_router(w1, 96, synth.x_bits(96, 1, w1.d)))
+    out1 = torch.empty_like(x1)
+    opt = fm.Options(path=fm.FLINT_PATH_AUTO, use_pdl=1)
+    for _ in range(4095):
+        fm.flint_moe_forward_ex(x1, 1, wr1, layer.weights, layer.shape, None, out1, layer.ws, opt)
+    torch.cuda.synchronize()
+    assert fm.flint_moe_get_status(layer.ws) == (0, 0)
+    x = synth.x_bits(97, 8, w8.d)
+    _run_and_check(layer, x, synth.make_router(w8, 97, x), what="batch 8, 4096 launches later")
+
+
 @pytest.mark.parametrize("T", [2, 3, 5, 9, 13, 31])
 def test_forward_ragged_tokens(T):
     w = synth.CONFIGS["cfg1"]
