@@ -62,10 +62,10 @@ def _tensor_peak(wdtype: str):
 
 
 # DRAM bytes (read + write) of one k_layer launch at batch 1, from an ncu
-# capture of `bench.py --profile t1` (dram__bytes_read.sum 13,565,440 B,
+# capture of `bench.py --profile t1` (dram__bytes_read.sum 13,561,088 B,
 # dram__bytes_write.sum 0 B); set to None whenever the kernel changes until it
 # is captured again.
-TRAFFIC_K_LAYER_T1 = 13565440
+TRAFFIC_K_LAYER_T1 = 13561088
 
 
 def _host_cores():
