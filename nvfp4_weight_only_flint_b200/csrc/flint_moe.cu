@@ -436,6 +436,8 @@ size_t down_smem(const LayerParams& p) {
 // everything after the routing descriptor. Returns the dynamic shared-memory
 // bytes, or 0 if the call does not fit.
 size_t configure_fused_tc(LayerParams& p, const Dims& s, int T, int sms) {
+  // the kernel's balanced tile split gives each CTA at most one shared-expert tile
+  if (s.S * (s.I / kTcUnits) > sms) return 0;
   const size_t a128 = 127;
   auto al = [&](size_t v) { return (v + a128) & ~a128; };
   const int rps = 32 / (s.I / 32);
