@@ -11,9 +11,11 @@
 //                   -> the bf16 rows as they are
 //   k_mma_ffn<GATEUP>  persistent: work item (active expert, 64 units = 128
 //                   interleaved gate/up rows). Weights reach shared memory by
-//                   TMA; NVFP4 codes and scales are dequantised there to f16
-//                   (e2m1 * e4m3 is exact in f16) in the 128-byte-swizzled
-//                   K-major operand layout; tcgen05.mma (kind::f16, M=128,
+//                   TMA; NVFP4 codes and scales are dequantised to f16 (e2m1 *
+//                   e4m3 is exact in f16) straight into tensor memory
+//                   (tcgen05.st), where the MMA reads its A operand; bf16
+//                   weight tiles are the A operand in shared memory (128-byte
+//                   swizzled K-major layout); tcgen05.mma (kind::f16, M=128,
 //                   N = the expert's tokens rounded up to 16, fp32 accumulators
 //                   in tensor memory, double-buffered) and an epilogue warpgroup
 //                   that applies the tensor scales, 1/sigma_t and SiLU*mul and
@@ -331,38 +333,6 @@ struct MmaMaps {
   CUtensorMap scales;
   CUtensorMap brows;
 };
-
-// Dequantise one 64-element slice of K of the 128-row A tile (256 threads):
-// thread (row r, half h) turns 32 codes and their 2 scales into 32 f16 values
-// written to the swizzled operand (16-byte chunk c of row r at c ^ (r % 8)).
-__device__ __forceinline__ void dequant_slice(const uint8_t* raw, int sub, uint8_t* a16, int dt) {
-  const int w = dt >> 5, l = dt & 31;
-  const int half = (l >> 3) & 1;
-  const int r = 16 * w + 8 * (l >> 4) + (l & 7);
-  const int chunk = 2 * sub + half;  // 16-byte code chunk of the 128-byte raw row
-  const uint4 cv = lds128(raw + r * 128 + ((chunk ^ (r & 7)) << 4));
-  const uint32_t s2 = *reinterpret_cast<const uint16_t*>(raw + 128 * 128 + r * 16 + 4 * sub + 2 * half);
-  uint32_t sh;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(sh) : "h"(static_cast<uint16_t>(s2)));
-  const __half2 hs = *reinterpret_cast<const __half2*>(&sh);
-  const __half2 sc[2] = {__low2half2(hs), __high2half2(hs)};
-  const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
-  uint8_t* row = a16 + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {  // 8 elements per q; words 0,1 -> block 0, words 2,3 -> block 1
-    uint32_t f[4];
-    e2m1x8_to_f16x2(cw[q], *reinterpret_cast<uint32_t(*)[4]>(&f[0]));
-    uint4 o;
-    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&f[j]), sc[q >> 1]);
-      ow[j] = *reinterpret_cast<const uint32_t*>(&v);
-    }
-    const int c8 = 4 * half + q;  // 16-byte chunk of the 128-byte f16 row
-    *reinterpret_cast<uint4*>(row + ((c8 ^ (r & 7)) << 4)) = o;
-  }
-}
 
 // Dequantise one 64-element slice of K of the 128-row A tile straight into
 // tensor memory (NVFP4 weights): dequantiser warp w (8..15) owns the lanes of
