@@ -377,13 +377,21 @@ def _barrier():
 
 
 def _max_over_ranks(v: float) -> float:
+    """The largest v over the ranks (a device time: the job is as slow as its
+    slowest rank). NCCL reduces a device tensor, gloo a host one."""
     if not _DIST["on"]:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: float, world: int, steps: int, max_ms: float) -> float:
+    """Units all ranks processed per second, over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (max_ms / 1e3)
 
 
 def main():
@@ -430,7 +438,7 @@ def main():
     ms, clocks = run_chain(stack, routers1, 1, args.steps, args.warmup, sampler=sampler, norm=1)
     ms = _max_over_ranks(ms)
     K = args.steps
-    tok_s = world * 1 * K / (ms / 1e3)
+    tok_s = whole_job_rate(1, world, K, ms)
     ms_step = ms / K
 
     # per-kernel timing of the dominant kernel and byte counts
