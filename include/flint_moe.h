@@ -181,7 +181,7 @@ size_t flint_moe_workspace_bytes(const flint_moe_shape* shape, int32_t max_token
 
 /* Zeroes the whole workspace (ws_bytes bytes): the control block at its head
  * (status word, router arrival counter, the single-kernel path's launch
- * generation and grid-barrier counters) and the single-kernel path's tagged
+ * generation) and the single-kernel path's tagged
  * router logits and SwiGLU values, which follow it at offsets that depend on
  * the shape only. Call
  * once after allocating a workspace, before its first use. Kernels only ever

@@ -243,10 +243,10 @@ constexpr size_t kCtrlBytes = 1024;
 
 // Workspace carve-up for calls of up to maxT tokens. The first kCtrlBytes hold
 // the control block: the status word (byte 0), the router's arrival counter
-// (byte 4, left at zero by every call), the persistent layer kernel's launch
-// generation (byte 8) and its four grid-barrier counters (bytes 132, 260, 388,
-// 516; one 128-byte line each). The tagged logits start with a tag of 0, which
-// no launch uses. flint_moe_workspace_init zeroes the whole workspace.
+// (byte 4, left at zero by every call) and the persistent layer kernel's
+// launch generation (byte 8); the rest is reserved. The tagged regions start
+// with a tag of 0, which no launch uses. flint_moe_workspace_init zeroes the
+// whole workspace.
 // Regions of the tensor-core path are laid out only when `mma` (the call takes
 // that path; flint_moe_workspace_bytes reports the size with them).
 WsLayout ws_layout(const Dims& s, int maxT, bool mma) {

@@ -39,8 +39,7 @@ struct LayerParams {
   uint16_t* out;             // [T][d] bf16
   int* status;               // workspace status word
   unsigned* counter;         // control block word 1: router arrival counter (self-resetting);
-                             // word 2: launch generation of the persistent kernel;
-                             // words 32*(i+1), i < 4: its grid-barrier arrival counters
+                             // word 2: launch generation of the persistent kernel
   RouteDesc* desc;           // routing descriptor (workspace)
   float* logits;             // [T][E]
   unsigned long long* tlogits;  // [8 tokens][replicas][E] tagged logits of the persistent kernel
