@@ -583,8 +583,8 @@ def run_reference(args, world):
     import oracle
     w = synth.CONFIGS["cfg1"]
     cores = _host_cores()
-    K = min(args.steps, 12)
-    W = min(args.warmup, 1)
+    K = min(args.steps, 12)             # a bounded sample: ~0.1 s of fp64 work per step
+    W = max(3, min(args.warmup, 5))     # at least 3 warm-up steps, as for the GPU arm
     prepared = []
     for i in range(K + W):
         x = synth.x_bits(args.seed + 50 + i, 1, w.d)
