@@ -209,14 +209,18 @@ int flint_moe_forward(const uint16_t* x, int32_t T, const uint16_t* router_w,
 
 /* As flint_moe_forward, with options (path choice, PDL, routing outputs).
  * options == NULL behaves as flint_moe_forward.
- * The tensor-core path (FLINT_PATH_MMA, or AUTO from 32 tokens) multiplies on
- * tcgen05 (kind::f16, fp32 accumulators in tensor memory): NVFP4 weights are
- * dequantised in shared memory to f16, exactly (an e2m1 code times an e4m3
- * scale has at most 6 significant bits), against x scaled per token by a power
- * of two into f16; bf16 weights multiply bf16 x directly. SwiGLU intermediates
- * are kept in fp32 and fed to the down projection as f16 (NVFP4, power-of-two
- * row scale) or bf16 (bf16 weights). Its profile events bracket the gate/up
- * kernel. */
+ * Arithmetic: every NVFP4 path forms the exact f16 value of an e2m1 code times
+ * its e4m3 block scale (at most 6 significant bits) and multiplies it with x
+ * scaled per token by a power of two into f16 (h likewise per row), products
+ * exact, accumulating in fp32; outputs bf16, round to nearest even. The
+ * single-kernel path (batch <= 8) does so with CUDA-core fma.rn.f32.f16 or
+ * register-fragment mma.sync (layer_variant). The tensor-core path
+ * (FLINT_PATH_MMA, or AUTO from 32 tokens) multiplies on tcgen05 (kind::f16,
+ * fp32 accumulators in tensor memory): NVFP4 weights are dequantised to f16
+ * straight into tensor memory; bf16 weights multiply bf16 x directly. SwiGLU
+ * intermediates are kept in fp32 and fed to the down projection as f16 (NVFP4,
+ * power-of-two row scale) or bf16 (bf16 weights). Its profile events bracket
+ * the gate/up kernel. */
 int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
                          const flint_moe_weights* weights, const flint_moe_shape* shape,
                          const uint16_t* residual, uint16_t* out, void* workspace,
