@@ -54,6 +54,14 @@ def test_sizes(L):
     assert fm.flint_packed_bytes(sb) == 257 * 3 * 512 * 2048 * 2
     assert fm.flint_block_scale_bytes(sb) == 0
     assert fm.flint_moe_workspace_bytes(s, 8) > fm.flint_moe_workspace_bytes(s, 1) > 0
+    # the single-kernel path's tagged regions are sized for its largest batch
+    # whatever max_tokens is: 8 tokens x 8 replicas x E tagged logits and
+    # 8 x (k+S) x inter tagged SwiGLU values, 8 bytes each, after the 1 KiB
+    # control block
+    tagged = 8 * 8 * 256 * 8 + 8 * (6 + 1) * 512 * 8
+    assert fm.flint_moe_workspace_bytes(s, 1) >= 1024 + tagged
+    sizes = [fm.flint_moe_workspace_bytes(s, t) for t in (1, 2, 8, 32, 128)]
+    assert sizes == sorted(sizes)
 
 
 @pytest.mark.parametrize("bad", [dict(d=1000), dict(d=8192), dict(inter=96), dict(E=0), dict(E=513),
