@@ -172,3 +172,99 @@ def test_input_norm_router_sees_normalised_x():
     xf = synth.bf16_bits_to_f64(x)
     rms = np.sqrt(np.mean(xf ** 2, axis=1, keepdims=True) + 1e-6)
     np.testing.assert_allclose(r["logits"], (xf / rms) @ synth.bf16_bits_to_f64(wr).T, rtol=1e-12)
+
+
+# ---------------------------------------------------------------- bf16 weights
+def _np_bf16(bits):
+    """bf16 bit patterns -> fp64 by widening the pattern to an fp32 one (numpy
+    only, independent of the oracle's decoder)."""
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _bf16_experts(n, d, inter, seed=0, layer=0):
+    out = []
+    for e in range(n):
+        g, u, dn = synth.expert_weights_np(seed, layer, e, d, inter)
+        out.append(tuple(oracle.BF16Matrix(synth.to_bf16_bits(m), m.shape[0], m.shape[1]) for m in (g, u, dn)))
+    return out
+
+
+def _np_dense_swiglu_bf16(trip, x):
+    g, u, dn = (_np_bf16(m.bits) for m in trip)
+    a, b = g @ x, u @ x
+    return dn @ (a / (1.0 + np.exp(-a)) * b)
+
+
+def test_bf16_decode_is_exact_widening():
+    # +0, -0, smallest subnormal, a subnormal, 1, -1.5, largest finite, 2^-126,
+    # 3.140625 (0x4049), -65280 (0xC77F)
+    bits = np.array([[0x0000, 0x8000, 0x0001, 0x0050, 0x3F80],
+                     [0xBFC0, 0x7F7F, 0x0080, 0x4049, 0xC77F]], np.uint16)
+    got = oracle.decode(oracle.BF16Matrix(bits, 2, 5))
+    want = np.array([[0.0, -0.0, 2.0 ** -133, 80 * 2.0 ** -133, 1.0],
+                     [-1.5, (2 - 2 ** -7) * 2.0 ** 127, 2.0 ** -126, 3.140625, -65280.0]])
+    assert np.array_equal(got, want)
+    assert np.signbit(got[0, 1])
+    # random patterns of finite values: the decode is the fp32 widening
+    rng = np.random.default_rng(3)
+    r = rng.integers(0, 1 << 16, size=(16, 32), dtype=np.uint32).astype(np.uint16)
+    r[(r & 0x7F80) == 0x7F80] = 0x3F80  # no inf/NaN patterns
+    assert np.array_equal(oracle.decode(oracle.BF16Matrix(r, 16, 32)), _np_bf16(r))
+
+
+def test_bf16_single_expert_layer_equals_dense_ffn():
+    d, inter = 64, 32
+    ex = _bf16_experts(1, d, inter, seed=12)
+    x = synth.x_bits(12, 3, d)
+    wr = synth.to_bf16_bits(np.random.default_rng(12).standard_normal((1, d)) * 0.02)
+    r = oracle.moe_forward(x, wr, ex, d=d, inter=inter, E=1, k=1, S=0)
+    xf = _np_bf16(x)
+    for t in range(3):
+        np.testing.assert_allclose(r["out"][t], _np_dense_swiglu_bf16(ex[0], xf[t]), rtol=1e-12, atol=1e-14)
+
+
+def test_bf16_layer_is_renormalised_mixture_plus_shared():
+    d, inter, E, k = 64, 32, 6, 2
+    ex = _bf16_experts(E + 1, d, inter, seed=13)
+    x = synth.x_bits(13, 2, d)
+    wr = synth.to_bf16_bits(np.random.default_rng(13).standard_normal((E, d)) * 0.3)
+    r = oracle.moe_forward(x, wr, ex, d=d, inter=inter, E=E, k=k, S=1)
+    xf, wrf = _np_bf16(x), _np_bf16(wr)
+    for t in range(2):
+        l = wrf @ xf[t]
+        sel = sorted(range(E), key=lambda e: (-l[e], e))[:k]
+        p = np.exp(l[sel] - l.max())
+        p /= p.sum()
+        want = sum(p[j] * _np_dense_swiglu_bf16(ex[e], xf[t]) for j, e in enumerate(sel))
+        want = want + _np_dense_swiglu_bf16(ex[E], xf[t])
+        assert r["ids"][t].tolist() == sel
+        np.testing.assert_allclose(r["out"][t], want, rtol=1e-11, atol=1e-13)
+
+
+def test_packed_layout_bf16_offsets():
+    # d=32, I=32, two experts, every element a distinct pattern: unit u of
+    # expert e = [gate row u | up row u] at element e*3*I*d + u*2d; down row n
+    # at e*3*I*d + 2*I*d + n*I
+    d, inter = 32, 32
+    ex = []
+    for e in range(2):
+        trip = []
+        for m in range(3):
+            rows, cols = (inter, d) if m < 2 else (d, inter)
+            bits = ((np.arange(rows * cols, dtype=np.int64) * 3 + 4096 * m + 12288 * e) % 65536).astype(np.uint16)
+            trip.append(oracle.BF16Matrix(bits.reshape(rows, cols), rows, cols))
+        ex.append(tuple(trip))
+    out = oracle.pack_layout_bf16(ex, d, inter)
+    per = 3 * inter * d
+    assert out.size == 2 * per
+    for e in range(2):
+        g, u, dn = ex[e]
+        for i in (0, 5, 31):
+            for j in (0, 7, 31):
+                assert out[e * per + i * 2 * d + j] == g.bits[i, j]
+                assert out[e * per + i * 2 * d + d + j] == u.bits[i, j]
+        for n in (0, 9, 31):
+            for j in (0, 16, 31):
+                assert out[e * per + 2 * inter * d + n * inter + j] == dn.bits[n, j]
+    # every element placed exactly once
+    assert np.array_equal(np.sort(out), np.sort(np.concatenate([m.bits.ravel() for t in ex for m in t])))
