@@ -118,9 +118,17 @@ typedef enum flint_path {
 } flint_path;
 
 typedef enum flint_layer_variant {
-  FLINT_LAYER_AUTO = 0, /* tensor-core inner loops from 2 tokens, CUDA-core at 1 */
-  FLINT_LAYER_FMA = 1,  /* CUDA-core dot products (fma.rn.f32.f16) */
-  FLINT_LAYER_MMA = 2   /* register-fragment mma.sync m16n8k16 */
+  FLINT_LAYER_AUTO = 0,   /* one token: the cluster kernel when the shape fits it;
+                             2..8 tokens: the persistent kernel's tensor-core loops */
+  FLINT_LAYER_FMA = 1,    /* persistent kernel, CUDA-core dot products (fma.rn.f32.f16) */
+  FLINT_LAYER_MMA = 2,    /* persistent kernel, register-fragment mma.sync m16n8k16 */
+  FLINT_LAYER_CLUSTER = 3 /* one token only: one 16-CTA cluster per selected expert and
+                             one for the shared expert; routing, the SwiGLU exchange
+                             and the down rows stay inside a cluster (distributed
+                             shared memory), and the last CTA to finish a block of
+                             output rows sums the experts' gated partials in slot
+                             order. FLINT_ERR_UNSUPPORTED_SHAPE if the shape does
+                             not fit it on the device */
 } flint_layer_variant;
 
 typedef struct flint_moe_options {
@@ -239,11 +247,16 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
  *  Arguments as for flint_moe_forward. A call whose scratch would exceed 1 MiB
  *  (flint_moe_workspace_bytes(shape, T) > 1048576) returns FLINT_ERR_WORKSPACE
  *  with a message, before any launch.
- *  The first call on each device looks up the array's device address
- *  (cudaGetSymbolAddress, with that device current) and caches it; make that
- *  first call before any stream capture. Each call first zeroes the part of
- *  the array it uses (an asynchronous memset on `stream`), so device check
- *  flags are not kept between calls.
+ *  The first call in each CUDA context (each device's primary context, or any
+ *  other context the caller made current) looks up the array's device address
+ *  in that context (cudaGetSymbolAddress) and caches it by the context's id;
+ *  make that first call before any stream capture.
+ *  The array keeps its contents between calls. Calls of one shape rely on the
+ *  launch tags of the single-kernel path, so nothing is cleared; when the
+ *  shape differs from the previous call's in that context, the call first
+ *  zeroes the array (an asynchronous memset on `stream`) except its status
+ *  word. Device check flags accumulate in that status word until
+ *  flint_moe_noalloc_get_status reads and clears them.
  *  All calls share the one array:
  *  calls that may run at the same time on the GPU (different streams, or
  *  different host threads) race on it and corrupt each other's results;
@@ -251,6 +264,18 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
 int flint_moe_forward_noalloc(const uint16_t* x, int32_t T, const uint16_t* router_w,
                               const flint_moe_weights* weights, const flint_moe_shape* shape,
                               const uint16_t* residual, uint16_t* out, void* stream);
+
+/* flint_moe_noalloc_get_status -- flint_moe_get_status for the built-in
+ * scratch of flint_moe_forward_noalloc in the current context: synchronises
+ * `stream`, reads the status word into *device_flags (may be NULL) and clears
+ * it. Returns FLINT_OK, or FLINT_ERR_TIMEOUT / FLINT_ERR_DEVICE_CHECK when a
+ * flag was set. (No counterpart in the pages.) */
+int flint_moe_noalloc_get_status(int32_t* device_flags, void* stream);
+
+/* Debug helper: the device address of the built-in scratch in the current
+ * context (looked up as flint_moe_forward_noalloc does), e.g. to pass it to
+ * flint_debug_wait_timeout. */
+int flint_debug_noalloc_scratch(void** addr);
 
 /* Synchronises `stream`, reads the workspace status word into *device_flags
  * (FLINT_DEVCHECK_* bits, may be NULL) and clears it. Returns FLINT_OK, or

@@ -19,13 +19,14 @@ __all__ = [
     "FLINT_W_NVFP4", "FLINT_W_BF16", "FLINT_PATH_AUTO", "FLINT_PATH_GEMV", "FLINT_PATH_MMA",
     "flint_packed_bytes", "flint_block_scale_bytes", "flint_tensor_scale_bytes",
     "flint_moe_workspace_bytes", "flint_moe_workspace_init", "flint_pack_nvfp4", "flint_pack_bf16", "flint_moe_route",
-    "flint_moe_forward", "flint_moe_forward_ex", "flint_moe_forward_noalloc", "flint_moe_get_status", "flint_last_error",
+    "flint_moe_forward", "flint_moe_forward_ex", "flint_moe_forward_noalloc", "flint_moe_noalloc_get_status",
+    "flint_moe_get_status", "flint_last_error", "flint_debug_noalloc_scratch",
     "flint_debug_dequant", "flint_debug_wait_timeout", "flint_version",
 ]
 
 FLINT_W_NVFP4, FLINT_W_BF16 = 0, 1
 FLINT_PATH_AUTO, FLINT_PATH_GEMV, FLINT_PATH_MMA = 0, 1, 2
-FLINT_LAYER_AUTO, FLINT_LAYER_FMA, FLINT_LAYER_MMA = 0, 1, 2
+FLINT_LAYER_AUTO, FLINT_LAYER_FMA, FLINT_LAYER_MMA, FLINT_LAYER_CLUSTER = 0, 1, 2, 3
 STATUS_NAMES = {0: "FLINT_OK", -1: "FLINT_ERR_INVALID_ARG", -2: "FLINT_ERR_UNSUPPORTED_SHAPE",
                 -3: "FLINT_ERR_MISALIGNED", -4: "FLINT_ERR_WORKSPACE", -5: "FLINT_ERR_CUDA",
                 -6: "FLINT_ERR_DEVICE_CHECK", -7: "FLINT_ERR_TIMEOUT"}
@@ -87,6 +88,10 @@ def lib() -> ctypes.CDLL:
         L.flint_moe_forward_ex.restype = i32
         L.flint_moe_forward_noalloc.argtypes = [vp, i32, vp, P(Weights), P(Shape), vp, vp, vp]
         L.flint_moe_forward_noalloc.restype = i32
+        L.flint_moe_noalloc_get_status.argtypes = [P(i32), vp]
+        L.flint_moe_noalloc_get_status.restype = i32
+        L.flint_debug_noalloc_scratch.argtypes = [P(vp)]
+        L.flint_debug_noalloc_scratch.restype = i32
         L.flint_moe_workspace_init.argtypes = [vp, sz, vp]
         L.flint_moe_workspace_init.restype = i32
         L.flint_moe_get_status.argtypes = [vp, P(i32), vp]
@@ -199,6 +204,21 @@ def flint_moe_forward_noalloc(x, T: int, router_w, weights: Weights, shape: Shap
     _check(lib().flint_moe_forward_noalloc(_ptr(x), int(T), _ptr(router_w), ctypes.byref(weights),
                                            ctypes.byref(shape), _ptr(residual), _ptr(out),
                                            _stream(stream)))
+
+
+def flint_moe_noalloc_get_status(stream=None) -> tuple[int, int]:
+    """Status of the built-in scratch of flint_moe_forward_noalloc: (status,
+    device_flags) without raising."""
+    flags = ctypes.c_int32(0)
+    rc = lib().flint_moe_noalloc_get_status(ctypes.byref(flags), _stream(stream))
+    return rc, flags.value
+
+
+def flint_debug_noalloc_scratch() -> int:
+    """Device address of the built-in scratch in the current context."""
+    addr = ctypes.c_void_p(0)
+    _check(lib().flint_debug_noalloc_scratch(ctypes.byref(addr)))
+    return addr.value
 
 
 def flint_moe_get_status(workspace, stream=None) -> tuple[int, int]:

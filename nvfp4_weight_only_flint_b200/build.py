@@ -10,9 +10,11 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 SO = os.path.join(PKG, "libflint_moe.so")
-SOURCES = ["flint_moe.cu"]
-NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
-              "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]
+OBJ_DIR = os.path.join(PKG, "_build")
+# translation units, compiled in parallel and linked into one shared library
+SOURCES = ["flint_moe.cu", "tok1.cu"]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+NVCC_FLAGS = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
 
 
 def _inputs():
@@ -27,11 +29,28 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if all(os.path.getmtime(f) <= so_time for f in _inputs()):
             return SO
     nvcc = os.environ.get("NVCC", "nvcc")
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    objs, procs = [], []
+    for src in SOURCES:
+        obj = os.path.join(OBJ_DIR, os.path.splitext(src)[0] + f".{os.getpid()}.o")
+        cmd = [nvcc, *NVCC_FLAGS, f"-I{INCLUDE}", "-c", os.path.join(CSRC, src), "-o", obj]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        objs.append(obj)
+        procs.append(subprocess.Popen(cmd))
+    failed = [p.wait() for p in procs]
+    if any(failed):
+        for o in objs:
+            if os.path.exists(o):
+                os.unlink(o)
+        raise subprocess.CalledProcessError(max(failed), "nvcc")
     tmp = SO + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, f"-I{INCLUDE}", *[os.path.join(CSRC, s) for s in SOURCES], "-o", tmp]
+    cmd = [nvcc, *ARCH, "-shared", *objs, "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
+    for o in objs:
+        os.unlink(o)
     os.replace(tmp, SO)
     return SO
 

@@ -13,6 +13,7 @@
 
 #include "fused_layer.cuh"
 #include "mma_path.cuh"
+#include "tok1.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -233,7 +234,7 @@ int check_shape(const flint_moe_shape* s, Dims* out) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct WsLayout {
-  size_t status, counter, amax, desc, logits, tlogits, ids, gates, h, htag;
+  size_t status, counter, rb_count, amax, desc, logits, tlogits, ids, gates, h, htag, tok1_part;
   size_t mma_n, mma_act, mma_off, mma_pair, xinv, hinv, xrows, hrows, y;  // tensor-core path
   size_t total;
 };
@@ -243,8 +244,9 @@ constexpr size_t kCtrlBytes = 1024;
 
 // Workspace carve-up for calls of up to maxT tokens. The first kCtrlBytes hold
 // the control block: the status word (byte 0), the router's arrival counter
-// (byte 4, left at zero by every call) and the persistent layer kernel's
-// launch generation (byte 8); the rest is reserved. The tagged regions start
+// (byte 4, left at zero by every call), the persistent layer kernel's launch
+// generation (byte 8) and the batch-1 cluster kernel's per-row-block arrival
+// counters (bytes 64..127, left at zero by every call); the rest is reserved. The tagged regions start
 // with a tag of 0, which no launch uses. flint_moe_workspace_init zeroes the
 // whole workspace.
 // Regions of the tensor-core path are laid out only when `mma` (the call takes
@@ -254,6 +256,7 @@ WsLayout ws_layout(const Dims& s, int maxT, bool mma) {
   size_t o = 0;
   w.status = 0;
   w.counter = 4;
+  w.rb_count = 64;
   o += kCtrlBytes;
   // the persistent kernel's tagged regions sit at offsets that do not depend
   // on the call's token count, so they only ever hold zeros or tagged words
@@ -262,6 +265,8 @@ WsLayout ws_layout(const Dims& s, int maxT, bool mma) {
   o += al256(sizeof(unsigned long long) * kLogitReplicas * static_cast<size_t>(kFusedMaxTokens) * s.E);
   w.htag = o;
   o += al256(sizeof(unsigned long long) * static_cast<size_t>(kFusedMaxTokens) * (s.k + s.S) * s.I);
+  w.tok1_part = o;  // the batch-1 cluster kernel's gated partial outputs [k+S][d]
+  o += al256(sizeof(float) * static_cast<size_t>(s.k + s.S) * s.d);
   w.amax = o;
   o += al256(sizeof(float) * (s.E + s.S) * 3);
   w.desc = o;
@@ -926,7 +931,10 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
   if (options && ((options->topk_ids == nullptr) != (options->topk_weights == nullptr)))
     return fail(FLINT_ERR_INVALID_ARG, "topk_ids and topk_weights go together");
   const int variant = options ? options->layer_variant : FLINT_LAYER_AUTO;
-  if (variant < FLINT_LAYER_AUTO || variant > FLINT_LAYER_MMA) return fail(FLINT_ERR_INVALID_ARG, "layer_variant %d", variant);
+  if (variant < FLINT_LAYER_AUTO || variant > FLINT_LAYER_CLUSTER)
+    return fail(FLINT_ERR_INVALID_ARG, "layer_variant %d", variant);
+  if (variant == FLINT_LAYER_CLUSTER && (T != 1 || path == FLINT_PATH_MMA || s.wd != FLINT_W_NVFP4))
+    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "the cluster kernel takes one token and NVFP4 weights (T=%d)", T);
   const bool use_gemv = (path == FLINT_PATH_GEMV) ||
                         (path == FLINT_PATH_AUTO && T < kMaxGemvTokens && s.wd == FLINT_W_NVFP4);
   if (use_gemv) {
@@ -964,6 +972,48 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
   cudaEvent_t* ev = options ? static_cast<cudaEvent_t*>(options->profile_events) : nullptr;
   if (!use_gemv) return run_mma_path(p, s, lay, static_cast<uint8_t*>(workspace), weights, ev, pdl, st);
   const bool split = options && options->split_kernels;
+  if (T == 1 && !split && (variant == FLINT_LAYER_AUTO || variant == FLINT_LAYER_CLUSTER)) {
+    // one token: one cluster of CTAs per selected expert and one for the shared
+    // expert (tok1.cuh), when the shape fits it on this device
+    Tok1Params t{};
+    t.x = x;
+    t.wr = router_w;
+    t.codes = p.codes;
+    t.scales = p.scales;
+    t.tscale = p.tscale;
+    t.residual = residual;
+    t.out = out;
+    t.status = p.status;
+    t.rb_count = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + lay.rb_count);
+    t.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + lay.tok1_part);
+    t.ids = p.ids;
+    t.gates = p.gates;
+    t.ids_out = p.ids_out;
+    t.gates_out = p.gates_out;
+    t.cpe = p.cpe;
+    t.spe = p.spe;
+    t.E = s.E;
+    t.k = s.k;
+    t.S = s.S;
+    t.input_norm = p.input_norm;
+    t.trigger_early = 1;
+    if (tok1_dispatch(s.d, s.I, s.E, false, &t, pdl, st, nullptr)) {
+      if (ev) {
+        cudaError_t e = cudaEventRecord(ev[0], st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+      }
+      cudaError_t e = cudaSuccess;
+      tok1_dispatch(s.d, s.I, s.E, true, &t, pdl && !ev, st, &e);
+      if (e != cudaSuccess) return cuda_fail(e, "k_tok1 launch");
+      if (ev) {
+        e = cudaEventRecord(ev[1], st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+      }
+      return FLINT_OK;
+    }
+    if (variant == FLINT_LAYER_CLUSTER)
+      return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "the cluster kernel does not fit this shape on this device");
+  }
   if (T <= kFusedMaxTokens && !split) {
     bool tc = variant == FLINT_LAYER_MMA || (variant == FLINT_LAYER_AUTO && T >= kTcMinTokens);
     size_t smem = configure_fused(p, s, T, tc);
@@ -1094,8 +1144,88 @@ namespace flint {
 namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB, held by every device that loads the library
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// The scratch's device address per CUDA context, keyed by the context's
+// unique id (cuCtxGetId never repeats an id within a process, so a context
+// created after cudaDeviceReset, or another driver context of the same
+// device, gets its own entry and its own lookup), with the shape of the last
+// call that ran on it.
+struct NoAllocSlot {
+  unsigned long long ctx_id;
+  void* addr;
+  bool have_shape;
+  Dims last;
+};
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[64] = {nullptr};
+NoAllocSlot g_noalloc_slots[64];
+int g_noalloc_n = 0;
+
+typedef CUresult (*PFN_ctx_get_current)(CUcontext*);
+typedef CUresult (*PFN_ctx_get_id)(CUcontext, unsigned long long*);
+
+int current_context_id(unsigned long long* id) {
+  static PFN_ctx_get_current get_current = nullptr;
+  static PFN_ctx_get_id get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_ctx_get_current>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_ctx_get_id>(f);
+  });
+  if (get_current == nullptr || get_id == nullptr)
+    return fail(FLINT_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId are not available");
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return fail(FLINT_ERR_CUDA, "cuCtxGetCurrent failed");
+  if (ctx == nullptr) {
+    // nothing current yet: bind the current device's primary context, as the
+    // runtime's first call on this thread would
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaSetDevice(dev);
+    if (e != cudaSuccess) return cuda_fail(e, "context set-up");
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return fail(FLINT_ERR_CUDA, "no current CUDA context");
+  }
+  if (get_id(ctx, id) != CUDA_SUCCESS) return fail(FLINT_ERR_CUDA, "cuCtxGetId failed");
+  return FLINT_OK;
+}
+
+// The slot of the current context, created (with the symbol lookup, done with
+// that context current) on first use. Called with g_noalloc_mu held.
+int noalloc_slot(NoAllocSlot** out) {
+  unsigned long long id = 0;
+  int rc = current_context_id(&id);
+  if (rc != FLINT_OK) return rc;
+  for (int i = 0; i < g_noalloc_n; ++i)
+    if (g_noalloc_slots[i].ctx_id == id) {
+      *out = &g_noalloc_slots[i];
+      return FLINT_OK;
+    }
+  // Host code cannot use the array's name as a device address: look the
+  // address up in this context.
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+  const bool evict = g_noalloc_n >= 64;
+  NoAllocSlot* s = &g_noalloc_slots[evict ? (id % 64) : g_noalloc_n++];
+  s->ctx_id = id;
+  s->addr = p;
+  // a context seen for the first time has a freshly loaded (zero) array; one
+  // whose slot was evicted earlier may not, so its next call zeroes it
+  s->have_shape = evict;
+  s->last = Dims{0, 0, 0, 0, 0, 0};
+  *out = s;
+  return FLINT_OK;
+}
+
+bool same_dims(const Dims& a, const Dims& b) {
+  return a.d == b.d && a.I == b.I && a.E == b.E && a.k == b.k && a.S == b.S && a.wd == b.wd;
+}
 }  // namespace
 }  // namespace flint
 
@@ -1117,30 +1247,51 @@ int flint_moe_forward_noalloc(const uint16_t* x, int32_t T, const uint16_t* rout
                 "flint_moe_forward_noalloc: this call needs %zu bytes of scratch; the built-in scratch holds %zu "
                 "(use flint_moe_forward with a caller workspace)",
                 need, kNoAllocScratchBytes);
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) return fail(FLINT_ERR_INVALID_ARG, "device ordinal %d out of range", dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (g_noalloc_addr[dev] == nullptr) {
-      // Host code cannot use the array's name as a device address: look the
-      // address up once per device, with that device current.
-      void* p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
-      g_noalloc_addr[dev] = p;
+    NoAllocSlot* slot = nullptr;
+    rc = noalloc_slot(&slot);
+    if (rc != FLINT_OK) return rc;
+    scratch = slot->addr;
+    // The persistent kernel's launch tags need the control block's generation
+    // word and the tagged regions (at offsets that depend on the shape) to
+    // hold only older tags. The array is zero when the module loads; after a
+    // shape change, everything but the status word (byte 0, kept for
+    // flint_moe_noalloc_get_status) is zeroed again. Calls of one shape keep
+    // the contents: the tags of later launches are newer.
+    if (slot->have_shape && !same_dims(slot->last, s)) {
+      cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(scratch) + 4, 0, kNoAllocScratchBytes - 4, st);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     }
-    scratch = g_noalloc_addr[dev];
+    slot->last = s;
+    slot->have_shape = true;
   }
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // Every call starts from a zeroed scratch (the control block and the tagged
-  // logits must; the rest is rewritten before it is read).
-  e = cudaMemsetAsync(scratch, 0, need, st);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   return flint_moe_forward_ex(x, T, router_w, weights, shape, residual, out, scratch, kNoAllocScratchBytes,
                               nullptr, stream);
+}
+
+int flint_moe_noalloc_get_status(int32_t* device_flags, void* stream) {
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    NoAllocSlot* slot = nullptr;
+    const int rc = noalloc_slot(&slot);
+    if (rc != FLINT_OK) return rc;
+    scratch = slot->addr;
+  }
+  return flint_moe_get_status(scratch, device_flags, stream);
+}
+
+int flint_debug_noalloc_scratch(void** addr) {
+  if (!addr) return fail(FLINT_ERR_INVALID_ARG, "addr is NULL");
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  NoAllocSlot* slot = nullptr;
+  const int rc = noalloc_slot(&slot);
+  if (rc != FLINT_OK) return rc;
+  *addr = slot->addr;
+  return FLINT_OK;
 }
 
 int flint_debug_wait_timeout(void* workspace, int64_t cycles, void* stream) {

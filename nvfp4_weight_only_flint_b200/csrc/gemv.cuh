@@ -267,7 +267,7 @@ struct Grouping {
   unsigned emask[kMaxExperts];  // scratch: per-expert token bitmask
 };
 
-__device__ void build_grouping(Grouping& g, const int* ids, int T, int k, int E, int S, int* status) {
+inline __device__ void build_grouping(Grouping& g, const int* ids, int T, int k, int E, int S, int* status) {
   const int tid = threadIdx.x;
   for (int e = tid; e < E; e += blockDim.x) {
     g.ecount[e] = 0;
@@ -351,7 +351,7 @@ __device__ void build_grouping(Grouping& g, const int* ids, int T, int k, int E,
 // Warp-synchronous token grouping for T*k <= 64 pairs: a bitonic sort of the
 // keys (expert << 16 | token << 8 | slot), two per lane, then run boundaries
 // by ballot. Writes the same descriptor fields as build_grouping.
-__device__ void warp_grouping(const int* ids, int T, int k, int E, int S, RouteDesc* d, int lane,
+inline __device__ void warp_grouping(const int* ids, int T, int k, int E, int S, RouteDesc* d, int lane,
                               int* status) {
   const int n = T * k;
   uint32_t key[2];

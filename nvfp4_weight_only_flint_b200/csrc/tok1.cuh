@@ -1,0 +1,385 @@
+// tok1.cuh -- the layer at decode batch 1 as one cluster-per-expert kernel.
+//
+// The grid is (k + S) clusters of kTok1Cluster CTAs. Cluster j < k serves
+// the expert the token routes to in top-k slot j; cluster k (when S = 1)
+// serves the shared expert. Inside a cluster every exchange goes through
+// distributed shared memory, so the only step that crosses clusters is the
+// final gated sum, done by whichever CTA arrives last at a per-row-block
+// counter (no CTA ever waits on another cluster):
+//   P0  (before the dependency wait of programmatic dependent launch) bulk
+//       copies of this CTA's slice of the router rows (routed clusters), or of
+//       its slice of the shared expert (shared cluster): routing-independent
+//   P1  the token's statistics, x staged as f16 in registers; this CTA's
+//       router logits, written into every CTA of the cluster (DSMEM)
+//   P2  cluster barrier; each CTA selects the top-k from its full copy of the
+//       logits and issues one burst of bulk copies: its I/CS gate/up units and
+//       its d/CS down rows of the cluster's expert
+//   P3  gate/up + SwiGLU of its units as their copies land; each h value is
+//       written into every CTA of the cluster (DSMEM); cluster barrier
+//   P4  down rows of its block against the whole h, times the slot's gate:
+//       fp32 partial sums of rows [rank*d/CS, (rank+1)*d/CS) of this slot
+//   P5  the CTA that arrives last at its row block's counter adds the k + S
+//       partials in slot order (+ residual), rounds to bf16 and resets it.
+// The cluster barriers are hardware barriers that every CTA of a cluster
+// reaches on every path; every mbarrier wait is bounded (FLINT_DEVCHECK_WAIT)
+// and a CTA whose wait gave up still takes every later barrier and counter
+// step, drains its copies and reports through the status word.
+#pragma once
+
+#include "gemv.cuh"
+
+namespace flint {
+
+constexpr int kTok1Cluster = 16;   // CTAs per cluster (non-portable size)
+constexpr int kTok1Warps = 16;
+constexpr int kTok1MaxChunks = 16;  // gate/up copy chunks (one per warp at most)
+
+struct Tok1Params {
+  const uint16_t* x;         // [1][d] bf16
+  const uint16_t* wr;        // [E][d] bf16
+  const uint8_t* codes;      // packed E2M1 codes
+  const uint8_t* scales;     // packed E4M3 block scales
+  const float* tscale;       // [E+S][3]
+  const uint16_t* residual;  // [1][d] bf16 or null
+  uint16_t* out;             // [1][d] bf16
+  int* status;               // workspace status word
+  unsigned* rb_count;        // [kTok1Cluster] arrival counters per row block (workspace, zero between launches)
+  float* partial;            // [k+S][d] gated fp32 partial outputs per slot (workspace)
+  int* ids;                  // [k] routed ids (workspace)
+  float* gates;              // [k]
+  int* ids_out;              // optional public copies
+  float* gates_out;
+  long long cpe, spe;        // code / scale bytes per expert
+  int E, k, S;
+  int input_norm;
+  int trigger_early;         // 1: allow the next kernel to launch at once
+};
+
+// Dynamic shared-memory bytes of k_tok1: the larger of the router-row slice and
+// the expert slice (they share the region), then the cluster's logits and h.
+__host__ __device__ constexpr size_t tok1_region_bytes(int D, int I, int E) {
+  const size_t rows = static_cast<size_t>((E + kTok1Cluster - 1) / kTok1Cluster) * D * 2;
+  const size_t ex = static_cast<size_t>(I / kTok1Cluster) * (D + D / 8) +
+                    static_cast<size_t>(D / kTok1Cluster) * (I / 2 + I / 16);
+  return ((rows > ex ? rows : ex) + 127) & ~static_cast<size_t>(127);
+}
+__host__ __device__ constexpr size_t tok1_smem_bytes(int D, int I, int E) {
+  return tok1_region_bytes(D, I, E) + ((static_cast<size_t>(E) * 4 + 127) & ~static_cast<size_t>(127)) +
+         static_cast<size_t>(I) * 4;
+}
+
+__device__ __forceinline__ unsigned cluster_rank() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ unsigned cluster_index() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Store v into the same shared-memory variable of CTA `rank` of this cluster.
+__device__ __forceinline__ void st_cluster_f32(float* local, unsigned rank, float v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
+
+template <int D, int I>
+__global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
+  constexpr int CS = kTok1Cluster;
+  constexpr int VPR = D / 32;                     // 16-byte code vectors per gate/up row
+  constexpr int XV = VPR >= 32 ? VPR / 32 : 1;    // x vectors (32 elements) per lane
+  constexpr int UV = 2 * VPR / 32 > 0 ? 2 * VPR / 32 : 1;  // code vectors per lane per unit
+  constexpr int UPC = I / CS;                     // gate/up units per CTA
+  constexpr int CU = UPC >= kTok1Warps ? UPC / kTok1Warps : 1;  // units per chunk
+  constexpr int NCH = UPC / CU;                   // chunks (<= 16)
+  constexpr int RPC = D / CS;                     // down rows per CTA
+  constexpr int LPR = I / 32;                     // lanes per down row (one 16-byte vector each)
+  constexpr int RPS = 32 / LPR;                   // down rows per warp step
+  constexpr int UNIT_C = D, UNIT_S = D / 8;       // bytes of a unit's codes / scales
+  constexpr int DROW_C = I / 2, DROW_S = I / 16;  // bytes of a down row's codes / scales
+  static_assert(NCH <= kTok1MaxChunks && NCH * CU == UPC, "chunking");
+  static_assert(RPC % RPS == 0 || RPC < RPS, "down rows");
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t s_bar[kTok1MaxChunks + 2];  // chunks, down rows, router rows
+  __shared__ int s_ids[kMaxTopK];
+  __shared__ float s_gates[kMaxTopK];
+  __shared__ int s_fail, s_last, s_burst;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int E = p.E, k = p.k, KS = k + p.S;
+  const unsigned rank = cluster_rank();
+  const int slot = static_cast<int>(cluster_index());  // top-k slot served, or k = shared
+  const bool shared = slot >= k;
+  uint8_t* region = smem;
+  float* s_logits = reinterpret_cast<float*>(smem + tok1_region_bytes(D, I, E));
+  float* s_h = s_logits + ((E + 31) & ~31);
+  uint8_t* gu_codes = region;                                   // [UPC][D]
+  uint8_t* gu_scales = region + UPC * UNIT_C;                   // [UPC][D/8]
+  uint8_t* dn_codes = gu_scales + UPC * UNIT_S;                 // [RPC][I/2]
+  uint8_t* dn_scales = dn_codes + RPC * DROW_C;                 // [RPC][I/16]
+  uint64_t* bar_chunk = s_bar;
+  uint64_t* bar_down = s_bar + kTok1MaxChunks;
+  uint64_t* bar_rows = s_bar + kTok1MaxChunks + 1;
+  const int r0 = static_cast<int>(rank) * E / CS, r1 = (static_cast<int>(rank) + 1) * E / CS;
+
+  // issue this CTA's slice of expert e (one lane per chunk, one for the down rows)
+  auto issue_expert = [&](int e) {
+    const uint8_t* cb = p.codes + static_cast<long long>(e) * p.cpe;
+    const uint8_t* sb = p.scales + static_cast<long long>(e) * p.spe;
+    const int u0 = static_cast<int>(rank) * UPC;
+    if (lane < NCH) {
+      const int u = u0 + lane * CU;
+      mbar_arrive_expect_tx(&bar_chunk[lane], CU * (UNIT_C + UNIT_S));
+      bulk_g2s(gu_codes + lane * CU * UNIT_C, cb + static_cast<long long>(u) * UNIT_C, CU * UNIT_C, &bar_chunk[lane]);
+      bulk_g2s(gu_scales + lane * CU * UNIT_S, sb + static_cast<long long>(u) * UNIT_S, CU * UNIT_S, &bar_chunk[lane]);
+    } else if (lane == NCH) {
+      const long long n0 = static_cast<long long>(rank) * RPC;
+      mbar_arrive_expect_tx(bar_down, RPC * (DROW_C + DROW_S));
+      bulk_g2s(dn_codes, cb + static_cast<long long>(I) * D + n0 * DROW_C, RPC * DROW_C, bar_down);
+      bulk_g2s(dn_scales, sb + static_cast<long long>(I) * D / 8 + n0 * DROW_S, RPC * DROW_S, bar_down);
+    }
+  };
+
+  // ---- P0: routing-independent copies, before the dependency wait
+  if (tid == 0) {
+    for (int i = 0; i < kTok1MaxChunks + 2; ++i) mbar_init(&s_bar[i], 1);
+    fence_barrier_init();
+    s_fail = 0;
+    s_burst = shared ? 1 : 0;
+    if (!shared) {
+      const uint32_t rbytes = static_cast<uint32_t>(r1 - r0) * D * 2;
+      mbar_arrive_expect_tx(bar_rows, rbytes);
+      if (rbytes) bulk_g2s(region, p.wr + static_cast<size_t>(r0) * D, rbytes, bar_rows);
+    }
+  }
+  __syncthreads();
+  if (shared && warp == 0) issue_expert(E);
+  // every CTA of the cluster must be running before any writes into its
+  // shared memory: arrive now, wait just before the first remote store
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  if (p.trigger_early) pdl_trigger();
+  pdl_wait();  // x (and the workspace) are written by the preceding kernel
+
+  // ---- P1: x -> statistics, f16 registers (lane's vectors v = lane + 32 j, j < XV
+  // of a gate/up row; at D = 512 lanes 16..31 repeat lanes 0..15)
+  bool ok = true;
+  const int xl = lane % VPR;  // first x vector of this lane
+  uint32_t xr[XV][16];        // bf16 pairs, then f16 pairs scaled by sigma
+  float amax = 0.f, ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < XV; ++j) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.x) + (xl + 32 * j) * 4;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = __ldcg(src + q);
+      xr[j][4 * q + 0] = v.x;
+      xr[j][4 * q + 1] = v.y;
+      xr[j][4 * q + 2] = v.z;
+      xr[j][4 * q + 3] = v.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float a = bf16_bits_to_f32(xr[j][i] & 0xFFFFu), b = __uint_as_float(xr[j][i] & 0xFFFF0000u);
+      amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+      ss = fmaf(a, a, ss);
+      ss = fmaf(b, b, ss);
+    }
+  }
+  if (lane >= VPR) ss = 0.f;  // repeated lanes count once
+  amax = segment_max<32>(amax);
+  ss = warp_sum(ss);
+  const float irms = p.input_norm ? 1.f / sqrtf(ss / static_cast<float>(D) + kRmsEps) : 1.f;
+  const float sigma = pow2_scale_for(amax);
+  const float fx = irms / sigma;  // dot(q, x*sigma) * fx = dot(q, x) * irms
+
+  // router rows of this CTA: warp w takes rows r0 + w, r0 + w + 16, ...; the
+  // lane covers the same elements as its x registers
+  // (warp-uniform outcomes: the reductions below need every lane)
+  if (!shared && r1 > r0 && !__all_sync(0xffffffffu, mbar_wait(bar_rows, 0, p.status))) ok = false;
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  if (!shared) {
+    for (int r = r0 + warp; r < r1 && ok; r += kTok1Warps) {
+      const uint8_t* row = region + static_cast<size_t>(r - r0) * D * 2;
+      float a = 0.f;
+      if (lane < VPR) {
+#pragma unroll
+        for (int j = 0; j < XV; ++j) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 wv = lds128(row + (xl + 32 * j) * 64 + 16 * q);
+            const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t xx = xr[j][4 * q + i];
+              a = fmaf(bf16_bits_to_f32(ww[i] & 0xFFFFu), bf16_bits_to_f32(xx & 0xFFFFu), a);
+              a = fmaf(__uint_as_float(ww[i] & 0xFFFF0000u), __uint_as_float(xx & 0xFFFF0000u), a);
+            }
+          }
+        }
+      }
+      const float logit = warp_sum(a) * irms;
+      if (lane < CS) st_cluster_f32(s_logits + r, static_cast<unsigned>(lane), logit);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < XV; ++j)
+#pragma unroll
+    for (int i = 0; i < 16; ++i) xr[j][i] = bf16x2_to_f16x2_scaled(xr[j][i], sigma);
+  if (!ok && lane == 0) s_fail = 1;
+
+  // ---- P2: every CTA of the cluster holds all E logits; select, then issue
+  cluster_sync_all();
+  if (s_fail) ok = false;
+  if (!shared && warp == 0 && ok) {
+    if (E <= 256) {
+      uint32_t code[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        code[i] = (e < E) ? max(route_code(s_logits[e]), 1u) : 0u;
+      }
+      topk_select<8>(code, k, s_ids, s_gates, lane);
+    } else {
+      uint32_t code[kMaxExperts / 32];
+#pragma unroll
+      for (int i = 0; i < kMaxExperts / 32; ++i) {
+        const int e = lane + 32 * i;
+        code[i] = (e < E) ? max(route_code(s_logits[e]), 1u) : 0u;
+      }
+      topk_select<kMaxExperts / 32>(code, k, s_ids, s_gates, lane);
+    }
+    __syncwarp();
+    // the router rows were read before the cluster barrier; order those
+    // generic reads before the copies that overwrite them
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    const int e = s_ids[slot];
+    if (e < 0 || e >= E) {
+      if (lane == 0) atomicOr(p.status, FLINT_DEVCHECK_EXPERT_ID);
+    } else {
+      issue_expert(e);
+      if (lane == 0) s_burst = 1;
+    }
+    if (slot == 0 && rank == 0 && lane < k) {
+      p.ids[lane] = s_ids[lane];
+      p.gates[lane] = s_gates[lane];
+      if (p.ids_out != nullptr) {
+        p.ids_out[lane] = s_ids[lane];
+        p.gates_out[lane] = s_gates[lane];
+      }
+    }
+  }
+  __syncthreads();
+  const bool issued = s_burst != 0;  // this CTA's slice of an expert is on its way
+  const int expert = shared ? E : (issued ? s_ids[slot] : 0);
+  const float gate = shared ? 1.f : s_gates[slot];
+  float sg = 0.f, su = 0.f, sd = 0.f;
+  if (issued) {
+    sg = __ldg(p.tscale + 3 * expert + 0);
+    su = __ldg(p.tscale + 3 * expert + 1);
+    sd = __ldg(p.tscale + 3 * expert + 2);
+  }
+
+  // ---- P3: gate/up of chunk `warp` (CU units), h into every CTA of the cluster
+  bool ok3 = issued;
+  if (warp < NCH && issued) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar_chunk[warp], 0, p.status))) ok3 = false;
+    if (ok3) {
+#pragma unroll 1
+      for (int c = 0; c < CU; ++c) {
+        const int ul = warp * CU + c;
+        const uint8_t* uc = gu_codes + ul * UNIT_C;
+        const uint8_t* us = gu_scales + ul * UNIT_S;
+        float g = 0.f, u = 0.f;
+#pragma unroll
+        for (int j = 0; j < UV; ++j) {
+          const int v = lane + 32 * j;  // vector of the unit (gate row: v < VPR)
+          const uint4 cv = lds128(uc + 16 * v);
+          const uint32_t s2 = *reinterpret_cast<const uint16_t*>(us + 2 * v);
+          float acc = 0.f;
+          dot32_strided<1, 16>(cv, s2, xr[VPR >= 32 ? j % XV : 0], &acc);
+          if (v < VPR) g += acc;
+          else u += acc;
+        }
+        g = warp_sum(g);
+        u = warp_sum(u);
+        const float hv = swiglu(g * fx * sg, u * fx * su);
+        if (lane < CS) st_cluster_f32(s_h + static_cast<int>(rank) * UPC + ul, static_cast<unsigned>(lane), hv);
+      }
+    }
+  }
+  if (!ok3 && issued && lane == 0) s_fail = 1;
+  cluster_sync_all();
+  if (s_fail) ok = false;
+  ok = ok && issued;
+
+  // ---- P4: down rows of this CTA's block against the whole h
+  float* part = p.partial + static_cast<size_t>(slot) * D + static_cast<size_t>(rank) * RPC;
+  if (ok && !__all_sync(0xffffffffu, mbar_wait(bar_down, 0, p.status))) ok = false;
+  if (ok) {
+    // h slice of this lane (elements 32 * (lane % LPR) ..), scaled by a power
+    // of two into f16; every warp derives the same scale from the whole h
+    float hm = 0.f;
+    for (int i = lane; i < I; i += 32) hm = fmaxf(hm, fabsf(s_h[i]));
+    hm = segment_max<32>(hm);
+    const float hs = pow2_scale_for(hm);
+    const int hv0 = (lane % LPR) * 32;
+    uint32_t hr[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) hr[i] = pack_f16x2(s_h[hv0 + 2 * i] * hs, s_h[hv0 + 2 * i + 1] * hs);
+    const float ys = sd * gate / hs;
+    for (int r = warp * RPS + lane / LPR; r < RPC; r += kTok1Warps * RPS) {
+      const uint4 cv = lds128(dn_codes + r * DROW_C + 16 * (lane % LPR));
+      const uint32_t s2 = *reinterpret_cast<const uint16_t*>(dn_scales + r * DROW_S + 2 * (lane % LPR));
+      float acc = 0.f;
+      dot32_strided<1, 16>(cv, s2, hr, &acc);
+      acc = segment_sum<LPR>(acc);
+      if (lane % LPR == 0) __stcg(part + r, acc * ys);
+    }
+  } else {
+    for (int r = tid; r < RPC; r += blockDim.x) __stcg(part + r, 0.f);
+  }
+
+  // ---- P5: the last of the k + S CTAs of this row block sums the slots
+  __threadfence();  // this thread's partial stores before the CTA's arrival
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned old = atomicAdd(p.rb_count + rank, 1u);
+    const int last = old == static_cast<unsigned>(KS - 1);
+    if (last) atomicExch(p.rb_count + rank, 0u);  // no other CTA of this launch touches it again
+    s_last = last;
+  }
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    for (int r = tid; r < RPC; r += blockDim.x) {
+      const int n = static_cast<int>(rank) * RPC + r;
+      float y = 0.f;
+      for (int j = 0; j < KS; ++j) y += __ldcg(p.partial + static_cast<size_t>(j) * D + n);
+      if (p.residual != nullptr) y += bf16_bits_to_f32(__ldcg(p.residual + n));
+      const __nv_bfloat16 b = __float2bfloat16_rn(y);
+      p.out[n] = *reinterpret_cast<const uint16_t*>(&b);
+    }
+  }
+  if (!p.trigger_early) pdl_trigger();
+  // copies still in flight after a failed wait land before the CTA exits
+  if (!ok && !shared && r1 > r0 && tid == 0) mbar_wait(bar_rows, 0, p.status);
+  if (!ok && issued) {
+    for (int c = tid; c < NCH; c += blockDim.x) mbar_wait(&bar_chunk[c], 0, p.status);
+    if (tid == 0) mbar_wait(bar_down, 0, p.status);
+  }
+}
+
+// Host side (tok1.cu): whether the cluster kernel serves (d, inter, E) on the
+// current device (its shared memory fits, a 16-CTA cluster can be resident);
+// with `launch`, also launches it for `t` on `st` and stores the launch status
+// in *err.
+bool tok1_dispatch(int d, int I, int E, bool launch, const Tok1Params* t, bool pdl, cudaStream_t st,
+                   cudaError_t* err);
+
+}  // namespace flint

@@ -103,10 +103,15 @@ def test_host_validation_errors(L):
     assert L.flint_moe_forward_ex(0x40000, 4, 0x40000, ctypes.byref(w), ctypes.byref(s), None, 0x50000,
                                   0x60000, ws_need, ctypes.byref(opt), None) == -1
     # bad layer variant option
-    opt = fm.Options(path=0, use_pdl=1, layer_variant=3)
+    opt = fm.Options(path=0, use_pdl=1, layer_variant=4)
     assert L.flint_moe_forward_ex(0x40000, 4, 0x40000, ctypes.byref(w), ctypes.byref(s), None, 0x50000,
                                   0x60000, ws_need, ctypes.byref(opt), None) == -1
     assert "layer_variant" in fm.flint_last_error()
+    # the cluster kernel takes one token only (refused before any launch)
+    opt = fm.Options(path=0, use_pdl=1, layer_variant=fm.FLINT_LAYER_CLUSTER)
+    assert L.flint_moe_forward_ex(0x40000, 4, 0x40000, ctypes.byref(w), ctypes.byref(s), None, 0x50000,
+                                  0x60000, ws_need, ctypes.byref(opt), None) == -2
+    assert "cluster" in fm.flint_last_error()
     # NVFP4 weights without scales
     w2 = fm.Weights(0x10000, None, None)
     assert L.flint_moe_forward(0x40000, 4, 0x40000, ctypes.byref(w2), ctypes.byref(s), None, 0x50000,
