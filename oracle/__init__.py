@@ -69,6 +69,8 @@ def lib():
         L.oracle_bf16_to_double.restype = f64
         L.oracle_quantize_nvfp4.argtypes = [vp, i32, i32, vp, vp, vp]
         L.oracle_quantize_nvfp4.restype = i32
+        L.oracle_quantize_nvfp4_rows.argtypes = [vp, i32, i32, f32, vp, vp, vp]
+        L.oracle_quantize_nvfp4_rows.restype = i32
         L.oracle_decode_matrix.argtypes = [ctypes.POINTER(OracleMatrix), vp]
         L.oracle_decode_matrix.restype = i32
         L.oracle_pack_layout.argtypes = [ctypes.POINTER(OracleMatrix), i32, i32, i32, vp, vp, vp]
@@ -85,6 +87,10 @@ def lib():
                                          ctypes.POINTER(OracleMatrix), vp, vp, i32, i32,
                                          vp, vp, vp, vp, vp]
         L.oracle_moe_forward.restype = i32
+        L.oracle_dense_gemv.argtypes = [ctypes.POINTER(OracleMatrix), vp, i32, vp, i32, vp]
+        L.oracle_dense_gemv.restype = i32
+        L.oracle_group.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
+        L.oracle_group.restype = i32
         _lib = L
     return _lib
 
@@ -153,6 +159,20 @@ def quantize(w: np.ndarray) -> NVFP4Matrix:
     rc = lib().oracle_quantize_nvfp4(_ptr(w), rows, cols, _ptr(codes), _ptr(scales), _ptr(ts))
     if rc != 0:
         raise ValueError("oracle_quantize_nvfp4 rejected the input")
+    return NVFP4Matrix(codes, scales, float(ts[0]), rows, cols)
+
+
+def quantize_with_tensor_scale(w: np.ndarray, amax: float) -> NVFP4Matrix:
+    """Rows of a larger tensor whose largest |w| is amax (its tensor scale is
+    amax / 2688), quantised with the same recipe."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    codes = np.zeros((rows, cols // 2), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 16), dtype=np.uint8)
+    ts = np.zeros(1, dtype=np.float32)
+    if lib().oracle_quantize_nvfp4_rows(_ptr(w), rows, cols, float(np.float32(amax)), _ptr(codes), _ptr(scales),
+                                        _ptr(ts)) != 0:
+        raise ValueError("oracle_quantize_nvfp4_rows rejected the input")
     return NVFP4Matrix(codes, scales, float(ts[0]), rows, cols)
 
 
@@ -227,6 +247,34 @@ def topk(logits: np.ndarray, k: int):
     if lib().oracle_topk(_ptr(logits), T, E, k, _ptr(ids), _ptr(gates), _ptr(gap)) != 0:
         raise ValueError("oracle_topk failed")
     return ids, gates, gap
+
+
+def dense_gemv(m: NVFP4Matrix, x_bits: np.ndarray, rows=None) -> np.ndarray:
+    """out [T][len(rows)] = decoded m[rows] . x in fp64 (all rows when None)."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    T = x_bits.shape[0]
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    n = m.rows if r is None else r.size
+    out = np.zeros((T, n), dtype=np.float64)
+    s = _as_struct(m)
+    if lib().oracle_dense_gemv(ctypes.byref(s), _ptr(x_bits), T, _ptr(r), n, _ptr(out)) != 0:
+        raise ValueError("oracle_dense_gemv failed")
+    return out
+
+
+def group(ids: np.ndarray, E: int, S: int):
+    """Grouping by expert of ids [T][k]: (act, off, pair, n_routed), or None
+    when an id lies outside [0, E)."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, k = ids.shape
+    act = np.zeros(E + S, dtype=np.int32)
+    off = np.zeros(E + S + 1, dtype=np.int32)
+    pair = np.zeros(max(1, T * (k + S)), dtype=np.int32)
+    nr = np.zeros(1, dtype=np.int32)
+    n = lib().oracle_group(_ptr(ids), T, k, E, S, _ptr(act), _ptr(off), _ptr(pair), _ptr(nr))
+    if n < 0:
+        return None
+    return act[:n].copy(), off[:n + 1].copy(), pair[:T * (k + S)].copy(), int(nr[0])
 
 
 def expert_ffn(trip, x: np.ndarray) -> np.ndarray:

@@ -140,6 +140,14 @@ int oracle_quantize_nvfp4(const float* w, int32_t rows, int32_t cols, uint8_t* c
     const float a = std::fabs(w[i]);
     if (a > amax) amax = a;
   }
+  return oracle_quantize_nvfp4_rows(w, rows, cols, amax, codes, scales, tensor_scale);
+}
+
+int oracle_quantize_nvfp4_rows(const float* w, int32_t rows, int32_t cols, float amax, uint8_t* codes,
+                               uint8_t* scales, float* tensor_scale) {
+  if (rows <= 0 || cols <= 0 || cols % 16 != 0 || !(amax >= 0.0f) || !std::isfinite(amax)) return -1;
+  for (size_t i = 0; i < static_cast<size_t>(rows) * cols; ++i)
+    if (!std::isfinite(w[i]) || std::fabs(w[i]) > amax) return -1;
   // 2688 = 6 (largest E2M1) * 448 (largest E4M3)
   const float s_t = (amax > 0.0f) ? amax / 2688.0f : 1.0f;
   *tensor_scale = s_t;
@@ -443,6 +451,65 @@ int oracle_moe_forward(int32_t T, int32_t d, int32_t inter, int32_t E, int32_t k
   if (gates_out) std::memcpy(gates_out, gates.data(), gates.size() * sizeof(double));
   if (gap_out) std::memcpy(gap_out, gap.data(), gap.size() * sizeof(double));
   if (logits_out) std::memcpy(logits_out, logits.data(), logits.size() * sizeof(double));
+  return 0;
+}
+
+// Grouping by expert, written from its definition: scan the experts in
+// ascending id order and, for each one some token selected, list its
+// selections token by token; the shared experts follow with every token.
+int32_t oracle_group(const int32_t* ids, int32_t T, int32_t k, int32_t E, int32_t S, int32_t* act,
+                     int32_t* off, int32_t* pair, int32_t* n_routed) {
+  if (T < 0 || T > 256 || k < 1 || E < 1 || S < 0) return -1;
+  for (int i = 0; i < T * k; ++i)
+    if (ids[i] < 0 || ids[i] >= E) return -1;
+  int n = 0, p = 0;
+  for (int e = 0; e < E; ++e) {
+    const int first = p;
+    for (int t = 0; t < T; ++t)
+      for (int j = 0; j < k; ++j)
+        if (ids[t * k + j] == e) pair[p++] = (t << 8) | j;
+    if (p > first) {
+      act[n] = e;
+      off[n] = first;
+      ++n;
+    }
+  }
+  *n_routed = n;
+  for (int s = 0; s < S; ++s) {
+    act[n] = E + s;
+    off[n] = p;
+    ++n;
+    for (int t = 0; t < T; ++t) pair[p++] = (t << 8) | (k + s);
+  }
+  off[n] = p;
+  return n;
+}
+
+// Dense NVFP4 matrix times bf16 vectors: each selected row decoded
+// element by element (as oracle_decode_matrix does) and dotted with x in fp64.
+int oracle_dense_gemv(const oracle_matrix* m, const uint16_t* x, int32_t T, const int32_t* rows,
+                      int32_t n_rows, double* out) {
+  if (!m || !x || !out || m->kind != 0 || !m->codes || !m->scales || m->cols % 16 != 0 || T < 0 || n_rows < 0)
+    return -1;
+  const int cols = m->cols;
+  const double s_t = static_cast<double>(m->tensor_scale);
+  std::vector<double> w(cols), xd(static_cast<size_t>(T) * cols);
+  for (size_t i = 0; i < xd.size(); ++i) xd[i] = bf16_bits_to_double(x[i]);
+  for (int i = 0; i < n_rows; ++i) {
+    const int r = rows ? rows[i] : i;
+    if (r < 0 || r >= m->rows) return -1;
+    for (int c = 0; c < cols; ++c) {
+      const uint8_t byte = m->codes[static_cast<size_t>(r) * (cols / 2) + c / 2];
+      const uint8_t q = (c % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+      const uint8_t sb = m->scales[static_cast<size_t>(r) * (cols / 16) + c / 16];
+      w[c] = oracle_e2m1_decode(q) * oracle_e4m3_decode(sb) * s_t;
+    }
+    for (int t = 0; t < T; ++t) {
+      double acc = 0.0;
+      for (int c = 0; c < cols; ++c) acc += w[c] * xd[static_cast<size_t>(t) * cols + c];
+      out[static_cast<size_t>(t) * n_rows + i] = acc;
+    }
+  }
   return 0;
 }
 

@@ -72,6 +72,12 @@ double oracle_bf16_to_double(uint16_t bits);
 int oracle_quantize_nvfp4(const float* w, int32_t rows, int32_t cols,
                           uint8_t* codes, uint8_t* scales, float* tensor_scale);
 
+/* The same recipe for some rows of a larger tensor whose amax (the largest
+ * |w| over the whole tensor) is given: s_t = amax/2688, then the rows' blocks
+ * as above. Returns -1 if a row value is non-finite or exceeds amax. */
+int oracle_quantize_nvfp4_rows(const float* w, int32_t rows, int32_t cols, float amax,
+                               uint8_t* codes, uint8_t* scales, float* tensor_scale);
+
 /* Decode one matrix to fp64 [rows][cols] (NVFP4: e2m1*e4m3*s_t; BF16: exact). */
 int oracle_decode_matrix(const oracle_matrix* m, double* out);
 
@@ -100,6 +106,26 @@ int oracle_router_logits(const uint16_t* x, int32_t T, const uint16_t* wr,
  * or +inf when k == E. */
 int oracle_topk(const double* logits, int32_t T, int32_t E, int32_t k,
                 int32_t* ids, double* gates, double* gap);
+
+/* Grouping of the routed selections by expert (the layer contract's "expert
+ * histogram + token permutation"): the experts that at least one token
+ * selected, in ascending id order, then the n_shared shared experts E..E+S-1;
+ * for each, its (token, slot) pairs as token << 8 | slot in ascending token
+ * order (a token selects an expert at most once), the shared experts serving
+ * every token in slot k + s; off[a] = index of expert a's first pair, off[n]
+ * = total. ids [T][k]. act holds up to E + S entries, off up to E + S + 1,
+ * pair T*(k+S). Writes *n_routed (routed experts in use) and returns the
+ * number of active experts, or -1 if an id lies outside [0, E) or T > 256. */
+int32_t oracle_group(const int32_t* ids, int32_t T, int32_t k, int32_t E, int32_t S,
+                     int32_t* act, int32_t* off, int32_t* pair, int32_t* n_routed);
+
+/* ---- dense NVFP4 matrix-vector product (the 4-bit output head) ----
+ * out[t][i] = sum_c w[rows[i]][c] * x[t][c] in fp64, w = e2m1 * e4m3 * s_t of
+ * the NVFP4 matrix m (natural layout), x bf16 [T][m->cols]. rows (nullable)
+ * picks n_rows of the matrix's rows (all rows in order when NULL, n_rows =
+ * m->rows). Returns 0, or -1 on a bad argument. */
+int oracle_dense_gemv(const oracle_matrix* m, const uint16_t* x, int32_t T, const int32_t* rows,
+                      int32_t n_rows, double* out);
 
 /* ---- experts ---- */
 /* Dense SwiGLU FFN of one expert: y = W_d (silu(W_g x) * (W_u x)).

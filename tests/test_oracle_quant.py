@@ -112,3 +112,17 @@ def test_rejects_non_finite():
     w[0, 5] = np.inf
     with pytest.raises(ValueError):
         oracle.quantize(w)
+
+
+def test_rows_of_a_larger_tensor_match_the_whole():
+    # quantising a subset of rows with the whole tensor's amax gives exactly
+    # those rows of the whole tensor's quantisation
+    rng = np.random.default_rng(21)
+    w = (rng.standard_normal((50, 64)) * 0.02).astype(np.float32)
+    whole = oracle.quantize(w)
+    rows = [3, 0, 49, 17]
+    part = oracle.quantize_with_tensor_scale(w[rows], float(np.abs(w).max()))
+    assert part.tensor_scale == whole.tensor_scale
+    assert np.array_equal(part.codes, whole.codes[rows]) and np.array_equal(part.scales, whole.scales[rows])
+    with pytest.raises(ValueError):  # a value above the stated amax
+        oracle.quantize_with_tensor_scale(w[rows], float(np.abs(w[rows]).max()) / 2)
