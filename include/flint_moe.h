@@ -277,6 +277,33 @@ int flint_moe_noalloc_get_status(int32_t* device_flags, void* stream);
  * flint_debug_wait_timeout. */
 int flint_debug_noalloc_scratch(void** addr);
 
+/* ---- the 4-bit output head ("Recursive Flint: 40B Local Coding Model,
+ * Benchmarks": architecture table, row "Vocabulary", and section "How
+ * Recursive built Flint", the 4-bit output head) ----
+ * A dense NVFP4 matrix W [rows][cols] (rows = vocabulary, cols = hidden size)
+ * in plain row-major planes: codes [rows][cols/2] (element 2j in the low
+ * nibble of byte j), E4M3 scales [rows][cols/16] (byte b covers elements
+ * 16b..16b+15), one fp32 tensor scale; w = e2m1(q) * e4m3(sb) * s_t. */
+
+/* flint_pack_nvfp4_dense -- quantise W (device, fp32 or bf16 bits when
+ * w_is_bf16, row-major [rows][cols]) with the experts' recipe (s_t =
+ * amax/2688, per-16 E4M3 scale, E2M1 codes; fp32 round to nearest, no fused
+ * multiply-add) into the planes above. cols one of 512, 1024, 2048, 4096;
+ * workspace >= 1280 bytes (status word at byte 0; a non-finite weight sets
+ * FLINT_DEVCHECK_NONFINITE there). Asynchronous on `stream`. */
+int flint_pack_nvfp4_dense(const void* w, int32_t w_is_bf16, int32_t rows, int32_t cols, uint8_t* codes,
+                           uint8_t* scales, float* tensor_scale, void* workspace, size_t ws_bytes, void* stream);
+
+/* flint_lm_head -- out[t][v] = sum_c w[v][c] x[t][c] for T decode tokens
+ * (T <= 2; T = 1 at cols = 4096). x: device bf16 [T][cols]; out: device fp32
+ * [T][rows]. Products of the exact e2m1*e4m3 value with x scaled per token
+ * by a power of two into f16 are exact; fp32 accumulation; the tensor scale
+ * is applied once per logit. workspace >= 4 bytes (status word, read it with
+ * flint_moe_get_status). Asynchronous on `stream`. */
+int flint_lm_head(const uint16_t* x, int32_t T, const uint8_t* codes, const uint8_t* scales,
+                  const float* tensor_scale, int32_t rows, int32_t cols, float* out, void* workspace,
+                  size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, reads the workspace status word into *device_flags
  * (FLINT_DEVCHECK_* bits, may be NULL) and clears it. Returns FLINT_OK, or
  * FLINT_ERR_TIMEOUT / FLINT_ERR_DEVICE_CHECK when a flag was set. */
@@ -295,6 +322,34 @@ const char* flint_last_error(void);
 int flint_debug_dequant(const flint_moe_weights* weights, const flint_moe_shape* shape,
                         int32_t expert, int32_t matrix, int32_t row0, int32_t rows,
                         float* out, float* tensor_scale_out, void* stream);
+
+/* Debug helper: decoded weights e2m1(q) * e4m3(sb) (no tensor scale) of a
+ * tile of one expert matrix, produced by the tensor-core decoders themselves:
+ * decoder 0 the tcgen05 path's decode into tensor memory (dequant_slice_tmem,
+ * read back with tcgen05.ld; tiles of 128 rows x 256 K), decoder 1 the
+ * register-fragment decode of the persistent kernel's mma.sync variant
+ * (tc_segment, extracted through the MMA with one-hot B columns; tiles of 16
+ * rows x 128 K). matrix 0: the 2*inter interleaved gate/up rows of the packed
+ * layout (row 2u = gate row u, 2u+1 = up row u); 1: the d down rows. Rows
+ * [row0, row0+rows) and K columns [k0, k0+kn) in whole tiles; out: device fp32
+ * [rows][kn]. Synchronises the stream. */
+int flint_debug_decode(const flint_moe_weights* weights, const flint_moe_shape* shape, int32_t expert,
+                       int32_t matrix, int32_t decoder, int32_t row0, int32_t rows, int32_t k0, int32_t kn,
+                       float* out, void* stream);
+
+/* Debug helper: the grouping of routed ids by expert (active experts in
+ * ascending id order, then the shared experts; per expert its pairs
+ * token << 8 | slot in ascending token order; offsets), computed on the
+ * device by one of the layer's grouping routines: impl 0 the CTA grouping of
+ * the persistent single-kernel path and the tensor-core path (T <= 128),
+ * impl 1 the warp grouping of the three-kernel path (T * top_k <= 64), impl 2
+ * its CTA grouping (T <= 32). ids: device int32 [T][top_k]. Outputs (device):
+ * act int32 [E+S], off int32 [E+S+1], pair int32 [T*(top_k+S)], counts int32
+ * [2] = {routed experts in use, active experts}. An id outside [0, E) is
+ * skipped and sets FLINT_DEVCHECK_EXPERT_ID in the workspace status word (read
+ * it with flint_moe_get_status). Asynchronous on `stream`. */
+int flint_debug_group(const int32_t* ids, int32_t T, const flint_moe_shape* shape, int32_t impl, int32_t* act,
+                      int32_t* off, int32_t* pair, int32_t* counts, void* workspace, size_t ws_bytes, void* stream);
 
 /* Failure-detection hook: launches one kernel whose bounded wait on a
  * shared-memory barrier that nothing completes gives up after `cycles` SM clock

@@ -21,7 +21,8 @@ __all__ = [
     "flint_moe_workspace_bytes", "flint_moe_workspace_init", "flint_pack_nvfp4", "flint_pack_bf16", "flint_moe_route",
     "flint_moe_forward", "flint_moe_forward_ex", "flint_moe_forward_noalloc", "flint_moe_noalloc_get_status",
     "flint_moe_get_status", "flint_last_error", "flint_debug_noalloc_scratch",
-    "flint_debug_dequant", "flint_debug_wait_timeout", "flint_version",
+    "flint_pack_nvfp4_dense", "flint_lm_head",
+    "flint_debug_dequant", "flint_debug_decode", "flint_debug_group", "flint_debug_wait_timeout", "flint_version",
 ]
 
 FLINT_W_NVFP4, FLINT_W_BF16 = 0, 1
@@ -92,6 +93,10 @@ def lib() -> ctypes.CDLL:
         L.flint_moe_noalloc_get_status.restype = i32
         L.flint_debug_noalloc_scratch.argtypes = [P(vp)]
         L.flint_debug_noalloc_scratch.restype = i32
+        L.flint_pack_nvfp4_dense.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+        L.flint_pack_nvfp4_dense.restype = i32
+        L.flint_lm_head.argtypes = [vp, i32, vp, vp, vp, i32, i32, vp, vp, sz, vp]
+        L.flint_lm_head.restype = i32
         L.flint_moe_workspace_init.argtypes = [vp, sz, vp]
         L.flint_moe_workspace_init.restype = i32
         L.flint_moe_get_status.argtypes = [vp, P(i32), vp]
@@ -100,6 +105,10 @@ def lib() -> ctypes.CDLL:
         L.flint_last_error.restype = ctypes.c_char_p
         L.flint_debug_dequant.argtypes = [P(Weights), P(Shape), i32, i32, i32, i32, vp, vp, vp]
         L.flint_debug_dequant.restype = i32
+        L.flint_debug_decode.argtypes = [P(Weights), P(Shape), i32, i32, i32, i32, i32, i32, i32, vp, vp]
+        L.flint_debug_decode.restype = i32
+        L.flint_debug_group.argtypes = [vp, i32, P(Shape), i32, vp, vp, vp, vp, vp, sz, vp]
+        L.flint_debug_group.restype = i32
         L.flint_debug_wait_timeout.argtypes = [vp, ctypes.c_int64, vp]
         L.flint_debug_wait_timeout.restype = i32
         L.flint_version.argtypes = []
@@ -221,6 +230,18 @@ def flint_debug_noalloc_scratch() -> int:
     return addr.value
 
 
+def flint_pack_nvfp4_dense(w, w_is_bf16: int, rows: int, cols: int, codes, scales, tensor_scale, workspace,
+                           stream=None) -> None:
+    _check(lib().flint_pack_nvfp4_dense(_ptr(w), int(w_is_bf16), int(rows), int(cols), _ptr(codes), _ptr(scales),
+                                        _ptr(tensor_scale), _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def flint_lm_head(x, T: int, codes, scales, tensor_scale, rows: int, cols: int, out, workspace,
+                  stream=None) -> None:
+    _check(lib().flint_lm_head(_ptr(x), int(T), _ptr(codes), _ptr(scales), _ptr(tensor_scale), int(rows),
+                               int(cols), _ptr(out), _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
 def flint_moe_get_status(workspace, stream=None) -> tuple[int, int]:
     """Returns (status, device_flags) without raising."""
     flags = ctypes.c_int32(0)
@@ -235,6 +256,20 @@ def flint_debug_dequant(weights: Weights, shape: Shape, expert: int, matrix: int
                                      int(matrix), int(row0), int(rows), _ptr(out), ts,
                                      _stream(stream)))
     return (ts[0], ts[1]) if matrix == 0 else (ts[0],)
+
+
+def flint_debug_decode(weights: Weights, shape: Shape, expert: int, matrix: int, decoder: int, row0: int,
+                       rows: int, k0: int, kn: int, out, stream=None) -> None:
+    _check(lib().flint_debug_decode(ctypes.byref(weights), ctypes.byref(shape), int(expert), int(matrix),
+                                    int(decoder), int(row0), int(rows), int(k0), int(kn), _ptr(out),
+                                    _stream(stream)))
+
+
+def flint_debug_group(ids, T: int, shape: Shape, impl: int, act, off, pair, counts, workspace,
+                      stream=None) -> None:
+    _check(lib().flint_debug_group(_ptr(ids), int(T), ctypes.byref(shape), int(impl), _ptr(act), _ptr(off),
+                                   _ptr(pair), _ptr(counts), _ptr(workspace), _nbytes(workspace),
+                                   _stream(stream)))
 
 
 def flint_debug_wait_timeout(workspace, cycles: int, stream=None) -> None:

@@ -14,6 +14,7 @@
 #include "fused_layer.cuh"
 #include "mma_path.cuh"
 #include "tok1.cuh"
+#include "lmhead.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -126,6 +127,60 @@ __global__ void k_pack_quant(const void* w, int d, int I, long long n_blocks, lo
   if (r == 0 && b == 0) ts[mat] = s_t;
 }
 
+// One dense matrix [rows][cols], row-major planes: codes [rows][cols/2],
+// scales [rows][cols/16], one tensor scale (the same recipe as k_pack_quant).
+template <bool BF16IN>
+__global__ void k_pack_dense_quant(const void* w, long long rows, int cols, const unsigned* amax_bits, uint8_t* codes,
+                                   uint8_t* scales, float* ts) {
+  const long long gb = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  const long long n_blocks = rows * (cols / 16);
+  if (gb >= n_blocks) return;
+  float v[16];
+  if (BF16IN) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(w) + 16 * gb);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint4 u = src[q];
+      const uint32_t ww[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[8 * q + 2 * i] = bf16_bits_to_f32(ww[i] & 0xFFFFu);
+        v[8 * q + 2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u);
+      }
+    }
+  } else {
+    const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(w) + 16 * gb);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 f = src[q];
+      v[4 * q] = f.x;
+      v[4 * q + 1] = f.y;
+      v[4 * q + 2] = f.z;
+      v[4 * q + 3] = f.w;
+    }
+  }
+  const float amax = __uint_as_float(amax_bits[0]);
+  const float s_t = (amax > 0.f) ? __fdiv_rn(amax, 2688.f) : 1.f;
+  float amax_b = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
+  const uint32_t sb = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax_b, 6.f), s_t));
+  const float dec = e4m3x2_to_f32x2(sb).x;
+  const float denom = __fmul_rn(dec, s_t);
+  uint32_t lo = 0, hi = 0;
+  if (denom != 0.f) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      lo |= f32x2_to_e2m1x2(__fdiv_rn(v[2 * i], denom), __fdiv_rn(v[2 * i + 1], denom)) << (8 * i);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      hi |= f32x2_to_e2m1x2(__fdiv_rn(v[8 + 2 * i], denom), __fdiv_rn(v[8 + 2 * i + 1], denom)) << (8 * i);
+  }
+  *reinterpret_cast<uint2*>(codes + 8 * gb) = make_uint2(lo, hi);
+  scales[gb] = static_cast<uint8_t>(sb);
+  if (gb == 0) ts[0] = s_t;
+}
+
 // bf16 weights in the same expert-major row order (16-byte vectors).
 __global__ void k_pack_bf16(const uint16_t* w, int d, int I, long long n_vec, uint16_t* out) {
   const long long gv = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
@@ -169,6 +224,142 @@ __global__ void k_debug_dequant(const uint8_t* codes, const uint8_t* scales, int
       out[r * K + v * 32 + wi * 8 + 2 * i] = f.x * sc;
       out[r * K + v * 32 + wi * 8 + 2 * i + 1] = f.y * sc;
     }
+  }
+}
+
+// The tensor-core path's NVFP4 decode (dequant_slice_tmem) on one tile of 128
+// rows x 256 K: the tile is staged the way its TMA copy lands (code rows of
+// 128 bytes with the 128-byte swizzle, then 16 scale bytes per row), decoded
+// into tensor memory by warps 8..15 exactly as in k_mma_ffn, read back with
+// tcgen05.ld by warps 4..7 (lanes 32*(w%4)..) and written as fp32. Column c of
+// the tile's 128 tensor-memory columns holds K elements 2c, 2c+1 as f16x2.
+// Grid (row tiles, K tiles); `codes`/`scales` point at the matrix's first row.
+__global__ void __launch_bounds__(512, 1) k_debug_decode_tmem(const uint8_t* codes, const uint8_t* scales, int K,
+                                                              int k0, float* out, int ldo) {
+  __shared__ __align__(1024) uint8_t raw[kMmaRawBytes];
+  __shared__ uint32_t s_tmem;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long r0 = 128LL * blockIdx.x;
+  const int kb = k0 + 256 * blockIdx.y;
+  for (int i = tid; i < 128 * 8; i += blockDim.x) {  // 16-byte code chunks, swizzled as TMA writes them
+    const int r = i >> 3, c = i & 7;
+    *reinterpret_cast<uint4*>(raw + r * 128 + ((c ^ (r & 7)) << 4)) =
+        *reinterpret_cast<const uint4*>(codes + (r0 + r) * (K / 2) + kb / 2 + 16 * c);
+  }
+  for (int i = tid; i < 128; i += blockDim.x)
+    *reinterpret_cast<uint4*>(raw + 128 * 128 + 16 * i) =
+        *reinterpret_cast<const uint4*>(scales + (r0 + i) * (K / 16) + kb / 16);
+  if (warp == 1) tmem_alloc(&s_tmem, 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  if (warp >= 8)
+    for (int sub = 0; sub < 4; ++sub) dequant_slice_tmem(raw, sub, tmem + 32u * sub, warp, lane);
+  tmem_wait_st();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp >= 4 && warp < 8) {
+    const int row = 32 * (warp & 3) + lane;
+    for (int c0 = 0; c0 < 128; c0 += 16) {
+      float v[16];
+      tmem_ld16(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + static_cast<uint32_t>(c0), v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t w = __float_as_uint(v[i]);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+        float* o = out + (r0 + row) * ldo + 256 * blockIdx.y + 2 * (c0 + i);
+        o[0] = f.x;
+        o[1] = f.y;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// The persistent kernel's register-fragment decode (tc_segment) on tiles of
+// 16 rows x 128 K, extracted through the MMA itself: in step q, B column n is
+// one-hot on the logical k that the segment's K permutation gives physical
+// element 8q + n, so D[row][n] = A[row][8q + n], the decoded weight of that
+// element (exact in f16, multiplied by 1 and accumulated in f32). One warp per
+// tile; grid (row tiles, K tiles).
+__global__ void __launch_bounds__(32) k_debug_decode_frag(const uint8_t* codes, const uint8_t* scales, int K, int k0,
+                                                          float* out, int ldo) {
+  const int lane = threadIdx.x, g = lane >> 2, t = lane & 3;
+  const long long r0 = 16LL * blockIdx.x;
+  const int kb = k0 + 128 * blockIdx.y;
+  const uint4 ra = *reinterpret_cast<const uint4*>(codes + (r0 + g) * (K / 2) + kb / 2 + 16 * t);
+  const uint4 rb = *reinterpret_cast<const uint4*>(codes + (r0 + g + 8) * (K / 2) + kb / 2 + 16 * t);
+  const uint32_t sa2 = *reinterpret_cast<const uint16_t*>(scales + (r0 + g) * (K / 16) + kb / 16 + 2 * t);
+  const uint32_t sb2 = *reinterpret_cast<const uint16_t*>(scales + (r0 + g + 8) * (K / 16) + kb / 16 + 2 * t);
+  for (int q = 0; q < 16; ++q) {
+    // this lane holds B rows k = 2t, 2t+1 (b[2j]) and 2t+8, 2t+9 (b[2j+1]) of
+    // column g; physical element p = 32t' + 4j + 2h + e sits in b[2j+h], half e,
+    // of the lanes with t = t'
+    const int p = 8 * q + g, tp = p >> 5, j = (p & 31) >> 2, h = (p >> 1) & 1, e = p & 1;
+    uint32_t b[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) b[i] = (tp == t && i == 2 * j + h) ? (e ? 0x3C000000u : 0x00003C00u) : 0u;
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+    tc_segment(c0, c1, ra, rb, sa2, sb2, b);
+    // c[0..1]: row g, columns 2t, 2t+1; c[2..3]: row g + 8
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int row = g + 8 * (i >> 1), col = 2 * t + (i & 1);
+      out[(r0 + row) * ldo + 128 * blockIdx.y + 8 * q + col] = c0[i] + c1[i];
+    }
+  }
+}
+
+// One of the grouping routines on given ids (debug entry flint_debug_group):
+// impl 0 the CTA grouping of the persistent kernel and the tensor-core path
+// (T <= 128), 1 the warp grouping of the three-kernel path (T*k <= 64), 2 its
+// CTA grouping (T <= 32). One CTA of 512 threads; outputs as int arrays.
+__global__ void __launch_bounds__(512) k_debug_group(const int* ids, int T, int k, int E, int S, int impl, int* act,
+                                                     int* off, int* pair, int* counts, int* status) {
+  __shared__ int s_ids[kMmaMaxTokens * kMaxTopK];
+  __shared__ __align__(8) uint8_t s_scratch[20 * kMaxExperts];
+  __shared__ Grouping g;
+  __shared__ RouteDesc dsc;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < T * k; i += blockDim.x) s_ids[i] = ids[i];
+  __syncthreads();
+  if (impl == 0) {
+    cta_grouping(s_ids, T, k, E, S, act, off, pair, counts, counts + 1, s_scratch, status);
+    return;
+  }
+  const int* a;
+  const int* o;
+  const unsigned short* pr;
+  int n_active, n_routed;
+  if (impl == 1) {
+    if (tid < 32) warp_grouping(s_ids, T, k, E, S, &dsc, tid, status);
+    __syncthreads();
+    a = dsc.act;
+    o = dsc.off;
+    pr = dsc.pair;
+    n_active = dsc.n_active;
+    n_routed = dsc.n_routed;
+  } else {
+    build_grouping(g, s_ids, T, k, E, S, status);
+    a = g.act;
+    o = g.off;
+    pr = g.pair;
+    n_active = g.n_active;
+    n_routed = g.n_routed;
+  }
+  for (int i = tid; i < n_active; i += blockDim.x) act[i] = a[i];
+  for (int i = tid; i <= n_active; i += blockDim.x) off[i] = o[i];
+  for (int i = tid; i < o[n_active]; i += blockDim.x) pair[i] = pr[i];
+  if (tid == 0) {
+    counts[0] = n_routed;
+    counts[1] = n_active;
   }
 }
 
@@ -879,6 +1070,69 @@ int flint_pack_bf16(const uint16_t* w, const flint_moe_shape* shape, uint16_t* p
   return FLINT_OK;
 }
 
+int flint_pack_nvfp4_dense(const void* w, int32_t w_is_bf16, int32_t rows, int32_t cols, uint8_t* codes,
+                           uint8_t* scales, float* tensor_scale, void* workspace, size_t ws_bytes, void* stream) {
+  if (!w || !codes || !scales || !tensor_scale || !workspace)
+    return fail(FLINT_ERR_INVALID_ARG, "flint_pack_nvfp4_dense: NULL pointer");
+  if (rows < 1 || !(cols == 512 || cols == 1024 || cols == 2048 || cols == 4096))
+    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "flint_pack_nvfp4_dense: rows=%d cols=%d (cols one of 512..4096)", rows, cols);
+  if (!aligned16(w) || !aligned16(codes) || !aligned16(scales) || !aligned16(tensor_scale) || !aligned16(workspace))
+    return fail(FLINT_ERR_MISALIGNED, "flint_pack_nvfp4_dense: pointers must be 16-byte aligned");
+  if (ws_bytes < kCtrlBytes + 256) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kCtrlBytes + 256);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  unsigned* amax = reinterpret_cast<unsigned*>(ws + kCtrlBytes);
+  int* status = reinterpret_cast<int*>(ws);
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned), st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  const long long n = static_cast<long long>(rows) * cols;
+  if (w_is_bf16)
+    k_pack_amax<true><<<dim3(1024, 1), 256, 0, st>>>(w, n, amax, status);
+  else
+    k_pack_amax<false><<<dim3(1024, 1), 256, 0, st>>>(w, n, amax, status);
+  const long long n_blocks = n / 16;
+  const unsigned g = static_cast<unsigned>((n_blocks + 255) / 256);
+  if (w_is_bf16)
+    k_pack_dense_quant<true><<<g, 256, 0, st>>>(w, rows, cols, amax, codes, scales, tensor_scale);
+  else
+    k_pack_dense_quant<false><<<g, 256, 0, st>>>(w, rows, cols, amax, codes, scales, tensor_scale);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "flint_pack_nvfp4_dense launch");
+  return FLINT_OK;
+}
+
+int flint_lm_head(const uint16_t* x, int32_t T, const uint8_t* codes, const uint8_t* scales,
+                  const float* tensor_scale, int32_t rows, int32_t cols, float* out, void* workspace,
+                  size_t ws_bytes, void* stream) {
+  if (!x || !codes || !scales || !tensor_scale || !out || !workspace)
+    return fail(FLINT_ERR_INVALID_ARG, "flint_lm_head: NULL pointer");
+  if (T < 0) return fail(FLINT_ERR_INVALID_ARG, "T=%d", T);
+  if (T == 0) return FLINT_OK;
+  if (rows < 1 || !(cols == 512 || cols == 1024 || cols == 2048 || cols == 4096))
+    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "flint_lm_head: rows=%d cols=%d (cols one of 512..4096)", rows, cols);
+  if (T > (cols == 4096 ? 1 : kLmMaxTokens))
+    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "flint_lm_head: at most %d tokens at cols=%d", cols == 4096 ? 1 : kLmMaxTokens, cols);
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(tensor_scale) || !aligned16(out) ||
+      !aligned16(workspace))
+    return fail(FLINT_ERR_MISALIGNED, "flint_lm_head: pointers must be 16-byte aligned");
+  if (ws_bytes < 4) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < 4 bytes", ws_bytes);
+  LmHeadParams p{};
+  p.x = x;
+  p.codes = codes;
+  p.scales = scales;
+  p.tscale = tensor_scale;
+  p.out = out;
+  p.status = static_cast<int*>(workspace);
+  p.T = T;
+  p.V = rows;
+  // as many 16-row stages as fit next to the staged x (at most 8)
+  const size_t budget = 200 * 1024 - static_cast<size_t>(kLmMaxTokens) * cols * 2;
+  p.stages = static_cast<int>(std::min<size_t>(kLmMaxStages, budget / lm_stage_bytes(cols)));
+  cudaError_t e = lm_head_launch(cols, p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "k_lm_head launch");
+  return FLINT_OK;
+}
+
 int flint_moe_route(const uint16_t* x, int32_t T, const uint16_t* router_w, const flint_moe_shape* shape,
                     int32_t* topk_ids, float* topk_weights, void* workspace, size_t ws_bytes, void* stream) {
   Dims s;
@@ -1086,6 +1340,55 @@ int flint_moe_get_status(void* workspace, int32_t* device_flags, void* stream) {
   if (device_flags) *device_flags = flags;
   if (flags & FLINT_DEVCHECK_WAIT) return fail(FLINT_ERR_TIMEOUT, "a bounded device wait ran out");
   if (flags) return fail(FLINT_ERR_DEVICE_CHECK, "device check flags 0x%x", flags);
+  return FLINT_OK;
+}
+
+int flint_debug_decode(const flint_moe_weights* weights, const flint_moe_shape* shape, int32_t expert,
+                       int32_t matrix, int32_t decoder, int32_t row0, int32_t rows, int32_t k0, int32_t kn, float* out,
+                       void* stream) {
+  Dims s;
+  int rc = check_shape(shape, &s);
+  if (rc != FLINT_OK) return rc;
+  if (s.wd != FLINT_W_NVFP4 || !weights || !weights->packed || !weights->block_scales || !out)
+    return fail(FLINT_ERR_INVALID_ARG, "flint_debug_decode: NVFP4 weights and output needed");
+  if (expert < 0 || expert >= s.E + s.S || (matrix != 0 && matrix != 1) || decoder < 0 || decoder > 1)
+    return fail(FLINT_ERR_INVALID_ARG, "flint_debug_decode: bad expert/matrix/decoder");
+  const int K = matrix == 0 ? s.d : s.I, nrows = matrix == 0 ? 2 * s.I : s.d;
+  const int th = decoder == 0 ? 128 : 16, tw = decoder == 0 ? 256 : 128;
+  if (row0 < 0 || rows <= 0 || rows % th || row0 + rows > nrows || k0 < 0 || kn <= 0 || kn % tw || k0 % tw ||
+      k0 + kn > K)
+    return fail(FLINT_ERR_INVALID_ARG, "flint_debug_decode: tiles of %d rows x %d K inside the matrix", th, tw);
+  const long long cpe = 3LL * s.I * s.d / 2, spe = 3LL * s.I * s.d / 16;
+  const uint8_t* codes = static_cast<const uint8_t*>(weights->packed) + expert * cpe +
+                         (matrix == 0 ? 0 : static_cast<long long>(s.I) * s.d) + static_cast<long long>(row0) * (K / 2);
+  const uint8_t* scales = weights->block_scales + expert * spe +
+                          (matrix == 0 ? 0 : static_cast<long long>(s.I) * s.d / 8) + static_cast<long long>(row0) * (K / 16);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (decoder == 0)
+    k_debug_decode_tmem<<<dim3(rows / 128, kn / 256), 512, 0, st>>>(codes, scales, K, k0, out, kn);
+  else
+    k_debug_decode_frag<<<dim3(rows / 16, kn / 128), 32, 0, st>>>(codes, scales, K, k0, out, kn);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "flint_debug_decode");
+  return FLINT_OK;
+}
+
+int flint_debug_group(const int32_t* ids, int32_t T, const flint_moe_shape* shape, int32_t impl, int32_t* act,
+                      int32_t* off, int32_t* pair, int32_t* counts, void* workspace, size_t ws_bytes, void* stream) {
+  Dims s;
+  int rc = check_shape(shape, &s);
+  if (rc != FLINT_OK) return rc;
+  if (!ids || !act || !off || !pair || !counts || !workspace)
+    return fail(FLINT_ERR_INVALID_ARG, "flint_debug_group: NULL pointer");
+  if (impl < 0 || impl > 2) return fail(FLINT_ERR_INVALID_ARG, "flint_debug_group: impl %d", impl);
+  const int max_t = impl == 0 ? kMmaMaxTokens : (impl == 1 ? 64 / s.k : kMaxGemvTokens);
+  if (T < 1 || T > max_t) return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "flint_debug_group: impl %d takes 1..%d tokens", impl, max_t);
+  if (ws_bytes < kCtrlBytes) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kCtrlBytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  k_debug_group<<<1, 512, 0, st>>>(ids, T, s.k, s.E, s.S, impl, act, off, pair, counts, static_cast<int*>(workspace));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "k_debug_group launch");
   return FLINT_OK;
 }
 

@@ -56,7 +56,8 @@ struct Tok1Params {
 };
 
 // Dynamic shared-memory bytes of k_tok1: the larger of the router-row slice and
-// the expert slice (they share the region), then the cluster's logits and h.
+// the expert slice (they share the region), then the cluster's logits and h,
+// then the token's x (bf16).
 __host__ __device__ constexpr size_t tok1_region_bytes(int D, int I, int E) {
   const size_t rows = static_cast<size_t>((E + kTok1Cluster - 1) / kTok1Cluster) * D * 2;
   const size_t ex = static_cast<size_t>(I / kTok1Cluster) * (D + D / 8) +
@@ -65,7 +66,7 @@ __host__ __device__ constexpr size_t tok1_region_bytes(int D, int I, int E) {
 }
 __host__ __device__ constexpr size_t tok1_smem_bytes(int D, int I, int E) {
   return tok1_region_bytes(D, I, E) + ((static_cast<size_t>(E) * 4 + 127) & ~static_cast<size_t>(127)) +
-         static_cast<size_t>(I) * 4;
+         static_cast<size_t>(I) * 4 + static_cast<size_t>(D) * 2;
 }
 
 __device__ __forceinline__ unsigned cluster_rank() {
@@ -106,7 +107,7 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   static_assert(RPC % RPS == 0 || RPC < RPS, "down rows");
 
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t s_bar[kTok1MaxChunks + 2];  // chunks, down rows, router rows
+  __shared__ __align__(8) uint64_t s_bar[kTok1MaxChunks + 3];  // chunks, down rows, router rows, x
   __shared__ int s_ids[kMaxTopK];
   __shared__ float s_gates[kMaxTopK];
   __shared__ int s_fail, s_last, s_burst;
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   uint8_t* region = smem;
   float* s_logits = reinterpret_cast<float*>(smem + tok1_region_bytes(D, I, E));
   float* s_h = s_logits + ((E + 31) & ~31);
+  const uint16_t* s_x = reinterpret_cast<const uint16_t*>(s_h + I);
   uint8_t* gu_codes = region;                                   // [UPC][D]
   uint8_t* gu_scales = region + UPC * UNIT_C;                   // [UPC][D/8]
   uint8_t* dn_codes = gu_scales + UPC * UNIT_S;                 // [RPC][I/2]
@@ -126,6 +128,7 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   uint64_t* bar_chunk = s_bar;
   uint64_t* bar_down = s_bar + kTok1MaxChunks;
   uint64_t* bar_rows = s_bar + kTok1MaxChunks + 1;
+  uint64_t* bar_x = s_bar + kTok1MaxChunks + 2;
   const int r0 = static_cast<int>(rank) * E / CS, r1 = (static_cast<int>(rank) + 1) * E / CS;
 
   // issue this CTA's slice of expert e (one lane per chunk, one for the down rows)
@@ -148,7 +151,7 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
 
   // ---- P0: routing-independent copies, before the dependency wait
   if (tid == 0) {
-    for (int i = 0; i < kTok1MaxChunks + 2; ++i) mbar_init(&s_bar[i], 1);
+    for (int i = 0; i < kTok1MaxChunks + 3; ++i) mbar_init(&s_bar[i], 1);
     fence_barrier_init();
     s_fail = 0;
     s_burst = shared ? 1 : 0;
@@ -165,19 +168,25 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   if (p.trigger_early) pdl_trigger();
   pdl_wait();  // x (and the workspace) are written by the preceding kernel
+  // one copy of x per CTA: every warp reading it from L2 would make its 32
+  // lines a hot spot of thousands of requests
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_x, D * 2);
+    bulk_g2s(const_cast<uint16_t*>(s_x), p.x, D * 2, bar_x);
+  }
 
   // ---- P1: x -> statistics, f16 registers (lane's vectors v = lane + 32 j, j < XV
   // of a gate/up row; at D = 512 lanes 16..31 repeat lanes 0..15)
-  bool ok = true;
+  bool ok = __all_sync(0xffffffffu, mbar_wait(bar_x, 0, p.status));
   const int xl = lane % VPR;  // first x vector of this lane
   uint32_t xr[XV][16];        // bf16 pairs, then f16 pairs scaled by sigma
   float amax = 0.f, ss = 0.f;
 #pragma unroll
   for (int j = 0; j < XV; ++j) {
-    const uint4* src = reinterpret_cast<const uint4*>(p.x) + (xl + 32 * j) * 4;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(s_x) + (xl + 32 * j) * 64;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const uint4 v = __ldcg(src + q);
+      const uint4 v = lds128(src + 16 * q);
       xr[j][4 * q + 0] = v.x;
       xr[j][4 * q + 1] = v.y;
       xr[j][4 * q + 2] = v.z;
@@ -345,18 +354,21 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
     for (int r = tid; r < RPC; r += blockDim.x) __stcg(part + r, 0.f);
   }
 
-  // ---- P5: the last of the k + S CTAs of this row block sums the slots
-  __threadfence();  // this thread's partial stores before the CTA's arrival
+  // ---- P5: the last of the k + S CTAs of this row block sums the slots.
+  // The barrier orders every thread's partial stores before thread 0's
+  // arrival, whose release (cumulative) publishes them at GPU scope; its
+  // acquire makes the other slots' partials visible to the last arriver, and
+  // the barrier after it to all of its threads.
   __syncthreads();
   if (tid == 0) {
-    const unsigned old = atomicAdd(p.rb_count + rank, 1u);
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.rb_count + rank) : "memory");
     const int last = old == static_cast<unsigned>(KS - 1);
     if (last) atomicExch(p.rb_count + rank, 0u);  // no other CTA of this launch touches it again
     s_last = last;
   }
   __syncthreads();
   if (s_last) {
-    __threadfence();
     for (int r = tid; r < RPC; r += blockDim.x) {
       const int n = static_cast<int>(rank) * RPC + r;
       float y = 0.f;
@@ -368,7 +380,10 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   }
   if (!p.trigger_early) pdl_trigger();
   // copies still in flight after a failed wait land before the CTA exits
-  if (!ok && !shared && r1 > r0 && tid == 0) mbar_wait(bar_rows, 0, p.status);
+  if (!ok && tid == 0) {
+    mbar_wait(bar_x, 0, p.status);
+    if (!shared && r1 > r0) mbar_wait(bar_rows, 0, p.status);
+  }
   if (!ok && issued) {
     for (int c = tid; c < NCH; c += blockDim.x) mbar_wait(&bar_chunk[c], 0, p.status);
     if (tid == 0) mbar_wait(bar_down, 0, p.status);

@@ -171,6 +171,18 @@ def zipf_bias(seed: int, E: int, s: float) -> np.ndarray:
     return np.log(p)
 
 
+def router_for_targets(w: Workload, seed: int, x_bits_: np.ndarray, sets, boost: float = 8.0,
+                       layer: int = 0) -> np.ndarray:
+    """Router weights [E][d] as bf16 bits that steer token t to the experts in
+    sets[t]: +boost on their logits through a rank-T change of W_r."""
+    wr = router_plain(seed, w.d, w.E, layer, w.std)
+    x = bf16_bits_to_f64(x_bits_)
+    bias = np.zeros((x.shape[0], w.E))
+    for t, s in enumerate(sets):
+        bias[t, list(s)] = boost
+    return to_bf16_bits(_shape_router(wr, x, bias))
+
+
 def make_router(w: Workload, seed: int, x_bits_: np.ndarray, layer: int = 0) -> np.ndarray:
     """Router weights [E][d] as bf16 bits, shaped for the workload's routing structure."""
     wr = router_plain(seed, w.d, w.E, layer, w.std)
