@@ -351,6 +351,68 @@ def run_e2e(stack: Stack, routers, T: int, K: int, norm: int = 0):
     return T * K / (ms / 1e3), T * d * 2, T * d * 2
 
 
+LM_VOCAB = 150144
+
+
+def run_lm_head(world: int, n_heads: int = 3, calls: int = 60):
+    """The 4-bit output head (150,144 x 2048 NVFP4, 173 MB): a graph of `calls`
+    launches cycling through `n_heads` independently drawn heads (more than
+    L2 holds), per launch time from CUDA events on the launching stream."""
+    import torch
+    import nvfp4_weight_only_flint_b200 as fm
+    rows, cols = LM_VOCAB, 2048
+    ws = torch.zeros(2048, dtype=torch.uint8, device="cuda")
+    heads = []
+    for h in range(n_heads):
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(synth.key(0, "experts", 10000 + h) & 0x7FFFFFFFFFFFFFFF)
+        w = torch.randn((rows, cols), generator=gen, device="cuda", dtype=torch.float32).mul_(0.02)
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device="cuda")
+        scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device="cuda")
+        ts = torch.empty(4, dtype=torch.float32, device="cuda")
+        fm.flint_pack_nvfp4_dense(w, 0, rows, cols, codes, scales, ts, ws)
+        torch.cuda.synchronize()
+        del w
+        heads.append((codes, scales, ts))
+    peak, peak_kind = _peaks()
+    res = {"workload": f"dense NVFP4 output head {rows} x {cols} (173 MB), {n_heads} heads used in turn",
+           "kernel": "k_lm_head"}
+    st = torch.cuda.Stream()
+    for T in (1, 8):
+        x = _bits_to_cuda(synth.x_bits(4242, T, cols))
+        out = torch.empty((T, rows), dtype=torch.float32, device="cuda")
+        with torch.cuda.stream(st):
+            for i in range(2 * n_heads):
+                c, s_, t_ = heads[i % n_heads]
+                fm.flint_lm_head(x, T, c, s_, t_, rows, cols, out, ws)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            for i in range(calls):
+                c, s_, t_ = heads[i % n_heads]
+                fm.flint_lm_head(x, T, c, s_, t_, rows, cols, out, ws)
+        with torch.cuda.stream(st):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(st):
+            e0.record(st)
+            g.replay()
+            e1.record(st)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / calls * 1e3
+        byt = rows * cols // 2 + rows * cols // 16 + T * cols * 2 + T * rows * 4
+        res[f"batch{T}"] = {"us": us, "bytes": byt, "gbs": byt / us / 1e3, "frac_of_peak": byt / us / 1e3 / peak,
+                            "tokens_per_s": world * T / (us / 1e6)}
+        del g
+    rc, flags = fm.flint_moe_get_status(ws)
+    if rc != 0:
+        raise RuntimeError(f"lm head status {rc} flags {flags}")
+    del heads
+    torch.cuda.empty_cache()
+    return res
+
+
 def cpu_baseline(n_tokens: int = 3, seed: int = 0):
     """The fp64 oracle as it stands, on host cores: T=1 layer decodes of the
     default workload (quantisation of the needed experts is untimed set-up)."""
@@ -522,6 +584,7 @@ def main():
                                   "tensor_peak_tflops": tf_peak, "tensor_peak_kind": tf_kind}}
             del st64, fx64, r64
             torch.cuda.empty_cache()
+        extras["lm_head"] = run_lm_head(world)
         extras["stack47"] = {
             "workload": "cfg3: 47 resident layers (21.4 GB NVFP4), residual chain, no attention",
             "batch1_tokens_per_s": tok_s / N_LAYERS, "batch1_us_per_layer": ms_step * 1e3,

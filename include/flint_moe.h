@@ -294,12 +294,13 @@ int flint_debug_noalloc_scratch(void** addr);
 int flint_pack_nvfp4_dense(const void* w, int32_t w_is_bf16, int32_t rows, int32_t cols, uint8_t* codes,
                            uint8_t* scales, float* tensor_scale, void* workspace, size_t ws_bytes, void* stream);
 
-/* flint_lm_head -- out[t][v] = sum_c w[v][c] x[t][c] for T decode tokens
- * (T <= 2; T = 1 at cols = 4096). x: device bf16 [T][cols]; out: device fp32
- * [T][rows]. Products of the exact e2m1*e4m3 value with x scaled per token
- * by a power of two into f16 are exact; fp32 accumulation; the tensor scale
- * is applied once per logit. workspace >= 4 bytes (status word, read it with
- * flint_moe_get_status). Asynchronous on `stream`. */
+/* flint_lm_head -- out[t][v] = sum_c w[v][c] x[t][c] for T <= 8 decode
+ * tokens. x: device bf16 [T][cols]; out: device fp32 [T][rows]. The exact
+ * e2m1*e4m3 values (f16) multiply x scaled per token by a power of two into
+ * f16 on the register-fragment tensor cores (mma.sync, fp32 accumulation);
+ * the partial sums of a row's 512-column parts are added in part order; the
+ * tensor scale and 1/sigma are applied once per logit. workspace >= 4 bytes
+ * (status word; read it with flint_moe_get_status). Asynchronous on `stream`. */
 int flint_lm_head(const uint16_t* x, int32_t T, const uint8_t* codes, const uint8_t* scales,
                   const float* tensor_scale, int32_t rows, int32_t cols, float* out, void* workspace,
                   size_t ws_bytes, void* stream);

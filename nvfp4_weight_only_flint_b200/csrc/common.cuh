@@ -177,11 +177,12 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) {
 // row fits f16 without overflow (sigma = 1 when amax is 0).
 __device__ __forceinline__ float pow2_scale_for(float amax) {
   if (!(amax > 0.f) || !isfinite(amax)) return 1.f;
-  int e;
-  frexpf(amax, &e);  // amax = m * 2^e, m in [0.5, 1)  =>  amax <= 2^e
+  // amax = m * 2^e with m in [0.5, 1) (for subnormal amax e <= -126, and the
+  // clamp below gives the same 2^127): e = biased exponent - 126
+  const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 126;
   int p = 15 - e;
   p = max(-126, min(p, 127));
-  return ldexpf(1.f, p);
+  return __uint_as_float(static_cast<uint32_t>(p + 127) << 23);
 }
 
 // Pack two floats (already scaled) into f16x2, element a in the low half.

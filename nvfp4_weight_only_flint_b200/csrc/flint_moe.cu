@@ -399,6 +399,9 @@ int fail(int code, const char* fmt, ...) {
 }
 
 int cuda_fail(cudaError_t e, const char* what) {
+  // a failed launch or call also stays in the runtime's last-error slot; take
+  // it out so that a later, unrelated check does not report it again
+  cudaGetLastError();
   return fail(FLINT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
@@ -1110,25 +1113,30 @@ int flint_lm_head(const uint16_t* x, int32_t T, const uint8_t* codes, const uint
   if (T == 0) return FLINT_OK;
   if (rows < 1 || !(cols == 512 || cols == 1024 || cols == 2048 || cols == 4096))
     return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "flint_lm_head: rows=%d cols=%d (cols one of 512..4096)", rows, cols);
-  if (T > (cols == 4096 ? 1 : kLmMaxTokens))
-    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "flint_lm_head: at most %d tokens at cols=%d", cols == 4096 ? 1 : kLmMaxTokens, cols);
+  if (T > kLmMaxTokens) return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "flint_lm_head: at most %d tokens", kLmMaxTokens);
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(tensor_scale) || !aligned16(out) ||
       !aligned16(workspace))
     return fail(FLINT_ERR_MISALIGNED, "flint_lm_head: pointers must be 16-byte aligned");
   if (ws_bytes < 4) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < 4 bytes", ws_bytes);
   LmHeadParams p{};
   p.x = x;
-  p.codes = codes;
-  p.scales = scales;
   p.tscale = tensor_scale;
   p.out = out;
   p.status = static_cast<int*>(workspace);
   p.T = T;
   p.V = rows;
-  // as many 16-row stages as fit next to the staged x (at most 8)
-  const size_t budget = 200 * 1024 - static_cast<size_t>(kLmMaxTokens) * cols * 2;
-  p.stages = static_cast<int>(std::min<size_t>(kLmMaxStages, budget / lm_stage_bytes(cols)));
-  cudaError_t e = lm_head_launch(cols, p, static_cast<cudaStream_t>(stream));
+  LmMaps maps;
+  const cuuint64_t cdims[2] = {static_cast<cuuint64_t>(cols / 2), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t cstr[1] = {static_cast<cuuint64_t>(cols / 2)};
+  const cuuint32_t cbox[2] = {128, 16};
+  int rc = encode_map(&maps.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, cdims, cstr, cbox, true);
+  if (rc != FLINT_OK) return rc;
+  const cuuint64_t sdims[2] = {static_cast<cuuint64_t>(cols / 16), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t sstr[1] = {static_cast<cuuint64_t>(cols / 16)};
+  const cuuint32_t sbox[2] = {32, 16};
+  rc = encode_map(&maps.scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, scales, sdims, sstr, sbox, false);
+  if (rc != FLINT_OK) return rc;
+  cudaError_t e = lm_head_launch(cols, p, maps, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "k_lm_head launch");
   return FLINT_OK;
 }

@@ -5,137 +5,160 @@
 namespace flint {
 namespace {
 
-template <int D, int T>
-__global__ void __launch_bounds__(kLmWarps * 32, 1) k_lm_head(LmHeadParams p) {
-  constexpr int VPR = D / 32;                  // 16-byte code vectors per row
-  constexpr int XV = VPR >= 32 ? VPR / 32 : 1;  // vectors per lane
-  constexpr int ROWC = D / 2, ROWS = D / 16;
-  constexpr int STC = kLmRows * ROWC;          // code bytes of a stage
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t full[kLmMaxStages], empty[kLmMaxStages];
+template <int D>
+__global__ void __launch_bounds__(kLmWarps * 32, 1) k_lm_head(LmHeadParams p, const __grid_constant__ LmMaps maps) {
+  constexpr int KP = D / 512;          // K parts (warps) per tile
+  constexpr int TPI = kLmWarps / KP;   // tiles in flight per CTA
+  constexpr int XSTR = tc_b_stride(D);
+  constexpr int NS = lm_stages(D);
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bars[kLmWarps * NS];
+  __shared__ int s_fail;
   __shared__ float s_f[kLmMaxTokens];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* codes = base;                                              // [warp][stage][4096], 1 KiB aligned
+  uint8_t* scales = codes + kLmWarps * NS * kTcStageCodes;             // [warp][stage][512]
+  uint8_t* x16 = scales + kLmWarps * NS * kTcStageScales;              // [8][XSTR] f16, B-fragment order
+  float* part = reinterpret_cast<float*>(x16 + kLmMaxTokens * XSTR);   // [TPI groups][2][KP][128]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int NS = p.stages, G = gridDim.x, c = blockIdx.x;
-  const size_t stb = lm_stage_bytes(D);
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + NS * stb);
-  const int row0 = static_cast<int>(static_cast<long long>(c) * p.V / G);
-  const int row1 = static_cast<int>(static_cast<long long>(c + 1) * p.V / G);
-  const int n_st = (row1 - row0 + kLmRows - 1) / kLmRows;
+  const int n_tiles = (p.V + 15) / 16, G = gridDim.x, c = blockIdx.x;
+  const int tile0 = static_cast<int>(static_cast<long long>(c) * n_tiles / G);
+  const int L = static_cast<int>(static_cast<long long>(c + 1) * n_tiles / G) - tile0;
+  const int kp = warp % KP, m = warp / KP;
+  const int n_q = L > m ? (L - 1 - m) / TPI + 1 : 0;  // this warp's stages: local tile m + TPI*q, part kp
+  uint64_t* wb = bars + warp * NS;
 
-  auto issue = [&](int i) {  // stage i of this CTA's rows into slot i % NS
-    const int r = row0 + i * kLmRows, n = min(kLmRows, row1 - r);
-    uint8_t* st = smem + (i % NS) * stb;
-    mbar_arrive_expect_tx(&full[i % NS], n * (ROWC + ROWS));
-    bulk_g2s(st, p.codes + static_cast<long long>(r) * ROWC, n * ROWC, &full[i % NS]);
-    bulk_g2s(st + STC, p.scales + static_cast<long long>(r) * ROWS, n * ROWS, &full[i % NS]);
+  auto issue = [&](int q) {
+    const int slot = q % NS, y = (tile0 + m + TPI * q) * 16;
+    uint8_t* cs = codes + (warp * NS + slot) * kTcStageCodes;
+    mbar_arrive_expect_tx(&wb[slot], kTcStageCodes + kTcStageScales);
+    tma_load_2d(cs, &maps.codes, kp * 256, y, &wb[slot]);
+    tma_load_2d(cs + 2048, &maps.codes, kp * 256 + 128, y, &wb[slot]);
+    tma_load_2d(scales + (warp * NS + slot) * kTcStageScales, &maps.scales, kp * 32, y, &wb[slot]);
   };
   if (tid == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kLmWarps);
-    }
+    for (int i = 0; i < kLmWarps * NS; ++i) mbar_init(&bars[i], 1);
     fence_barrier_init();
-    for (int i = 0; i < NS && i < n_st; ++i) issue(i);  // weights do not depend on earlier kernels
   }
+  if (tid == 0) s_fail = 0;
+  __syncthreads();
+  int issued = 0;
+  if (lane == 0)  // weights do not depend on earlier kernels
+    for (; issued < NS && issued < n_q; ++issued) issue(issued);
+  issued = __shfl_sync(0xffffffffu, issued, 0);
   pdl_wait();
-  // the tokens' x, scaled per token by a power of two into f16 (warp t: token t)
-  if (warp < T) {
-    const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(warp) * D);
+  // the tokens' x as f16 after a power-of-two scale each (warp t: token t);
+  // rows of unused columns are zero
+  if (warp < kLmMaxTokens) {
+    const int t = warp;
+    const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t) * D);
     float amax = 0.f;
-    for (int i = lane; i < D / 8; i += 32) {
-      const uint4 v = __ldcg(src + i);
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    if (t < p.T) {
+      for (int i = lane; i < D / 8; i += 32) {
+        const uint4 v = __ldcg(src + i);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_f32(w4[q] & 0xFFFFu)), fabsf(__uint_as_float(w4[q] & 0xFFFF0000u))));
+        for (int q = 0; q < 4; ++q)
+          amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_f32(w4[q] & 0xFFFFu)), fabsf(__uint_as_float(w4[q] & 0xFFFF0000u))));
+      }
     }
     amax = segment_max<32>(amax);
     const float sg = pow2_scale_for(amax);
-    if (lane == 0) s_f[warp] = __ldg(p.tscale) / sg;
+    if (lane == 0) s_f[t] = (t < p.T) ? __ldg(p.tscale) / sg : 0.f;
     for (int i = lane; i < D / 8; i += 32) {
-      const uint4 v = __ldcg(src + i);
-      uint4 o;
-      o.x = pack_f16x2(bf16_bits_to_f32(v.x & 0xFFFFu) * sg, __uint_as_float(v.x & 0xFFFF0000u) * sg);
-      o.y = pack_f16x2(bf16_bits_to_f32(v.y & 0xFFFFu) * sg, __uint_as_float(v.y & 0xFFFF0000u) * sg);
-      o.z = pack_f16x2(bf16_bits_to_f32(v.z & 0xFFFFu) * sg, __uint_as_float(v.z & 0xFFFF0000u) * sg);
-      o.w = pack_f16x2(bf16_bits_to_f32(v.w & 0xFFFFu) * sg, __uint_as_float(v.w & 0xFFFF0000u) * sg);
-      *reinterpret_cast<uint4*>(xs + static_cast<size_t>(warp) * D + 8 * i) = o;
+      uint4 o = make_uint4(0u, 0u, 0u, 0u);
+      if (t < p.T) {
+        const uint4 v = __ldcg(src + i);
+        o.x = pack_f16x2(bf16_bits_to_f32(v.x & 0xFFFFu) * sg, __uint_as_float(v.x & 0xFFFF0000u) * sg);
+        o.y = pack_f16x2(bf16_bits_to_f32(v.y & 0xFFFFu) * sg, __uint_as_float(v.y & 0xFFFF0000u) * sg);
+        o.z = pack_f16x2(bf16_bits_to_f32(v.z & 0xFFFFu) * sg, __uint_as_float(v.z & 0xFFFF0000u) * sg);
+        o.w = pack_f16x2(bf16_bits_to_f32(v.w & 0xFFFFu) * sg, __uint_as_float(v.w & 0xFFFF0000u) * sg);
+      }
+      // elements 8i + 2j, +1 (j = 0..3) sit 16 bytes apart in the B-fragment order
+      uint8_t* b = x16 + static_cast<size_t>(t) * XSTR + tc_b_offset(8 * i);
+      *reinterpret_cast<uint32_t*>(b) = o.x;
+      *reinterpret_cast<uint32_t*>(b + 16) = o.y;
+      *reinterpret_cast<uint32_t*>(b + 32) = o.z;
+      *reinterpret_cast<uint32_t*>(b + 48) = o.w;
     }
   }
   __syncthreads();
   pdl_trigger();
-  // x of the lane's vectors v = lane + 32 j (lanes beyond VPR repeat)
-  const int xl = lane % VPR;
-  uint32_t xr[T][XV][16];
+  float f[2];
+  const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-  for (int t = 0; t < T; ++t)
-#pragma unroll
-    for (int j = 0; j < XV; ++j)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 v = lds128(xs + static_cast<size_t>(t) * D + (xl + 32 * j) * 32 + 8 * q);
-        xr[t][j][4 * q + 0] = v.x;
-        xr[t][j][4 * q + 1] = v.y;
-        xr[t][j][4 * q + 2] = v.z;
-        xr[t][j][4 * q + 3] = v.w;
-      }
-  float f[T];
-#pragma unroll
-  for (int t = 0; t < T; ++t) f[t] = s_f[t];
+  for (int h = 0; h < 2; ++h) f[h] = s_f[2 * t4 + h];
+  const uint8_t* xrow = x16 + static_cast<size_t>(lane & 7) * XSTR;
 
+  // The KP warps of a tile group take the same steps in lockstep (a named
+  // barrier per step, so no warp runs ahead of its group); step q's partial
+  // sums use buffer q & 1 of the group, which the group's part-0 warp adds in
+  // part order after the barrier; the next step's barrier orders that read
+  // before the buffer is written again two steps later. A warp whose wait
+  // gives up keeps taking every step and barrier (later waits are skipped)
+  // so that its group never waits on it.
   bool ok = true;
-  int i = 0;
-  for (; i < n_st && ok; ++i) {
-    const int slot = i % NS;
-    if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], (i / NS) & 1, p.status))) {
-      ok = false;
-      break;
-    }
-    const int r = row0 + i * kLmRows + warp;
-    if (r < row1) {
-      const uint8_t* st = smem + slot * stb;
-      float acc[T];
-#pragma unroll
-      for (int t = 0; t < T; ++t) acc[t] = 0.f;
-      if (lane < VPR) {
-#pragma unroll
-        for (int j = 0; j < XV; ++j) {
-          const int v = xl + 32 * j;
-          const uint4 cv = lds128(st + warp * ROWC + 16 * v);
-          const uint32_t s2 = *reinterpret_cast<const uint16_t*>(st + STC + warp * ROWS + 2 * v);
-#pragma unroll
-          for (int t = 0; t < T; ++t) dot32_strided<1, 16>(cv, s2, xr[t][j], &acc[t]);
-        }
-      }
-#pragma unroll
-      for (int t = 0; t < T; ++t) {
-        const float s = warp_sum(acc[t]);
-        if (lane == 0) p.out[static_cast<size_t>(t) * p.V + r] = s * f[t];
-      }
-    }
-    __syncwarp();
-    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&empty[slot])) : "memory");
-    // the producer refills the slot once every warp is done with it
-    if (tid == 0 && i + NS < n_st) {
-      if (!mbar_wait(&empty[slot], (i / NS) & 1, p.status)) {
+  int q_fail = n_q;  // stages [q_fail, issued) may still be in flight after a failure
+  float* gp = part + static_cast<size_t>(m) * 2 * KP * 128;  // [2][KP][128]
+  for (int q = 0; q < n_q; ++q) {
+    const int slot = q % NS;
+    const int fail_now = __shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s_fail), 0);
+    if (ok && fail_now == 0) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&wb[slot], (q / NS) & 1, p.status))) {
         ok = false;
-      } else {
+        q_fail = q;
+        if (lane == 0) s_fail = 1;
+      }
+    } else if (ok) {
+      ok = false;  // another warp's wait gave up: skip the rest
+      q_fail = q;
+    }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+    if (ok) {
+      const uint8_t* cs = codes + (warp * NS + slot) * kTcStageCodes;
+      const uint8_t* ss = scales + (warp * NS + slot) * kTcStageScales;
+#pragma unroll 2
+      for (int seg = 0; seg < 4; ++seg) {
+        uint32_t b[16];
+        tc_load_b(xrow, (kp * 4 + seg) * 256, lane, b);
+        const uint4 ca = lds128(tc_code_chunk(cs, g, seg, t4)), cb = lds128(tc_code_chunk(cs, g + 8, seg, t4));
+        const uint32_t sa = *reinterpret_cast<const uint16_t*>(ss + g * 32 + seg * 8 + 2 * t4);
+        const uint32_t sb = *reinterpret_cast<const uint16_t*>(ss + (g + 8) * 32 + seg * 8 + 2 * t4);
+        tc_segment(acc, acc1, ca, cb, sa, sb, b);
+      }
+      __syncwarp();
+      if (q + NS < n_q && lane == 0) {  // the slot is read: refill it
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue(i + NS);
+        issue(q + NS);
+        ++issued;
+      }
+    }
+    float* pp = gp + (q & 1) * KP * 128;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) pp[kp * 128 + r * 32 + lane] = acc[r] + acc1[r];
+    if constexpr (KP > 1) asm volatile("bar.sync %0, %1;" ::"r"(m + 1), "r"(32 * KP) : "memory");
+    else __syncwarp();
+    if (kp == 0) {
+      const int row_base = (tile0 + m + TPI * q) * 16;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        float v = 0.f;
+#pragma unroll
+        for (int k2 = 0; k2 < KP; ++k2) v += pp[k2 * 128 + r * 32 + lane];
+        const int row = row_base + g + 8 * (r >> 1), col = 2 * t4 + (r & 1);
+        if (ok && col < p.T && row < p.V) p.out[static_cast<size_t>(col) * p.V + row] = v * f[r & 1];
       }
     }
   }
   // copies still in flight after a failed wait land before the CTA exits
-  if (!ok && tid == 0) {
-    const int issued = min(n_st, i + NS);
-    for (int k = i; k < issued; ++k) mbar_wait(&full[k % NS], (k / NS) & 1, p.status);
-  }
+  if (!ok && lane == 0)
+    for (int k2 = q_fail; k2 < issued; ++k2) mbar_wait(&wb[k2 % NS], (k2 / NS) & 1, p.status);
 }
 
-template <int D, int T>
-cudaError_t launch_dt(const LmHeadParams& p, cudaStream_t st) {
-  auto kern = k_lm_head<D, T>;
-  const size_t smem = lm_smem_bytes(D, p.stages);
+template <int D>
+cudaError_t launch_d(const LmHeadParams& p, const LmMaps& maps, cudaStream_t st) {
+  auto kern = k_lm_head<D>;
+  const size_t smem = lm_smem_bytes(D);
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -151,22 +174,17 @@ cudaError_t launch_dt(const LmHeadParams& p, cudaStream_t st) {
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
-}
-
-template <int D>
-cudaError_t launch_d(const LmHeadParams& p, cudaStream_t st) {
-  return p.T == 1 ? launch_dt<D, 1>(p, st) : launch_dt<D, 2>(p, st);
+  return cudaLaunchKernelEx(&cfg, kern, p, maps);
 }
 
 }  // namespace
 
-cudaError_t lm_head_launch(int d, const LmHeadParams& p, cudaStream_t st) {
+cudaError_t lm_head_launch(int d, const LmHeadParams& p, const LmMaps& maps, cudaStream_t st) {
   switch (d) {
-    case 512: return launch_d<512>(p, st);
-    case 1024: return launch_d<1024>(p, st);
-    case 2048: return launch_d<2048>(p, st);
-    default: return launch_dt<4096, 1>(p, st);
+    case 512: return launch_d<512>(p, maps, st);
+    case 1024: return launch_d<1024>(p, maps, st);
+    case 2048: return launch_d<2048>(p, maps, st);
+    default: return launch_d<4096>(p, maps, st);
   }
 }
 

@@ -10,9 +10,9 @@ namespace {
 // ----------------------------------------------------------------- batch-1 cluster kernel (host)
 // Whether the batch-1 cluster kernel serves this shape on the current device:
 // its shared memory fits and at least one 16-CTA cluster can be resident.
-template <int D, int I>
+template <int D, int I, int NE>
 bool tok1_ready(int E, size_t* smem_out) {
-  auto kern = k_tok1<D, I>;
+  auto kern = k_tok1<D, I, NE>;
   static std::mutex mu;
   static int cache_dev[64];
   static int cache_E[64];
@@ -33,8 +33,10 @@ bool tok1_ready(int E, size_t* smem_out) {
       smem + fa.sharedSizeBytes <= static_cast<size_t>(optin) &&
       cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
           cudaSuccess &&
+      // the limit is the function's, shared by every E this instantiation
+      // serves: the device's whole opt-in budget
       cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) == cudaSuccess) {
+                           optin - static_cast<int>(fa.sharedSizeBytes)) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kTok1Cluster);
     cfg.blockDim = dim3(kTok1Warps * 32);
@@ -59,7 +61,7 @@ bool tok1_ready(int E, size_t* smem_out) {
   return ok;
 }
 
-template <int D, int I>
+template <int D, int I, int NE>
 cudaError_t launch_tok1_di(const Tok1Params& t, size_t smem, bool pdl, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((t.k + t.S) * kTok1Cluster);
@@ -75,30 +77,30 @@ cudaError_t launch_tok1_di(const Tok1Params& t, size_t smem, bool pdl, cudaStrea
   at[1].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, k_tok1<D, I>, t);
+  return cudaLaunchKernelEx(&cfg, k_tok1<D, I, NE>, t);
 }
 
-// Dispatch over (d, inter): `ready` checks the shape, else launches.
+// Dispatch over (d, inter, E class): `ready` checks the shape, else launches.
+template <int D, int I>
+bool tok1_dispatch_e(int E, bool launch, const Tok1Params* t, bool pdl, cudaStream_t st, cudaError_t* err) {
+  size_t smem = 0;
+  if (E <= 256) {
+    if (!tok1_ready<D, I, 8>(E, &smem)) return false;
+    if (launch) *err = launch_tok1_di<D, I, 8>(*t, smem, pdl, st);
+  } else {
+    if (!tok1_ready<D, I, kMaxExperts / 32>(E, &smem)) return false;
+    if (launch) *err = launch_tok1_di<D, I, kMaxExperts / 32>(*t, smem, pdl, st);
+  }
+  return true;
+}
+
 template <int D>
 bool tok1_dispatch_i(int I, int E, bool launch, const Tok1Params* t, bool pdl, cudaStream_t st, cudaError_t* err) {
-  size_t smem = 0;
   switch (I) {
-    case 128:
-      if (!tok1_ready<D, 128>(E, &smem)) return false;
-      if (launch) *err = launch_tok1_di<D, 128>(*t, smem, pdl, st);
-      return true;
-    case 256:
-      if (!tok1_ready<D, 256>(E, &smem)) return false;
-      if (launch) *err = launch_tok1_di<D, 256>(*t, smem, pdl, st);
-      return true;
-    case 512:
-      if (!tok1_ready<D, 512>(E, &smem)) return false;
-      if (launch) *err = launch_tok1_di<D, 512>(*t, smem, pdl, st);
-      return true;
-    default:
-      if (!tok1_ready<D, 1024>(E, &smem)) return false;
-      if (launch) *err = launch_tok1_di<D, 1024>(*t, smem, pdl, st);
-      return true;
+    case 128: return tok1_dispatch_e<D, 128>(E, launch, t, pdl, st, err);
+    case 256: return tok1_dispatch_e<D, 256>(E, launch, t, pdl, st, err);
+    case 512: return tok1_dispatch_e<D, 512>(E, launch, t, pdl, st, err);
+    default: return tok1_dispatch_e<D, 1024>(E, launch, t, pdl, st, err);
   }
 }
 

@@ -57,7 +57,9 @@ struct Tok1Params {
 
 // Dynamic shared-memory bytes of k_tok1: the larger of the router-row slice and
 // the expert slice (they share the region), then the cluster's logits and h,
-// then the token's x (bf16).
+// the token's x (bf16), x as f16 and h as f16 in the lane-interleaved order
+// (element i of 32-element vector v at chunk (i % 32) / 8 * V + v, so the
+// lanes of a warp read consecutive 16-byte chunks).
 __host__ __device__ constexpr size_t tok1_region_bytes(int D, int I, int E) {
   const size_t rows = static_cast<size_t>((E + kTok1Cluster - 1) / kTok1Cluster) * D * 2;
   const size_t ex = static_cast<size_t>(I / kTok1Cluster) * (D + D / 8) +
@@ -66,7 +68,7 @@ __host__ __device__ constexpr size_t tok1_region_bytes(int D, int I, int E) {
 }
 __host__ __device__ constexpr size_t tok1_smem_bytes(int D, int I, int E) {
   return tok1_region_bytes(D, I, E) + ((static_cast<size_t>(E) * 4 + 127) & ~static_cast<size_t>(127)) +
-         static_cast<size_t>(I) * 4 + static_cast<size_t>(D) * 2;
+         static_cast<size_t>(I) * 4 + static_cast<size_t>(D) * 4 + static_cast<size_t>(I) * 2;
 }
 
 __device__ __forceinline__ unsigned cluster_rank() {
@@ -89,7 +91,54 @@ __device__ __forceinline__ void st_cluster_f32(float* local, unsigned rank, floa
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
 }
 
-template <int D, int I>
+// Top-k of one token's E <= 32*NE logits by one warp, in k rolled rounds
+// (every phase of this kernel runs once per launch, so its code size, not its
+// loop overhead, is what costs: an unrolled sorting network would be fetched
+// from L2 at every launch). Lane l holds the order-preserving codes of
+// experts l + 32 i (0 = absent). A round takes each lane's best (largest code,
+// the lowest i on ties), the warp maximum of those with redux.sync, then among
+// the lanes holding it the lowest expert index (a second redux over
+// 0xFFFFFFFF - e); the owner clears it. Ties go to the lower expert index,
+// -0 equals +0 (route_code). Gates: exp(l_j - l_max) / sum over the selected.
+template <int NE>
+__device__ __forceinline__ void topk_rounds(uint32_t (&code)[NE], int k, int* ids, float* gates, int lane) {
+  float my_val = 0.f, v0 = 0.f;
+  int my_sel = 0;
+#pragma unroll 1
+  for (int r = 0; r < k; ++r) {
+    uint32_t best = 0u;
+    int bi = 0;
+#pragma unroll
+    for (int i = 0; i < NE; ++i)
+      if (code[i] > best) {
+        best = code[i];
+        bi = i;
+      }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+    const uint32_t w = __reduce_max_sync(0xffffffffu, best == m ? 0xFFFFFFFFu - static_cast<uint32_t>(lane + 32 * bi) : 0u);
+    const int e = static_cast<int>(0xFFFFFFFFu - w);
+    if ((e & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i < NE; ++i)
+        if (i == (e >> 5)) code[i] = 0u;
+    }
+    const float v = route_code_value(m);
+    if (r == 0) v0 = v;
+    if (lane == r) {
+      my_val = v;
+      my_sel = e;
+    }
+  }
+  const float ex = (lane < k) ? __expf(my_val - v0) : 0.f;
+  const float sum = warp_sum(ex);
+  if (lane < k) {
+    ids[lane] = my_sel;
+    gates[lane] = ex * (1.f / sum);
+  }
+}
+
+// NE: logit slots per lane of the top-k (E <= 32 * NE), 8 or 16.
+template <int D, int I, int NE>
 __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   constexpr int CS = kTok1Cluster;
   constexpr int VPR = D / 32;                     // 16-byte code vectors per gate/up row
@@ -121,6 +170,9 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   float* s_logits = reinterpret_cast<float*>(smem + tok1_region_bytes(D, I, E));
   float* s_h = s_logits + ((E + 31) & ~31);
   const uint16_t* s_x = reinterpret_cast<const uint16_t*>(s_h + I);
+  uint16_t* x16 = const_cast<uint16_t*>(s_x) + D;  // f16, lane-interleaved
+  uint16_t* h16 = x16 + D;                         // f16, lane-interleaved
+  __shared__ float s_raw[kMaxExperts / kTok1Cluster], s_stat[4];
   uint8_t* gu_codes = region;                                   // [UPC][D]
   uint8_t* gu_scales = region + UPC * UNIT_C;                   // [UPC][D/8]
   uint8_t* dn_codes = gu_scales + UPC * UNIT_S;                 // [RPC][I/2]
@@ -175,94 +227,96 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
     bulk_g2s(const_cast<uint16_t*>(s_x), p.x, D * 2, bar_x);
   }
 
-  // ---- P1: x -> statistics, f16 registers (lane's vectors v = lane + 32 j, j < XV
-  // of a gate/up row; at D = 512 lanes 16..31 repeat lanes 0..15)
+  // ---- P1: the token's statistics (warp 0) and this CTA's router dots
+  // (other warps) from the bf16 copy; then x as f16 (power-of-two scale) in
+  // the lane-interleaved order, and each lane's x vectors v = lane + 32 j
+  // (j < XV) of a gate/up row in registers (at D = 512 lanes 16..31 repeat
+  // lanes 0..15). Shared memory is read once per CTA, conflict-free.
   bool ok = __all_sync(0xffffffffu, mbar_wait(bar_x, 0, p.status));
-  const int xl = lane % VPR;  // first x vector of this lane
-  uint32_t xr[XV][16];        // bf16 pairs, then f16 pairs scaled by sigma
-  float amax = 0.f, ss = 0.f;
+  if (!shared && r1 > r0 && !__all_sync(0xffffffffu, mbar_wait(bar_rows, 0, p.status))) ok = false;
+  if (warp == 0) {
+    float amax = 0.f, ss = 0.f;
+    for (int i = lane; i < D / 8; i += 32) {
+      const uint4 v = lds128(s_x + 8 * i);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int j = 0; j < XV; ++j) {
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(s_x) + (xl + 32 * j) * 64;
+      for (int q = 0; q < 4; ++q) {
+        const float a = bf16_bits_to_f32(w4[q] & 0xFFFFu), b = __uint_as_float(w4[q] & 0xFFFF0000u);
+        amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+        ss = fmaf(a, a, ss);
+        ss = fmaf(b, b, ss);
+      }
+    }
+    amax = segment_max<32>(amax);
+    ss = warp_sum(ss);
+    if (lane == 0) {
+      s_stat[0] = pow2_scale_for(amax);
+      s_stat[1] = p.input_norm ? 1.f / sqrtf(ss / static_cast<float>(D) + kRmsEps) : 1.f;
+    }
+  } else if (!shared && ok) {
+    // warp w >= 1: rows r0 + w - 1, + 15, ...; lane l reads the row's 16-byte
+    // vectors l + 32 i and the same vectors of x
+    for (int r = r0 + warp - 1; r < r1; r += kTok1Warps - 1) {
+      const uint8_t* row = region + static_cast<size_t>(r - r0) * D * 2;
+      float a = 0.f;
+#pragma unroll 4
+      for (int i = lane; i < D / 8; i += 32) {
+        const uint4 wv = lds128(row + 16 * i), xv = lds128(s_x + 8 * i);
+        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w}, xx[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          a = fmaf(bf16_bits_to_f32(ww[q] & 0xFFFFu), bf16_bits_to_f32(xx[q] & 0xFFFFu), a);
+          a = fmaf(__uint_as_float(ww[q] & 0xFFFF0000u), __uint_as_float(xx[q] & 0xFFFF0000u), a);
+        }
+      }
+      a = warp_sum(a);
+      if (lane == 0) s_raw[r - r0] = a;
+    }
+  }
+  if (!ok && lane == 0) s_fail = 1;
+  __syncthreads();
+  const float sigma = s_stat[0], irms = s_stat[1];
+  const float fx = irms / sigma;  // dot(q, x*sigma) * fx = dot(q, x) * irms
+  // logits into every CTA of the cluster (each must be running: the cluster
+  // arrival of P0 is waited for here)
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  if (!shared && !s_fail)
+    for (int i = tid; i < (r1 - r0) * CS; i += blockDim.x)
+      st_cluster_f32(s_logits + r0 + i / CS, static_cast<unsigned>(i % CS), s_raw[i / CS] * irms);
+  for (int i = tid; i < D / 8; i += blockDim.x) {
+    const uint4 v = lds128(s_x + 8 * i);
+    uint4 o;
+    o.x = bf16x2_to_f16x2_scaled(v.x, sigma);
+    o.y = bf16x2_to_f16x2_scaled(v.y, sigma);
+    o.z = bf16x2_to_f16x2_scaled(v.z, sigma);
+    o.w = bf16x2_to_f16x2_scaled(v.w, sigma);
+    *reinterpret_cast<uint4*>(x16 + (((i & 3) * VPR) + (i >> 2)) * 8) = o;  // vector i/4, chunk i%4
+  }
+  __syncthreads();
+  const int xl = lane % VPR;  // first x vector of this lane
+  uint32_t xr[XV][16];
+#pragma unroll
+  for (int j = 0; j < XV; ++j)
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const uint4 v = lds128(src + 16 * q);
+      const uint4 v = lds128(x16 + ((q * VPR) + xl + 32 * j) * 8);
       xr[j][4 * q + 0] = v.x;
       xr[j][4 * q + 1] = v.y;
       xr[j][4 * q + 2] = v.z;
       xr[j][4 * q + 3] = v.w;
     }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float a = bf16_bits_to_f32(xr[j][i] & 0xFFFFu), b = __uint_as_float(xr[j][i] & 0xFFFF0000u);
-      amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
-      ss = fmaf(a, a, ss);
-      ss = fmaf(b, b, ss);
-    }
-  }
-  if (lane >= VPR) ss = 0.f;  // repeated lanes count once
-  amax = segment_max<32>(amax);
-  ss = warp_sum(ss);
-  const float irms = p.input_norm ? 1.f / sqrtf(ss / static_cast<float>(D) + kRmsEps) : 1.f;
-  const float sigma = pow2_scale_for(amax);
-  const float fx = irms / sigma;  // dot(q, x*sigma) * fx = dot(q, x) * irms
-
-  // router rows of this CTA: warp w takes rows r0 + w, r0 + w + 16, ...; the
-  // lane covers the same elements as its x registers
-  // (warp-uniform outcomes: the reductions below need every lane)
-  if (!shared && r1 > r0 && !__all_sync(0xffffffffu, mbar_wait(bar_rows, 0, p.status))) ok = false;
-  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-  if (!shared) {
-    for (int r = r0 + warp; r < r1 && ok; r += kTok1Warps) {
-      const uint8_t* row = region + static_cast<size_t>(r - r0) * D * 2;
-      float a = 0.f;
-      if (lane < VPR) {
-#pragma unroll
-        for (int j = 0; j < XV; ++j) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 wv = lds128(row + (xl + 32 * j) * 64 + 16 * q);
-            const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint32_t xx = xr[j][4 * q + i];
-              a = fmaf(bf16_bits_to_f32(ww[i] & 0xFFFFu), bf16_bits_to_f32(xx & 0xFFFFu), a);
-              a = fmaf(__uint_as_float(ww[i] & 0xFFFF0000u), __uint_as_float(xx & 0xFFFF0000u), a);
-            }
-          }
-        }
-      }
-      const float logit = warp_sum(a) * irms;
-      if (lane < CS) st_cluster_f32(s_logits + r, static_cast<unsigned>(lane), logit);
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < XV; ++j)
-#pragma unroll
-    for (int i = 0; i < 16; ++i) xr[j][i] = bf16x2_to_f16x2_scaled(xr[j][i], sigma);
-  if (!ok && lane == 0) s_fail = 1;
 
   // ---- P2: every CTA of the cluster holds all E logits; select, then issue
   cluster_sync_all();
   if (s_fail) ok = false;
   if (!shared && warp == 0 && ok) {
-    if (E <= 256) {
-      uint32_t code[8];
+    uint32_t code[NE];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int e = lane + 32 * i;
-        code[i] = (e < E) ? max(route_code(s_logits[e]), 1u) : 0u;
-      }
-      topk_select<8>(code, k, s_ids, s_gates, lane);
-    } else {
-      uint32_t code[kMaxExperts / 32];
-#pragma unroll
-      for (int i = 0; i < kMaxExperts / 32; ++i) {
-        const int e = lane + 32 * i;
-        code[i] = (e < E) ? max(route_code(s_logits[e]), 1u) : 0u;
-      }
-      topk_select<kMaxExperts / 32>(code, k, s_ids, s_gates, lane);
+    for (int i = 0; i < NE; ++i) {
+      const int e = lane + 32 * i;
+      code[i] = (e < E) ? max(route_code(s_logits[e]), 1u) : 0u;
     }
+    topk_rounds<NE>(code, k, s_ids, s_gates, lane);
     __syncwarp();
     // the router rows were read before the cluster barrier; order those
     // generic reads before the copies that overwrite them
@@ -329,18 +383,36 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
 
   // ---- P4: down rows of this CTA's block against the whole h
   float* part = p.partial + static_cast<size_t>(slot) * D + static_cast<size_t>(rank) * RPC;
-  if (ok && !__all_sync(0xffffffffu, mbar_wait(bar_down, 0, p.status))) ok = false;
-  if (ok) {
-    // h slice of this lane (elements 32 * (lane % LPR) ..), scaled by a power
-    // of two into f16; every warp derives the same scale from the whole h
+  // h as f16 with a power-of-two scale, once per CTA in the lane-interleaved
+  // order; each lane then holds the 32 elements of vector lane % LPR
+  if (warp == 0) {
     float hm = 0.f;
     for (int i = lane; i < I; i += 32) hm = fmaxf(hm, fabsf(s_h[i]));
     hm = segment_max<32>(hm);
-    const float hs = pow2_scale_for(hm);
-    const int hv0 = (lane % LPR) * 32;
+    if (lane == 0) s_stat[2] = pow2_scale_for(hm);
+  }
+  __syncthreads();
+  const float hs = s_stat[2];
+  for (int i = tid; i < I / 8; i += blockDim.x) {
+    uint4 o;
+    o.x = pack_f16x2(s_h[8 * i + 0] * hs, s_h[8 * i + 1] * hs);
+    o.y = pack_f16x2(s_h[8 * i + 2] * hs, s_h[8 * i + 3] * hs);
+    o.z = pack_f16x2(s_h[8 * i + 4] * hs, s_h[8 * i + 5] * hs);
+    o.w = pack_f16x2(s_h[8 * i + 6] * hs, s_h[8 * i + 7] * hs);
+    *reinterpret_cast<uint4*>(h16 + (((i & 3) * LPR) + (i >> 2)) * 8) = o;
+  }
+  __syncthreads();
+  if (ok && !__all_sync(0xffffffffu, mbar_wait(bar_down, 0, p.status))) ok = false;
+  if (ok) {
     uint32_t hr[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) hr[i] = pack_f16x2(s_h[hv0 + 2 * i] * hs, s_h[hv0 + 2 * i + 1] * hs);
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = lds128(h16 + ((q * LPR) + lane % LPR) * 8);
+      hr[4 * q + 0] = v.x;
+      hr[4 * q + 1] = v.y;
+      hr[4 * q + 2] = v.z;
+      hr[4 * q + 3] = v.w;
+    }
     const float ys = sd * gate / hs;
     for (int r = warp * RPS + lane / LPR; r < RPC; r += kTok1Warps * RPS) {
       const uint4 cv = lds128(dn_codes + r * DROW_C + 16 * (lane % LPR));

@@ -2,8 +2,8 @@
 against the oracle: packed planes bit-exact with the oracle's quantiser, and
 logits within rel L2 <= 5e-3, max-abs <= 2e-2 * rms on all rows of a small
 head and on sampled rows (plus the first and last) of the full-size head,
-at one and two tokens; shape edges (rows not a multiple of the stage, one
-row); wide-range x."""
+at one, two and eight tokens; shape edges (rows not a multiple of the 16-row
+tile, one row); wide-range x."""
 import numpy as np
 import pytest
 import torch
@@ -47,8 +47,8 @@ def _check(got, ref, what):
         assert np.abs(d).max() <= 2e-2 * np.sqrt(np.mean(ref[t] ** 2)), what
 
 
-@pytest.mark.parametrize("rows,cols,T", [(1, 512, 1), (37, 512, 2), (5000, 1024, 2), (2367, 2048, 1),
-                                         (300, 4096, 1)])
+@pytest.mark.parametrize("rows,cols,T", [(1, 512, 1), (37, 512, 2), (5000, 1024, 8), (2367, 2048, 1),
+                                         (2367, 2048, 5), (300, 4096, 1), (300, 4096, 8)])
 def test_small_heads_all_rows(rows, cols, T):
     ws = _ws()
     rng = np.random.default_rng(rows + cols)
@@ -61,7 +61,7 @@ def test_small_heads_all_rows(rows, cols, T):
     _check(_run(codes, scales, ts, x, rows, cols, ws), oracle.dense_gemv(m, x), f"{rows}x{cols} T={T}")
 
 
-@pytest.mark.parametrize("T", [1, 2])
+@pytest.mark.parametrize("T", [1, 2, 8])
 def test_flint_head_sampled_rows(T):
     rows, cols = VOCAB, 2048
     ws = _ws()
@@ -99,8 +99,8 @@ def test_head_rejects_bad_shapes():
     ws = _ws()
     z = torch.zeros(64, dtype=torch.uint8, device="cuda")
     f = torch.zeros(64, dtype=torch.float32, device="cuda")
-    x = torch.zeros((3, 2048), dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros((9, 2048), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(fm.FlintError):
-        fm.flint_lm_head(x, 3, z, z, f, 16, 2048, f, ws)   # three tokens
+        fm.flint_lm_head(x, 9, z, z, f, 16, 2048, f, ws)   # nine tokens
     with pytest.raises(fm.FlintError):
         fm.flint_lm_head(x, 1, z, z, f, 16, 1000, f, ws)   # cols not supported

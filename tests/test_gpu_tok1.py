@@ -111,6 +111,21 @@ def test_cluster_kernel_shape_variants(d, inter, E, k, S):
         _check(layer, x, wr, what=f"shape {d},{inter},{E},{k},{S} seed {s}")
 
 
+def test_cluster_kernel_after_other_expert_counts():
+    # one kernel instantiation serves every E up to 256 (and another up to
+    # 512): calls at E = 13, then 256, then 13 again at the same (d, inter)
+    # must all launch (the shared-memory limit is the function's, not the
+    # first call's)
+    for E in (13, 256, 13, 40):
+        w = synth.Workload("var", d=2048, inter=512, E=E, k=6, S=1, T=1)
+        layer = GpuLayer(w, seed=E + 1, max_tokens=1, keep_f32=False)
+        x = synth.x_bits(E + 3, 1, 2048)
+        wr = synth.to_bf16_bits(np.random.default_rng(E + 3).standard_normal((E, 2048)) * 0.02)
+        _check(layer, x, wr, what=f"E={E}")
+        del layer
+        torch.cuda.empty_cache()
+
+
 def test_cluster_kernel_refuses_shapes_it_cannot_hold():
     # d=4096, inter=1024: a CTA's slice of one expert is 432 KB, above the
     # shared memory of an SM; the forced variant is refused, AUTO falls back
