@@ -122,13 +122,18 @@ typedef enum flint_layer_variant {
                              2..8 tokens: the persistent kernel's tensor-core loops */
   FLINT_LAYER_FMA = 1,    /* persistent kernel, CUDA-core dot products (fma.rn.f32.f16) */
   FLINT_LAYER_MMA = 2,    /* persistent kernel, register-fragment mma.sync m16n8k16 */
-  FLINT_LAYER_CLUSTER = 3 /* one token only: one 16-CTA cluster per selected expert and
-                             one for the shared expert; routing, the SwiGLU exchange
-                             and the down rows stay inside a cluster (distributed
-                             shared memory), and the last CTA to finish a block of
-                             output rows sums the experts' gated partials in slot
-                             order. FLINT_ERR_UNSUPPORTED_SHAPE if the shape does
-                             not fit it on the device */
+  FLINT_LAYER_CLUSTER = 3 /* 16-CTA cluster kernels, NVFP4 weights. One token: one
+                             cluster per selected expert and one for the shared
+                             expert. 2..8 tokens: persistent clusters that each
+                             route the batch and take the active experts in turn
+                             (register-fragment mma.sync, d in {512, 1024, 2048},
+                             inter in {256, 512, 1024}, E <= 256). Routing, the
+                             SwiGLU exchange and the down rows stay inside a
+                             cluster (distributed shared memory), and the last CTA
+                             to finish a block of output rows sums the experts'
+                             gated partials in slot order. More than 8 tokens, or a
+                             shape that does not fit on the device:
+                             FLINT_ERR_UNSUPPORTED_SHAPE */
 } flint_layer_variant;
 
 typedef struct flint_moe_options {

@@ -14,6 +14,7 @@
 #include "fused_layer.cuh"
 #include "mma_path.cuh"
 #include "tok1.cuh"
+#include "tokn.cuh"
 #include "lmhead.cuh"
 
 #include <cudaTypedefs.h>
@@ -439,8 +440,8 @@ constexpr size_t kCtrlBytes = 1024;
 // Workspace carve-up for calls of up to maxT tokens. The first kCtrlBytes hold
 // the control block: the status word (byte 0), the router's arrival counter
 // (byte 4, left at zero by every call), the persistent layer kernel's launch
-// generation (byte 8) and the batch-1 cluster kernel's per-row-block arrival
-// counters (bytes 64..127, left at zero by every call); the rest is reserved. The tagged regions start
+// generation (byte 8) and the cluster kernels' per-row-block arrival counters
+// (bytes 64..127, left at zero by every call); the rest is reserved. The tagged regions start
 // with a tag of 0, which no launch uses. flint_moe_workspace_init zeroes the
 // whole workspace.
 // Regions of the tensor-core path are laid out only when `mma` (the call takes
@@ -459,8 +460,8 @@ WsLayout ws_layout(const Dims& s, int maxT, bool mma) {
   o += al256(sizeof(unsigned long long) * kLogitReplicas * static_cast<size_t>(kFusedMaxTokens) * s.E);
   w.htag = o;
   o += al256(sizeof(unsigned long long) * static_cast<size_t>(kFusedMaxTokens) * (s.k + s.S) * s.I);
-  w.tok1_part = o;  // the batch-1 cluster kernel's gated partial outputs [k+S][d]
-  o += al256(sizeof(float) * static_cast<size_t>(s.k + s.S) * s.d);
+  w.tok1_part = o;  // the cluster kernels' gated partial outputs [min(T, 8) * (k+S)][d]
+  o += al256(sizeof(float) * static_cast<size_t>(maxT < kTnMaxTokens ? maxT : kTnMaxTokens) * (s.k + s.S) * s.d);
   w.amax = o;
   o += al256(sizeof(float) * (s.E + s.S) * 3);
   w.desc = o;
@@ -880,6 +881,38 @@ int fused_maps(FusedMaps* m, const Dims& s, const flint_moe_weights* wts) {
   return encode_map(&m->scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, wts->block_scales, sdims, sstr, sbox, false);
 }
 
+// Tensor maps of the batch-2..8 cluster kernel: gate/up codes [E+S][2*inter]
+// [d/2] bytes (box 128 x 16, 128-byte swizzle) and block scales [E+S][2*inter]
+// [d/16] (box 16 x 16); the down rows likewise from inter*d/2 code bytes and
+// inter*d/16 scale bytes past each expert's base: codes [E+S][d][inter/2],
+// scales [E+S][d][inter/16].
+int tokn_maps(TokNMaps* m, const Dims& s, const flint_moe_weights* wts) {
+  const cuuint64_t ne = static_cast<cuuint64_t>(s.E + s.S);
+  const cuuint64_t cexp = 3ull * s.I * s.d / 2, sexp = 3ull * s.I * s.d / 16;
+  const cuuint32_t cbox[3] = {128, 16, 1}, sbox[3] = {16, 16, 1};
+  const uint8_t* codes = static_cast<const uint8_t*>(wts->packed);
+  const uint8_t* scales = wts->block_scales;
+  {
+    const cuuint64_t cdims[3] = {static_cast<cuuint64_t>(s.d / 2), static_cast<cuuint64_t>(2 * s.I), ne};
+    const cuuint64_t cstr[2] = {static_cast<cuuint64_t>(s.d / 2), cexp};
+    int rc = encode_map(&m->gu_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, codes, cdims, cstr, cbox, true);
+    if (rc != FLINT_OK) return rc;
+    const cuuint64_t sdims[3] = {static_cast<cuuint64_t>(s.d / 16), static_cast<cuuint64_t>(2 * s.I), ne};
+    const cuuint64_t sstr[2] = {static_cast<cuuint64_t>(s.d / 16), sexp};
+    rc = encode_map(&m->gu_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, scales, sdims, sstr, sbox, false);
+    if (rc != FLINT_OK) return rc;
+  }
+  const cuuint64_t cdims[3] = {static_cast<cuuint64_t>(s.I / 2), static_cast<cuuint64_t>(s.d), ne};
+  const cuuint64_t cstr[2] = {static_cast<cuuint64_t>(s.I / 2), cexp};
+  int rc = encode_map(&m->dn_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, codes + static_cast<size_t>(s.I) * s.d, cdims,
+                      cstr, cbox, true);
+  if (rc != FLINT_OK) return rc;
+  const cuuint64_t sdims[3] = {static_cast<cuuint64_t>(s.I / 16), static_cast<cuuint64_t>(s.d), ne};
+  const cuuint64_t sstr[2] = {static_cast<cuuint64_t>(s.I / 16), sexp};
+  return encode_map(&m->dn_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, scales + static_cast<size_t>(s.I) * s.d / 8,
+                    sdims, sstr, sbox, false);
+}
+
 // Ring depths of the tensor-core kernels for a call of T tokens: B stages hold
 // the largest expert's rows (T rounded up to 16), four of them; NVFP4 keeps
 // four A stages and as many raw-weight stages as fit; bf16 weights as many A
@@ -1195,8 +1228,9 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
   const int variant = options ? options->layer_variant : FLINT_LAYER_AUTO;
   if (variant < FLINT_LAYER_AUTO || variant > FLINT_LAYER_CLUSTER)
     return fail(FLINT_ERR_INVALID_ARG, "layer_variant %d", variant);
-  if (variant == FLINT_LAYER_CLUSTER && (T != 1 || path == FLINT_PATH_MMA || s.wd != FLINT_W_NVFP4))
-    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "the cluster kernel takes one token and NVFP4 weights (T=%d)", T);
+  if (variant == FLINT_LAYER_CLUSTER && (T > kTnMaxTokens || path == FLINT_PATH_MMA || s.wd != FLINT_W_NVFP4))
+    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "the cluster kernels take 1..%d tokens and NVFP4 weights (T=%d)",
+                kTnMaxTokens, T);
   const bool use_gemv = (path == FLINT_PATH_GEMV) ||
                         (path == FLINT_PATH_AUTO && T < kMaxGemvTokens && s.wd == FLINT_W_NVFP4);
   if (use_gemv) {
@@ -1267,6 +1301,48 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
       cudaError_t e = cudaSuccess;
       tok1_dispatch(s.d, s.I, s.E, true, &t, pdl && !ev, st, &e);
       if (e != cudaSuccess) return cuda_fail(e, "k_tok1 launch");
+      if (ev) {
+        e = cudaEventRecord(ev[1], st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+      }
+      return FLINT_OK;
+    }
+    if (variant == FLINT_LAYER_CLUSTER)
+      return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "the cluster kernel does not fit this shape on this device");
+  }
+  if (T >= 2 && T <= kTnMaxTokens && !split && variant == FLINT_LAYER_CLUSTER) {
+    // 2..8 tokens, on request: persistent 16-CTA clusters taking the selected
+    // experts in turn (tokn.cuh), when the shape fits it on this device (AUTO
+    // keeps the persistent layer kernel, measured faster at these batches)
+    TokNParams t{};
+    t.x = x;
+    t.wr = router_w;
+    t.tscale = p.tscale;
+    t.residual = residual;
+    t.out = out;
+    t.status = p.status;
+    t.rb_count = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + lay.rb_count);
+    t.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + lay.tok1_part);
+    t.ids = p.ids;
+    t.gates = p.gates;
+    t.ids_out = p.ids_out;
+    t.gates_out = p.gates_out;
+    t.T = T;
+    t.E = s.E;
+    t.k = s.k;
+    t.S = s.S;
+    t.input_norm = p.input_norm;
+    if (tokn_dispatch(s.d, s.I, s.E, T, false, &t, nullptr, pdl, st, nullptr)) {
+      TokNMaps maps;
+      const int rc = tokn_maps(&maps, s, weights);
+      if (rc != FLINT_OK) return rc;
+      if (ev) {
+        cudaError_t e = cudaEventRecord(ev[0], st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+      }
+      cudaError_t e = cudaSuccess;
+      tokn_dispatch(s.d, s.I, s.E, T, true, &t, &maps, pdl && !ev, st, &e);
+      if (e != cudaSuccess) return cuda_fail(e, "k_tokn launch");
       if (ev) {
         e = cudaEventRecord(ev[1], st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");

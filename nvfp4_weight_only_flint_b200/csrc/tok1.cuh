@@ -32,7 +32,8 @@ namespace flint {
 
 constexpr int kTok1Cluster = 16;   // CTAs per cluster (non-portable size)
 constexpr int kTok1Warps = 16;
-constexpr int kTok1MaxChunks = 16;  // gate/up copy chunks (one per warp at most)
+constexpr int kTok1MaxChunks = 16;  // gate/up chunks (one per warp at most)
+constexpr int kTok1ChunksPerCopy = 1;  // gate/up chunks one bulk copy (and its barrier) covers
 
 struct Tok1Params {
   const uint16_t* x;         // [1][d] bf16
@@ -56,10 +57,11 @@ struct Tok1Params {
 };
 
 // Dynamic shared-memory bytes of k_tok1: the larger of the router-row slice and
-// the expert slice (they share the region), then the cluster's logits and h,
-// the token's x (bf16), x as f16 and h as f16 in the lane-interleaved order
-// (element i of 32-element vector v at chunk (i % 32) / 8 * V + v, so the
-// lanes of a warp read consecutive 16-byte chunks).
+// the expert slice (they share the region), then the cluster's logits, h
+// (fp32, lane-interleaved: unit u at (u % 32) * (I/32) + u / 32), the token's
+// x (bf16) and x as f16 in the lane-interleaved order (8-element chunk q of
+// 32-element vector v at q * (d/32) + v), so that the lanes of a warp read
+// consecutive words or 16-byte chunks.
 __host__ __device__ constexpr size_t tok1_region_bytes(int D, int I, int E) {
   const size_t rows = static_cast<size_t>((E + kTok1Cluster - 1) / kTok1Cluster) * D * 2;
   const size_t ex = static_cast<size_t>(I / kTok1Cluster) * (D + D / 8) +
@@ -68,7 +70,7 @@ __host__ __device__ constexpr size_t tok1_region_bytes(int D, int I, int E) {
 }
 __host__ __device__ constexpr size_t tok1_smem_bytes(int D, int I, int E) {
   return tok1_region_bytes(D, I, E) + ((static_cast<size_t>(E) * 4 + 127) & ~static_cast<size_t>(127)) +
-         static_cast<size_t>(I) * 4 + static_cast<size_t>(D) * 4 + static_cast<size_t>(I) * 2;
+         static_cast<size_t>(I) * 4 + static_cast<size_t>(D) * 4;
 }
 
 __device__ __forceinline__ unsigned cluster_rank() {
@@ -89,6 +91,12 @@ __device__ __forceinline__ void st_cluster_f32(float* local, unsigned rank, floa
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_u32(unsigned* local, unsigned rank, unsigned v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
 }
 
 // Top-k of one token's E <= 32*NE logits by one warp, in k rolled rounds
@@ -152,7 +160,9 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   constexpr int RPS = 32 / LPR;                   // down rows per warp step
   constexpr int UNIT_C = D, UNIT_S = D / 8;       // bytes of a unit's codes / scales
   constexpr int DROW_C = I / 2, DROW_S = I / 16;  // bytes of a down row's codes / scales
-  static_assert(NCH <= kTok1MaxChunks && NCH * CU == UPC, "chunking");
+  constexpr int CPC = kTok1ChunksPerCopy < NCH ? kTok1ChunksPerCopy : NCH;  // chunks per copy
+  constexpr int NCP = NCH / CPC;                  // gate/up copies
+  static_assert(NCH <= kTok1MaxChunks && NCH * CU == UPC && NCP * CPC == NCH, "chunking");
   static_assert(RPC % RPS == 0 || RPC < RPS, "down rows");
 
   extern __shared__ __align__(128) uint8_t smem[];
@@ -171,8 +181,6 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   float* s_h = s_logits + ((E + 31) & ~31);
   const uint16_t* s_x = reinterpret_cast<const uint16_t*>(s_h + I);
   uint16_t* x16 = const_cast<uint16_t*>(s_x) + D;  // f16, lane-interleaved
-  uint16_t* h16 = x16 + D;                         // f16, lane-interleaved
-  __shared__ float s_raw[kMaxExperts / kTok1Cluster], s_stat[4];
   uint8_t* gu_codes = region;                                   // [UPC][D]
   uint8_t* gu_scales = region + UPC * UNIT_C;                   // [UPC][D/8]
   uint8_t* dn_codes = gu_scales + UPC * UNIT_S;                 // [RPC][I/2]
@@ -188,12 +196,14 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
     const uint8_t* cb = p.codes + static_cast<long long>(e) * p.cpe;
     const uint8_t* sb = p.scales + static_cast<long long>(e) * p.spe;
     const int u0 = static_cast<int>(rank) * UPC;
-    if (lane < NCH) {
-      const int u = u0 + lane * CU;
-      mbar_arrive_expect_tx(&bar_chunk[lane], CU * (UNIT_C + UNIT_S));
-      bulk_g2s(gu_codes + lane * CU * UNIT_C, cb + static_cast<long long>(u) * UNIT_C, CU * UNIT_C, &bar_chunk[lane]);
-      bulk_g2s(gu_scales + lane * CU * UNIT_S, sb + static_cast<long long>(u) * UNIT_S, CU * UNIT_S, &bar_chunk[lane]);
-    } else if (lane == NCH) {
+    if (lane < NCP) {
+      constexpr int CCU = CPC * CU;  // units of one copy
+      const int u = u0 + lane * CCU;
+      mbar_arrive_expect_tx(&bar_chunk[lane], CCU * (UNIT_C + UNIT_S));
+      bulk_g2s(gu_codes + lane * CCU * UNIT_C, cb + static_cast<long long>(u) * UNIT_C, CCU * UNIT_C, &bar_chunk[lane]);
+      bulk_g2s(gu_scales + lane * CCU * UNIT_S, sb + static_cast<long long>(u) * UNIT_S, CCU * UNIT_S,
+               &bar_chunk[lane]);
+    } else if (lane == NCP) {
       const long long n0 = static_cast<long long>(rank) * RPC;
       mbar_arrive_expect_tx(bar_down, RPC * (DROW_C + DROW_S));
       bulk_g2s(dn_codes, cb + static_cast<long long>(I) * D + n0 * DROW_C, RPC * DROW_C, bar_down);
@@ -227,14 +237,17 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
     bulk_g2s(const_cast<uint16_t*>(s_x), p.x, D * 2, bar_x);
   }
 
-  // ---- P1: the token's statistics (warp 0) and this CTA's router dots
-  // (other warps) from the bf16 copy; then x as f16 (power-of-two scale) in
-  // the lane-interleaved order, and each lane's x vectors v = lane + 32 j
-  // (j < XV) of a gate/up row in registers (at D = 512 lanes 16..31 repeat
-  // lanes 0..15). Shared memory is read once per CTA, conflict-free.
+  // ---- P1: every warp derives the token's statistics from the bf16 copy of
+  // x (16-byte lanes, conflict-free; the same values in every warp, so no
+  // barrier); warp w computes router rows r0 + w, r0 + w + 16, ... and stores
+  // each logit into every CTA of the cluster; x is converted once into a
+  // lane-interleaved f16 copy, from which each lane loads its x vectors
+  // v = lane + 32 j (j < XV) of a gate/up row (at D = 512 lanes 16..31 repeat
+  // lanes 0..15).
   bool ok = __all_sync(0xffffffffu, mbar_wait(bar_x, 0, p.status));
   if (!shared && r1 > r0 && !__all_sync(0xffffffffu, mbar_wait(bar_rows, 0, p.status))) ok = false;
-  if (warp == 0) {
+  float sigma, irms;
+  {
     float amax = 0.f, ss = 0.f;
     for (int i = lane; i < D / 8; i += 32) {
       const uint4 v = lds128(s_x + 8 * i);
@@ -249,14 +262,15 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
     }
     amax = segment_max<32>(amax);
     ss = warp_sum(ss);
-    if (lane == 0) {
-      s_stat[0] = pow2_scale_for(amax);
-      s_stat[1] = p.input_norm ? 1.f / sqrtf(ss / static_cast<float>(D) + kRmsEps) : 1.f;
-    }
-  } else if (!shared && ok) {
-    // warp w >= 1: rows r0 + w - 1, + 15, ...; lane l reads the row's 16-byte
-    // vectors l + 32 i and the same vectors of x
-    for (int r = r0 + warp - 1; r < r1; r += kTok1Warps - 1) {
+    sigma = pow2_scale_for(amax);
+    irms = p.input_norm ? 1.f / sqrtf(ss / static_cast<float>(D) + kRmsEps) : 1.f;
+  }
+  const float fx = irms / sigma;  // dot(q, x*sigma) * fx = dot(q, x) * irms
+  // every CTA of the cluster must be running before the remote stores: the
+  // cluster arrival of P0 is waited for here
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  if (!shared && ok) {
+    for (int r = r0 + warp; r < r1; r += kTok1Warps) {
       const uint8_t* row = region + static_cast<size_t>(r - r0) * D * 2;
       float a = 0.f;
 #pragma unroll 4
@@ -269,20 +283,10 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
           a = fmaf(__uint_as_float(ww[q] & 0xFFFF0000u), __uint_as_float(xx[q] & 0xFFFF0000u), a);
         }
       }
-      a = warp_sum(a);
-      if (lane == 0) s_raw[r - r0] = a;
+      const float logit = warp_sum(a) * irms;
+      if (lane < CS) st_cluster_f32(s_logits + r, static_cast<unsigned>(lane), logit);
     }
   }
-  if (!ok && lane == 0) s_fail = 1;
-  __syncthreads();
-  const float sigma = s_stat[0], irms = s_stat[1];
-  const float fx = irms / sigma;  // dot(q, x*sigma) * fx = dot(q, x) * irms
-  // logits into every CTA of the cluster (each must be running: the cluster
-  // arrival of P0 is waited for here)
-  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-  if (!shared && !s_fail)
-    for (int i = tid; i < (r1 - r0) * CS; i += blockDim.x)
-      st_cluster_f32(s_logits + r0 + i / CS, static_cast<unsigned>(i % CS), s_raw[i / CS] * irms);
   for (int i = tid; i < D / 8; i += blockDim.x) {
     const uint4 v = lds128(s_x + 8 * i);
     uint4 o;
@@ -292,6 +296,7 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
     o.w = bf16x2_to_f16x2_scaled(v.w, sigma);
     *reinterpret_cast<uint4*>(x16 + (((i & 3) * VPR) + (i >> 2)) * 8) = o;  // vector i/4, chunk i%4
   }
+  if (!ok && lane == 0) s_fail = 1;
   __syncthreads();
   const int xl = lane % VPR;  // first x vector of this lane
   uint32_t xr[XV][16];
@@ -351,7 +356,7 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   // ---- P3: gate/up of chunk `warp` (CU units), h into every CTA of the cluster
   bool ok3 = issued;
   if (warp < NCH && issued) {
-    if (!__all_sync(0xffffffffu, mbar_wait(&bar_chunk[warp], 0, p.status))) ok3 = false;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar_chunk[warp / CPC], 0, p.status))) ok3 = false;
     if (ok3) {
 #pragma unroll 1
       for (int c = 0; c < CU; ++c) {
@@ -372,7 +377,10 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
         g = warp_sum(g);
         u = warp_sum(u);
         const float hv = swiglu(g * fx * sg, u * fx * su);
-        if (lane < CS) st_cluster_f32(s_h + static_cast<int>(rank) * UPC + ul, static_cast<unsigned>(lane), hv);
+        // stored lane-interleaved: unit u at (u % 32) * (I / 32) + u / 32, so
+        // that the lanes of a down step read consecutive words
+        const int uu = static_cast<int>(rank) * UPC + ul;
+        if (lane < CS) st_cluster_f32(s_h + (uu & 31) * LPR + (uu >> 5), static_cast<unsigned>(lane), hv);
       }
     }
   }
@@ -383,36 +391,22 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
 
   // ---- P4: down rows of this CTA's block against the whole h
   float* part = p.partial + static_cast<size_t>(slot) * D + static_cast<size_t>(rank) * RPC;
-  // h as f16 with a power-of-two scale, once per CTA in the lane-interleaved
-  // order; each lane then holds the 32 elements of vector lane % LPR
-  if (warp == 0) {
+  // every warp scales h by the same power of two (from its own pass over the
+  // interleaved words, conflict-free) and takes the 32 elements of vector
+  // lane % LPR as f16 pairs
+  float hs;
+  {
     float hm = 0.f;
     for (int i = lane; i < I; i += 32) hm = fmaxf(hm, fabsf(s_h[i]));
     hm = segment_max<32>(hm);
-    if (lane == 0) s_stat[2] = pow2_scale_for(hm);
+    hs = pow2_scale_for(hm);
   }
-  __syncthreads();
-  const float hs = s_stat[2];
-  for (int i = tid; i < I / 8; i += blockDim.x) {
-    uint4 o;
-    o.x = pack_f16x2(s_h[8 * i + 0] * hs, s_h[8 * i + 1] * hs);
-    o.y = pack_f16x2(s_h[8 * i + 2] * hs, s_h[8 * i + 3] * hs);
-    o.z = pack_f16x2(s_h[8 * i + 4] * hs, s_h[8 * i + 5] * hs);
-    o.w = pack_f16x2(s_h[8 * i + 6] * hs, s_h[8 * i + 7] * hs);
-    *reinterpret_cast<uint4*>(h16 + (((i & 3) * LPR) + (i >> 2)) * 8) = o;
-  }
-  __syncthreads();
   if (ok && !__all_sync(0xffffffffu, mbar_wait(bar_down, 0, p.status))) ok = false;
   if (ok) {
     uint32_t hr[16];
+    const int hv = lane % LPR;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 v = lds128(h16 + ((q * LPR) + lane % LPR) * 8);
-      hr[4 * q + 0] = v.x;
-      hr[4 * q + 1] = v.y;
-      hr[4 * q + 2] = v.z;
-      hr[4 * q + 3] = v.w;
-    }
+    for (int i = 0; i < 16; ++i) hr[i] = pack_f16x2(s_h[(2 * i) * LPR + hv] * hs, s_h[(2 * i + 1) * LPR + hv] * hs);
     const float ys = sd * gate / hs;
     for (int r = warp * RPS + lane / LPR; r < RPC; r += kTok1Warps * RPS) {
       const uint4 cv = lds128(dn_codes + r * DROW_C + 16 * (lane % LPR));
@@ -457,7 +451,7 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
     if (!shared && r1 > r0) mbar_wait(bar_rows, 0, p.status);
   }
   if (!ok && issued) {
-    for (int c = tid; c < NCH; c += blockDim.x) mbar_wait(&bar_chunk[c], 0, p.status);
+    for (int c = tid; c < NCP; c += blockDim.x) mbar_wait(&bar_chunk[c], 0, p.status);
     if (tid == 0) mbar_wait(bar_down, 0, p.status);
   }
 }

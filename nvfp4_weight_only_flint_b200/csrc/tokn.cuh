@@ -1,0 +1,466 @@
+// tokn.cuh -- the layer at decode batch 2..8 as persistent 16-CTA clusters.
+//
+// The grid is NC clusters of kTok1Cluster CTAs (as many as can be resident,
+// at most the number of (expert) items a call can have). Every cluster routes
+// the batch itself -- router logits through distributed shared memory as in
+// the one-token kernel, top-k per token, the grouping by expert (the experts
+// the tokens selected, ascending, then the shared expert) -- and then takes
+// the items a = cluster, cluster + NC, ... in turn. An item is one expert
+// with its tokens (1..T of them): CTA r of the cluster owns units
+// [r*I/16, (r+1)*I/16) of its gate/up and rows [r*d/16, (r+1)*d/16) of its
+// down projection. Both go through the register-fragment tensor cores
+// (mma.sync m16n8k16: 16 weight rows x the item's tokens as the 8 columns,
+// the in-register NVFP4 decode of fused_tc.cuh), fed by per-warp rings of
+// 256-column stages (one 128-byte-swizzled TMA box of codes, one box of
+// scales) that run ahead across item boundaries:
+//   gate/up  warp w < TL*KP takes tile w / KP (8 units = 16 rows) and K part
+//            w % KP (512 columns, two stages); the KP parts of a tile meet in
+//            shared memory (named barrier per tile group, double-buffered by
+//            item parity) and the group's first warp applies SwiGLU and stores
+//            h into every CTA of the cluster (DSMEM, double-buffered by item)
+//   cluster barrier: the item's h is complete everywhere
+//   h -> f16 with a power-of-two scale per token row, in the B-fragment order
+//   down     warp w < DT*DKP takes row tile w / DKP and K part w % DKP (one
+//            256-column stage); parts summed as above; the first warp writes
+//            gate * s_d * W_d h for the item's (token, slot) pairs: fp32
+//            partials [token * (k+S) + slot][d] in the workspace
+//   arrival  after its last item, one release/acquire atomic per CTA at its
+//            row block's counter; the CTA that brings it to the number of
+//            clusters adds, per token, the k + S partials of its rows in slot
+//            order (+ residual), rounds to bf16 and resets the counter.
+// No CTA waits on another cluster. Cluster barriers are reached by every CTA
+// of a cluster on every path; every mbarrier wait is bounded; a warp whose
+// wait gives up keeps taking every barrier (its work skipped).
+#pragma once
+
+#include <cuda.h>
+
+#include "fused_tc.cuh"
+#include "tok1.cuh"
+
+namespace flint {
+
+constexpr int kTnWarps = 16;
+constexpr int kTnMaxTokens = 8;
+constexpr int kTnSlots = 2;            // ring slots per warp
+constexpr int kTnStageCodes = 2048;    // 16 rows x 128 code bytes (256 columns), 128-byte swizzle
+constexpr int kTnStageScales = 256;    // 16 rows x 16 scale bytes
+constexpr int kTnMaxExperts = 256;     // router rows of a CTA fit the rings' 64 KiB
+
+struct TokNParams {
+  const uint16_t* x;         // [T][d] bf16
+  const uint16_t* wr;        // [E][d] bf16
+  const float* tscale;       // [E+S][3]
+  const uint16_t* residual;  // [T][d] bf16 or null
+  uint16_t* out;             // [T][d] bf16
+  int* status;
+  unsigned* rb_count;        // [kTok1Cluster] arrival counters (workspace control block)
+  float* partial;            // [T*(k+S)][d] gated partial outputs (workspace)
+  int* ids;                  // [T][k] routed ids (workspace)
+  float* gates;              // [T][k]
+  int* ids_out;
+  float* gates_out;
+  int T, E, k, S;
+  int input_norm;
+};
+
+// Gate/up: codes [E+S][2I][d/2] bytes, box 128 x 16 x 1, 128-byte swizzle;
+// scales [E+S][2I][d/16], box 16 x 16 x 1. Down (from the expert's I*d/2-th
+// code byte): codes [E+S][d][I/2], scales [E+S][d][I/16], same boxes.
+struct TokNMaps {
+  CUtensorMap gu_codes, gu_scales, dn_codes, dn_scales;
+};
+
+template <int D, int I>
+struct TnShape {
+  static constexpr int UPC = I / kTok1Cluster;   // gate/up units per CTA
+  static constexpr int TL = UPC / 8;             // gate/up tiles (16 rows) per CTA
+  static constexpr int KP = D / 512;             // gate/up K parts (512 columns)
+  static constexpr int GU = TL * KP;             // gate/up warps
+  static constexpr int RPC = D / kTok1Cluster;   // down rows per CTA
+  static constexpr int DT = RPC / 16;            // down tiles per CTA
+  static constexpr int DKP = I / 256;            // down K parts (256 columns)
+  static constexpr int DN = DT * DKP;            // down warps
+  static constexpr int XSTR = tc_b_stride(D), HSTR = tc_b_stride(I);
+  static constexpr bool ok = (I >= 256) && (UPC % 8 == 0) && GU >= 1 && GU <= kTnWarps && DN >= 1 &&
+                             DN <= kTnWarps && (TL + DT) <= 14;
+};
+
+// Dynamic shared memory (after 1 KiB alignment slack): rings' codes and
+// scales (the router rows use the codes area before the first item), x as
+// f16 in the B-fragment order, h fp32 [2][8][I] (x's bf16 copy before the
+// first item), h as f16 [8][HSTR] (the grouping's scratch before), the K-part
+// partial sums of gate/up and down (2 buffers each), logits [8][E].
+__host__ __device__ constexpr size_t tn_h32_bytes(int D, int I) {
+  return (2 * kTnMaxTokens * static_cast<size_t>(I) * 4 > kTnMaxTokens * static_cast<size_t>(D) * 2)
+             ? 2 * kTnMaxTokens * static_cast<size_t>(I) * 4
+             : kTnMaxTokens * static_cast<size_t>(D) * 2;
+}
+__host__ __device__ constexpr size_t tn_smem_bytes(int D, int I) {
+  return 1024 + static_cast<size_t>(kTnWarps) * kTnSlots * (kTnStageCodes + kTnStageScales) +
+         static_cast<size_t>(kTnMaxTokens) * tc_b_stride(D) + tn_h32_bytes(D, I) +
+         ((static_cast<size_t>(kTnMaxTokens) * tc_b_stride(I) > 20 * kTnMaxExperts)
+              ? static_cast<size_t>(kTnMaxTokens) * tc_b_stride(I)
+              : 20 * kTnMaxExperts) +
+         2 * 2 * static_cast<size_t>(kTnWarps) * 128 * 4 + static_cast<size_t>(kTnMaxTokens) * kTnMaxExperts * 4;
+}
+
+__device__ __forceinline__ void named_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+template <int D, int I>
+__global__ void __launch_bounds__(kTnWarps * 32, 1) k_tokn(TokNParams p, const __grid_constant__ TokNMaps maps) {
+  using SH = TnShape<D, I>;
+  constexpr int CS = kTok1Cluster, TL = SH::TL, KP = SH::KP, GU = SH::GU, DKP = SH::DKP, DN = SH::DN;
+  constexpr int RPC = SH::RPC, XSTR = SH::XSTR, HSTR = SH::HSTR;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bars[kTnWarps * kTnSlots];
+  __shared__ __align__(8) uint64_t bar_x, bar_rows;
+  __shared__ int s_ids[kTnMaxTokens * kMaxTopK];
+  __shared__ float s_gates[kTnMaxTokens * kMaxTopK];
+  __shared__ int s_act[kTnMaxExperts + 1], s_off[kTnMaxExperts + 2], s_pair[kTnMaxTokens * (kMaxTopK + 1)];
+  __shared__ int s_nr, s_na, s_fail, s_last;
+  __shared__ float s_sig[kTnMaxTokens], s_irms[kTnMaxTokens], s_hsig[kTnMaxTokens];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int T = p.T, E = p.E, k = p.k, KS = k + p.S;
+  const unsigned rank = cluster_rank();
+  const int cl = static_cast<int>(cluster_index()), NC = static_cast<int>(gridDim.x) / CS;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* rcodes = base;                                             // [warp][slot][2048]
+  uint8_t* rscales = rcodes + kTnWarps * kTnSlots * kTnStageCodes;     // [warp][slot][256]
+  uint8_t* x16 = rscales + kTnWarps * kTnSlots * kTnStageScales;       // [8][XSTR]
+  float* h32 = reinterpret_cast<float*>(x16 + kTnMaxTokens * XSTR);    // [2][8][I]
+  uint8_t* h16 = reinterpret_cast<uint8_t*>(h32) + tn_h32_bytes(D, I);  // [8][HSTR]
+  float* pgu = reinterpret_cast<float*>(h16 + ((kTnMaxTokens * HSTR > 20 * kTnMaxExperts) ? kTnMaxTokens * HSTR
+                                                                                          : 20 * kTnMaxExperts));
+  float* pdn = pgu + 2 * kTnWarps * 128;                               // [2][DN][128]
+  float* s_logits = pdn + 2 * kTnWarps * 128;                          // [8][E]
+  const uint16_t* s_x = reinterpret_cast<const uint16_t*>(h32);       // bf16 copy of x, before the first item
+  const int r0 = static_cast<int>(rank) * E / CS, r1 = (static_cast<int>(rank) + 1) * E / CS;
+  uint64_t* wb = bars + warp * kTnSlots;
+
+  // ---- P0
+  if (tid == 0) {
+    for (int i = 0; i < kTnWarps * kTnSlots; ++i) mbar_init(&bars[i], 1);
+    mbar_init(&bar_x, 1);
+    mbar_init(&bar_rows, 1);
+    fence_barrier_init();
+    s_fail = 0;
+    const uint32_t rbytes = static_cast<uint32_t>(r1 - r0) * D * 2;
+    mbar_arrive_expect_tx(&bar_rows, rbytes);
+    if (rbytes) bulk_g2s(rcodes, p.wr + static_cast<size_t>(r0) * D, rbytes, &bar_rows);
+  }
+  __syncthreads();
+  // release: a CTA's barrier and flag initialisation is visible to the remote
+  // stores that follow the matching wait
+  asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");
+  pdl_trigger();
+  pdl_wait();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bar_x, static_cast<uint32_t>(T) * D * 2);
+    bulk_g2s(const_cast<uint16_t*>(s_x), p.x, static_cast<uint32_t>(T) * D * 2, &bar_x);
+  }
+
+  // ---- P1: per-token statistics (warp t), router dots for every token,
+  // logits into every CTA of the cluster; x as f16 in the B-fragment order
+  bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_x, 0, p.status));
+  if (!__all_sync(0xffffffffu, mbar_wait(&bar_rows, 0, p.status))) ok = false;
+  if (warp < T) {
+    float amax = 0.f, ss = 0.f;
+    for (int i = lane; i < D / 8; i += 32) {
+      const uint4 v = lds128(s_x + static_cast<size_t>(warp) * D + 8 * i);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float a = bf16_bits_to_f32(w4[q] & 0xFFFFu), b = __uint_as_float(w4[q] & 0xFFFF0000u);
+        amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+        ss = fmaf(a, a, ss);
+        ss = fmaf(b, b, ss);
+      }
+    }
+    amax = segment_max<32>(amax);
+    ss = warp_sum(ss);
+    if (lane == 0) {
+      s_sig[warp] = pow2_scale_for(amax);
+      s_irms[warp] = p.input_norm ? 1.f / sqrtf(ss / static_cast<float>(D) + kRmsEps) : 1.f;
+    }
+  }
+  __syncthreads();
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every CTA runs: remote stores allowed
+  // a failed wait is made known to the whole cluster, so that every CTA of it
+  // takes the same items (and cluster barriers) below
+  if (!ok && lane < CS) st_cluster_u32(reinterpret_cast<unsigned*>(&s_fail), static_cast<unsigned>(lane), 1u);
+  if (ok) {
+    for (int r = r0 + warp; r < r1; r += kTnWarps) {
+      const uint8_t* row = rcodes + static_cast<size_t>(r - r0) * D * 2;
+      float a[kTnMaxTokens];
+#pragma unroll
+      for (int t = 0; t < kTnMaxTokens; ++t) a[t] = 0.f;
+#pragma unroll 2
+      for (int i = lane; i < D / 8; i += 32) {
+        const uint4 wv = lds128(row + 16 * i);
+        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int t = 0; t < kTnMaxTokens; ++t) {
+          if (t < T) {
+            const uint4 xv = lds128(s_x + static_cast<size_t>(t) * D + 8 * i);
+            const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              a[t] = fmaf(bf16_bits_to_f32(ww[q] & 0xFFFFu), bf16_bits_to_f32(xx[q] & 0xFFFFu), a[t]);
+              a[t] = fmaf(__uint_as_float(ww[q] & 0xFFFF0000u), __uint_as_float(xx[q] & 0xFFFF0000u), a[t]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < kTnMaxTokens; ++t) {
+        if (t < T) {
+          const float logit = warp_sum(a[t]) * s_irms[t];
+          if (lane < CS) st_cluster_f32(s_logits + t * E + r, static_cast<unsigned>(lane), logit);
+        }
+      }
+    }
+  }
+  for (int i = tid; i < kTnMaxTokens * (D / 8); i += blockDim.x) {
+    const int t = i / (D / 8), c = i % (D / 8);
+    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+    if (t < T) {
+      const float sg = s_sig[t];
+      const uint4 v = lds128(s_x + static_cast<size_t>(t) * D + 8 * c);
+      o.x = bf16x2_to_f16x2_scaled(v.x, sg);
+      o.y = bf16x2_to_f16x2_scaled(v.y, sg);
+      o.z = bf16x2_to_f16x2_scaled(v.z, sg);
+      o.w = bf16x2_to_f16x2_scaled(v.w, sg);
+    }
+    uint8_t* b = x16 + static_cast<size_t>(t) * XSTR + tc_b_offset(8 * c);
+    *reinterpret_cast<uint32_t*>(b) = o.x;
+    *reinterpret_cast<uint32_t*>(b + 16) = o.y;
+    *reinterpret_cast<uint32_t*>(b + 32) = o.z;
+    *reinterpret_cast<uint32_t*>(b + 48) = o.w;
+  }
+
+  // ---- P2: all logits everywhere; top-k per token (warp t), grouping
+  cluster_sync_all();
+  if (s_fail) ok = false;
+  if (warp < T && ok) {
+    uint32_t code[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      code[i] = (e < E) ? max(route_code(s_logits[warp * E + e]), 1u) : 0u;
+    }
+    topk_rounds<8>(code, k, s_ids + warp * k, s_gates + warp * k, lane);
+  }
+  __syncthreads();
+  if (ok) cta_grouping(s_ids, T, k, E, p.S, s_act, s_off, s_pair, &s_nr, &s_na, h16, p.status);
+  __syncthreads();
+  if (cl == 0 && rank == 0 && ok) {
+    for (int i = tid; i < T * k; i += blockDim.x) {
+      p.ids[i] = s_ids[i];
+      p.gates[i] = s_gates[i];
+      if (p.ids_out != nullptr) {
+        p.ids_out[i] = s_ids[i];
+        p.gates_out[i] = s_gates[i];
+      }
+    }
+  }
+  const int n_items = ok ? s_na : 0;
+  const int n_my = n_items > cl ? (n_items - 1 - cl) / NC + 1 : 0;  // items cl, cl + NC, ...
+  // this warp's stage stream: per item its two gate/up stages, then its down stage
+  const int gsw = warp < GU ? 2 : 0, dsw = warp < DN ? 1 : 0, NSW = gsw + dsw;
+  const int n_st = n_my * NSW;
+  const int gt = warp / KP, gp = warp % KP;   // gate/up tile and K part
+  const int dt = warp / DKP, dp = warp % DKP; // down tile and K part
+  auto issue = [&](int q) {
+    const int it = q / NSW, kk = q % NSW, e = s_act[cl + NC * it], slot = q % kTnSlots;
+    uint8_t* cs = rcodes + (warp * kTnSlots + slot) * kTnStageCodes;
+    uint8_t* sc = rscales + (warp * kTnSlots + slot) * kTnStageScales;
+    mbar_arrive_expect_tx(&wb[slot], kTnStageCodes + kTnStageScales);
+    if (kk < gsw) {
+      const int kc = gp * 512 + kk * 256, y = (static_cast<int>(rank) * TL + gt) * 16;
+      tma_load_3d(cs, &maps.gu_codes, kc / 2, y, e, &wb[slot]);
+      tma_load_3d(sc, &maps.gu_scales, kc / 16, y, e, &wb[slot]);
+    } else {
+      const int kc = dp * 256, y = static_cast<int>(rank) * RPC + dt * 16;
+      tma_load_3d(cs, &maps.dn_codes, kc / 2, y, e, &wb[slot]);
+      tma_load_3d(sc, &maps.dn_scales, kc / 16, y, e, &wb[slot]);
+    }
+  };
+  int issued = 0;
+  if (lane == 0) {
+    // the router rows in the codes area are read: order those reads first
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    for (; issued < kTnSlots && issued < n_st; ++issued) issue(issued);
+  }
+  int q = 0, q_fail = -1;  // stages consumed; first stage whose wait gave up
+  auto wait_stage = [&]() -> bool {
+    bool good = ok && (*reinterpret_cast<volatile int*>(&s_fail) == 0);
+    good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+    if (good) good = __all_sync(0xffffffffu, mbar_wait(&wb[q % kTnSlots], (q / kTnSlots) & 1, p.status));
+    if (!good) {
+      if (ok) q_fail = q;
+      ok = false;
+      if (lane == 0) s_fail = 1;
+    }
+    return good;
+  };
+  auto release_stage = [&]() {  // the slot's data is read: refill it
+    __syncwarp();
+    if (lane == 0 && ok && issued < n_st) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue(issued);
+      ++issued;
+    }
+    ++q;
+  };
+  const int g = lane >> 2, t4 = lane & 3;
+
+  for (int it = 0; it < n_my; ++it) {
+    const int a = cl + NC * it, buf = it & 1;
+    const int e = s_act[a], pb = s_off[a], ne = s_off[a + 1] - pb;
+    // the lane's ldmatrix row: the token of column lane % 8 (unused columns repeat column 0)
+    const int my_pair = s_pair[pb + ((lane & 7) < ne ? (lane & 7) : 0)];
+    // ---- gate/up
+    if (warp < GU) {
+      const float sgt = __ldg(p.tscale + 3 * e + 0), sut = __ldg(p.tscale + 3 * e + 1);
+      const uint8_t* xrow = x16 + static_cast<size_t>(my_pair >> 8) * XSTR;
+      const int rg = 2 * tc_unit_of(g), ru = rg + 1;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int s = 0; s < 2; ++s) {
+        if (wait_stage()) {
+          const uint8_t* cs = rcodes + (warp * kTnSlots + (q % kTnSlots)) * kTnStageCodes;
+          const uint8_t* ss = rscales + (warp * kTnSlots + (q % kTnSlots)) * kTnStageScales;
+#pragma unroll
+          for (int seg = 0; seg < 2; ++seg) {
+            uint32_t b[16];
+            tc_load_b(xrow, (gp * 4 + s * 2 + seg) * 256, lane, b);
+            const uint4 ca = lds128(tc_code_chunk(cs, rg, seg, t4)), cb = lds128(tc_code_chunk(cs, ru, seg, t4));
+            const uint32_t sa = *reinterpret_cast<const uint16_t*>(ss + rg * 16 + seg * 8 + 2 * t4);
+            const uint32_t sb = *reinterpret_cast<const uint16_t*>(ss + ru * 16 + seg * 8 + 2 * t4);
+            tc_segment(acc, acc1, ca, cb, sa, sb, b);
+          }
+        }
+        release_stage();
+      }
+      float* pp = pgu + (static_cast<size_t>(buf) * kTnWarps + gt * KP) * 128;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) pp[gp * 128 + r * 32 + lane] = acc[r] + acc1[r];
+      if constexpr (KP > 1) named_sync(1 + gt, 32 * KP);
+      else __syncwarp();
+      if (gp == 0) {
+        float v[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          v[r] = 0.f;
+#pragma unroll
+          for (int k2 = 0; k2 < KP; ++k2) v[r] += pp[k2 * 128 + r * 32 + lane];
+        }
+        const int u = (static_cast<int>(rank) * TL + gt) * 8 + tc_unit_of(g);  // unit within the expert
+        float* hb = h32 + static_cast<size_t>(buf) * kTnMaxTokens * I;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int col = 2 * t4 + h2;
+          if (col < ne) {
+            const int tok = s_pair[pb + col] >> 8;
+            const float f = s_irms[tok] / s_sig[tok];
+            const float hv = swiglu(v[h2] * f * sgt, v[2 + h2] * f * sut);
+#pragma unroll 4
+            for (int dst = 0; dst < CS; ++dst) st_cluster_f32(hb + col * I + u, static_cast<unsigned>(dst), hv);
+          }
+        }
+      }
+    }
+    // ---- the item's h is complete in every CTA of the cluster
+    cluster_sync_all();
+    // h as f16 in the B-fragment order with a power-of-two scale per token row
+    // (warp n: column n)
+    if (warp < ne) {
+      const float* hr = h32 + (static_cast<size_t>(buf) * kTnMaxTokens + warp) * I;
+      float hm = 0.f;
+      for (int i = lane; i < I; i += 32) hm = fmaxf(hm, fabsf(hr[i]));
+      hm = segment_max<32>(hm);
+      const float hs = pow2_scale_for(hm);
+      if (lane == 0) s_hsig[warp] = hs;
+      for (int i = lane; i < I / 2; i += 32) {
+        const uint32_t v = pack_f16x2(hr[2 * i] * hs, hr[2 * i + 1] * hs);
+        *reinterpret_cast<uint32_t*>(h16 + static_cast<size_t>(warp) * HSTR + tc_b_offset(2 * i)) = v;
+      }
+    }
+    __syncthreads();
+    // ---- down
+    if (warp < DN) {
+      const float sdt = __ldg(p.tscale + 3 * e + 2);
+      const uint8_t* hrow = h16 + static_cast<size_t>((lane & 7) < ne ? (lane & 7) : 0) * HSTR;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+      if (wait_stage()) {
+        const uint8_t* cs = rcodes + (warp * kTnSlots + (q % kTnSlots)) * kTnStageCodes;
+        const uint8_t* ss = rscales + (warp * kTnSlots + (q % kTnSlots)) * kTnStageScales;
+#pragma unroll
+        for (int seg = 0; seg < 2; ++seg) {
+          uint32_t b[16];
+          tc_load_b(hrow, (dp * 2 + seg) * 256, lane, b);
+          const uint4 ca = lds128(tc_code_chunk(cs, g, seg, t4)), cb = lds128(tc_code_chunk(cs, g + 8, seg, t4));
+          const uint32_t sa = *reinterpret_cast<const uint16_t*>(ss + g * 16 + seg * 8 + 2 * t4);
+          const uint32_t sb = *reinterpret_cast<const uint16_t*>(ss + (g + 8) * 16 + seg * 8 + 2 * t4);
+          tc_segment(acc, acc1, ca, cb, sa, sb, b);
+        }
+      }
+      release_stage();
+      float* pp = pdn + (static_cast<size_t>(buf) * kTnWarps + dt * DKP) * 128;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) pp[dp * 128 + r * 32 + lane] = acc[r] + acc1[r];
+      if constexpr (DKP > 1) named_sync(1 + TL + dt, 32 * DKP);
+      else __syncwarp();
+      if (dp == 0) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          float v = 0.f;
+#pragma unroll
+          for (int k2 = 0; k2 < DKP; ++k2) v += pp[k2 * 128 + r * 32 + lane];
+          const int col = 2 * t4 + (r & 1), row = static_cast<int>(rank) * RPC + dt * 16 + g + 8 * (r >> 1);
+          if (col < ne && ok) {
+            const int pr = s_pair[pb + col], tok = pr >> 8, j = pr & 0xFF;
+            const float gate = j < k ? s_gates[tok * k + j] : 1.f;
+            __stcg(p.partial + static_cast<size_t>(tok * KS + j) * D + row, v * sdt * gate / s_hsig[col]);
+          }
+        }
+      }
+    }
+  }
+  // copies still in flight after a failed wait land before the CTA goes on
+  if (!ok && lane == 0 && q_fail >= 0)
+    for (int k2 = q_fail; k2 < issued; ++k2) mbar_wait(&wb[k2 % kTnSlots], (k2 / kTnSlots) & 1, p.status);
+  // ---- arrival at this CTA's row block: once per CTA, whatever happened
+  // above, so the counter returns to zero; the CTA that brings it to the
+  // number of clusters adds the row block's partials
+  __syncthreads();
+  if (tid == 0) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.rb_count + rank) : "memory");
+    const int last = old == static_cast<unsigned>(NC - 1);
+    if (last) atomicExch(p.rb_count + rank, 0u);
+    s_last = last;
+  }
+  __syncthreads();
+  if (s_last) {
+    for (int idx = tid; idx < T * RPC; idx += blockDim.x) {
+      const int t = idx / RPC, n = static_cast<int>(rank) * RPC + idx % RPC;
+      float y = 0.f;
+      for (int j = 0; j < KS; ++j) y += __ldcg(p.partial + static_cast<size_t>(t * KS + j) * D + n);
+      const size_t o = static_cast<size_t>(t) * D + n;
+      if (p.residual != nullptr) y += bf16_bits_to_f32(__ldcg(p.residual + o));
+      const __nv_bfloat16 bv = __float2bfloat16_rn(y);
+      p.out[o] = *reinterpret_cast<const uint16_t*>(&bv);
+    }
+  }
+}
+
+// Host side (tokn.cu): whether the kernel serves (d, inter, E, T) on the
+// current device and, with `launch`, its launch for `t` on `st` (status in
+// *err). `maps` as TokNMaps.
+bool tokn_dispatch(int d, int I, int E, int T, bool launch, const TokNParams* t, const TokNMaps* maps, bool pdl,
+                   cudaStream_t st, cudaError_t* err);
+
+}  // namespace flint

@@ -107,9 +107,9 @@ def test_host_validation_errors(L):
     assert L.flint_moe_forward_ex(0x40000, 4, 0x40000, ctypes.byref(w), ctypes.byref(s), None, 0x50000,
                                   0x60000, ws_need, ctypes.byref(opt), None) == -1
     assert "layer_variant" in fm.flint_last_error()
-    # the cluster kernel takes one token only (refused before any launch)
+    # the cluster kernels take at most 8 tokens (refused before any launch)
     opt = fm.Options(path=0, use_pdl=1, layer_variant=fm.FLINT_LAYER_CLUSTER)
-    assert L.flint_moe_forward_ex(0x40000, 4, 0x40000, ctypes.byref(w), ctypes.byref(s), None, 0x50000,
+    assert L.flint_moe_forward_ex(0x40000, 9, 0x40000, ctypes.byref(w), ctypes.byref(s), None, 0x50000,
                                   0x60000, ws_need, ctypes.byref(opt), None) == -2
     assert "cluster" in fm.flint_last_error()
     # NVFP4 weights without scales

@@ -139,9 +139,9 @@ def test_cluster_kernel_refuses_shapes_it_cannot_hold():
     _check(layer, x, wr, what="auto fallback", variant=fm.FLINT_LAYER_AUTO)
 
 
-def test_cluster_kernel_rejects_more_than_one_token():
+def test_cluster_kernels_reject_more_than_eight_tokens():
     layer = _flint_layer()
-    x = bits_to_cuda(synth.x_bits(240, 2, 2048))
+    x = bits_to_cuda(synth.x_bits(240, 9, 2048))
     wr = bits_to_cuda(synth.make_router(synth.CONFIGS["cfg1"], 240, synth.x_bits(240, 1, 2048)))
     with pytest.raises(fm.FlintError) as ei:
         layer.forward(x, wr, variant=CLUSTER)
