@@ -139,6 +139,16 @@ __device__ __forceinline__ void fma2_f16_f32(uint32_t q, uint32_t x, float& acc)
       : "r"(q), "r"(x));
 }
 
+// acc (f32) += w.lo * x.lo + w.hi * x.hi with bf16 operands, products exact
+// in f32, one rounding per step (sm_100 mixed-precision fma): the same result
+// as fmaf on the widened values, without the widening instructions.
+__device__ __forceinline__ void fma2_bf16_f32(uint32_t w, uint32_t x, float& acc) {
+  asm("{\n .reg .b16 wl, wh, xl, xh;\n mov.b32 {wl, wh}, %1;\n mov.b32 {xl, xh}, %2;\n"
+      " fma.rn.f32.bf16 %0, wl, xl, %0;\n fma.rn.f32.bf16 %0, wh, xh, %0;\n}"
+      : "+f"(acc)
+      : "r"(w), "r"(x));
+}
+
 // One 16-byte code vector (32 elements = two 16-element blocks) against TG
 // activation vectors (16 f16x2 registers each, XS registers apart, pre-scaled
 // by a power of two):

@@ -860,7 +860,7 @@ int mma_maps(MmaMaps* mp, const Dims& s, const flint_moe_weights* wts, bool gate
   }
   const cuuint64_t bdims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(P)};
   const cuuint64_t bstr[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t bbox[2] = {64, 16};
+  const cuuint32_t bbox[2] = {64, 64};  // one copy per 64 rows: a thread issues a copy in ~0.25 us
   return encode_map(&mp->brows, s.wd == FLINT_W_NVFP4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                     2, brows, bdims, bstr, bbox, true);
 }
@@ -920,7 +920,7 @@ int tokn_maps(TokNMaps* m, const Dims& s, const flint_moe_weights* wts) {
 size_t mma_configure(MmaParams& m, int T) {
   constexpr size_t kBudget = 220 * 1024 - 1024;
   const int npad = std::min(kMmaMaxTokens, (T + 15) & ~15);
-  m.b_bytes = npad * 128;
+  m.b_bytes = ((npad + 63) & ~63) * 128;  // whole 64-row boxes
   m.ksplit = (npad <= kMmaMaxTokens / 2) ? 2 : 1;
   // A stages are recycled only after their MMAs complete, so the A ring must
   // cover that round trip: NVFP4 keeps 8 stages in tensor memory (columns
@@ -1317,6 +1317,10 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
     TokNParams t{};
     t.x = x;
     t.wr = router_w;
+    t.codes = p.codes;
+    t.scales = p.scales;
+    t.cpe = p.cpe;
+    t.spe = p.spe;
     t.tscale = p.tscale;
     t.residual = residual;
     t.out = out;

@@ -79,7 +79,7 @@ struct MmaParams {
   int T, d, I, E, k, S;
   int nvfp4;                // 1: NVFP4 weights, f16 operands; 0: bf16 weights, bf16 operands
   int n_raw, n_a, n_b;      // ring depths (raw NVFP4 stages, A stages, B stages)
-  int b_bytes;              // B stage: (tokens rounded up to 16, at most 128) x 128 bytes
+  int b_bytes;              // B stage: (tokens rounded up to 64, at most 128) x 128 bytes
   int ksplit;               // accumulators per item (1 or 2), fed alternate K steps, summed in the epilogue
 };
 
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(256) k_mma_combine(MmaParams p) {
 // Tensor maps of one call. Raw NVFP4: codes [experts][rows][K/2] bytes, box
 // (128 B, 128 rows, 1), 128-byte swizzle; scales [experts][rows][K/16], box
 // (16 B, 128, 1). bf16 weights: [experts][rows][K] bf16, box (64, 128, 1),
-// 128-byte swizzle. B rows: [P][K] 16-bit, box (64, 16), 128-byte swizzle.
+// 128-byte swizzle. B rows: [P][K] 16-bit, box (64, 64), 128-byte swizzle.
 struct MmaMaps {
   CUtensorMap codes;
   CUtensorMap scales;
@@ -425,58 +425,64 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     for (int i = max(0, n - ns); i < n; ++i) mbar_wait(&full[i % ns], (i / ns) & 1, p.status);
   };
 
+  // The producers issue a stage's operations from several lanes at once (the
+  // barrier's byte count from lane 0, each copy from a lane of its own): one
+  // thread takes ~0.25 us per operation. Every lane waits for the slot; the
+  // warp goes on only if all lanes saw it free.
   if (warp == 0) {
     // ------------------------------------------------ A producer: weights
-    if (lane == 0) {
-      int rc = 0, ac = 0;  // stages issued: raw NVFP4, A (bf16 weights)
-      bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const int a = it / tiles, t = it % tiles;
-        const int e = p.rt.act[a];
-        for (int s = 0; s < n_sub && ok; ++s) {
-          if (fp4) {
-            if ((s & 3) != 0) continue;
-            const int slot = rc % NR;
-            if (!(ok = mma_wait(&raw_empty[slot], ((rc / NR) & 1) ^ 1, abort_flag, p.status))) break;
-            uint8_t* st = raw + slot * kMmaRawBytes;
-            mbar_arrive_expect_tx(&raw_full[slot], kMmaRawBytes);
-            tma_load_3d(st, &maps.codes, (s / 4) * 128, t * 128, e, &raw_full[slot]);
-            tma_load_3d(st + 128 * 128, &maps.scales, (s / 4) * 16, t * 128, e, &raw_full[slot]);
-            ++rc;
-          } else {
-            const int slot = ac % NA;
-            if (!(ok = mma_wait(&a_empty[slot], ((ac / NA) & 1) ^ 1, abort_flag, p.status))) break;
-            mbar_arrive_expect_tx(&a_full[slot], kMmaABytes);
-            tma_load_3d(abuf + slot * kMmaABytes, &maps.codes, s * 64, t * 128, e, &a_full[slot]);
-            ++ac;
-          }
+    int rc = 0, ac = 0;  // stages issued: raw NVFP4, A (bf16 weights)
+    bool ok = true;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const int a = it / tiles, t = it % tiles;
+      const int e = p.rt.act[a];
+      for (int s = 0; s < n_sub && ok; ++s) {
+        if (fp4) {
+          if ((s & 3) != 0) continue;
+          const int slot = rc % NR;
+          if (!(ok = __all_sync(0xffffffffu, mma_wait(&raw_empty[slot], ((rc / NR) & 1) ^ 1, abort_flag, p.status))))
+            break;
+          uint8_t* st = raw + slot * kMmaRawBytes;
+          if (lane == 0) mbar_arrive_expect_tx(&raw_full[slot], kMmaRawBytes);
+          else if (lane == 1) tma_load_3d(st, &maps.codes, (s / 4) * 128, t * 128, e, &raw_full[slot]);
+          else if (lane == 2) tma_load_3d(st + 128 * 128, &maps.scales, (s / 4) * 16, t * 128, e, &raw_full[slot]);
+          ++rc;
+        } else {
+          const int slot = ac % NA;
+          if (!(ok = __all_sync(0xffffffffu, mma_wait(&a_empty[slot], ((ac / NA) & 1) ^ 1, abort_flag, p.status))))
+            break;
+          if (lane == 0) mbar_arrive_expect_tx(&a_full[slot], kMmaABytes);
+          else if (lane == 1) tma_load_3d(abuf + slot * kMmaABytes, &maps.codes, s * 64, t * 128, e, &a_full[slot]);
+          ++ac;
         }
       }
-      if (!ok) {
-        drain(raw_full, NR, rc);
-        drain(a_full, NA, ac);
-      }
+    }
+    if (!ok && lane == 0) {
+      drain(raw_full, NR, rc);
+      drain(a_full, NA, ac);
     }
   } else if (warp == 2) {
     // ------------------------------------------------ B producer: activation rows
-    if (lane == 0) {
-      int bc = 0;
-      bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const int a = it / tiles;
-        const int off = p.rt.off[a], nt = p.rt.off[a + 1] - off;
-        const int npad = (nt + 15) & ~15;
-        for (int s = 0; s < n_sub && ok; ++s) {
-          const int slot = bc % NB;
-          if (!(ok = mma_wait(&b_empty[slot], ((bc / NB) & 1) ^ 1, abort_flag, p.status))) break;
-          mbar_arrive_expect_tx(&b_full[slot], npad * 128);
-          for (int j = 0; j < npad / 16; ++j)
-            tma_load_2d(bbuf + slot * BB + j * 2048, &maps.brows, s * 64, off + 16 * j, &b_full[slot]);
-          ++bc;
-        }
+    int bc = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const int a = it / tiles;
+      const int off = p.rt.off[a], nt = p.rt.off[a + 1] - off;
+      const int npad = (nt + 15) & ~15;
+      for (int s = 0; s < n_sub && ok; ++s) {
+        const int slot = bc % NB;
+        if (!(ok = __all_sync(0xffffffffu, mma_wait(&b_empty[slot], ((bc / NB) & 1) ^ 1, abort_flag, p.status))))
+          break;
+        // 64-row boxes (rows past the expert's tokens are loaded but not
+        // multiplied; rows past the last pair are zero-filled)
+        const int nbox = (npad + 63) / 64;
+        if (lane == 0) mbar_arrive_expect_tx(&b_full[slot], nbox * 8192);
+        else if (lane <= nbox)
+          tma_load_2d(bbuf + slot * BB + (lane - 1) * 8192, &maps.brows, s * 64, off + 64 * (lane - 1), &b_full[slot]);
+        ++bc;
       }
-      if (!ok) drain(b_full, NB, bc);
     }
+    if (!ok && lane == 0) drain(b_full, NB, bc);
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {

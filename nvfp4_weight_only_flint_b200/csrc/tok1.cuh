@@ -86,6 +86,14 @@ __device__ __forceinline__ unsigned cluster_index() {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// Named CTA barriers (id > 0) over `threads` threads, whole warps.
+__device__ __forceinline__ void named_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id, int threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // Store v into the same shared-memory variable of CTA `rank` of this cluster.
 __device__ __forceinline__ void st_cluster_f32(float* local, unsigned rank, float v) {
   uint32_t remote;
@@ -112,24 +120,26 @@ template <int NE>
 __device__ __forceinline__ void topk_rounds(uint32_t (&code)[NE], int k, int* ids, float* gates, int lane) {
   float my_val = 0.f, v0 = 0.f;
   int my_sel = 0;
+  // slots already selected, as a bit mask: the code array is only read, so it
+  // stays in registers (clearing a slot by a computed index had put it in
+  // local memory)
+  uint32_t taken = 0u;
 #pragma unroll 1
   for (int r = 0; r < k; ++r) {
     uint32_t best = 0u;
     int bi = 0;
 #pragma unroll
-    for (int i = 0; i < NE; ++i)
-      if (code[i] > best) {
-        best = code[i];
+    for (int i = 0; i < NE; ++i) {
+      const uint32_t c = ((taken >> i) & 1u) ? 0u : code[i];
+      if (c > best) {
+        best = c;
         bi = i;
       }
+    }
     const uint32_t m = __reduce_max_sync(0xffffffffu, best);
     const uint32_t w = __reduce_max_sync(0xffffffffu, best == m ? 0xFFFFFFFFu - static_cast<uint32_t>(lane + 32 * bi) : 0u);
     const int e = static_cast<int>(0xFFFFFFFFu - w);
-    if ((e & 31) == lane) {
-#pragma unroll
-      for (int i = 0; i < NE; ++i)
-        if (i == (e >> 5)) code[i] = 0u;
-    }
+    if ((e & 31) == lane) taken |= 1u << (e >> 5);
     const float v = route_code_value(m);
     if (r == 0) v0 = v;
     if (lane == r) {
@@ -169,7 +179,7 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   __shared__ __align__(8) uint64_t s_bar[kTok1MaxChunks + 3];  // chunks, down rows, router rows, x
   __shared__ int s_ids[kMaxTopK];
   __shared__ float s_gates[kMaxTopK];
-  __shared__ int s_fail, s_last, s_burst;
+  __shared__ int s_fail, s_last, s_burst, s_expert;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = p.E, k = p.k, KS = k + p.S;
@@ -191,23 +201,29 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   uint64_t* bar_x = s_bar + kTok1MaxChunks + 2;
   const int r0 = static_cast<int>(rank) * E / CS, r1 = (static_cast<int>(rank) + 1) * E / CS;
 
-  // issue this CTA's slice of expert e (one lane per chunk, one for the down rows)
-  auto issue_expert = [&](int e) {
+  // This CTA's slice of expert e: one copy per chunk and one for the down
+  // rows, each from a lane of its own; `codes` selects the code copies (warp
+  // 0) or the scale copies (warp 1), so that the two go out in parallel (a
+  // thread takes ~0.25 us per bulk-copy operation). The barriers' byte counts
+  // are set in P0: they do not depend on the routing.
+  auto issue_expert = [&](int e, bool codes) {
     const uint8_t* cb = p.codes + static_cast<long long>(e) * p.cpe;
     const uint8_t* sb = p.scales + static_cast<long long>(e) * p.spe;
     const int u0 = static_cast<int>(rank) * UPC;
+    constexpr int CCU = CPC * CU;  // units of one copy
     if (lane < NCP) {
-      constexpr int CCU = CPC * CU;  // units of one copy
       const int u = u0 + lane * CCU;
-      mbar_arrive_expect_tx(&bar_chunk[lane], CCU * (UNIT_C + UNIT_S));
-      bulk_g2s(gu_codes + lane * CCU * UNIT_C, cb + static_cast<long long>(u) * UNIT_C, CCU * UNIT_C, &bar_chunk[lane]);
-      bulk_g2s(gu_scales + lane * CCU * UNIT_S, sb + static_cast<long long>(u) * UNIT_S, CCU * UNIT_S,
-               &bar_chunk[lane]);
+      if (codes)
+        bulk_g2s(gu_codes + lane * CCU * UNIT_C, cb + static_cast<long long>(u) * UNIT_C, CCU * UNIT_C, &bar_chunk[lane]);
+      else
+        bulk_g2s(gu_scales + lane * CCU * UNIT_S, sb + static_cast<long long>(u) * UNIT_S, CCU * UNIT_S,
+                 &bar_chunk[lane]);
     } else if (lane == NCP) {
       const long long n0 = static_cast<long long>(rank) * RPC;
-      mbar_arrive_expect_tx(bar_down, RPC * (DROW_C + DROW_S));
-      bulk_g2s(dn_codes, cb + static_cast<long long>(I) * D + n0 * DROW_C, RPC * DROW_C, bar_down);
-      bulk_g2s(dn_scales, sb + static_cast<long long>(I) * D / 8 + n0 * DROW_S, RPC * DROW_S, bar_down);
+      if (codes)
+        bulk_g2s(dn_codes, cb + static_cast<long long>(I) * D + n0 * DROW_C, RPC * DROW_C, bar_down);
+      else
+        bulk_g2s(dn_scales, sb + static_cast<long long>(I) * D / 8 + n0 * DROW_S, RPC * DROW_S, bar_down);
     }
   };
 
@@ -224,7 +240,16 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
     }
   }
   __syncthreads();
-  if (shared && warp == 0) issue_expert(E);
+  if (warp == 0) {  // byte counts of the expert slice's barriers
+    constexpr int CCU = CPC * CU;
+    if (lane < NCP) mbar_arrive_expect_tx(&bar_chunk[lane], CCU * (UNIT_C + UNIT_S));
+    else if (lane == NCP) mbar_arrive_expect_tx(bar_down, RPC * (DROW_C + DROW_S));
+    else if (lane == NCP + 1) mbar_arrive_expect_tx(bar_x, D * 2);
+  }
+  if (shared && warp < 2) {  // the shared expert's slice needs no routing
+    named_sync(1, 64);  // after the byte counts
+    issue_expert(E, warp == 0);
+  }
   // every CTA of the cluster must be running before any writes into its
   // shared memory: arrive now, wait just before the first remote store
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -232,10 +257,7 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   pdl_wait();  // x (and the workspace) are written by the preceding kernel
   // one copy of x per CTA: every warp reading it from L2 would make its 32
   // lines a hot spot of thousands of requests
-  if (tid == 0) {
-    mbar_arrive_expect_tx(bar_x, D * 2);
-    bulk_g2s(const_cast<uint16_t*>(s_x), p.x, D * 2, bar_x);
-  }
+  if (tid == 0) bulk_g2s(const_cast<uint16_t*>(s_x), p.x, D * 2, bar_x);
 
   // ---- P1: every warp derives the token's statistics from the bf16 copy of
   // x (16-byte lanes, conflict-free; the same values in every warp, so no
@@ -276,12 +298,10 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
 #pragma unroll 4
       for (int i = lane; i < D / 8; i += 32) {
         const uint4 wv = lds128(row + 16 * i), xv = lds128(s_x + 8 * i);
-        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w}, xx[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          a = fmaf(bf16_bits_to_f32(ww[q] & 0xFFFFu), bf16_bits_to_f32(xx[q] & 0xFFFFu), a);
-          a = fmaf(__uint_as_float(ww[q] & 0xFFFF0000u), __uint_as_float(xx[q] & 0xFFFF0000u), a);
-        }
+        fma2_bf16_f32(wv.x, xv.x, a);
+        fma2_bf16_f32(wv.y, xv.y, a);
+        fma2_bf16_f32(wv.z, xv.z, a);
+        fma2_bf16_f32(wv.w, xv.w, a);
       }
       const float logit = warp_sum(a) * irms;
       if (lane < CS) st_cluster_f32(s_logits + r, static_cast<unsigned>(lane), logit);
@@ -314,32 +334,46 @@ __global__ void __launch_bounds__(kTok1Warps * 32, 1) k_tok1(Tok1Params p) {
   // ---- P2: every CTA of the cluster holds all E logits; select, then issue
   cluster_sync_all();
   if (s_fail) ok = false;
-  if (!shared && warp == 0 && ok) {
-    uint32_t code[NE];
+  if (!shared && warp == 0) {
+    int e = -1;
+    if (ok) {
+      uint32_t code[NE];
 #pragma unroll
-    for (int i = 0; i < NE; ++i) {
-      const int e = lane + 32 * i;
-      code[i] = (e < E) ? max(route_code(s_logits[e]), 1u) : 0u;
+      for (int i = 0; i < NE; ++i) {
+        const int ei = lane + 32 * i;
+        code[i] = (ei < E) ? max(route_code(s_logits[ei]), 1u) : 0u;
+      }
+      topk_rounds<NE>(code, k, s_ids, s_gates, lane);
+      __syncwarp();
+      e = s_ids[slot];
+      if (e < 0 || e >= E) {
+        if (lane == 0) atomicOr(p.status, FLINT_DEVCHECK_EXPERT_ID);
+        e = -1;
+      }
     }
-    topk_rounds<NE>(code, k, s_ids, s_gates, lane);
-    __syncwarp();
+    if (lane == 0) {
+      s_expert = e;
+      s_burst = e >= 0 ? 1 : 0;
+    }
     // the router rows were read before the cluster barrier; order those
     // generic reads before the copies that overwrite them
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    const int e = s_ids[slot];
-    if (e < 0 || e >= E) {
-      if (lane == 0) atomicOr(p.status, FLINT_DEVCHECK_EXPERT_ID);
-    } else {
-      issue_expert(e);
-      if (lane == 0) s_burst = 1;
-    }
-    if (slot == 0 && rank == 0 && lane < k) {
+    named_arrive(1, 64);  // warp 1 takes the scale copies
+    if (e >= 0) issue_expert(e, true);
+    if (ok && slot == 0 && rank == 0 && lane < k) {
       p.ids[lane] = s_ids[lane];
       p.gates[lane] = s_gates[lane];
       if (p.ids_out != nullptr) {
         p.ids_out[lane] = s_ids[lane];
         p.gates_out[lane] = s_gates[lane];
       }
+    }
+  } else if (!shared && warp == 1) {
+    named_sync(1, 64);
+    const int e = s_expert;
+    if (e >= 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue_expert(e, false);
     }
   }
   __syncthreads();

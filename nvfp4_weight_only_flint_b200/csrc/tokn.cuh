@@ -2,9 +2,10 @@
 //
 // The grid is NC clusters of kTok1Cluster CTAs (as many as can be resident,
 // at most the number of (expert) items a call can have). Every cluster routes
-// the batch itself -- router logits through distributed shared memory as in
-// the one-token kernel, top-k per token, the grouping by expert (the experts
-// the tokens selected, ascending, then the shared expert) -- and then takes
+// the batch itself -- router logits on the register-fragment tensor cores,
+// shared through distributed shared memory as in the one-token kernel, top-k
+// per token, the grouping by expert (the experts the tokens selected,
+// ascending, then the shared expert) -- and then takes
 // the items a = cluster, cluster + NC, ... in turn. An item is one expert
 // with its tokens (1..T of them): CTA r of the cluster owns units
 // [r*I/16, (r+1)*I/16) of its gate/up and rows [r*d/16, (r+1)*d/16) of its
@@ -50,6 +51,9 @@ constexpr int kTnMaxExperts = 256;     // router rows of a CTA fit the rings' 64
 struct TokNParams {
   const uint16_t* x;         // [T][d] bf16
   const uint16_t* wr;        // [E][d] bf16
+  const uint8_t* codes;      // packed E2M1 codes (L2 prefetch of upcoming items)
+  const uint8_t* scales;     // packed E4M3 block scales
+  long long cpe, spe;        // code / scale bytes per expert
   const float* tscale;       // [E+S][3]
   const uint16_t* residual;  // [T][d] bf16 or null
   uint16_t* out;             // [T][d] bf16
@@ -105,15 +109,23 @@ __host__ __device__ constexpr size_t tn_smem_bytes(int D, int I) {
          2 * 2 * static_cast<size_t>(kTnWarps) * 128 * 4 + static_cast<size_t>(kTnMaxTokens) * kTnMaxExperts * 4;
 }
 
-__device__ __forceinline__ void named_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+// mma.sync m16n8k16, A row-major bf16, B column-major bf16, f32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ uint32_t lds32(const void* p) { return *reinterpret_cast<const uint32_t*>(p); }
+
 
 template <int D, int I>
 __global__ void __launch_bounds__(kTnWarps * 32, 1) k_tokn(TokNParams p, const __grid_constant__ TokNMaps maps) {
   using SH = TnShape<D, I>;
   constexpr int CS = kTok1Cluster, TL = SH::TL, KP = SH::KP, GU = SH::GU, DKP = SH::DKP, DN = SH::DN;
-  constexpr int RPC = SH::RPC, XSTR = SH::XSTR, HSTR = SH::HSTR;
+  constexpr int RPC = SH::RPC, XSTR = SH::XSTR, HSTR = SH::HSTR, UPC = SH::UPC;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars[kTnWarps * kTnSlots];
   __shared__ __align__(8) uint64_t bar_x, bar_rows;
@@ -191,36 +203,39 @@ __global__ void __launch_bounds__(kTnWarps * 32, 1) k_tokn(TokNParams p, const _
   // a failed wait is made known to the whole cluster, so that every CTA of it
   // takes the same items (and cluster barriers) below
   if (!ok && lane < CS) st_cluster_u32(reinterpret_cast<unsigned*>(&s_fail), static_cast<unsigned>(lane), 1u);
+  // router logits on the tensor cores: the CTA's rows r0..r1 (at most 16, the
+  // MMA's M) x the batch's tokens (the 8 columns, unused ones repeat token 0),
+  // K split over the 16 warps; bf16 products are exact, fp32 accumulation; the
+  // warps' partial sums are added in warp order
+  float* red = pgu;  // [16 warps][16 rows x 8 columns], free until the first item
   if (ok) {
-    for (int r = r0 + warp; r < r1; r += kTnWarps) {
-      const uint8_t* row = rcodes + static_cast<size_t>(r - r0) * D * 2;
-      float a[kTnMaxTokens];
+    const int g = lane >> 2, t4 = lane & 3;
+    const uint8_t* arow0 = rcodes + static_cast<size_t>(g) * D * 2;
+    const uint8_t* arow1 = rcodes + static_cast<size_t>(g + 8) * D * 2;
+    const uint8_t* brow = reinterpret_cast<const uint8_t*>(s_x) + static_cast<size_t>(g < T ? g : 0) * D * 2;
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    constexpr int KW = D / kTnWarps;
 #pragma unroll
-      for (int t = 0; t < kTnMaxTokens; ++t) a[t] = 0.f;
-#pragma unroll 2
-      for (int i = lane; i < D / 8; i += 32) {
-        const uint4 wv = lds128(row + 16 * i);
-        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-        for (int t = 0; t < kTnMaxTokens; ++t) {
-          if (t < T) {
-            const uint4 xv = lds128(s_x + static_cast<size_t>(t) * D + 8 * i);
-            const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              a[t] = fmaf(bf16_bits_to_f32(ww[q] & 0xFFFFu), bf16_bits_to_f32(xx[q] & 0xFFFFu), a[t]);
-              a[t] = fmaf(__uint_as_float(ww[q] & 0xFFFF0000u), __uint_as_float(xx[q] & 0xFFFF0000u), a[t]);
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int t = 0; t < kTnMaxTokens; ++t) {
-        if (t < T) {
-          const float logit = warp_sum(a[t]) * s_irms[t];
-          if (lane < CS) st_cluster_f32(s_logits + t * E + r, static_cast<unsigned>(lane), logit);
-        }
-      }
+    for (int s = 0; s < KW / 16; ++s) {
+      const int kb = (warp * KW + 16 * s + 2 * t4) * 2;  // byte offset of the lane's k pair
+      mma_bf16_16816(c, lds32(arow0 + kb), lds32(arow1 + kb), lds32(arow0 + kb + 16), lds32(arow1 + kb + 16),
+                     lds32(brow + kb), lds32(brow + kb + 16));
+    }
+    float* rw = red + warp * 128;
+    rw[g * 8 + 2 * t4] = c[0];
+    rw[g * 8 + 2 * t4 + 1] = c[1];
+    rw[(g + 8) * 8 + 2 * t4] = c[2];
+    rw[(g + 8) * 8 + 2 * t4 + 1] = c[3];
+  }
+  __syncthreads();
+  if (ok && tid < 128) {
+    const int rr = tid >> 3, t = tid & 7;
+    if (rr < r1 - r0 && t < T) {
+      float v = 0.f;
+      for (int w = 0; w < kTnWarps; ++w) v += red[w * 128 + tid];
+      const float logit = v * s_irms[t];
+#pragma unroll 4
+      for (int dst = 0; dst < CS; ++dst) st_cluster_f32(s_logits + t * E + r0 + rr, static_cast<unsigned>(dst), logit);
     }
   }
   for (int i = tid; i < kTnMaxTokens * (D / 8); i += blockDim.x) {
@@ -273,27 +288,43 @@ __global__ void __launch_bounds__(kTnWarps * 32, 1) k_tokn(TokNParams p, const _
   const int n_st = n_my * NSW;
   const int gt = warp / KP, gp = warp % KP;   // gate/up tile and K part
   const int dt = warp / DKP, dp = warp % DKP; // down tile and K part
-  auto issue = [&](int q) {
+  // a stage's three operations (the barrier's byte count, the codes box, the
+  // scales box) go out from lanes 0, 1, 2 at once: one thread takes ~0.25 us
+  // per operation, so lane 0 alone made every stage cost three of those (the
+  // barrier's phase completes only when the arrival and all bytes are in,
+  // whatever their order)
+  auto issue = [&](int q) {  // lanes 0..2
     const int it = q / NSW, kk = q % NSW, e = s_act[cl + NC * it], slot = q % kTnSlots;
     uint8_t* cs = rcodes + (warp * kTnSlots + slot) * kTnStageCodes;
     uint8_t* sc = rscales + (warp * kTnSlots + slot) * kTnStageScales;
-    mbar_arrive_expect_tx(&wb[slot], kTnStageCodes + kTnStageScales);
-    if (kk < gsw) {
-      const int kc = gp * 512 + kk * 256, y = (static_cast<int>(rank) * TL + gt) * 16;
-      tma_load_3d(cs, &maps.gu_codes, kc / 2, y, e, &wb[slot]);
-      tma_load_3d(sc, &maps.gu_scales, kc / 16, y, e, &wb[slot]);
-    } else {
-      const int kc = dp * 256, y = static_cast<int>(rank) * RPC + dt * 16;
-      tma_load_3d(cs, &maps.dn_codes, kc / 2, y, e, &wb[slot]);
-      tma_load_3d(sc, &maps.dn_scales, kc / 16, y, e, &wb[slot]);
-    }
+    const bool gu = kk < gsw;
+    const int kc = gu ? gp * 512 + kk * 256 : dp * 256;
+    const int y = gu ? (static_cast<int>(rank) * TL + gt) * 16 : static_cast<int>(rank) * RPC + dt * 16;
+    if (lane == 0) mbar_arrive_expect_tx(&wb[slot], kTnStageCodes + kTnStageScales);
+    else if (lane == 1) tma_load_3d(cs, gu ? &maps.gu_codes : &maps.dn_codes, kc / 2, y, e, &wb[slot]);
+    else tma_load_3d(sc, gu ? &maps.gu_scales : &maps.dn_scales, kc / 16, y, e, &wb[slot]);
   };
-  int issued = 0;
-  if (lane == 0) {
-    // the router rows in the codes area are read: order those reads first
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    for (; issued < kTnSlots && issued < n_st; ++issued) issue(issued);
+  // this CTA's slices of its items two ahead are prefetched into L2, so that
+  // the HBM stream runs ahead of the per-warp rings across the cluster barriers
+  auto prefetch_item = [&](int it) {
+    if (it >= n_my) return;
+    const int e = s_act[cl + NC * it];
+    const uint8_t* cb = p.codes + static_cast<long long>(e) * p.cpe;
+    const uint8_t* sb = p.scales + static_cast<long long>(e) * p.spe;
+    prefetch_l2(cb + static_cast<size_t>(rank) * UPC * D, UPC * D);
+    prefetch_l2(sb + static_cast<size_t>(rank) * UPC * (D / 8), UPC * (D / 8));
+    prefetch_l2(cb + static_cast<size_t>(I) * D + static_cast<size_t>(rank) * RPC * (I / 2), RPC * (I / 2));
+    prefetch_l2(sb + static_cast<size_t>(I) * (D / 8) + static_cast<size_t>(rank) * RPC * (I / 16), RPC * (I / 16));
+  };
+  if (tid == 0) {
+    prefetch_item(0);
+    prefetch_item(1);
   }
+  int issued = 0;  // stages issued (the same in every lane)
+  // the router rows in the codes area are read: order those reads first
+  if (lane < 3) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  for (; issued < kTnSlots && issued < n_st; ++issued)
+    if (lane < 3) issue(issued);
   int q = 0, q_fail = -1;  // stages consumed; first stage whose wait gave up
   auto wait_stage = [&]() -> bool {
     bool good = ok && (*reinterpret_cast<volatile int*>(&s_fail) == 0);
@@ -308,9 +339,11 @@ __global__ void __launch_bounds__(kTnWarps * 32, 1) k_tokn(TokNParams p, const _
   };
   auto release_stage = [&]() {  // the slot's data is read: refill it
     __syncwarp();
-    if (lane == 0 && ok && issued < n_st) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue(issued);
+    if (ok && issued < n_st) {
+      if (lane < 3) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue(issued);
+      }
       ++issued;
     }
     ++q;
@@ -319,6 +352,7 @@ __global__ void __launch_bounds__(kTnWarps * 32, 1) k_tokn(TokNParams p, const _
 
   for (int it = 0; it < n_my; ++it) {
     const int a = cl + NC * it, buf = it & 1;
+    if (tid == 0) prefetch_item(it + 2);
     const int e = s_act[a], pb = s_off[a], ne = s_off[a + 1] - pb;
     // the lane's ldmatrix row: the token of column lane % 8 (unused columns repeat column 0)
     const int my_pair = s_pair[pb + ((lane & 7) < ne ? (lane & 7) : 0)];
