@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(512, 1) k_debug_decode_tmem(const uint8_t* cod
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   if (warp >= 8)
-    for (int sub = 0; sub < 4; ++sub) dequant_slice_tmem(raw, sub, tmem + 32u * sub, warp, lane);
+    for (int sub = 0; sub < 4; ++sub) dequant_slice_tmem(raw, sub, tmem + 32u * sub, warp & 3, (warp - 8) >> 2, lane);
   tmem_wait_st();
   tc_fence_before();
   __syncthreads();
@@ -913,29 +913,30 @@ int tokn_maps(TokNMaps* m, const Dims& s, const flint_moe_weights* wts) {
                     sdims, sstr, sbox, false);
 }
 
-// Ring depths of the tensor-core kernels for a call of T tokens: B stages hold
-// the largest expert's rows (T rounded up to 16), four of them; NVFP4 keeps
-// four A stages and as many raw-weight stages as fit; bf16 weights as many A
-// stages as fit. Returns the dynamic shared-memory bytes.
+// Ring depths of the tensor-core kernels for a call of T tokens: a B stage
+// holds the largest expert's rows (T rounded up to whole 64-row boxes), and
+// items with at most 64 tokens get two accumulators (and two MMA issuers).
+// Returns the dynamic shared-memory bytes.
 size_t mma_configure(MmaParams& m, int T) {
   constexpr size_t kBudget = 220 * 1024 - 1024;
   const int npad = std::min(kMmaMaxTokens, (T + 15) & ~15);
   m.b_bytes = ((npad + 63) & ~63) * 128;  // whole 64-row boxes
   m.ksplit = (npad <= kMmaMaxTokens / 2) ? 2 : 1;
-  // A stages are recycled only after their MMAs complete, so the A ring must
-  // cover that round trip: NVFP4 keeps 8 stages in tensor memory (columns
-  // 256..511) fed by 4 raw stages; bf16 weights take the shared memory left
-  // after 6 activation-row stages
-  m.n_b = 6;
-  const size_t bbytes = static_cast<size_t>(m.n_b) * m.b_bytes;
-  size_t wbytes;
+  // A and B rings have the same depth (one stage of each per 64-wide K slice,
+  // freed together). A stages are recycled only after their MMAs complete, so
+  // the rings must cover that round trip: NVFP4 keeps 8 A stages in tensor
+  // memory (columns 256..511) fed by raw stages in the shared memory left after
+  // 8 activation-row stages; bf16 weights take as many A + B stage pairs as fit
+  size_t wbytes, bbytes;
   if (m.nvfp4) {
-    m.n_a = 8;
+    m.n_a = m.n_b = 8;
+    bbytes = static_cast<size_t>(m.n_b) * m.b_bytes;
     m.n_raw = static_cast<int>(std::min<size_t>(8, (kBudget - bbytes) / kMmaRawBytes));
     wbytes = static_cast<size_t>(m.n_raw) * kMmaRawBytes;
   } else {
     m.n_raw = 1;
-    m.n_a = static_cast<int>(std::min<size_t>(kMmaMaxStages, (kBudget - bbytes) / kMmaABytes));
+    m.n_a = m.n_b = static_cast<int>(std::min<size_t>(kMmaMaxStages, kBudget / (kMmaABytes + m.b_bytes)));
+    bbytes = static_cast<size_t>(m.n_b) * m.b_bytes;
     wbytes = static_cast<size_t>(m.n_a) * kMmaABytes;
   }
   return 1024 + wbytes + bbytes;

@@ -334,13 +334,13 @@ struct MmaMaps {
   CUtensorMap brows;
 };
 
-// Dequantise one 64-element slice of K of the 128-row A tile straight into
-// tensor memory (NVFP4 weights): dequantiser warp w (8..15) owns the lanes of
-// its quarter (rows 32*(w%4)..+31) and half (w-8)/4 of the slice's K: 32 codes
-// and their 2 scales of its row -> 16 columns of two f16 values each. The
-// operand never passes through shared memory.
-__device__ __forceinline__ void dequant_slice_tmem(const uint8_t* raw, int sub, uint32_t a_tmem, int warp, int lane) {
-  const int qtr = warp & 3, half = (warp - 8) >> 2;
+// Dequantise one half (32 elements) of a 64-element slice of K of the 128-row
+// A tile straight into tensor memory (NVFP4 weights): the warp owns the lanes
+// of its quarter (rows 32*qtr..+31, qtr = warp % 4): 32 codes and their 2
+// scales of its row -> 16 columns of two f16 values each. The operand never
+// passes through shared memory.
+__device__ __forceinline__ void dequant_slice_tmem(const uint8_t* raw, int sub, uint32_t a_tmem, int qtr, int half,
+                                                   int lane) {
   const int r = 32 * qtr + lane;
   const int chunk = 2 * sub + half;  // 16-byte code chunk of the 128-byte raw row
   const uint4 cv = lds128(raw + r * 128 + ((chunk ^ (r & 7)) << 4));
@@ -369,15 +369,20 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     k_mma_ffn(MmaParams p, const __grid_constant__ MmaMaps maps, int ncols) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t raw_full[kMmaMaxStages], raw_empty[kMmaMaxStages];
-  __shared__ __align__(8) uint64_t a_full[kMmaMaxStages], a_empty[kMmaMaxStages];
-  __shared__ __align__(8) uint64_t b_full[kMmaMaxStages], b_empty[kMmaMaxStages];
+  // A and B stages advance together (one of each per 64-wide K slice, rings
+  // of the same depth), so one barrier says both of a slot are free
+  __shared__ __align__(8) uint64_t a_full[kMmaMaxStages], b_full[kMmaMaxStages], ab_empty[kMmaMaxStages];
   __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_nact;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool fp4 = p.nvfp4 != 0;
-  const int NR = p.n_raw, NA = p.n_a, NB = p.n_b, BB = p.b_bytes;
+  const int NR = p.n_raw, NA = p.n_a, BB = p.b_bytes;  // p.n_b == p.n_a
+  // MMA issuers: with two accumulators per item, each has its own thread
+  // (warps 1 and 3), issuing the K steps of its accumulator (a thread takes
+  // ~60 ns per tcgen05.mma, more than the MMA itself at these N)
+  const int NI = p.ksplit;
   // 1024-aligned carve-up: [raw stages (NVFP4 only)][A stages][B stages]
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* raw = base;
@@ -395,16 +400,15 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     for (int i = 0; i < kMmaMaxStages; ++i) {
       mbar_init(&raw_full[i], 1);
       mbar_init(&raw_empty[i], 8);
-      mbar_init(&a_full[i], fp4 ? 8 : 1);
-      mbar_init(&a_empty[i], 1);
+      mbar_init(&a_full[i], fp4 ? 4 : 1);
       mbar_init(&b_full[i], 1);
-      mbar_init(&b_empty[i], 1);
+      mbar_init(&ab_empty[i], NI);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_full[i], NI);
       mbar_init(&acc_empty[i], 4);
     }
-    mbar_init(&mma_done, 1);
+    mbar_init(&mma_done, NI);
     fence_barrier_init();
     s_abort = 0;
   }
@@ -449,7 +453,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
           ++rc;
         } else {
           const int slot = ac % NA;
-          if (!(ok = __all_sync(0xffffffffu, mma_wait(&a_empty[slot], ((ac / NA) & 1) ^ 1, abort_flag, p.status))))
+          if (!(ok = __all_sync(0xffffffffu, mma_wait(&ab_empty[slot], ((ac / NA) & 1) ^ 1, abort_flag, p.status))))
             break;
           if (lane == 0) mbar_arrive_expect_tx(&a_full[slot], kMmaABytes);
           else if (lane == 1) tma_load_3d(abuf + slot * kMmaABytes, &maps.codes, s * 64, t * 128, e, &a_full[slot]);
@@ -470,8 +474,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
       const int off = p.rt.off[a], nt = p.rt.off[a + 1] - off;
       const int npad = (nt + 15) & ~15;
       for (int s = 0; s < n_sub && ok; ++s) {
-        const int slot = bc % NB;
-        if (!(ok = __all_sync(0xffffffffu, mma_wait(&b_empty[slot], ((bc / NB) & 1) ^ 1, abort_flag, p.status))))
+        const int slot = bc % NA;
+        if (!(ok = __all_sync(0xffffffffu, mma_wait(&ab_empty[slot], ((bc / NA) & 1) ^ 1, abort_flag, p.status))))
           break;
         // 64-row boxes (rows past the expert's tokens are loaded but not
         // multiplied; rows past the last pair are zero-filled)
@@ -482,11 +486,12 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
         ++bc;
       }
     }
-    if (!ok && lane == 0) drain(b_full, NB, bc);
-  } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer
+    if (!ok && lane == 0) drain(b_full, NA, bc);
+  } else if (warp == 1 || (warp == 3 && NI == 2)) {
+    // ------------------------------------------------ MMA issuers
     if (lane == 0) {
-      int sc = 0, bcount = 0, icount = 0;
+      const int iss = warp == 1 ? 0 : 1;  // accumulator (K steps iss, iss + NI, ...)
+      int sc = 0, icount = 0;
       bool ok = true;
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++icount) {
         const int a = it / tiles;
@@ -496,38 +501,31 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
         const int ab = icount & 1;
         if (!(ok = mma_wait(&acc_empty[ab], ((icount >> 1) & 1) ^ 1, abort_flag, p.status))) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * kMmaMaxTokens);
-        // consecutive K steps alternate between `ksplit` accumulators of
-        // kMmaMaxTokens / ksplit columns: independent accumulation chains
-        const uint32_t dstep = static_cast<uint32_t>(kMmaMaxTokens / p.ksplit);
-        const int kmask = p.ksplit - 1;
+        // the NI accumulators of an item are kMmaMaxTokens / NI columns apart;
+        // independent accumulation chains, summed in the epilogue
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * kMmaMaxTokens + iss * (kMmaMaxTokens / NI));
         for (int s = 0; s < n_sub; ++s) {
-          const int as = sc % NA, bs = bcount % NB;
+          const int as = sc % NA;
           if (!(ok = mma_wait(&a_full[as], (sc / NA) & 1, abort_flag, p.status))) break;
-          if (!(ok = mma_wait(&b_full[bs], (bcount / NB) & 1, abort_flag, p.status))) break;
+          if (!(ok = mma_wait(&b_full[as], (sc / NA) & 1, abort_flag, p.status))) break;
           tc_fence_after();
-          const uint32_t baddr = smem_addr(bbuf + bs * BB);
+          const uint32_t baddr = smem_addr(bbuf + as * BB);
           if (fp4) {
             const uint32_t a_tmem = tmem + kAccCols + static_cast<uint32_t>(32 * as);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_ts(d_tmem + dstep * (kk & kmask), a_tmem + 8 * kk, sw128_desc(baddr + 32 * kk), idesc,
-                         (s > 0 || kk > kmask) ? 1u : 0u);
+            for (int kk = iss; kk < 4; kk += NI)
+              mma_f16_ts(d_tmem, a_tmem + 8 * kk, sw128_desc(baddr + 32 * kk), idesc, (s > 0 || kk >= NI) ? 1u : 0u);
           } else {
             const uint32_t aaddr = smem_addr(abuf + as * kMmaABytes);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16(d_tmem + dstep * (kk & kmask), sw128_desc(aaddr + 32 * kk), sw128_desc(baddr + 32 * kk), idesc,
-                      (s > 0 || kk > kmask) ? 1u : 0u);
+            for (int kk = iss; kk < 4; kk += NI)
+              mma_f16(d_tmem, sw128_desc(aaddr + 32 * kk), sw128_desc(baddr + 32 * kk), idesc,
+                      (s > 0 || kk >= NI) ? 1u : 0u);
           }
-          mma_commit(&a_empty[as]);
-          mma_commit(&b_empty[bs]);
+          mma_commit(&ab_empty[as]);
           ++sc;
-          ++bcount;
         }
         if (ok) mma_commit(&acc_full[ab]);
       }
-      // every MMA this thread issued completes before tensor memory is freed
+      // every MMA of both issuers completes before tensor memory is freed
       mma_commit(&mma_done);
       mbar_wait(&mma_done, 0, p.status);
     }
@@ -599,22 +597,29 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     }
   } else if (warp >= 8 && fp4) {
     // ------------------------------------------------ dequantisers (NVFP4)
+    // two groups of four warps (one per tensor-memory lane quarter) take the
+    // even and the odd slices, so that two slices are converted at once; a
+    // warp converts both halves of its slices' K for its quarter
+    const int grp = (warp - 8) >> 2, qtr = warp & 3;
     int rc = 0, sc = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       for (int s = 0; s < n_sub; ++s) {
         const int rs = rc % NR, as = sc % NA;
-        if (!(ok = mma_wait(&raw_full[rs], (rc / NR) & 1, abort_flag, p.status))) break;
-        if (!(ok = mma_wait(&a_empty[as], ((sc / NA) & 1) ^ 1, abort_flag, p.status))) break;
-        tc_fence_after();  // the stage's previous MMAs are done (a_empty) before it is rewritten
-        dequant_slice_tmem(raw + rs * kMmaRawBytes, s & 3, tmem + kAccCols + static_cast<uint32_t>(32 * as), warp,
-                           lane);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[as]);
+        if ((s & 1) == grp) {
+          if (!(ok = mma_wait(&raw_full[rs], (rc / NR) & 1, abort_flag, p.status))) break;
+          if (!(ok = mma_wait(&ab_empty[as], ((sc / NA) & 1) ^ 1, abort_flag, p.status))) break;
+          tc_fence_after();  // the stage's previous MMAs are done before it is rewritten
+          const uint32_t a_tmem = tmem + kAccCols + static_cast<uint32_t>(32 * as);
+          dequant_slice_tmem(raw + rs * kMmaRawBytes, s & 3, a_tmem, qtr, 0, lane);
+          dequant_slice_tmem(raw + rs * kMmaRawBytes, s & 3, a_tmem, qtr, 1, lane);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[as]);
+        }
         ++sc;
-        if ((s & 3) == 3) {
+        if ((s & 3) == 3) {  // both groups are done with this raw stage
           if (lane == 0) mbar_arrive(&raw_empty[rs]);
           ++rc;
         }
