@@ -62,9 +62,10 @@ def _tensor_peak(wdtype: str):
 
 
 # DRAM bytes (read + write) of one launch of the batch-1 cluster kernel
-# (k_tok1<2048, 512>), from an ncu capture of `bench.py --profile t1`; None
-# whenever the kernel changes until it is captured again.
-TRAFFIC_K_TOK1 = None
+# (k_tok1<2048, 512>), from an ncu capture of `bench.py --profile t1`
+# (13,482,752 read + 0 written: the seven experts, the router rows and x);
+# None whenever the kernel changes until it is captured again.
+TRAFFIC_K_TOK1 = 13482752
 
 
 def _host_cores():
@@ -533,6 +534,9 @@ def main():
         K8 = 2 * N_LAYERS * 40
         ms8, _ = run_chain(stack, r8, w2.T, K8, 2 * N_LAYERS, fixed_inputs=fx8)
         ms8 = _max_over_ranks(ms8)
+        # the same steps through the batch-2..8 cluster kernel (layer_variant CLUSTER)
+        ms8c, _ = run_chain(stack, r8, w2.T, K8, 2 * N_LAYERS, fixed_inputs=fx8, variant=stack.fm.FLINT_LAYER_CLUSTER)
+        ms8c = _max_over_ranks(ms8c)
         g8_ms, g8_bytes, _, ids8 = kernel_timing(stack, r8, w2.T, 2 * N_LAYERS, fixed_inputs=fx8)
         sb8 = np.mean([step_bytes(w2, ids8[i]) for i in range(ids8.shape[0])])
         unions = [len(np.unique(ids8[i])) for i in range(ids8.shape[0])]
@@ -547,7 +551,10 @@ def main():
                             "union_experts_mean": float(np.mean(unions)), "overlap_mean": float(np.mean(ov)),
                             "layer_kernel": {"name": "k_layer (tensor-core variant)", "us": g8_ms * 1e3, "bytes": g8_bytes,
                                              "gbs": g8_bytes / (g8_ms / 1e3) / 1e9,
-                                             "frac_of_peak": g8_bytes / (g8_ms / 1e3) / 1e9 / peak}}
+                                             "frac_of_peak": g8_bytes / (g8_ms / 1e3) / 1e9 / peak},
+                            "cluster_kernel": {"name": "k_tokn (layer_variant CLUSTER, not the default)",
+                                               "us_per_layer": ms8c / K8 * 1e3,
+                                               "frac_of_peak": sb8 / (ms8c / K8 / 1e3) / 1e9 / peak}}
         # 47-layer stack at batch 4 (residual chain)
         w4 = synth.CONFIGS["cfg3_t4"]
         K4 = 2 * N_LAYERS * 40
