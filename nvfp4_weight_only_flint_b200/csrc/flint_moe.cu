@@ -920,16 +920,17 @@ int tokn_maps(TokNMaps* m, const Dims& s, const flint_moe_weights* wts) {
 size_t mma_configure(MmaParams& m, int T) {
   constexpr size_t kBudget = 220 * 1024 - 1024;
   const int npad = std::min(kMmaMaxTokens, (T + 15) & ~15);
-  m.b_bytes = ((npad + 63) & ~63) * 128;  // whole 64-row boxes
+  m.b_bytes = ((npad + 63) & ~63) * 2 * kMmaSliceK;  // whole 64-row boxes, one slice of K
   m.ksplit = (npad <= kMmaMaxTokens / 2) ? 2 : 1;
-  // A and B rings have the same depth (one stage of each per 64-wide K slice,
-  // freed together). A stages are recycled only after their MMAs complete, so
-  // the rings must cover that round trip: NVFP4 keeps 8 A stages in tensor
-  // memory (columns 256..511) fed by raw stages in the shared memory left after
-  // 8 activation-row stages; bf16 weights take as many A + B stage pairs as fit
+  // A and B rings have the same depth (one stage of each per 128-wide K
+  // slice, freed together). A stages are recycled only after their MMAs
+  // complete, so the rings must cover that round trip: NVFP4 keeps 4 A stages
+  // in tensor memory (columns 256..511, 64 each) fed by raw stages in the
+  // shared memory left after 4 activation-row stages; bf16 weights take as
+  // many A + B stage pairs as fit
   size_t wbytes, bbytes;
   if (m.nvfp4) {
-    m.n_a = m.n_b = 8;
+    m.n_a = m.n_b = 4;
     bbytes = static_cast<size_t>(m.n_b) * m.b_bytes;
     m.n_raw = static_cast<int>(std::min<size_t>(8, (kBudget - bbytes) / kMmaRawBytes));
     wbytes = static_cast<size_t>(m.n_raw) * kMmaRawBytes;

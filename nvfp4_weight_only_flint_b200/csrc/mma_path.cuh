@@ -47,7 +47,12 @@ constexpr int kMmaMaxTokens = 128;  // N of one MMA <= 128 (tokens of one expert
 constexpr int kMmaWarps = 16;
 constexpr int kMmaMaxStages = 16;   // ring depths are chosen per call, up to this
 constexpr int kMmaRawBytes = 128 * 128 + 128 * 16;  // NVFP4 stage, 256 of K: codes (swizzled) + scales
-constexpr int kMmaABytes = 128 * 128;               // A operand stage: 128 rows x 64 of K, 16-bit
+// A pipeline slice is 128 of K (8 MMAs of K = 16): every slice costs the MMA
+// thread a fixed ~0.25 us of waits, fence and commit besides its MMAs, so the
+// wider slice halves that overhead per weight (64-wide slices measured ~0.3 us
+// per slice of it)
+constexpr int kMmaSliceK = 128;
+constexpr int kMmaABytes = 128 * kMmaSliceK * 2;    // bf16 A stage: 128 rows x 128 of K (two 64-wide boxes)
 
 enum MmaEpi { kEpiGateUp = 0, kEpiDown = 1 };
 
@@ -79,7 +84,7 @@ struct MmaParams {
   int T, d, I, E, k, S;
   int nvfp4;                // 1: NVFP4 weights, f16 operands; 0: bf16 weights, bf16 operands
   int n_raw, n_a, n_b;      // ring depths (raw NVFP4 stages, A stages, B stages)
-  int b_bytes;              // B stage: (tokens rounded up to 64, at most 128) x 128 bytes
+  int b_bytes;              // B stage: (tokens rounded up to 64, at most 128) x 256 bytes (128 of K)
   int ksplit;               // accumulators per item (1 or 2), fed alternate K steps, summed in the epilogue
 };
 
@@ -393,7 +398,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
   constexpr uint32_t kAccCols = 2 * kMmaMaxTokens;
   const int K = EPI == kEpiGateUp ? p.d : p.I;
   const int tiles = EPI == kEpiGateUp ? p.I / 64 : p.d / 128;
-  const int n_sub = K / 64;
+  const int n_sub = K / kMmaSliceK;
   const int KS = p.k + p.S;
 
   if (tid == 0) {
@@ -442,21 +447,23 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
       const int e = p.rt.act[a];
       for (int s = 0; s < n_sub && ok; ++s) {
         if (fp4) {
-          if ((s & 3) != 0) continue;
+          if ((s & 1) != 0) continue;
           const int slot = rc % NR;
           if (!(ok = __all_sync(0xffffffffu, mma_wait(&raw_empty[slot], ((rc / NR) & 1) ^ 1, abort_flag, p.status))))
             break;
           uint8_t* st = raw + slot * kMmaRawBytes;
           if (lane == 0) mbar_arrive_expect_tx(&raw_full[slot], kMmaRawBytes);
-          else if (lane == 1) tma_load_3d(st, &maps.codes, (s / 4) * 128, t * 128, e, &raw_full[slot]);
-          else if (lane == 2) tma_load_3d(st + 128 * 128, &maps.scales, (s / 4) * 16, t * 128, e, &raw_full[slot]);
+          else if (lane == 1) tma_load_3d(st, &maps.codes, (s / 2) * 128, t * 128, e, &raw_full[slot]);
+          else if (lane == 2) tma_load_3d(st + 128 * 128, &maps.scales, (s / 2) * 16, t * 128, e, &raw_full[slot]);
           ++rc;
         } else {
           const int slot = ac % NA;
           if (!(ok = __all_sync(0xffffffffu, mma_wait(&ab_empty[slot], ((ac / NA) & 1) ^ 1, abort_flag, p.status))))
             break;
           if (lane == 0) mbar_arrive_expect_tx(&a_full[slot], kMmaABytes);
-          else if (lane == 1) tma_load_3d(abuf + slot * kMmaABytes, &maps.codes, s * 64, t * 128, e, &a_full[slot]);
+          else if (lane <= 2)  // the slice's two 64-wide K boxes
+            tma_load_3d(abuf + slot * kMmaABytes + (lane - 1) * (kMmaABytes / 2), &maps.codes,
+                        s * kMmaSliceK + (lane - 1) * 64, t * 128, e, &a_full[slot]);
           ++ac;
         }
       }
@@ -480,9 +487,13 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
         // 64-row boxes (rows past the expert's tokens are loaded but not
         // multiplied; rows past the last pair are zero-filled)
         const int nbox = (npad + 63) / 64;
-        if (lane == 0) mbar_arrive_expect_tx(&b_full[slot], nbox * 8192);
-        else if (lane <= nbox)
-          tma_load_2d(bbuf + slot * BB + (lane - 1) * 8192, &maps.brows, s * 64, off + 64 * (lane - 1), &b_full[slot]);
+        // two 64-wide K halves of the slice, each [rows][128 B] (half h at BB / 2 * h)
+        if (lane == 0) mbar_arrive_expect_tx(&b_full[slot], 2 * nbox * 8192);
+        else if (lane <= 2 * nbox) {
+          const int h = (lane - 1) / nbox, j = (lane - 1) % nbox;
+          tma_load_2d(bbuf + slot * BB + h * (BB / 2) + j * 8192, &maps.brows, s * kMmaSliceK + 64 * h, off + 64 * j,
+                      &b_full[slot]);
+        }
         ++bc;
       }
     }
@@ -511,14 +522,15 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
           tc_fence_after();
           const uint32_t baddr = smem_addr(bbuf + as * BB);
           if (fp4) {
-            const uint32_t a_tmem = tmem + kAccCols + static_cast<uint32_t>(32 * as);
-            for (int kk = iss; kk < 4; kk += NI)
-              mma_f16_ts(d_tmem, a_tmem + 8 * kk, sw128_desc(baddr + 32 * kk), idesc, (s > 0 || kk >= NI) ? 1u : 0u);
+            const uint32_t a_tmem = tmem + kAccCols + static_cast<uint32_t>(64 * as);
+            for (int kk = iss; kk < 8; kk += NI)
+              mma_f16_ts(d_tmem, a_tmem + 8 * kk, sw128_desc(baddr + (kk >> 2) * (BB / 2) + 32 * (kk & 3)), idesc,
+                         (s > 0 || kk >= NI) ? 1u : 0u);
           } else {
             const uint32_t aaddr = smem_addr(abuf + as * kMmaABytes);
-            for (int kk = iss; kk < 4; kk += NI)
-              mma_f16(d_tmem, sw128_desc(aaddr + 32 * kk), sw128_desc(baddr + 32 * kk), idesc,
-                      (s > 0 || kk >= NI) ? 1u : 0u);
+            for (int kk = iss; kk < 8; kk += NI)
+              mma_f16(d_tmem, sw128_desc(aaddr + (kk >> 2) * (kMmaABytes / 2) + 32 * (kk & 3)),
+                      sw128_desc(baddr + (kk >> 2) * (BB / 2) + 32 * (kk & 3)), idesc, (s > 0 || kk >= NI) ? 1u : 0u);
           }
           mma_commit(&ab_empty[as]);
           ++sc;
@@ -610,16 +622,19 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
           if (!(ok = mma_wait(&raw_full[rs], (rc / NR) & 1, abort_flag, p.status))) break;
           if (!(ok = mma_wait(&ab_empty[as], ((sc / NA) & 1) ^ 1, abort_flag, p.status))) break;
           tc_fence_after();  // the stage's previous MMAs are done before it is rewritten
-          const uint32_t a_tmem = tmem + kAccCols + static_cast<uint32_t>(32 * as);
-          dequant_slice_tmem(raw + rs * kMmaRawBytes, s & 3, a_tmem, qtr, 0, lane);
-          dequant_slice_tmem(raw + rs * kMmaRawBytes, s & 3, a_tmem, qtr, 1, lane);
+          const uint32_t a_tmem = tmem + kAccCols + static_cast<uint32_t>(64 * as);
+#pragma unroll
+          for (int sub2 = 0; sub2 < 2; ++sub2) {  // the slice's two 64-wide sub-slices of the raw stage
+            dequant_slice_tmem(raw + rs * kMmaRawBytes, 2 * (s & 1) + sub2, a_tmem + 32 * sub2, qtr, 0, lane);
+            dequant_slice_tmem(raw + rs * kMmaRawBytes, 2 * (s & 1) + sub2, a_tmem + 32 * sub2, qtr, 1, lane);
+          }
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&a_full[as]);
         }
         ++sc;
-        if ((s & 3) == 3) {  // both groups are done with this raw stage
+        if ((s & 1) == 1) {  // both groups are done with this raw stage (two slices)
           if (lane == 0) mbar_arrive(&raw_empty[rs]);
           ++rc;
         }
