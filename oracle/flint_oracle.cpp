@@ -459,7 +459,7 @@ int oracle_moe_forward(int32_t T, int32_t d, int32_t inter, int32_t E, int32_t k
 // selections token by token; the shared experts follow with every token.
 int32_t oracle_group(const int32_t* ids, int32_t T, int32_t k, int32_t E, int32_t S, int32_t* act,
                      int32_t* off, int32_t* pair, int32_t* n_routed) {
-  if (T < 0 || T > 256 || k < 1 || E < 1 || S < 0) return -1;
+  if (T < 0 || T > 65536 || k < 1 || E < 1 || S < 0) return -1;  // token << 8 stays within int32
   for (int i = 0; i < T * k; ++i)
     if (ids[i] < 0 || ids[i] >= E) return -1;
   int n = 0, p = 0;

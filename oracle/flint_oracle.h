@@ -115,7 +115,7 @@ int oracle_topk(const double* logits, int32_t T, int32_t E, int32_t k,
  * every token in slot k + s; off[a] = index of expert a's first pair, off[n]
  * = total. ids [T][k]. act holds up to E + S entries, off up to E + S + 1,
  * pair T*(k+S). Writes *n_routed (routed experts in use) and returns the
- * number of active experts, or -1 if an id lies outside [0, E) or T > 256. */
+ * number of active experts, or -1 if an id lies outside [0, E) or T > 65536. */
 int32_t oracle_group(const int32_t* ids, int32_t T, int32_t k, int32_t E, int32_t S,
                      int32_t* act, int32_t* off, int32_t* pair, int32_t* n_routed);
 
