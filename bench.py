@@ -414,6 +414,30 @@ def run_lm_head(world: int, n_heads: int = 3, calls: int = 60):
     return res
 
 
+def run_prefill(world: int, seed: int, T: int = 8192, n_layers: int = 4, calls: int = 12):
+    """One prefill-size call of 8192 tokens per layer on the tensor-core path
+    (counting-sort grouping, 128-token tiles), NVFP4 weights of the Flint
+    shape, 4 resident layers used in turn; the expert GEMMs' rate against the
+    16-bit tensor peak (the operands are f16, e2m1*e4m3 exact)."""
+    import torch
+    w = synth.CONFIGS["cfg1"]
+    st = Stack(w, n_layers, seed, max_tokens=T)
+    xs = [_bits_to_cuda(synth.x_bits(seed + 3000 + l, T, w.d)) for l in range(n_layers)]
+    rs = [_bits_to_cuda(synth.to_bf16_bits(synth.router_plain(seed, w.d, w.E, l))) for l in range(n_layers)]
+    ms, _ = run_chain(st, rs, T, calls, n_layers, fixed_inputs=xs)
+    ms = _max_over_ranks(ms)
+    per = ms / calls / 1e3
+    P = T * (w.k + w.S)
+    flops = 2.0 * P * 3 * w.inter * w.d
+    tf_peak, tf_kind = _tensor_peak("nvfp4")
+    del st, xs
+    torch.cuda.empty_cache()
+    return {"workload": f"{T} tokens through one d=2048/I=512/E=256+1 top-6 NVFP4 layer (prefill-size call)",
+            "ms_per_layer": per * 1e3, "tokens_per_s": world * T / per,
+            "expert_tflops": flops / per / 1e12, "frac_of_tensor_peak": flops / per / 1e12 / tf_peak,
+            "tensor_peak_tflops": tf_peak, "tensor_peak_kind": tf_kind}
+
+
 def cpu_baseline(n_tokens: int = 3, seed: int = 0):
     """The fp64 oracle as it stands, on host cores: T=1 layer decodes of the
     default workload (quantisation of the needed experts is untimed set-up),
@@ -603,6 +627,7 @@ def main():
             del st64, fx64, r64
             torch.cuda.empty_cache()
         extras["lm_head"] = run_lm_head(world)
+        extras["prefill"] = run_prefill(world, args.seed)
         extras["stack47"] = {
             "workload": "cfg3: 47 resident layers (21.4 GB NVFP4), residual chain, no attention",
             "batch1_tokens_per_s": tok_s / N_LAYERS, "batch1_us_per_layer": ms_step * 1e3,

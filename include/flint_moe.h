@@ -112,9 +112,11 @@ typedef enum flint_path {
   FLINT_PATH_AUTO = 0, /* NVFP4: GEMV kernels below 32 tokens, tensor-core path from
                           32; bf16 weights: tensor-core path */
   FLINT_PATH_GEMV = 1, /* CUDA-core dequant-GEMV kernels at any token count */
-  FLINT_PATH_MMA = 2   /* TMA-staged dequant-to-smem + tcgen05 MMA at any count up
-                          to 128 tokens; NVFP4 weights need inter >= 256; no
-                          input_rmsnorm */
+  FLINT_PATH_MMA = 2   /* TMA-staged dequant-to-tensor-memory + tcgen05 MMA at any
+                          count up to 16384 tokens (above 128 tokens the pairs
+                          are grouped by a counting sort and each expert's
+                          tokens are cut into tiles of 128; E + S <= 1024);
+                          NVFP4 weights need inter >= 256; no input_rmsnorm */
 } flint_path;
 
 typedef enum flint_layer_variant {
@@ -349,7 +351,10 @@ int flint_debug_decode(const flint_moe_weights* weights, const flint_moe_shape* 
  * device by one of the layer's grouping routines: impl 0 the CTA grouping of
  * the persistent single-kernel path and the tensor-core path (T <= 128),
  * impl 1 the warp grouping of the three-kernel path (T * top_k <= 64), impl 2
- * its CTA grouping (T <= 32). ids: device int32 [T][top_k]. Outputs (device):
+ * its CTA grouping (T <= 32), impl 3 the counting-sort grouping the
+ * tensor-core path uses above 128 tokens (T <= 16384, E + S <= 1024; its
+ * scratch needs a workspace of flint_moe_workspace_bytes for T tokens). ids:
+ * device int32 [T][top_k]. Outputs (device):
  * act int32 [E+S], off int32 [E+S+1], pair int32 [T*(top_k+S)], counts int32
  * [2] = {routed experts in use, active experts}. An id outside [0, E) is
  * skipped and sets FLINT_DEVCHECK_EXPERT_ID in the workspace status word (read

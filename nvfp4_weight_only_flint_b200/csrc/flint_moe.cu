@@ -322,6 +322,9 @@ __global__ void __launch_bounds__(32) k_debug_decode_frag(const uint8_t* codes, 
 // impl 0 the CTA grouping of the persistent kernel and the tensor-core path
 // (T <= 128), 1 the warp grouping of the three-kernel path (T*k <= 64), 2 its
 // CTA grouping (T <= 32). One CTA of 512 threads; outputs as int arrays.
+// counts[0] (routed experts in use) from counts[1] (active experts).
+__global__ void k_debug_routed_count(int* counts, int S) { counts[0] = counts[1] - S; }
+
 __global__ void __launch_bounds__(512) k_debug_group(const int* ids, int T, int k, int E, int S, int impl, int* act,
                                                      int* off, int* pair, int* counts, int* status) {
   __shared__ int s_ids[kMmaMaxTokens * kMaxTopK];
@@ -431,10 +434,18 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 struct WsLayout {
   size_t status, counter, rb_count, amax, desc, logits, tlogits, ids, gates, h, htag, tok1_part;
   size_t mma_n, mma_act, mma_off, mma_pair, xinv, hinv, xrows, hrows, y;  // tensor-core path
+  size_t mma_tiles, mma_mask, mma_wpre, mma_cnt;  // its token tiles and large-T grouping scratch
   size_t total;
 };
 
 size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Token tiles of a call of up to maxT tokens: each active expert's pairs in
+// runs of at most kMmaMaxTokens; at most P / kMmaMaxTokens + one per expert.
+size_t mma_max_tiles(const Dims& s, int maxT) {
+  const size_t P = static_cast<size_t>(maxT) * (s.k + s.S);
+  return P / kMmaMaxTokens + s.E + s.S + 1;
+}
 constexpr size_t kCtrlBytes = 1024;
 
 // Workspace carve-up for calls of up to maxT tokens. The first kCtrlBytes hold
@@ -477,6 +488,7 @@ WsLayout ws_layout(const Dims& s, int maxT, bool mma) {
   o += al256(sizeof(float) * P * s.I);
   if (!mma) {
     w.mma_n = w.mma_act = w.mma_off = w.mma_pair = w.xinv = w.hinv = w.xrows = w.hrows = w.y = 0;
+    w.mma_tiles = w.mma_mask = w.mma_wpre = w.mma_cnt = 0;
     w.total = o;
     return w;
   }
@@ -498,6 +510,18 @@ WsLayout ws_layout(const Dims& s, int maxT, bool mma) {
   o += al256(2 * P * s.I);
   w.y = o;
   o += al256(sizeof(float) * P * s.d);
+  // token tiles: [1 + 3 * max tiles] ints (count, then the three arrays)
+  w.mma_tiles = o;
+  o += al256(sizeof(int) * (1 + 3 * mma_max_tiles(s, maxT)));
+  // large-T grouping (more than kMmaGroupSmallT tokens): bit masks and word
+  // prefix counts [E][T/32], counts [E]
+  const size_t words = maxT > kMmaGroupSmallT ? static_cast<size_t>(s.E) * ((maxT + 31) / 32) : 0;
+  w.mma_mask = o;
+  o += al256(sizeof(uint32_t) * words);
+  w.mma_wpre = o;
+  o += al256(sizeof(int) * words);
+  w.mma_cnt = o;
+  o += al256(sizeof(int) * (words ? s.E : 0));
   w.total = o;
   return w;
 }
@@ -962,6 +986,14 @@ int run_mma_path(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, 
   m.rt.act = reinterpret_cast<int*>(ws + w.mma_act);
   m.rt.off = reinterpret_cast<int*>(ws + w.mma_off);
   m.rt.pair = reinterpret_cast<int*>(ws + w.mma_pair);
+  m.rt.n_tiles = reinterpret_cast<int*>(ws + w.mma_tiles);
+  const size_t max_tiles = mma_max_tiles(s, T);
+  m.rt.tile_a = m.rt.n_tiles + 1;
+  m.rt.tile_off = m.rt.tile_a + max_tiles;
+  m.rt.tile_n = m.rt.tile_off + max_tiles;
+  m.rt.mask = reinterpret_cast<uint32_t*>(ws + w.mma_mask);
+  m.rt.wpre = reinterpret_cast<int*>(ws + w.mma_wpre);
+  m.rt.cnt = reinterpret_cast<int*>(ws + w.mma_cnt);
   m.xrows = reinterpret_cast<uint16_t*>(ws + w.xrows);
   m.xinv = reinterpret_cast<float*>(ws + w.xinv);
   m.h = p.h;
@@ -985,8 +1017,19 @@ int run_mma_path(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, 
   if (e != cudaSuccess) return cuda_fail(e, "k_router_only launch");
   e = launch(k_topk, dim3((T + 7) / 8), dim3(256), 0, st, pdl, p);
   if (e != cudaSuccess) return cuda_fail(e, "k_topk launch");
-  e = launch(k_mma_group, dim3(1), dim3(512), 0, st, pdl, m);
-  if (e != cudaSuccess) return cuda_fail(e, "k_mma_group launch");
+  if (T <= kMmaGroupSmallT) {
+    e = launch(k_mma_group, dim3(1), dim3(512), 0, st, pdl, m);
+    if (e != cudaSuccess) return cuda_fail(e, "k_mma_group launch");
+  } else {
+    // prefill-size call: counting-sort grouping (mma_path.cuh)
+    const int g = std::max(1, std::min(4 * num_sms(), (T * s.k + 255) / 256));
+    e = launch(k_grp_zero, dim3(num_sms()), dim3(256), 0, st, pdl, m);
+    if (e == cudaSuccess) e = launch(k_grp_mask, dim3(g), dim3(256), 0, st, pdl, m);
+    if (e == cudaSuccess) e = launch(k_grp_scan, dim3((s.E + 7) / 8), dim3(256), 0, st, pdl, m);
+    if (e == cudaSuccess) e = launch(k_grp_final, dim3(1), dim3(1024), 0, st, pdl, m);
+    if (e == cudaSuccess) e = launch(k_grp_scatter, dim3(g), dim3(256), 0, st, pdl, m);
+    if (e != cudaSuccess) return cuda_fail(e, "grouping launch");
+  }
   e = launch(k_mma_prep, dim3((P + 7) / 8), dim3(256), 0, st, pdl, m);
   if (e != cudaSuccess) return cuda_fail(e, "k_mma_prep launch");
   const size_t smem = mma_configure(m, T);
@@ -1242,8 +1285,10 @@ int flint_moe_forward_ex(const uint16_t* x, int32_t T, const uint16_t* router_w,
     if (T > gemv_max_t)
       return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "GEMV path takes at most %d tokens at d=%d", gemv_max_t, s.d);
   } else {
-    if (T > kMmaMaxTokens)
-      return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "tensor-core path takes at most %d tokens (T=%d)", kMmaMaxTokens, T);
+    if (T > kMmaMaxCallTokens)
+      return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "tensor-core path takes at most %d tokens (T=%d)", kMmaMaxCallTokens, T);
+    if (T > kMmaGroupSmallT && s.E + s.S > 1024)
+      return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "more than %d tokens need E + S <= 1024", kMmaGroupSmallT);
     if (s.wd == FLINT_W_NVFP4 && s.I < 256)
       return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "tensor-core path with NVFP4 weights needs inter >= 256 (inter=%d)", s.I);
     if (options && options->input_rmsnorm)
@@ -1471,11 +1516,54 @@ int flint_debug_group(const int32_t* ids, int32_t T, const flint_moe_shape* shap
   if (rc != FLINT_OK) return rc;
   if (!ids || !act || !off || !pair || !counts || !workspace)
     return fail(FLINT_ERR_INVALID_ARG, "flint_debug_group: NULL pointer");
-  if (impl < 0 || impl > 2) return fail(FLINT_ERR_INVALID_ARG, "flint_debug_group: impl %d", impl);
-  const int max_t = impl == 0 ? kMmaMaxTokens : (impl == 1 ? 64 / s.k : kMaxGemvTokens);
+  if (impl < 0 || impl > 3) return fail(FLINT_ERR_INVALID_ARG, "flint_debug_group: impl %d", impl);
+  const int max_t = impl == 0 ? kMmaGroupSmallT
+                              : (impl == 1 ? 64 / s.k : (impl == 2 ? kMaxGemvTokens : kMmaMaxCallTokens));
   if (T < 1 || T > max_t) return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "flint_debug_group: impl %d takes 1..%d tokens", impl, max_t);
   if (ws_bytes < kCtrlBytes) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kCtrlBytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (impl == 3) {
+    // the tensor-core path's counting-sort grouping, scratch after the control block
+    if (s.E + s.S > 1024) return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "flint_debug_group: impl 3 needs E + S <= 1024");
+    const size_t tiles = mma_max_tiles(s, T), words = static_cast<size_t>(s.E) * ((T + 31) / 32);
+    const size_t need = kCtrlBytes + al256(sizeof(int) * (1 + 3 * tiles)) + 2 * al256(4 * words) + al256(4 * s.E);
+    if (ws_bytes < need) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    MmaParams m{};
+    m.ids = ids;
+    m.status = static_cast<int*>(workspace);
+    m.T = T;
+    m.E = s.E;
+    m.k = s.k;
+    m.S = s.S;
+    m.rt.act = act;
+    m.rt.off = off;
+    m.rt.pair = pair;
+    m.rt.n_active = counts + 1;
+    size_t o = kCtrlBytes;
+    m.rt.n_tiles = reinterpret_cast<int*>(w + o);
+    m.rt.tile_a = m.rt.n_tiles + 1;
+    m.rt.tile_off = m.rt.tile_a + tiles;
+    m.rt.tile_n = m.rt.tile_off + tiles;
+    o += al256(sizeof(int) * (1 + 3 * tiles));
+    m.rt.mask = reinterpret_cast<uint32_t*>(w + o);
+    o += al256(4 * words);
+    m.rt.wpre = reinterpret_cast<int*>(w + o);
+    o += al256(4 * words);
+    m.rt.cnt = reinterpret_cast<int*>(w + o);
+    const int g = std::max(1, std::min(4 * num_sms(), (T * s.k + 255) / 256));
+    cudaError_t e = launch(k_grp_zero, dim3(num_sms()), dim3(256), 0, st, false, m);
+    if (e == cudaSuccess) e = launch(k_grp_mask, dim3(g), dim3(256), 0, st, false, m);
+    if (e == cudaSuccess) e = launch(k_grp_scan, dim3((s.E + 7) / 8), dim3(256), 0, st, false, m);
+    if (e == cudaSuccess) e = launch(k_grp_final, dim3(1), dim3(1024), 0, st, false, m);
+    if (e == cudaSuccess) e = launch(k_grp_scatter, dim3(g), dim3(256), 0, st, false, m);
+    if (e == cudaSuccess) {
+      k_debug_routed_count<<<1, 1, 0, st>>>(counts, s.S);
+      e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "grouping launch");
+    return FLINT_OK;
+  }
   k_debug_group<<<1, 512, 0, st>>>(ids, T, s.k, s.E, s.S, impl, act, off, pair, counts, static_cast<int*>(workspace));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "k_debug_group launch");

@@ -43,7 +43,9 @@
 
 namespace flint {
 
-constexpr int kMmaMaxTokens = 128;  // N of one MMA <= 128 (tokens of one expert)
+constexpr int kMmaMaxTokens = 128;  // N of one MMA <= 128: an item's token tile
+constexpr int kMmaGroupSmallT = 128;     // up to this many tokens one CTA groups the pairs
+constexpr int kMmaMaxCallTokens = 16384; // tokens of one call on this path (prefill-size batches)
 constexpr int kMmaWarps = 16;
 constexpr int kMmaMaxStages = 16;   // ring depths are chosen per call, up to this
 constexpr int kMmaRawBytes = 128 * 128 + 128 * 16;  // NVFP4 stage, 256 of K: codes (swizzled) + scales
@@ -62,6 +64,17 @@ struct MmaRoute {
   int* act;       // [E+S] active experts (routed ascending, then shared)
   int* off;       // [E+S+1] first pair of each active expert
   int* pair;      // [T*(k+S)] token << 8 | slot, grouped by expert, token order
+  // token tiles: each active expert's pairs cut into runs of at most
+  // kMmaMaxTokens (the MMA's N); a work item is (tile, row tile)
+  int* n_tiles;   // [1]
+  int* tile_a;    // [max tiles] active index of the tile's expert
+  int* tile_off;  // [max tiles] first pair of the tile
+  int* tile_n;    // [max tiles] pairs in the tile
+  // large-T grouping scratch: per expert, a bit per token and the running
+  // count of set bits before each 32-token word
+  uint32_t* mask; // [E][T/32 rounded up]
+  int* wpre;      // [E][T/32 rounded up]
+  int* cnt;       // [E]
 };
 
 struct MmaParams {
@@ -203,6 +216,166 @@ __global__ void __launch_bounds__(512) k_mma_group(MmaParams p) {
   __shared__ int s_nrouted;
   cta_grouping(s_ids, p.T, p.k, p.E, p.S, p.rt.act, p.rt.off, p.rt.pair, &s_nrouted, p.rt.n_active, s_scratch,
                p.status);
+  // at most kMmaGroupSmallT tokens: one token tile per active expert
+  const int na = *p.rt.n_active;
+  for (int a = tid; a < na; a += blockDim.x) {
+    p.rt.tile_a[a] = a;
+    p.rt.tile_off[a] = p.rt.off[a];
+    p.rt.tile_n[a] = p.rt.off[a + 1] - p.rt.off[a];
+  }
+  if (tid == 0) *p.rt.n_tiles = na;
+}
+
+// ----------------------------------------------------------------- grouping, large T
+// For calls of more than kMmaGroupSmallT tokens (prefill-size batches) the
+// grouping is a counting sort that keeps token order, in five kernels:
+//   k_grp_zero     clears the per-expert token bitmasks and counts
+//   k_grp_mask     each routed (token, slot) pair sets its token's bit in its
+//                  expert's mask and counts once for its expert
+//   k_grp_scan     per expert (one warp): the number of set bits before each
+//                  32-token word of its mask
+//   k_grp_final    one CTA: active experts in ascending id (shared last), their
+//                  first pair, each expert's first pair by id, and the token
+//                  tiles (runs of at most kMmaMaxTokens pairs of one expert)
+//   k_grp_scatter  each pair's place: its expert's first pair + the set bits of
+//                  its expert's mask before its token
+// A token selects an expert at most once, so its bit is its pair's rank.
+__device__ __forceinline__ int grp_words(int T) { return (T + 31) >> 5; }
+
+__global__ void __launch_bounds__(256) k_grp_zero(MmaParams p) {
+  pdl_wait();  // the previous call's scatter has read the masks
+  pdl_trigger();
+  const int W = grp_words(p.T);
+  const int n = p.E * W;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p.rt.mask[i] = 0u;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.E; i += gridDim.x * blockDim.x) p.rt.cnt[i] = 0;
+}
+
+__global__ void __launch_bounds__(256) k_grp_mask(MmaParams p) {
+  pdl_wait();
+  pdl_trigger();
+  const int W = grp_words(p.T), n = p.T * p.k;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int e = p.ids[i], t = i / p.k;
+    if (p.ids_out != nullptr) {
+      p.ids_out[i] = e;
+      p.gates_out[i] = p.gates[i];
+    }
+    if (e < 0 || e >= p.E) {
+      atomicOr(p.status, FLINT_DEVCHECK_EXPERT_ID);
+      continue;
+    }
+    atomicOr(p.rt.mask + static_cast<size_t>(e) * W + (t >> 5), 1u << (t & 31));
+    atomicAdd(p.rt.cnt + e, 1);
+  }
+}
+
+__global__ void __launch_bounds__(256) k_grp_scan(MmaParams p) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31, e = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (e >= p.E) return;
+  const int W = grp_words(p.T);
+  const uint32_t* m = p.rt.mask + static_cast<size_t>(e) * W;
+  int* pre = p.rt.wpre + static_cast<size_t>(e) * W;
+  int run = 0;
+  for (int w0 = 0; w0 < W; w0 += 32) {
+    const int w = w0 + lane;
+    const int c = w < W ? __popc(m[w]) : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (w < W) pre[w] = run + incl - c;
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
+// Exclusive scan of one int per thread over a CTA of up to 1024 threads.
+__device__ __forceinline__ int cta_exclusive_scan(int v, int* s_warp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nw ? s_warp[lane] : 0;
+    const int x = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += u;
+    }
+    if (lane < nw) s_warp[lane] = w - x;
+    if (lane == 31) *total = w;
+  }
+  __syncthreads();
+  const int r = s_warp[warp] + incl - v;
+  __syncthreads();
+  return r;
+}
+
+// One CTA of 1024 threads; E <= 1024.
+__global__ void __launch_bounds__(1024) k_grp_final(MmaParams p) {
+  __shared__ int s_warp[32];
+  __shared__ int s_tot_pairs, s_tot_act, s_tot_tiles;
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x, E = p.E;
+  const int c = tid < E ? p.rt.cnt[tid] : 0;
+  const int base = cta_exclusive_scan(c, s_warp, &s_tot_pairs);   // expert's first pair (by id)
+  const int ai = cta_exclusive_scan(c > 0 ? 1 : 0, s_warp, &s_tot_act);  // active index
+  const int nr = s_tot_act, routed = s_tot_pairs;
+  if (tid < E) {
+    p.rt.cnt[tid] = base;
+    if (c > 0) {
+      p.rt.act[ai] = tid;
+      p.rt.off[ai] = base;
+    }
+  }
+  if (tid < p.S) {
+    p.rt.act[nr + tid] = E + tid;
+    p.rt.off[nr + tid] = routed + tid * p.T;
+  }
+  if (tid == 0) {
+    p.rt.off[nr + p.S] = routed + p.S * p.T;
+    *p.rt.n_active = nr + p.S;
+  }
+  for (int i = tid; i < p.S * p.T; i += blockDim.x)  // the shared experts' pairs, every token
+    p.rt.pair[routed + i] = ((i % p.T) << 8) | (p.k + i / p.T);
+  // token tiles of each active expert (routed: thread per expert id; shared:
+  // threads E.. E+S-1 stand for them)
+  const bool has = (tid < E && c > 0) || (tid >= E && tid < E + p.S);
+  const int a = tid < E ? ai : nr + (tid - E);
+  const int npairs = tid < E ? c : p.T;
+  const int ntt = has ? (npairs + kMmaMaxTokens - 1) / kMmaMaxTokens : 0;
+  const int t0 = cta_exclusive_scan(ntt, s_warp, &s_tot_tiles);
+  const int first = tid < E ? base : routed + (tid - E) * p.T;
+  for (int j = 0; j < ntt; ++j) {
+    p.rt.tile_a[t0 + j] = a;
+    p.rt.tile_off[t0 + j] = first + j * kMmaMaxTokens;
+    p.rt.tile_n[t0 + j] = min(kMmaMaxTokens, npairs - j * kMmaMaxTokens);
+  }
+  if (tid == 0) *p.rt.n_tiles = s_tot_tiles;
+}
+
+__global__ void __launch_bounds__(256) k_grp_scatter(MmaParams p) {
+  pdl_wait();
+  pdl_trigger();
+  const int W = grp_words(p.T), n = p.T * p.k, k = p.k;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int e = p.ids[i], t = i / k;
+    if (e < 0 || e >= p.E) continue;
+    const size_t wi = static_cast<size_t>(e) * W + (t >> 5);
+    const int pos = p.rt.cnt[e] + p.rt.wpre[wi] + __popc(p.rt.mask[wi] & ((1u << (t & 31)) - 1u));
+    p.rt.pair[pos] = (t << 8) | (i - t * k);
+  }
 }
 
 // ----------------------------------------------------------------- B rows of gate/up
@@ -422,11 +595,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
   __syncthreads();
   tc_fence_after();
   pdl_wait();
-  if (tid == 0) s_nact = p.rt.n_active[0];
+  if (tid == 0) s_nact = p.rt.n_tiles[0];
   __syncthreads();
   pdl_trigger();
   const uint32_t tmem = s_tmem;
-  const int n_items = s_nact * tiles;
+  const int n_items = s_nact * tiles;  // (token tile, row tile)
   volatile int* abort_flag = &s_abort;
   // on abort: wait (bounded) for every copy a producer started; stages older
   // than the ring depth were consumed, so they have landed
@@ -443,8 +616,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     int rc = 0, ac = 0;  // stages issued: raw NVFP4, A (bf16 weights)
     bool ok = true;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      const int a = it / tiles, t = it % tiles;
-      const int e = p.rt.act[a];
+      const int tt = it / tiles, t = it % tiles;  // token tile, row tile
+      const int e = p.rt.act[p.rt.tile_a[tt]];
       for (int s = 0; s < n_sub && ok; ++s) {
         if (fp4) {
           if ((s & 1) != 0) continue;
@@ -477,8 +650,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     int bc = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      const int a = it / tiles;
-      const int off = p.rt.off[a], nt = p.rt.off[a + 1] - off;
+      const int tt = it / tiles;
+      const int off = p.rt.tile_off[tt], nt = p.rt.tile_n[tt];
       const int npad = (nt + 15) & ~15;
       for (int s = 0; s < n_sub && ok; ++s) {
         const int slot = bc % NA;
@@ -505,8 +678,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
       int sc = 0, icount = 0;
       bool ok = true;
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++icount) {
-        const int a = it / tiles;
-        const int nt = p.rt.off[a + 1] - p.rt.off[a];
+        const int nt = p.rt.tile_n[it / tiles];
         const int npad = (nt + 15) & ~15;
         const uint32_t idesc = mma_idesc(128, npad, !fp4);
         const int ab = icount & 1;
@@ -546,9 +718,9 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     const int ew = warp - 4, m = 32 * ew + lane;  // accumulator lane = A tile row
     int icount = 0;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++icount) {
-      const int a = it / tiles, t = it % tiles;
-      const int e = p.rt.act[a];
-      const int off = p.rt.off[a], nt = p.rt.off[a + 1] - off;
+      const int tt = it / tiles, t = it % tiles;
+      const int e = p.rt.act[p.rt.tile_a[tt]];
+      const int off = p.rt.tile_off[tt], nt = p.rt.tile_n[tt];
       const int ab = icount & 1;
       if (!mma_wait(&acc_full[ab], (icount >> 1) & 1, abort_flag, p.status)) break;
       tc_fence_after();
