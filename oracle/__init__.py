@@ -91,6 +91,8 @@ def lib():
         L.oracle_dense_gemv.restype = i32
         L.oracle_group.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
         L.oracle_group.restype = i32
+        L.oracle_qk_norm_rope_kv.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, i32, vp, i32, f64, vp, vp, vp]
+        L.oracle_qk_norm_rope_kv.restype = i32
         _lib = L
     return _lib
 
@@ -260,6 +262,28 @@ def dense_gemv(m: NVFP4Matrix, x_bits: np.ndarray, rows=None) -> np.ndarray:
     if lib().oracle_dense_gemv(ctypes.byref(s), _ptr(x_bits), T, _ptr(r), n, _ptr(out)) != 0:
         raise ValueError("oracle_dense_gemv failed")
     return out
+
+
+def qk_norm_rope_kv(qkv_bits: np.ndarray, n_q_heads: int, n_kv_heads: int, q_w_bits, k_w_bits, cos_sin=None,
+                    positions=None, rope: bool = False, eps: float = 1e-6):
+    """Attention prologue of one layer in fp64 (see oracle_qk_norm_rope_kv):
+    qkv_bits bf16 [T][Hq + 2*Hkv][Dh]; returns (q [T][Hq][Dh], k, v [T][Hkv][Dh])."""
+    qkv = np.ascontiguousarray(qkv_bits, dtype=np.uint16)
+    T, H, Dh = qkv.shape
+    assert H == n_q_heads + 2 * n_kv_heads
+    qw = np.ascontiguousarray(q_w_bits, dtype=np.uint16)
+    kw = np.ascontiguousarray(k_w_bits, dtype=np.uint16)
+    cs = None if cos_sin is None else np.ascontiguousarray(cos_sin, dtype=np.float32)
+    pos = None if positions is None else np.ascontiguousarray(positions, dtype=np.int32)
+    max_pos = 0 if cs is None else cs.shape[0]
+    q = np.zeros((T, n_q_heads, Dh), dtype=np.float64)
+    k = np.zeros((T, n_kv_heads, Dh), dtype=np.float64)
+    v = np.zeros((T, n_kv_heads, Dh), dtype=np.float64)
+    rc = lib().oracle_qk_norm_rope_kv(T, n_q_heads, n_kv_heads, Dh, _ptr(qkv), _ptr(qw), _ptr(kw), _ptr(cs), max_pos,
+                                      _ptr(pos), int(bool(rope)), float(eps), _ptr(q), _ptr(k), _ptr(v))
+    if rc != 0:
+        raise ValueError("oracle_qk_norm_rope_kv failed")
+    return q, k, v
 
 
 def group(ids: np.ndarray, E: int, S: int):

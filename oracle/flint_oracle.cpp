@@ -513,4 +513,57 @@ int oracle_dense_gemv(const oracle_matrix* m, const uint16_t* x, int32_t T, cons
   return 0;
 }
 
+// Attention prologue of one layer, written from its definition (fp64): per
+// token and head of the fused projection qkv [T][Hq + 2*Hkv][Dh] (query heads,
+// then key heads, then value heads), query and key heads are RMS-normalised
+// over the head dimension and scaled by their weight vector,
+//   y_i = x_i / sqrt(mean_j x_j^2 + eps) * w_i,
+// then, when rope != 0, each pair (i, i + Dh/2), i < Dh/2, is rotated by the
+// token's position row of the cos/sin table cs [max_pos][Dh] (cos_i in column
+// i, sin_i in column Dh/2 + i):
+//   out_i = y_i cos_i - y_{i+Dh/2} sin_i,   out_{i+Dh/2} = y_{i+Dh/2} cos_i + y_i sin_i;
+// value heads pass unchanged. Outputs fp64: q [T][Hq][Dh], k and v
+// [T][Hkv][Dh] (the values a kernel rounds to bf16 and writes to its cache
+// slots). Returns 0, or -1 on a bad argument or a position outside the table.
+int oracle_qk_norm_rope_kv(int32_t T, int32_t Hq, int32_t Hkv, int32_t Dh, const uint16_t* qkv, const uint16_t* q_w,
+                           const uint16_t* k_w, const float* cs, int32_t max_pos, const int32_t* positions,
+                           int32_t rope, double eps, double* q_out, double* k_out, double* v_out) {
+  if (T < 0 || Hq < 1 || Hkv < 1 || Dh < 2 || Dh % 2 != 0 || !qkv || !q_w || !k_w || !q_out || !k_out || !v_out)
+    return -1;
+  if (rope && (!cs || !positions || max_pos < 1)) return -1;
+  const int H = Hq + 2 * Hkv, half = Dh / 2;
+  std::vector<double> x(Dh), y(Dh);
+  for (int t = 0; t < T; ++t) {
+    if (rope && (positions[t] < 0 || positions[t] >= max_pos)) return -1;
+    for (int h = 0; h < H; ++h) {
+      const uint16_t* src = qkv + (static_cast<size_t>(t) * H + h) * Dh;
+      for (int i = 0; i < Dh; ++i) x[i] = bf16_bits_to_double(src[i]);
+      if (h >= Hq + Hkv) {  // value head
+        double* dst = v_out + (static_cast<size_t>(t) * Hkv + (h - Hq - Hkv)) * Dh;
+        for (int i = 0; i < Dh; ++i) dst[i] = x[i];
+        continue;
+      }
+      const uint16_t* w = h < Hq ? q_w : k_w;
+      double ms = 0.0;
+      for (int i = 0; i < Dh; ++i) ms += x[i] * x[i];
+      ms /= Dh;
+      const double r = 1.0 / std::sqrt(ms + eps);
+      for (int i = 0; i < Dh; ++i) y[i] = x[i] * r * bf16_bits_to_double(w[i]);
+      double* dst = h < Hq ? q_out + (static_cast<size_t>(t) * Hq + h) * Dh
+                           : k_out + (static_cast<size_t>(t) * Hkv + (h - Hq)) * Dh;
+      if (!rope) {
+        for (int i = 0; i < Dh; ++i) dst[i] = y[i];
+        continue;
+      }
+      const float* row = cs + static_cast<size_t>(positions[t]) * Dh;
+      for (int i = 0; i < half; ++i) {
+        const double c = row[i], s = row[half + i];
+        dst[i] = y[i] * c - y[half + i] * s;
+        dst[half + i] = y[half + i] * c + y[i] * s;
+      }
+    }
+  }
+  return 0;
+}
+
 }  // extern "C"

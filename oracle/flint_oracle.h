@@ -22,6 +22,14 @@
  *    SwiGLU experts (gate/up d->I, down I->d, no biases).
  *  - E2M1 / E4M3 bit meanings follow the public OCP Microscaling (MX) v1.0
  *    element formats (FP4 E2M1; FP8 E4M3 "fn": no infinities, S.1111.111 NaN).
+ *  - The attention prologue (fused Q/K normalisation + rotary embedding +
+ *    KV-cache write): "[Model] Add Flint (RecursiveSI/flint)", section "What
+ *    happened"; grouped-query attention with 32 query and 4 key/value heads of
+ *    dimension 128, rotary positions on the sliding-window layers and none on
+ *    the full-attention layers: "Recursive Flint: 125 tok/s on an M4 Pro",
+ *    architecture table. The pages fix no norm type or rotary layout: RMS
+ *    normalisation over the head dimension with a learned weight, and rotation
+ *    of pairs (i, i + Dh/2) by a caller-supplied cos/sin table.
  *
  * Precision: every arithmetic step of the forward pass runs in fp64; weights
  * are decoded exactly (e2m1 * e4m3 * fp32 tensor scale fits in 53 bits).
@@ -147,6 +155,18 @@ int oracle_moe_forward(int32_t T, int32_t d, int32_t inter, int32_t E, int32_t k
                        const int32_t* ids_override, int32_t input_norm, int32_t n_threads,
                        int32_t* ids_out, double* gates_out, double* gap_out,
                        double* logits_out, double* out);
+
+/* ---- attention prologue ---- */
+/* Fused Q/K RMS normalisation + rotary embedding + key/value pass-through of
+ * one layer's QKV projection qkv [T][Hq + 2*Hkv][Dh] bf16 (query heads, key
+ * heads, value heads). Query/key heads: y = x / sqrt(mean(x^2) + eps) * w
+ * (w = q_w or k_w, bf16 [Dh]); with rope, pairs (i, i + Dh/2) rotated by the
+ * position's row of cs [max_pos][Dh] fp32 (cos in columns 0..Dh/2-1, sin in
+ * Dh/2..Dh-1). fp64 outputs q [T][Hq][Dh], k, v [T][Hkv][Dh]. Returns 0, or -1
+ * on a bad argument or a position outside [0, max_pos). */
+int oracle_qk_norm_rope_kv(int32_t T, int32_t Hq, int32_t Hkv, int32_t Dh, const uint16_t* qkv, const uint16_t* q_w,
+                           const uint16_t* k_w, const float* cs, int32_t max_pos, const int32_t* positions,
+                           int32_t rope, double eps, double* q_out, double* k_out, double* v_out);
 
 #ifdef __cplusplus
 }
