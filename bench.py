@@ -438,6 +438,57 @@ def run_prefill(world: int, seed: int, T: int = 8192, n_layers: int = 4, calls: 
             "tensor_peak_tflops": tf_peak, "tensor_peak_kind": tf_kind}
 
 
+def run_attn_prologue(seed: int, calls: int = 50):
+    """The attention prologue (flint_qk_norm_rope_kv) at the pages' heads (32
+    query, 4 key/value, dimension 128), rotary on: per-call device time from a
+    CUDA graph of `calls` launches, at decode and prefill sizes, with the
+    bytes it must move (qkv in, cos/sin row, q out, k and v into the cache)."""
+    import torch
+    import nvfp4_weight_only_flint_b200 as fm
+    hq, hkv, dh = 32, 4, 128
+    res = {"workload": "fused Q/K RMS norm + rotary + KV-cache write, 32 q / 4 kv heads x 128, bf16"}
+    peak, kind = _peaks()
+    for T in (1, 64, 8192):
+        g = torch.Generator(device="cuda").manual_seed(seed + T)
+        qkv = torch.randn((T, hq + 2 * hkv, dh), device="cuda", generator=g).to(torch.bfloat16)
+        w = torch.ones(dh, device="cuda").to(torch.bfloat16)
+        max_pos = max(T, 4096)
+        inv = 10000.0 ** (-torch.arange(0, dh, 2, device="cuda", dtype=torch.float64) / dh)
+        ang = torch.arange(max_pos, device="cuda", dtype=torch.float64)[:, None] * inv[None, :]
+        cs = torch.cat([ang.cos(), ang.sin()], dim=1).float().contiguous()
+        pos = torch.arange(T, device="cuda", dtype=torch.int32)
+        slots = torch.arange(T, device="cuda", dtype=torch.int32)
+        q_out = torch.empty((T, hq, dh), device="cuda", dtype=torch.bfloat16)
+        kc = torch.empty((T, hkv, dh), device="cuda", dtype=torch.bfloat16)
+        vc = torch.empty((T, hkv, dh), device="cuda", dtype=torch.bfloat16)
+        st = torch.cuda.Stream()
+
+        def call():
+            fm.flint_qk_norm_rope_kv(qkv, T, hq, hkv, w, w, cs, max_pos, pos, True, 1e-6, slots, T, q_out, kc, vc,
+                                     stream=st.cuda_stream)
+        with torch.cuda.stream(st):
+            for _ in range(5):
+                call()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=st):
+            for _ in range(calls):
+                call()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(st):  # replay and events on the captured stream
+            graph.replay()
+            torch.cuda.synchronize()
+            e0.record()
+            graph.replay()
+            e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / calls * 1e3
+        byt = T * ((hq + 2 * hkv) * dh * 2 + dh * 4 + (hq + 2 * hkv) * dh * 2 + 8)
+        res[f"T{T}"] = {"us": us, "bytes": byt, "gbs": byt / (us * 1e-6) / 1e9, "frac_of_peak": byt / (us * 1e-6) / 1e9 / peak}
+        del graph
+    return res
+
+
 def cpu_baseline(n_tokens: int = 3, seed: int = 0):
     """The fp64 oracle as it stands, on host cores: T=1 layer decodes of the
     default workload (quantisation of the needed experts is untimed set-up),
@@ -506,7 +557,7 @@ def main():
     ap.add_argument("--impl", choices=["flint", "reference"], default="flint")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-extras", action="store_true", help="skip the batch-8 / batch-4 / batch-64 lines")
-    ap.add_argument("--profile", choices=["t1", "t8", "t64_nvfp4", "t64_bf16"], default=None,
+    ap.add_argument("--profile", choices=["t1", "t8", "t64_nvfp4", "t64_bf16", "prefill"], default=None,
                     help="profiling case: one layer, --steps eager layer calls, no timing output")
     args = ap.parse_args()
     if args.profile:
@@ -628,6 +679,7 @@ def main():
             torch.cuda.empty_cache()
         extras["lm_head"] = run_lm_head(world)
         extras["prefill"] = run_prefill(world, args.seed)
+        extras["attn_prologue"] = run_attn_prologue(args.seed)
         extras["stack47"] = {
             "workload": "cfg3: 47 resident layers (21.4 GB NVFP4), residual chain, no attention",
             "batch1_tokens_per_s": tok_s / N_LAYERS, "batch1_us_per_layer": ms_step * 1e3,
@@ -682,16 +734,25 @@ def run_profile_case(args):
     import torch
     import nvfp4_weight_only_flint_b200 as fm
     fm.lib()
-    name = {"t1": "cfg1", "t8": "cfg2", "t64_nvfp4": "cfg4_nvfp4", "t64_bf16": "cfg4_bf16"}[args.profile]
-    w = synth.CONFIGS[name]
-    st = Stack(synth.CONFIGS["cfg1"], 1, args.seed, max_tokens=w.T, wdtype=w.wdtype)
-    xb = synth.x_bits(args.seed + 3000, w.T, w.d)
-    x = _bits_to_cuda(xb)
-    wr = _bits_to_cuda(synth.make_router(w, args.seed, xb))
+    if args.profile == "prefill":  # 8192 tokens, the Flint shape, NVFP4 (1.5 GB with the workspace)
+        w = synth.CONFIGS["cfg1"]
+        T = 8192
+        st = Stack(w, 1, args.seed, max_tokens=T)
+        xb = synth.x_bits(args.seed + 3000, T, w.d)
+        x = _bits_to_cuda(xb)
+        wr = _bits_to_cuda(synth.to_bf16_bits(synth.router_plain(args.seed, w.d, w.E, 0)))
+    else:
+        name = {"t1": "cfg1", "t8": "cfg2", "t64_nvfp4": "cfg4_nvfp4", "t64_bf16": "cfg4_bf16"}[args.profile]
+        w = synth.CONFIGS[name]
+        T = w.T
+        st = Stack(synth.CONFIGS["cfg1"], 1, args.seed, max_tokens=T, wdtype=w.wdtype)
+        xb = synth.x_bits(args.seed + 3000, T, w.d)
+        x = _bits_to_cuda(xb)
+        wr = _bits_to_cuda(synth.make_router(w, args.seed, xb))
     out = torch.empty_like(x)
     opt = fm.Options(path=fm.FLINT_PATH_AUTO, use_pdl=1)
     for _ in range(max(1, args.steps)):
-        fm.flint_moe_forward_ex(x, w.T, wr, st.layers[0][3], st.shape, None, out, st.ws, opt)
+        fm.flint_moe_forward_ex(x, T, wr, st.layers[0][3], st.shape, None, out, st.ws, opt)
     torch.cuda.synchronize()
     rc, flags = fm.flint_moe_get_status(st.ws)
     if rc != 0:

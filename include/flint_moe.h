@@ -105,7 +105,8 @@ enum {
   FLINT_DEVCHECK_EXPERT_ID = 1,   /* an expert id outside [0, E) reached a kernel */
   FLINT_DEVCHECK_NONFINITE = 2,   /* a non-finite weight reached the packer */
   FLINT_DEVCHECK_WAIT = 4,        /* a bounded wait gave up (FLINT_ERR_TIMEOUT) */
-  FLINT_DEVCHECK_MMA = 8          /* the tensor-core path rejected a tile */
+  FLINT_DEVCHECK_MMA = 8,         /* the tensor-core path rejected a tile */
+  FLINT_DEVCHECK_INDEX = 16       /* a position or cache slot outside its range (skipped) */
 };
 
 typedef enum flint_path {
@@ -311,6 +312,37 @@ int flint_pack_nvfp4_dense(const void* w, int32_t w_is_bf16, int32_t rows, int32
 int flint_lm_head(const uint16_t* x, int32_t T, const uint8_t* codes, const uint8_t* scales,
                   const float* tensor_scale, int32_t rows, int32_t cols, float* out, void* workspace,
                   size_t ws_bytes, void* stream);
+
+/* flint_qk_norm_rope_kv -- the attention prologue of one layer: fused Q/K
+ * normalisation + rotary embedding + KV-cache write ("[Model] Add Flint
+ * (RecursiveSI/flint)", section "What happened"; heads from "Recursive Flint:
+ * 125 tok/s on an M4 Pro", architecture table: 32 query, 4 key/value heads of
+ * dimension 128, rotary positions on the sliding-window layers, none on the
+ * full-attention layers).
+ *   qkv      device bf16 [T][n_q_heads + 2*n_kv_heads][head_dim]: the fused
+ *            projection, query heads, then key heads, then value heads
+ *   q_norm_w, k_norm_w  device bf16 [head_dim]
+ *   query/key heads: y = x / sqrt(mean(x^2) + eps) * w (fp32); with rope != 0,
+ *   pairs (i, i + head_dim/2) rotated by row positions[t] of cos_sin (device
+ *   fp32 [max_pos][head_dim], cos in the first half of a row, sin in the
+ *   second, 16-byte aligned): first = y_i cos - y_j sin, second = y_j cos + y_i
+ *   sin; outputs rounded to bf16.
+ *   q_out    device bf16 [T][n_q_heads][head_dim]
+ *   k_cache, v_cache  device bf16 [n_slots][n_kv_heads][head_dim]; token t's
+ *            key and value heads go to row slots[t] (device int32 [T]); other
+ *            rows are not touched.
+ *   status   nullable device int32: a slot outside [0, n_slots) (that token's
+ *            key and value are not written) or a position outside [0,
+ *            max_pos) (its rotation is skipped) sets FLINT_DEVCHECK_INDEX.
+ * head_dim must be 128. The caller owns all buffers; 8-byte aligned pointers.
+ * One kernel, asynchronous on `stream`; T = 0 launches nothing. The pages
+ * give no norm type or rotary layout: RMS normalisation with a learned weight
+ * and the rotate-half pairing are the readings taken. */
+int flint_qk_norm_rope_kv(const uint16_t* qkv, int32_t T, int32_t n_q_heads, int32_t n_kv_heads,
+                          int32_t head_dim, const uint16_t* q_norm_w, const uint16_t* k_norm_w,
+                          const float* cos_sin, int32_t max_pos, const int32_t* positions, int32_t rope,
+                          float eps, const int32_t* slots, int64_t n_slots, uint16_t* q_out, uint16_t* k_cache,
+                          uint16_t* v_cache, int32_t* status, void* stream);
 
 /* Synchronises `stream`, reads the workspace status word into *device_flags
  * (FLINT_DEVCHECK_* bits, may be NULL) and clears it. Returns FLINT_OK, or

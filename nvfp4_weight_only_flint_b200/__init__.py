@@ -28,6 +28,8 @@ __all__ = [
 FLINT_W_NVFP4, FLINT_W_BF16 = 0, 1
 FLINT_PATH_AUTO, FLINT_PATH_GEMV, FLINT_PATH_MMA = 0, 1, 2
 FLINT_LAYER_AUTO, FLINT_LAYER_FMA, FLINT_LAYER_MMA, FLINT_LAYER_CLUSTER = 0, 1, 2, 3
+FLINT_DEVCHECK_EXPERT_ID, FLINT_DEVCHECK_NONFINITE, FLINT_DEVCHECK_WAIT, FLINT_DEVCHECK_MMA = 1, 2, 4, 8
+FLINT_DEVCHECK_INDEX = 16
 STATUS_NAMES = {0: "FLINT_OK", -1: "FLINT_ERR_INVALID_ARG", -2: "FLINT_ERR_UNSUPPORTED_SHAPE",
                 -3: "FLINT_ERR_MISALIGNED", -4: "FLINT_ERR_WORKSPACE", -5: "FLINT_ERR_CUDA",
                 -6: "FLINT_ERR_DEVICE_CHECK", -7: "FLINT_ERR_TIMEOUT"}
@@ -97,6 +99,9 @@ def lib() -> ctypes.CDLL:
         L.flint_pack_nvfp4_dense.restype = i32
         L.flint_lm_head.argtypes = [vp, i32, vp, vp, vp, i32, i32, vp, vp, sz, vp]
         L.flint_lm_head.restype = i32
+        L.flint_qk_norm_rope_kv.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, i32, vp, i32, ctypes.c_float, vp,
+                                            ctypes.c_int64, vp, vp, vp, vp, vp]
+        L.flint_qk_norm_rope_kv.restype = i32
         L.flint_moe_workspace_init.argtypes = [vp, sz, vp]
         L.flint_moe_workspace_init.restype = i32
         L.flint_moe_get_status.argtypes = [vp, P(i32), vp]
@@ -240,6 +245,15 @@ def flint_lm_head(x, T: int, codes, scales, tensor_scale, rows: int, cols: int, 
                   stream=None) -> None:
     _check(lib().flint_lm_head(_ptr(x), int(T), _ptr(codes), _ptr(scales), _ptr(tensor_scale), int(rows),
                                int(cols), _ptr(out), _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def flint_qk_norm_rope_kv(qkv, T: int, n_q_heads: int, n_kv_heads: int, q_norm_w, k_norm_w, cos_sin, max_pos: int,
+                          positions, rope: bool, eps: float, slots, n_slots: int, q_out, k_cache, v_cache,
+                          status=None, head_dim: int = 128, stream=None) -> None:
+    _check(lib().flint_qk_norm_rope_kv(_ptr(qkv), int(T), int(n_q_heads), int(n_kv_heads), int(head_dim),
+                                       _ptr(q_norm_w), _ptr(k_norm_w), _ptr(cos_sin), int(max_pos), _ptr(positions),
+                                       int(bool(rope)), float(eps), _ptr(slots), int(n_slots), _ptr(q_out),
+                                       _ptr(k_cache), _ptr(v_cache), _ptr(status), _stream(stream)))
 
 
 def flint_moe_get_status(workspace, stream=None) -> tuple[int, int]:

@@ -12,6 +12,10 @@
 
 namespace flint {
 
+// Records msg in the library's last-error slot (flint_last_error) and returns
+// code; defined in flint_moe.cu.
+int flint_fail_external(int code, const char* msg);
+
 // A bounded device wait gives up after this many SM clock cycles (about one
 // second at the B200's boost clock) and records FLINT_DEVCHECK_WAIT.
 constexpr long long kWaitCycles = 2000000000LL;

@@ -402,6 +402,13 @@ int fail(int code, const char* fmt, ...) {
   return code;
 }
 
+}  // namespace
+
+// The last-error slot for the library's other translation units.
+int flint_fail_external(int code, const char* msg) { return fail(code, "%s", msg); }
+
+namespace {
+
 int cuda_fail(cudaError_t e, const char* what) {
   // a failed launch or call also stays in the runtime's last-error slot; take
   // it out so that a later, unrelated check does not report it again
@@ -1013,8 +1020,15 @@ int run_mma_path(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, 
   rc = mma_maps(&dn, s, wts, false, m.hrows, P);
   if (rc != FLINT_OK) return rc;
 
-  cudaError_t e = launch_router_only(p, st);
-  if (e != cudaSuccess) return cuda_fail(e, "k_router_only launch");
+  cudaError_t e;
+  if (T > kMmaGroupSmallT) {  // many tokens: the router on tensor cores
+    e = launch(k_router_tc, dim3((T + kRtTile - 1) / kRtTile, (s.E + kRtTile - 1) / kRtTile), dim3(256), 0, st,
+               false, p);
+    if (e != cudaSuccess) return cuda_fail(e, "k_router_tc launch");
+  } else {
+    e = launch_router_only(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "k_router_only launch");
+  }
   e = launch(k_topk, dim3((T + 7) / 8), dim3(256), 0, st, pdl, p);
   if (e != cudaSuccess) return cuda_fail(e, "k_topk launch");
   if (T <= kMmaGroupSmallT) {
@@ -1240,8 +1254,15 @@ int flint_moe_route(const uint16_t* x, int32_t T, const uint16_t* router_w, cons
   p.ids = topk_ids;
   p.gates = topk_weights;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_router_only(p, st);
-  if (e != cudaSuccess) return cuda_fail(e, "k_router_only launch");
+  cudaError_t e;
+  if (T > kMmaGroupSmallT) {  // many tokens: the router on tensor cores
+    e = launch(k_router_tc, dim3((T + kRtTile - 1) / kRtTile, (s.E + kRtTile - 1) / kRtTile), dim3(256), 0, st,
+               false, p);
+    if (e != cudaSuccess) return cuda_fail(e, "k_router_tc launch");
+  } else {
+    e = launch_router_only(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "k_router_only launch");
+  }
   e = launch(k_topk, dim3((T + 7) / 8), dim3(256), 0, st, true, p);
   if (e != cudaSuccess) return cuda_fail(e, "k_topk launch");
   return FLINT_OK;

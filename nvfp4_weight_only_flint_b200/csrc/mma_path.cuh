@@ -197,6 +197,66 @@ __device__ __forceinline__ bool mma_wait(uint64_t* bar, uint32_t parity, volatil
   return true;
 }
 
+// ----------------------------------------------------------------- router, large T
+// logits [T][E] = x [T][d] . W_r^T on the register-fragment tensor cores
+// (mma.sync m16n8k16, bf16 products exact, fp32 accumulation) for calls of
+// many tokens, where a CUDA-core router took a third of an 8192-token call. A
+// CTA computes a 64-token x 64-expert tile over K in steps of 64: both 64 x 64
+// operand tiles are staged in shared memory with rows padded to 72 elements
+// (the eight rows of a fragment load fall in distinct banks); warp w takes
+// tokens 16*(w/2).. and experts 32*(w%2).. (four 8-expert MMA columns).
+constexpr int kRtTile = 64, kRtPad = 72;
+
+__device__ __forceinline__ void mma_bf16_m16n8k16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                  uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(256) k_router_tc(LayerParams p) {
+  __shared__ __align__(16) uint16_t sx[kRtTile][kRtPad];
+  __shared__ __align__(16) uint16_t sw[kRtTile][kRtPad];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t0 = blockIdx.x * kRtTile, e0 = blockIdx.y * kRtTile, D = p.d;
+  const int mt = warp >> 1, nh = warp & 1, g = lane >> 2, t4 = lane & 3;
+  float acc[4][4] = {};
+  auto ld32 = [](const uint16_t* q) { return *reinterpret_cast<const uint32_t*>(q); };
+  for (int k0 = 0; k0 < D; k0 += kRtTile) {
+    for (int c = tid; c < kRtTile * kRtTile / 8; c += blockDim.x) {  // 16-byte chunks of both tiles
+      const int r = c >> 3, q = c & 7;
+      uint4 vx = make_uint4(0u, 0u, 0u, 0u), vw = make_uint4(0u, 0u, 0u, 0u);
+      if (t0 + r < p.T) vx = __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t0 + r) * D + k0) + q);
+      if (e0 + r < p.E) vw = __ldg(reinterpret_cast<const uint4*>(p.wr + static_cast<size_t>(e0 + r) * D + k0) + q);
+      *reinterpret_cast<uint4*>(&sx[r][8 * q]) = vx;
+      *reinterpret_cast<uint4*>(&sw[r][8 * q]) = vw;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kRtTile; kk += 16) {
+      const int ra = 16 * mt + g;
+      const uint32_t a0 = ld32(&sx[ra][kk + 2 * t4]), a1 = ld32(&sx[ra + 8][kk + 2 * t4]);
+      const uint32_t a2 = ld32(&sx[ra][kk + 8 + 2 * t4]), a3 = ld32(&sx[ra + 8][kk + 8 + 2 * t4]);
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+        const int rb = 32 * nh + 8 * n + g;
+        mma_bf16_m16n8k16(acc[n], a0, a1, a2, a3, ld32(&sw[rb][kk + 2 * t4]), ld32(&sw[rb][kk + 8 + 2 * t4]));
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int n = 0; n < 4; ++n) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int t = t0 + 16 * mt + g + 8 * (r >> 1), e = e0 + 32 * nh + 8 * n + 2 * t4 + (r & 1);
+      if (t < p.T && e < p.E) p.logits[static_cast<size_t>(t) * p.E + e] = acc[n][r];
+    }
+  }
+}
+
 // ----------------------------------------------------------------- grouping
 // One CTA of 512 threads (E <= 1024, T <= 128).
 __global__ void __launch_bounds__(512) k_mma_group(MmaParams p) {
