@@ -93,6 +93,8 @@ def lib():
         L.oracle_group.restype = i32
         L.oracle_qk_norm_rope_kv.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, i32, vp, i32, f64, vp, vp, vp]
         L.oracle_qk_norm_rope_kv.restype = i32
+        L.oracle_decode_attention.argtypes = [i32, i32, i32, i32, vp, vp, vp, ctypes.c_int64, vp, vp, f64, vp]
+        L.oracle_decode_attention.restype = i32
         _lib = L
     return _lib
 
@@ -284,6 +286,24 @@ def qk_norm_rope_kv(qkv_bits: np.ndarray, n_q_heads: int, n_kv_heads: int, q_w_b
     if rc != 0:
         raise ValueError("oracle_qk_norm_rope_kv failed")
     return q, k, v
+
+
+def decode_attention(q_bits, k_bits, v_bits, start, length, scale=None):
+    """fp64 decode attention: q_bits [T][Hq][Dh], k/v_bits [rows][Hkv][Dh]
+    (bf16 bits), start int64 [T], length int32 [T]; returns [T][Hq][Dh]."""
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    v = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    T, Hq, Dh = q.shape
+    rows, Hkv, _ = k.shape
+    st = np.ascontiguousarray(start, dtype=np.int64)
+    ln = np.ascontiguousarray(length, dtype=np.int32)
+    out = np.zeros((T, Hq, Dh), dtype=np.float64)
+    sc = 1.0 / np.sqrt(Dh) if scale is None else float(scale)
+    if lib().oracle_decode_attention(T, Hq, Hkv, Dh, _ptr(q), _ptr(k), _ptr(v), rows, _ptr(st), _ptr(ln), sc,
+                                     _ptr(out)) != 0:
+        raise ValueError("oracle_decode_attention failed")
+    return out
 
 
 def group(ids: np.ndarray, E: int, S: int):

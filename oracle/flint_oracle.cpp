@@ -566,4 +566,50 @@ int oracle_qk_norm_rope_kv(int32_t T, int32_t Hq, int32_t Hkv, int32_t Dh, const
   return 0;
 }
 
+// Decode attention of one layer, from its definition (fp64): query token t,
+// head h attends to the cache rows start[t] .. start[t] + len[t] - 1 of key
+// and value head g = h / (Hq / Hkv) (grouped-query attention):
+//   s_j = (q_h . k_{g,j}) * scale,  p_j = exp(s_j - max s) / sum_j exp(s_j - max s),
+//   o_h = sum_j p_j v_{g,j}.
+// q bf16 [T][Hq][Dh]; k, v bf16 [rows][Hkv][Dh]; out fp64 [T][Hq][Dh]; a token
+// with len 0 gets zeros. Returns 0, or -1 on a bad argument or a range outside
+// [0, rows).
+int oracle_decode_attention(int32_t T, int32_t Hq, int32_t Hkv, int32_t Dh, const uint16_t* q, const uint16_t* k,
+                            const uint16_t* v, int64_t rows, const int64_t* start, const int32_t* len, double scale,
+                            double* out) {
+  if (T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Dh < 1 || !q || !k || !v || !start || !len || !out) return -1;
+  const int group = Hq / Hkv;
+  std::vector<double> sc;
+  for (int t = 0; t < T; ++t) {
+    if (len[t] < 0 || start[t] < 0 || start[t] + len[t] > rows) return -1;
+    for (int h = 0; h < Hq; ++h) {
+      const int g = h / group;
+      const uint16_t* qh = q + (static_cast<size_t>(t) * Hq + h) * Dh;
+      double* oh = out + (static_cast<size_t>(t) * Hq + h) * Dh;
+      for (int i = 0; i < Dh; ++i) oh[i] = 0.0;
+      if (len[t] == 0) continue;
+      sc.assign(len[t], 0.0);
+      double mx = -INFINITY;
+      for (int j = 0; j < len[t]; ++j) {
+        const uint16_t* kj = k + (static_cast<size_t>(start[t] + j) * Hkv + g) * Dh;
+        double dot = 0.0;
+        for (int i = 0; i < Dh; ++i) dot += bf16_bits_to_double(qh[i]) * bf16_bits_to_double(kj[i]);
+        sc[j] = dot * scale;
+        mx = std::max(mx, sc[j]);
+      }
+      double sum = 0.0;
+      for (int j = 0; j < len[t]; ++j) {
+        sc[j] = std::exp(sc[j] - mx);
+        sum += sc[j];
+      }
+      for (int j = 0; j < len[t]; ++j) {
+        const uint16_t* vj = v + (static_cast<size_t>(start[t] + j) * Hkv + g) * Dh;
+        const double pj = sc[j] / sum;
+        for (int i = 0; i < Dh; ++i) oh[i] += pj * bf16_bits_to_double(vj[i]);
+      }
+    }
+  }
+  return 0;
+}
+
 }  // extern "C"

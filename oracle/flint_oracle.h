@@ -30,6 +30,9 @@
  *    architecture table. The pages fix no norm type or rotary layout: RMS
  *    normalisation over the head dimension with a learned weight, and rotation
  *    of pairs (i, i + Dh/2) by a caller-supplied cos/sin table.
+ *  - Decode attention over the cache (same page and table): grouped-query
+ *    softmax attention, query head h reading key/value head h / (Hq / Hkv),
+ *    scale 1/sqrt(Dh), over a caller-given range of cache rows per token.
  *
  * Precision: every arithmetic step of the forward pass runs in fp64; weights
  * are decoded exactly (e2m1 * e4m3 * fp32 tensor scale fits in 53 bits).
@@ -167,6 +170,15 @@ int oracle_moe_forward(int32_t T, int32_t d, int32_t inter, int32_t E, int32_t k
 int oracle_qk_norm_rope_kv(int32_t T, int32_t Hq, int32_t Hkv, int32_t Dh, const uint16_t* qkv, const uint16_t* q_w,
                            const uint16_t* k_w, const float* cs, int32_t max_pos, const int32_t* positions,
                            int32_t rope, double eps, double* q_out, double* k_out, double* v_out);
+
+/* Decode attention (fp64): query token t, head h attends to cache rows
+ * start[t] .. start[t] + len[t] - 1 of key/value head h / (Hq / Hkv):
+ * o = softmax(scale * q . k) v. q bf16 [T][Hq][Dh]; k, v bf16 [rows][Hkv][Dh];
+ * out fp64 [T][Hq][Dh] (zeros for len 0). Returns 0, or -1 on a bad argument
+ * or a range outside [0, rows). */
+int oracle_decode_attention(int32_t T, int32_t Hq, int32_t Hkv, int32_t Dh, const uint16_t* q, const uint16_t* k,
+                            const uint16_t* v, int64_t rows, const int64_t* start, const int32_t* len, double scale,
+                            double* out);
 
 #ifdef __cplusplus
 }
