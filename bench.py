@@ -489,6 +489,60 @@ def run_attn_prologue(seed: int, calls: int = 50):
     return res
 
 
+def run_decode_attention(seed: int, calls: int = 40):
+    """Decode attention (flint_decode_attention) at the pages' heads (32 query,
+    4 key/value, dimension 128) over bf16 caches: per-call device time from a
+    CUDA graph of `calls` launches, the calls cycling over cache regions of
+    more than 300 MB in all so that no call finds its rows in L2; bytes = the
+    key and value rows read (2 KB per row and token) plus q and out."""
+    import torch
+    import nvfp4_weight_only_flint_b200 as fm
+    hq, hkv, dh = 32, 4, 128
+    res = {"workload": "GQA decode attention, 32 q / 4 kv heads x 128, bf16 cache, split-K over the context"}
+    peak, kind = _peaks()
+    row_bytes = hkv * dh * 2 * 2
+    for T, L in ((1, 4096), (1, 32768), (1, 131072), (8, 32768), (64, 4096)):
+        regions = max(1, -(-(300 << 20) // (T * L * row_bytes)))
+        rows = regions * T * L
+        g = torch.Generator(device="cuda").manual_seed(seed + T * 7 + L)
+        kc = torch.randn((rows, hkv, dh), device="cuda", generator=g).to(torch.bfloat16)
+        vc = torch.randn((rows, hkv, dh), device="cuda", generator=g).to(torch.bfloat16)
+        q = torch.randn((T, hq, dh), device="cuda", generator=g).to(torch.bfloat16)
+        out = torch.empty((T, hq, dh), device="cuda", dtype=torch.bfloat16)
+        length = torch.full((T,), L, device="cuda", dtype=torch.int32)
+        starts = [torch.arange(T, device="cuda", dtype=torch.int64) * L + r * T * L for r in range(regions)]
+        nb = fm.flint_decode_attention_workspace_bytes(T, hkv, L)
+        ws = torch.empty(max(nb, 16), device="cuda", dtype=torch.uint8) if nb else None
+        st = torch.cuda.Stream()
+
+        def call(i):
+            fm.flint_decode_attention(q, kc, vc, rows, starts[i % regions], length, T, hq, hkv, L, dh ** -0.5, out,
+                                      ws, stream=st.cuda_stream)
+        with torch.cuda.stream(st):
+            for i in range(5):
+                call(i)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=st):
+            for i in range(calls):
+                call(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(st):
+            graph.replay()
+            torch.cuda.synchronize()
+            e0.record()
+            graph.replay()
+            e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / calls * 1e3
+        byt = T * L * row_bytes + 2 * T * hq * dh * 2
+        res[f"T{T}_L{L}"] = {"us": us, "bytes": byt, "gbs": byt / (us * 1e-6) / 1e9,
+                             "frac_of_peak": byt / (us * 1e-6) / 1e9 / peak}
+        del graph, kc, vc
+    res["peak_kind"] = kind
+    return res
+
+
 def cpu_baseline(n_tokens: int = 3, seed: int = 0):
     """The fp64 oracle as it stands, on host cores: T=1 layer decodes of the
     default workload (quantisation of the needed experts is untimed set-up),
@@ -680,6 +734,7 @@ def main():
         extras["lm_head"] = run_lm_head(world)
         extras["prefill"] = run_prefill(world, args.seed)
         extras["attn_prologue"] = run_attn_prologue(args.seed)
+        extras["decode_attention"] = run_decode_attention(args.seed)
         extras["stack47"] = {
             "workload": "cfg3: 47 resident layers (21.4 GB NVFP4), residual chain, no attention",
             "batch1_tokens_per_s": tok_s / N_LAYERS, "batch1_us_per_layer": ms_step * 1e3,

@@ -344,6 +344,41 @@ int flint_qk_norm_rope_kv(const uint16_t* qkv, int32_t T, int32_t n_q_heads, int
                           float eps, const int32_t* slots, int64_t n_slots, uint16_t* q_out, uint16_t* k_cache,
                           uint16_t* v_cache, int32_t* status, void* stream);
 
+/* flint_decode_attention -- grouped-query decode attention of one layer over
+ * the bf16 KV cache flint_qk_norm_rope_kv writes ("[Model] Add Flint
+ * (RecursiveSI/flint)", section "What happened": the attention step of the
+ * per-layer decode chain; heads from "Recursive Flint: 125 tok/s on an M4 Pro",
+ * architecture table: 32 query, 4 key/value heads of dimension 128; the
+ * sliding-window layers pass a window-sized range, the full-attention layers
+ * the whole history).
+ *   q        device bf16 [T][n_q_heads][head_dim]: one query per token
+ *   k_cache, v_cache  device bf16 [n_rows][n_kv_heads][head_dim]
+ *   start    device int64 [T], len device int32 [T]: token t attends rows
+ *            start[t] .. start[t] + len[t] - 1
+ *   out      device bf16 [T][n_q_heads][head_dim]:
+ *            out[t][h] = sum_j w_j v[start+j][g], w = softmax_j(scale *
+ *            q[t][h] . k[start+j][g]), g = h / (n_q_heads / n_kv_heads);
+ *            zeros for len 0. fp32 scores and sums; the weights enter the
+ *            value sum rounded to bf16.
+ *   max_len  host upper bound of len[t]; it sizes the split of each context
+ *            into chunks (about 296 CTAs in all) and the workspace.
+ *   workspace  device, 16-byte aligned, flint_decode_attention_workspace_bytes(
+ *            T, n_kv_heads, max_len) bytes (0 -- NULL allowed -- when each
+ *            context fits one chunk): per-chunk partial results, overwritten
+ *            by every call.
+ *   status   nullable device int32: len[t] > max_len (clamped to max_len) or
+ *            a range outside [0, n_rows) or len < 0 (that token's output is
+ *            zeros) sets FLINT_DEVCHECK_INDEX.
+ * head_dim must be 128, n_q_heads a multiple of n_kv_heads with at most 8
+ * query heads per kv head, T <= 65535, scale > 0 (1/sqrt(128) for the
+ * model). q, caches, out: 16-byte aligned. The caller owns all buffers. One or
+ * two kernels, asynchronous on `stream`; T = 0 launches nothing. */
+size_t flint_decode_attention_workspace_bytes(int32_t T, int32_t n_kv_heads, int32_t max_len);
+int flint_decode_attention(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache, int64_t n_rows,
+                           const int64_t* start, const int32_t* len, int32_t T, int32_t n_q_heads,
+                           int32_t n_kv_heads, int32_t head_dim, int32_t max_len, float scale, uint16_t* out,
+                           void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
+
 /* Synchronises `stream`, reads the workspace status word into *device_flags
  * (FLINT_DEVCHECK_* bits, may be NULL) and clears it. Returns FLINT_OK, or
  * FLINT_ERR_TIMEOUT / FLINT_ERR_DEVICE_CHECK when a flag was set. */

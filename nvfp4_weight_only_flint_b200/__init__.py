@@ -102,6 +102,11 @@ def lib() -> ctypes.CDLL:
         L.flint_qk_norm_rope_kv.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, i32, vp, i32, ctypes.c_float, vp,
                                             ctypes.c_int64, vp, vp, vp, vp, vp]
         L.flint_qk_norm_rope_kv.restype = i32
+        L.flint_decode_attention_workspace_bytes.argtypes = [i32, i32, i32]
+        L.flint_decode_attention_workspace_bytes.restype = sz
+        L.flint_decode_attention.argtypes = [vp, vp, vp, ctypes.c_int64, vp, vp, i32, i32, i32, i32, i32,
+                                             ctypes.c_float, vp, vp, sz, vp, vp]
+        L.flint_decode_attention.restype = i32
         L.flint_moe_workspace_init.argtypes = [vp, sz, vp]
         L.flint_moe_workspace_init.restype = i32
         L.flint_moe_get_status.argtypes = [vp, P(i32), vp]
@@ -148,7 +153,7 @@ def _check(rc: int):
 
 
 def _nbytes(t) -> int:
-    return t.numel() * t.element_size()
+    return 0 if t is None else t.numel() * t.element_size()
 
 
 def flint_last_error() -> str:
@@ -254,6 +259,19 @@ def flint_qk_norm_rope_kv(qkv, T: int, n_q_heads: int, n_kv_heads: int, q_norm_w
                                        _ptr(q_norm_w), _ptr(k_norm_w), _ptr(cos_sin), int(max_pos), _ptr(positions),
                                        int(bool(rope)), float(eps), _ptr(slots), int(n_slots), _ptr(q_out),
                                        _ptr(k_cache), _ptr(v_cache), _ptr(status), _stream(stream)))
+
+
+def flint_decode_attention_workspace_bytes(T: int, n_kv_heads: int, max_len: int) -> int:
+    return int(lib().flint_decode_attention_workspace_bytes(int(T), int(n_kv_heads), int(max_len)))
+
+
+def flint_decode_attention(q, k_cache, v_cache, n_rows: int, start, length, T: int, n_q_heads: int,
+                           n_kv_heads: int, max_len: int, scale: float, out, workspace=None, status=None,
+                           head_dim: int = 128, stream=None) -> None:
+    _check(lib().flint_decode_attention(_ptr(q), _ptr(k_cache), _ptr(v_cache), int(n_rows), _ptr(start),
+                                        _ptr(length), int(T), int(n_q_heads), int(n_kv_heads), int(head_dim),
+                                        int(max_len), float(scale), _ptr(out), _ptr(workspace),
+                                        _nbytes(workspace), _ptr(status), _stream(stream)))
 
 
 def flint_moe_get_status(workspace, stream=None) -> tuple[int, int]:

@@ -126,5 +126,28 @@ def test_host_validation_errors(L):
     assert L.flint_moe_get_status(None, None, None) == -1
 
 
+def test_decode_attention_host_validation(L):
+    # workspace: none when every context fits one chunk, else per-chunk partials
+    assert fm.flint_decode_attention_workspace_bytes(64, 4, 4096) == 0
+    assert fm.flint_decode_attention_workspace_bytes(1, 4, 32768) > 0
+    assert fm.flint_decode_attention_workspace_bytes(0, 4, 32768) == 0
+    need = fm.flint_decode_attention_workspace_bytes(1, 4, 32768)
+    a = 0x100000
+
+    def call(T=1, hq=32, hkv=4, dh=128, max_len=32768, scale=0.088, q=a, ws=a, ws_bytes=need):
+        return L.flint_decode_attention(q, a, a, 1 << 20, a, a, T, hq, hkv, dh, max_len, scale, a, ws, ws_bytes,
+                                        None, None)
+    assert call(dh=64) == -2
+    assert call(hq=64) == -2          # 16 query heads per kv head
+    assert call(hq=30) == -2          # not a multiple of the kv heads
+    assert call(T=-1) == -1
+    assert call(scale=0.0) == -1
+    assert call(T=0) == 0             # no-op
+    assert call(q=None) == -1
+    assert call(q=a + 8) == -3
+    assert call(ws_bytes=need - 16) == -4
+    assert call(ws=None) == -4
+
+
 def test_version(L):
     assert "sm_100a" in fm.flint_version()
