@@ -611,7 +611,7 @@ def main():
     ap.add_argument("--impl", choices=["flint", "reference"], default="flint")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-extras", action="store_true", help="skip the batch-8 / batch-4 / batch-64 lines")
-    ap.add_argument("--profile", choices=["t1", "t8", "t64_nvfp4", "t64_bf16", "prefill"], default=None,
+    ap.add_argument("--profile", choices=["t1", "t8", "t64_nvfp4", "t64_bf16", "prefill", "attn"], default=None,
                     help="profiling case: one layer, --steps eager layer calls, no timing output")
     args = ap.parse_args()
     if args.profile:
@@ -789,6 +789,8 @@ def run_profile_case(args):
     import torch
     import nvfp4_weight_only_flint_b200 as fm
     fm.lib()
+    if args.profile == "attn":
+        return run_profile_attn(args)
     if args.profile == "prefill":  # 8192 tokens, the Flint shape, NVFP4 (1.5 GB with the workspace)
         w = synth.CONFIGS["cfg1"]
         T = 8192
@@ -812,6 +814,43 @@ def run_profile_case(args):
     rc, flags = fm.flint_moe_get_status(st.ws)
     if rc != 0:
         raise RuntimeError(f"device status {rc} flags {flags}")
+    return 0
+
+
+def run_profile_attn(args):
+    """Small case for ncu of the attention kernels: the prologue over 8192
+    tokens, decode attention of 8 tokens over 32K cache rows each and of one
+    token over 32K rows (about 0.9 GB on the device), `--steps` eager calls
+    of each."""
+    import torch
+    import nvfp4_weight_only_flint_b200 as fm
+    hq, hkv, dh, T, L, Tp = 32, 4, 128, 8, 32768, 8192
+    g = torch.Generator(device="cuda").manual_seed(args.seed)
+    kc = torch.randn((T * L, hkv, dh), device="cuda", generator=g).to(torch.bfloat16)
+    vc = torch.randn((T * L, hkv, dh), device="cuda", generator=g).to(torch.bfloat16)
+    q = torch.randn((T, hq, dh), device="cuda", generator=g).to(torch.bfloat16)
+    out = torch.empty_like(q)
+    start = torch.arange(T, device="cuda", dtype=torch.int64) * L
+    length = torch.full((T,), L, device="cuda", dtype=torch.int32)
+    nb = fm.flint_decode_attention_workspace_bytes(T, hkv, L)
+    ws = torch.empty(max(nb, 16), device="cuda", dtype=torch.uint8)
+    ws1 = torch.empty(max(fm.flint_decode_attention_workspace_bytes(1, hkv, L), 16), device="cuda",
+                      dtype=torch.uint8)
+    qkv = torch.randn((Tp, hq + 2 * hkv, dh), device="cuda", generator=g).to(torch.bfloat16)
+    w1 = torch.ones(dh, device="cuda").to(torch.bfloat16)
+    cs = torch.zeros((Tp, dh), device="cuda", dtype=torch.float32)
+    cs[:, : dh // 2] = 1.0
+    pos = torch.arange(Tp, device="cuda", dtype=torch.int32)
+    q_out = torch.empty((Tp, hq, dh), device="cuda", dtype=torch.bfloat16)
+    status = torch.zeros(1, device="cuda", dtype=torch.int32)
+    for _ in range(max(1, args.steps)):
+        fm.flint_qk_norm_rope_kv(qkv, Tp, hq, hkv, w1, w1, cs, Tp, pos, True, 1e-6, pos, T * L, q_out, kc, vc,
+                                 status)
+        fm.flint_decode_attention(q, kc, vc, T * L, start, length, T, hq, hkv, L, dh ** -0.5, out, ws, status)
+        fm.flint_decode_attention(q, kc, vc, T * L, start, length, 1, hq, hkv, L, dh ** -0.5, out, ws1, status)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device check flags {int(status.item())}")
     return 0
 
 

@@ -23,8 +23,9 @@
 // The warps merge (max, sum, O) in shared memory. A token whose context fits
 // one chunk is finished there (divided by the sum, bf16 out); otherwise the CTA
 // writes the chunk's (max, sum) and unnormalised O, and k_attn_combine (one
-// CTA per (token, head), launched with programmatic dependent launch) rescales
-// the chunks to their common max and divides by the summed weights.
+// CTA of 16 warps per (token, head), launched with programmatic dependent
+// launch) rescales the chunks to their common max and divides by the summed
+// weights.
 // HBM-bound at long contexts: 512 bytes of key and value per cached row and kv
 // head (2 KB per row at 4 kv heads).
 #include <cuda_runtime.h>
@@ -262,13 +263,16 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_attn_partial(Params p) {
   }
 }
 
-// One CTA of 128 threads per (token, head): warp w takes chunks w, w + 4, ...;
-// lane holds 4 dimensions. The common max comes first (all threads over the
-// chunk maxima), so every chunk's loads are independent.
-__global__ void __launch_bounds__(128) k_attn_combine(Params p) {
-  __shared__ float s_red[kWarps];
-  __shared__ float s_acc[kWarps][kDh];
-  __shared__ float s_l[kWarps];
+// One CTA of 16 warps per (token, head). Warp w takes chunks w, w + 16, ...
+// eight at a time, all eight chunks' loads issued before any is used (one
+// round trip for up to 128 chunks), merged with a running max; lane l holds
+// dimensions 4l .. 4l + 3. The warps' (max, sum, O) then meet in shared memory.
+constexpr int kCombineWarps = 16;
+constexpr int kCombineBatch = 8;
+
+__global__ void __launch_bounds__(kCombineWarps * 32) k_attn_combine(Params p) {
+  __shared__ float s_m[kCombineWarps], s_l[kCombineWarps];
+  __shared__ __align__(16) float s_acc[kCombineWarps][kDh];
   pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int h = blockIdx.x, t = blockIdx.y;
@@ -277,33 +281,62 @@ __global__ void __launch_bounds__(128) k_attn_combine(Params p) {
   const int L = token_len(p, t, base, false);
   const int nc = (L + p.chunk - 1) / p.chunk;
   const size_t tg = (static_cast<size_t>(t) * p.Hkv + g) * p.n_chunks;
-  float M = -INFINITY;
-  for (int c = threadIdx.x; c < nc; c += 128) M = fmaxf(M, __ldcg(p.ml + ((tg + c) * kMaxGroup + hh) * 2));
-#pragma unroll
-  for (int s = 16; s > 0; s >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, s));
-  if (lane == 0) s_red[warp] = M;
-  __syncthreads();
-  M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
-  float lsum = 0.f;
+  float M = -INFINITY, lsum = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int c = warp; c < nc; c += kWarps) {
-    const size_t r = (tg + c) * kMaxGroup + hh;
-    const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.ml + r * 2));
-    const float4 ov = __ldcg(reinterpret_cast<const float4*>(p.po + r * kDh) + lane);
-    const float f = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-    lsum = fmaf(ml.y, f, lsum);
-    acc.x = fmaf(ov.x, f, acc.x);
-    acc.y = fmaf(ov.y, f, acc.y);
-    acc.z = fmaf(ov.z, f, acc.z);
-    acc.w = fmaf(ov.w, f, acc.w);
+  for (int c0 = warp; c0 < nc; c0 += kCombineWarps * kCombineBatch) {
+    float2 mlv[kCombineBatch];
+    float4 ov[kCombineBatch];
+#pragma unroll
+    for (int i = 0; i < kCombineBatch; ++i) {
+      const int c = c0 + i * kCombineWarps;
+      if (c < nc) {
+        const size_t r = (tg + c) * kMaxGroup + hh;
+        mlv[i] = __ldcg(reinterpret_cast<const float2*>(p.ml + r * 2));
+        ov[i] = __ldcg(reinterpret_cast<const float4*>(p.po + r * kDh) + lane);
+      } else {
+        mlv[i] = make_float2(-INFINITY, 0.f);
+        ov[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    float mb = M;
+#pragma unroll
+    for (int i = 0; i < kCombineBatch; ++i) mb = fmaxf(mb, mlv[i].x);
+    if (mb == -INFINITY) continue;  // nothing in this batch or before it
+    const float fo = M == -INFINITY ? 0.f : exp2f(M - mb);
+    lsum *= fo;
+    acc.x *= fo;
+    acc.y *= fo;
+    acc.z *= fo;
+    acc.w *= fo;
+#pragma unroll
+    for (int i = 0; i < kCombineBatch; ++i) {
+      const float f = mlv[i].x == -INFINITY ? 0.f : exp2f(mlv[i].x - mb);
+      lsum = fmaf(mlv[i].y, f, lsum);
+      acc.x = fmaf(ov[i].x, f, acc.x);
+      acc.y = fmaf(ov[i].y, f, acc.y);
+      acc.z = fmaf(ov[i].z, f, acc.z);
+      acc.w = fmaf(ov[i].w, f, acc.w);
+    }
+    M = mb;
+  }
+  if (lane == 0) {
+    s_m[warp] = M;
+    s_l[warp] = lsum;
   }
   *reinterpret_cast<float4*>(&s_acc[warp][4 * lane]) = acc;
-  if (lane == 0) s_l[warp] = lsum;
   __syncthreads();
+  if (threadIdx.x >= kDh) return;
   const int d = threadIdx.x;
-  const float tot = (s_l[0] + s_l[1]) + (s_l[2] + s_l[3]);
-  const float num = (s_acc[0][d] + s_acc[1][d]) + (s_acc[2][d] + s_acc[3][d]);
+  float Mx = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kCombineWarps; ++w) Mx = fmaxf(Mx, s_m[w]);
+  float tot = 0.f, num = 0.f;
+#pragma unroll
+  for (int w = 0; w < kCombineWarps; ++w) {
+    const float f = s_m[w] == -INFINITY ? 0.f : exp2f(s_m[w] - Mx);
+    tot = fmaf(s_l[w], f, tot);
+    num = fmaf(s_acc[w][d], f, num);
+  }
   const __nv_bfloat16 bv = __float2bfloat16_rn(tot > 0.f ? num / tot : 0.f);
   p.out[(static_cast<size_t>(t) * p.Hq + h) * kDh + d] = *reinterpret_cast<const uint16_t*>(&bv);
 }
@@ -394,7 +427,7 @@ extern "C" int flint_decode_attention(const uint16_t* q, const uint16_t* k_cache
   if (p.n_chunks > 1) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(n_q_heads, T);
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3(kCombineWarps * 32);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute at[1];
