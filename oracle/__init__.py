@@ -91,6 +91,8 @@ def lib():
         L.oracle_dense_gemv.restype = i32
         L.oracle_group.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
         L.oracle_group.restype = i32
+        L.oracle_ep_plan.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+        L.oracle_ep_plan.restype = i32
         L.oracle_qk_norm_rope_kv.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, i32, vp, i32, f64, vp, vp, vp]
         L.oracle_qk_norm_rope_kv.restype = i32
         L.oracle_decode_attention.argtypes = [i32, i32, i32, i32, vp, vp, vp, ctypes.c_int64, vp, vp, f64, vp]
@@ -319,6 +321,28 @@ def group(ids: np.ndarray, E: int, S: int):
     if n < 0:
         return None
     return act[:n].copy(), off[:n + 1].copy(), pair[:T * (k + S)].copy(), int(nr[0])
+
+
+def ep_plan(ids: np.ndarray, gates: np.ndarray, S: int, E: int, R: int, rank: int):
+    """Expert-parallel dispatch plan of ids/gates [T][k] on rank `rank` of R:
+    dict with send_ids, send_gates, send_token (send order), counts [R],
+    pair_pos [T][k+S], dropped."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    gates = np.ascontiguousarray(gates, dtype=np.float32)
+    T, k = ids.shape
+    P = T * (k + S)
+    send_ids = np.full(max(P, 1), -7, np.int32)
+    send_gates = np.zeros(max(P, 1), np.float32)
+    send_token = np.full(max(P, 1), -7, np.int32)
+    counts = np.zeros(R, np.int32)
+    pair_pos = np.zeros(max(P, 1), np.int32)
+    dropped = lib().oracle_ep_plan(_ptr(ids), _ptr(gates), T, k, S, E, R, rank, _ptr(send_ids), _ptr(send_gates),
+                                   _ptr(send_token), _ptr(counts), _ptr(pair_pos))
+    if dropped < 0:
+        raise ValueError("oracle_ep_plan: bad sizes")
+    n = int(counts.sum())
+    return {"send_ids": send_ids[:n].copy(), "send_gates": send_gates[:n].copy(), "send_token": send_token[:n].copy(),
+            "counts": counts, "pair_pos": pair_pos[:P].reshape(T, k + S).copy(), "dropped": int(dropped)}
 
 
 def expert_ffn(trip, x: np.ndarray) -> np.ndarray:

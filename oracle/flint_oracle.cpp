@@ -485,6 +485,56 @@ int32_t oracle_group(const int32_t* ids, int32_t T, int32_t k, int32_t E, int32_
   return n;
 }
 
+// Expert-parallel dispatch plan, from its definition: rank r of R holds the
+// routed experts [r E/R, (r+1) E/R) (local id e mod E/R) and the shared
+// experts (local ids E/R ..); pair i = t (k + S) + j goes to the rank holding
+// expert ids[t][j] (j < k) or, for a shared slot, to the token's own rank.
+// Send order: destination ranks in ascending order, each rank's pairs in
+// ascending pair index. An id outside [0, E) drops its pair (position -1).
+// Returns the number of dropped pairs, or -1 for bad sizes.
+int32_t oracle_ep_plan(const int32_t* ids, const float* gates, int32_t T, int32_t k, int32_t S, int32_t E,
+                       int32_t R, int32_t rank, int32_t* send_ids, float* send_gates, int32_t* send_token,
+                       int32_t* counts, int32_t* pair_pos) {
+  if (T < 0 || k < 1 || S < 0 || E < 1 || R < 1 || E % R != 0 || rank < 0 || rank >= R) return -1;
+  const int slots = k + S, el = E / R, P = T * slots;
+  int dropped = 0;
+  for (int i = 0; i < P; ++i) {
+    const int t = i / slots, j = i % slots;
+    if (j < k && (ids[t * k + j] < 0 || ids[t * k + j] >= E)) {
+      pair_pos[i] = -1;
+      ++dropped;
+    }
+  }
+  int pos = 0;
+  for (int r = 0; r < R; ++r) {
+    counts[r] = 0;
+    for (int i = 0; i < P; ++i) {
+      const int t = i / slots, j = i % slots;
+      int dest, lid;
+      float g;
+      if (j < k) {
+        const int e = ids[t * k + j];
+        if (e < 0 || e >= E) continue;
+        dest = e / el;
+        lid = e % el;
+        g = gates[t * k + j];
+      } else {
+        dest = rank;
+        lid = el + (j - k);
+        g = 1.0f;
+      }
+      if (dest != r) continue;
+      pair_pos[i] = pos;
+      send_ids[pos] = lid;
+      send_gates[pos] = g;
+      send_token[pos] = t;
+      ++pos;
+      ++counts[r];
+    }
+  }
+  return dropped;
+}
+
 // Dense NVFP4 matrix times bf16 vectors: each selected row decoded
 // element by element (as oracle_decode_matrix does) and dotted with x in fp64.
 int oracle_dense_gemv(const oracle_matrix* m, const uint16_t* x, int32_t T, const int32_t* rows,

@@ -130,6 +130,17 @@ int oracle_topk(const double* logits, int32_t T, int32_t E, int32_t k,
 int32_t oracle_group(const int32_t* ids, int32_t T, int32_t k, int32_t E, int32_t S,
                      int32_t* act, int32_t* off, int32_t* pair, int32_t* n_routed);
 
+/* Expert-parallel dispatch plan (expert parallelism over the GPUs of one node,
+ * "[Model] Add Flint (RecursiveSI/flint)", section "What happened"): the send
+ * order of the T (k + S) (token, slot) pairs by destination rank (rank r holds
+ * routed experts [r E/R, (r+1) E/R); shared slots stay on `rank`), ascending
+ * pair index within a rank; per send row its local expert id, gate and
+ * source token; per rank its row count; per pair its send position (-1 for an
+ * id outside [0, E)). Returns the dropped pairs, or -1 for bad sizes. */
+int32_t oracle_ep_plan(const int32_t* ids, const float* gates, int32_t T, int32_t k, int32_t S, int32_t E,
+                       int32_t R, int32_t rank, int32_t* send_ids, float* send_gates, int32_t* send_token,
+                       int32_t* counts, int32_t* pair_pos);
+
 /* ---- dense NVFP4 matrix-vector product (the 4-bit output head) ----
  * out[t][i] = sum_c w[rows[i]][c] * x[t][c] in fp64, w = e2m1 * e4m3 * s_t of
  * the NVFP4 matrix m (natural layout), x bf16 [T][m->cols]. rows (nullable)
