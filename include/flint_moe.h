@@ -313,6 +313,56 @@ int flint_lm_head(const uint16_t* x, int32_t T, const uint8_t* codes, const uint
                   const float* tensor_scale, int32_t rows, int32_t cols, float* out, void* workspace,
                   size_t ws_bytes, void* stream);
 
+/* flint_moe_forward_routed -- the layer's experts with the routing supplied
+ * by the caller instead of computed: out[t] = sum_{j<top_k} topk_weights[t][j]
+ * * FFN_{topk_ids[t][j]}(x_t) + shared expert(x_t) (+ residual[t]), bf16 out,
+ * on the tensor-core path (T <= 16384; more than 128 tokens need E + S <= 1024;
+ * NVFP4 weights need inter >= 256). The expert-parallel layer calls it with
+ * top_k = 1 and n_shared = 0 over the rows it receives, the shared expert seen
+ * as one more local expert (ids are validated on the device: an id outside
+ * [0, E) is skipped and sets FLINT_DEVCHECK_EXPERT_ID). topk_ids device int32
+ * [T][top_k], topk_weights device float [T][top_k] (4-byte aligned); the
+ * other pointers and the workspace as for flint_moe_forward (workspace of
+ * flint_moe_workspace_bytes(shape, >= T) bytes). Asynchronous on `stream`. */
+int flint_moe_forward_routed(const uint16_t* x, int32_t T, const int32_t* topk_ids, const float* topk_weights,
+                             const flint_moe_weights* weights, const flint_moe_shape* shape,
+                             const uint16_t* residual, uint16_t* out, void* workspace, size_t ws_bytes,
+                             void* stream);
+
+/* flint_ep_dispatch -- expert-parallel dispatch of one layer over n_ranks
+ * GPUs ("[Model] Add Flint (RecursiveSI/flint)", section "What happened":
+ * expert parallelism, left on stock layers there). Rank r holds routed
+ * experts [r E/R, (r+1) E/R) and the shared expert as local id E/R. Each of
+ * the T (top_k + n_shared) pairs (token t, slot j) goes to the rank holding
+ * its expert (the shared slot to `rank`, gate 1); pairs are ordered by
+ * destination rank, then by pair index t (top_k + n_shared) + j (a stable
+ * counting sort). Outputs (device, sized for P = T (top_k + n_shared) rows):
+ *   send_x      bf16 [P][d]: x row of each send position (positions >= the
+ *               total count are not written)
+ *   send_ids    int32 [P]: local expert id on the destination rank
+ *   send_gates  float [P]: the pair's gate
+ *   send_token  int32 [P]: source token
+ *   send_counts int32 [n_ranks]: rows for each rank (the send splits)
+ *   pair_pos    int32 [T][top_k + n_shared]: send position of each pair, -1
+ *               for a dropped pair (an id outside [0, E): sets
+ *               FLINT_DEVCHECK_EXPERT_ID in the nullable device `status`)
+ * n_ranks 1..8 dividing n_experts; top_k 1..8; n_shared 0 or 1; d a
+ * multiple of 8; x and send_x 16-byte aligned. Two kernels, asynchronous on
+ * `stream`. */
+int flint_ep_dispatch(const int32_t* topk_ids, const float* topk_weights, int32_t T, int32_t top_k,
+                      int32_t n_shared, int32_t n_experts, int32_t n_ranks, int32_t rank, const uint16_t* x,
+                      int32_t d, uint16_t* send_x, int32_t* send_ids, float* send_gates, int32_t* send_token,
+                      int32_t* send_counts, int32_t* pair_pos, int32_t* status, void* stream);
+
+/* flint_ep_combine -- the expert-parallel layer's output on the home rank:
+ * out[t] = bf16(sum_{j < slots, pair_pos[t][j] >= 0} y[pair_pos[t][j]] +
+ * residual[t]) in fp32. y: device bf16 [rows][d], the expert rows returned
+ * in send order (each already scaled by its gate); pair_pos as written by
+ * flint_ep_dispatch; residual nullable. slots 1..9; d a multiple of 8; y, out,
+ * residual 16-byte aligned. One kernel, asynchronous on `stream`. */
+int flint_ep_combine(const uint16_t* y, const int32_t* pair_pos, int32_t T, int32_t slots, int32_t d,
+                     const uint16_t* residual, uint16_t* out, void* stream);
+
 /* flint_qk_norm_rope_kv -- the attention prologue of one layer: fused Q/K
  * normalisation + rotary embedding + KV-cache write ("[Model] Add Flint
  * (RecursiveSI/flint)", section "What happened"; heads from "Recursive Flint:

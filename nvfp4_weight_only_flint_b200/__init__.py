@@ -107,6 +107,13 @@ def lib() -> ctypes.CDLL:
         L.flint_decode_attention.argtypes = [vp, vp, vp, ctypes.c_int64, vp, vp, i32, i32, i32, i32, i32,
                                              ctypes.c_float, vp, vp, sz, vp, vp]
         L.flint_decode_attention.restype = i32
+        L.flint_moe_forward_routed.argtypes = [vp, i32, vp, vp, P(Weights), P(Shape), vp, vp, vp, sz, vp]
+        L.flint_moe_forward_routed.restype = i32
+        L.flint_ep_dispatch.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp, vp,
+                                        vp]
+        L.flint_ep_dispatch.restype = i32
+        L.flint_ep_combine.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
+        L.flint_ep_combine.restype = i32
         L.flint_moe_workspace_init.argtypes = [vp, sz, vp]
         L.flint_moe_workspace_init.restype = i32
         L.flint_moe_get_status.argtypes = [vp, P(i32), vp]
@@ -272,6 +279,27 @@ def flint_decode_attention(q, k_cache, v_cache, n_rows: int, start, length, T: i
                                         _ptr(length), int(T), int(n_q_heads), int(n_kv_heads), int(head_dim),
                                         int(max_len), float(scale), _ptr(out), _ptr(workspace),
                                         _nbytes(workspace), _ptr(status), _stream(stream)))
+
+
+def flint_moe_forward_routed(x, T: int, topk_ids, topk_weights, weights: Weights, shape: Shape, residual, out,
+                             workspace, stream=None) -> None:
+    _check(lib().flint_moe_forward_routed(_ptr(x), int(T), _ptr(topk_ids), _ptr(topk_weights), ctypes.byref(weights),
+                                          ctypes.byref(shape), _ptr(residual), _ptr(out), _ptr(workspace),
+                                          _nbytes(workspace), _stream(stream)))
+
+
+def flint_ep_dispatch(topk_ids, topk_weights, T: int, top_k: int, n_shared: int, n_experts: int, n_ranks: int,
+                      rank: int, x, d: int, send_x, send_ids, send_gates, send_token, send_counts, pair_pos,
+                      status=None, stream=None) -> None:
+    _check(lib().flint_ep_dispatch(_ptr(topk_ids), _ptr(topk_weights), int(T), int(top_k), int(n_shared),
+                                   int(n_experts), int(n_ranks), int(rank), _ptr(x), int(d), _ptr(send_x),
+                                   _ptr(send_ids), _ptr(send_gates), _ptr(send_token), _ptr(send_counts),
+                                   _ptr(pair_pos), _ptr(status), _stream(stream)))
+
+
+def flint_ep_combine(y, pair_pos, T: int, slots: int, d: int, residual, out, stream=None) -> None:
+    _check(lib().flint_ep_combine(_ptr(y), _ptr(pair_pos), int(T), int(slots), int(d), _ptr(residual), _ptr(out),
+                                  _stream(stream)))
 
 
 def flint_moe_get_status(workspace, stream=None) -> tuple[int, int]:

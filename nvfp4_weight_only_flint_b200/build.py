@@ -12,7 +12,7 @@ INCLUDE = os.path.join(ROOT, "include")
 SO = os.path.join(PKG, "libflint_moe.so")
 OBJ_DIR = os.path.join(PKG, "_build")
 # translation units, compiled in parallel and linked into one shared library
-SOURCES = ["flint_moe.cu", "tok1.cu", "tokn.cu", "lmhead.cu", "attn.cu", "attn_decode.cu"]
+SOURCES = ["flint_moe.cu", "tok1.cu", "tokn.cu", "lmhead.cu", "attn.cu", "attn_decode.cu", "ep.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
 

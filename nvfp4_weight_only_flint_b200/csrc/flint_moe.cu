@@ -976,8 +976,11 @@ size_t mma_configure(MmaParams& m, int T) {
 
 // The tensor-core layer: router, top-k, grouping, B rows, gate/up, h rows,
 // down, combine.
+// ids_in / gates_in (both or neither): routing supplied by the caller, the
+// router and top-k are skipped and the grouping reads these arrays.
 int run_mma_path(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, const flint_moe_weights* wts,
-                 cudaEvent_t* ev, bool pdl, cudaStream_t st) {
+                 cudaEvent_t* ev, bool pdl, cudaStream_t st, const int32_t* ids_in = nullptr,
+                 const float* gates_in = nullptr) {
   const int T = p.T, P = T * (s.k + s.S);
   MmaParams m{};
   m.x = p.x;
@@ -985,8 +988,8 @@ int run_mma_path(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, 
   m.residual = p.residual;
   m.out = p.out;
   m.status = p.status;
-  m.ids = p.ids;
-  m.gates = p.gates;
+  m.ids = ids_in ? ids_in : p.ids;
+  m.gates = ids_in ? gates_in : p.gates;
   m.ids_out = p.ids_out;
   m.gates_out = p.gates_out;
   m.rt.n_active = reinterpret_cast<int*>(ws + w.mma_n);
@@ -1021,16 +1024,18 @@ int run_mma_path(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, 
   if (rc != FLINT_OK) return rc;
 
   cudaError_t e;
-  if (T > kMmaGroupSmallT) {  // many tokens: the router on tensor cores
-    e = launch(k_router_tc, dim3((T + kRtTile - 1) / kRtTile, (s.E + kRtTile - 1) / kRtTile), dim3(256), 0, st,
-               false, p);
-    if (e != cudaSuccess) return cuda_fail(e, "k_router_tc launch");
-  } else {
-    e = launch_router_only(p, st);
-    if (e != cudaSuccess) return cuda_fail(e, "k_router_only launch");
+  if (ids_in == nullptr) {
+    if (T > kMmaGroupSmallT) {  // many tokens: the router on tensor cores
+      e = launch(k_router_tc, dim3((T + kRtTile - 1) / kRtTile, (s.E + kRtTile - 1) / kRtTile), dim3(256), 0, st,
+                 false, p);
+      if (e != cudaSuccess) return cuda_fail(e, "k_router_tc launch");
+    } else {
+      e = launch_router_only(p, st);
+      if (e != cudaSuccess) return cuda_fail(e, "k_router_only launch");
+    }
+    e = launch(k_topk, dim3((T + 7) / 8), dim3(256), 0, st, pdl, p);
+    if (e != cudaSuccess) return cuda_fail(e, "k_topk launch");
   }
-  e = launch(k_topk, dim3((T + 7) / 8), dim3(256), 0, st, pdl, p);
-  if (e != cudaSuccess) return cuda_fail(e, "k_topk launch");
   if (T <= kMmaGroupSmallT) {
     e = launch(k_mma_group, dim3(1), dim3(512), 0, st, pdl, m);
     if (e != cudaSuccess) return cuda_fail(e, "k_mma_group launch");
@@ -1473,6 +1478,44 @@ int flint_moe_forward(const uint16_t* x, int32_t T, const uint16_t* router_w, co
                       size_t ws_bytes, void* stream) {
   return flint_moe_forward_ex(x, T, router_w, weights, shape, residual, out, workspace, ws_bytes, nullptr,
                               stream);
+}
+
+int flint_moe_forward_routed(const uint16_t* x, int32_t T, const int32_t* topk_ids, const float* topk_weights,
+                             const flint_moe_weights* weights, const flint_moe_shape* shape,
+                             const uint16_t* residual, uint16_t* out, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  Dims s;
+  int rc = check_shape(shape, &s);
+  if (rc != FLINT_OK) return rc;
+  if (T < 0) return fail(FLINT_ERR_INVALID_ARG, "T=%d", T);
+  if (T == 0) return FLINT_OK;
+  if (!x || !topk_ids || !topk_weights || !weights || !weights->packed || !out || !workspace)
+    return fail(FLINT_ERR_INVALID_ARG, "flint_moe_forward_routed: NULL pointer");
+  if (s.wd == FLINT_W_NVFP4 && (!weights->block_scales || !weights->tensor_scales))
+    return fail(FLINT_ERR_INVALID_ARG, "flint_moe_forward_routed: NVFP4 weights need block and tensor scales");
+  if (!aligned16(x) || !aligned16(weights->packed) || !aligned16(out) || !aligned16(workspace) ||
+      (residual && !aligned16(residual)) || (weights->block_scales && !aligned16(weights->block_scales)) ||
+      (weights->tensor_scales && !aligned16(weights->tensor_scales)) ||
+      (reinterpret_cast<uintptr_t>(topk_ids) & 3u) || (reinterpret_cast<uintptr_t>(topk_weights) & 3u))
+    return fail(FLINT_ERR_MISALIGNED, "flint_moe_forward_routed: misaligned pointer");
+  if (T > kMmaMaxCallTokens)
+    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "tensor-core path takes at most %d tokens (T=%d)", kMmaMaxCallTokens, T);
+  if (T > kMmaGroupSmallT && s.E + s.S > 1024)
+    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "more than %d tokens need E + S <= 1024", kMmaGroupSmallT);
+  if (s.wd == FLINT_W_NVFP4 && s.I < 256)
+    return fail(FLINT_ERR_UNSUPPORTED_SHAPE, "tensor-core path with NVFP4 weights needs inter >= 256 (inter=%d)", s.I);
+  const WsLayout lay = ws_layout(s, T, true);
+  if (ws_bytes < lay.total) return fail(FLINT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, lay.total);
+  LayerParams p{};
+  fill_common(p, s, lay, static_cast<uint8_t*>(workspace), T);
+  p.x = x;
+  p.codes = static_cast<const uint8_t*>(weights->packed);
+  p.scales = weights->block_scales;
+  p.tscale = weights->tensor_scales;
+  p.residual = residual;
+  p.out = out;
+  return run_mma_path(p, s, lay, static_cast<uint8_t*>(workspace), weights, nullptr, true,
+                      static_cast<cudaStream_t>(stream), topk_ids, topk_weights);
 }
 
 int flint_moe_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
