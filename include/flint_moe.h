@@ -384,7 +384,7 @@ int flint_ep_combine(const uint16_t* y, const int32_t* pair_pos, int32_t T, int3
  *   status   nullable device int32: a slot outside [0, n_slots) (that token's
  *            key and value are not written) or a position outside [0,
  *            max_pos) (its rotation is skipped) sets FLINT_DEVCHECK_INDEX.
- * head_dim must be 128. The caller owns all buffers; 8-byte aligned pointers.
+ * head_dim must be 128. The caller owns all buffers; 16-byte aligned pointers.
  * One kernel, asynchronous on `stream`; T = 0 launches nothing. The pages
  * give no norm type or rotary layout: RMS normalisation with a learned weight
  * and the rotate-half pairing are the readings taken. */

@@ -5,13 +5,13 @@
 // 32 query and 4 key/value heads of dimension 128; rotary positions on the
 // sliding-window layers, none on the full-attention layers (rope = 0).
 //
-// One warp per (token, head) of the fused projection qkv [T][Hq + 2*Hkv][128]
-// bf16: lane l holds elements 4l..4l+3 (one 8-byte load; a warp reads a head's
-// 256 contiguous bytes). Query/key heads: sum of squares by a warp reduction,
-// y = x / sqrt(mean + eps) * w in fp32; rotation partner of element i is
-// i +- 64, held by lane l ^ 16 in the same register, so one shuffle per
-// element; the cos/sin row of the token's position is read as two 16-byte
-// loads per lane. Query heads go to q_out [T][Hq][128]; key heads to
+// One half-warp per (token, head) of the fused projection qkv
+// [T][Hq + 2*Hkv][128] bf16: lane l of the half holds elements 8l..8l+7 (one
+// 16-byte load; a half-warp reads a head's 256 contiguous bytes). Query/key
+// heads: sum of squares by a 16-lane reduction, y = x / sqrt(mean + eps) * w
+// in fp32; rotation partner of element i is i +- 64, held by lane l ^ 8 in
+// the same register, so one shuffle per element; the cos/sin row of the
+// token's position is read as four 16-byte loads per lane. Query heads go to q_out [T][Hq][128]; key heads to
 // k_cache[slot][Hkv][128]; value heads are copied to v_cache[slot][Hkv][128].
 // HBM-bound: 21,000 bytes per token at Hq = 32, Hkv = 4 (read qkv 10,240, the
 // cos/sin row 512, position and slot 8; write q 8,192, k and v 1,024 each).
@@ -51,13 +51,13 @@ struct AttnPrologueParams {
 };
 
 __global__ void __launch_bounds__(256) k_qk_norm_rope_kv(AttnPrologueParams p) {
-  const int lane = threadIdx.x & 31;
+  // half-warp per (token, head): lane l of the half holds elements 8l .. 8l+7
+  const int lane = threadIdx.x & 15;
   const int H = p.Hq + 2 * p.Hkv;
-  const long long task = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (task >= static_cast<long long>(p.T) * H) return;
-  const int t = static_cast<int>(task / H), h = static_cast<int>(task % H);
-  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(p.qkv + task * kHeadDim) + lane);
-  float x[4] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y)};
+  const int task = blockIdx.x * 16 + (threadIdx.x >> 4);
+  if (task >= p.T * H) return;
+  const int t = task / H, h = task - t * H;
+  const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.qkv + static_cast<size_t>(task) * kHeadDim) + lane);
   long long slot = -1;
   if (h >= p.Hq) {
     slot = p.slots[t];
@@ -68,49 +68,73 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope_kv(AttnPrologueParams p) {
   }
   if (h >= p.Hq + p.Hkv) {  // value head: copied to its cache slot
     uint16_t* dst = p.v_cache + (slot * p.Hkv + (h - p.Hq - p.Hkv)) * kHeadDim;
-    reinterpret_cast<uint2*>(dst)[lane] = raw;
+    reinterpret_cast<uint4*>(dst)[lane] = raw;
     return;
   }
+  const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+  float x[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    x[2 * q] = bf16_lo(rw[q]);
+    x[2 * q + 1] = bf16_hi(rw[q]);
+  }
   const uint16_t* wv = h < p.Hq ? p.q_w : p.k_w;
-  const uint2 wr = __ldg(reinterpret_cast<const uint2*>(wv) + lane);
-  const float w[4] = {bf16_lo(wr.x), bf16_hi(wr.x), bf16_lo(wr.y), bf16_hi(wr.y)};
+  const uint4 wr = __ldg(reinterpret_cast<const uint4*>(wv) + lane);
+  const uint32_t ww[4] = {wr.x, wr.y, wr.z, wr.w};
   float ss = 0.f;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) ss = fmaf(x[j], x[j], ss);
-  ss = warp_sum(ss);
-  const float r = 1.f / sqrtf(ss / static_cast<float>(kHeadDim) + p.eps);
-  float y[4];
+  for (int j = 0; j < 8; ++j) ss = fmaf(x[j], x[j], ss);
+  // sum over the 16 lanes of this half-warp (xor offsets below 16 stay in it)
 #pragma unroll
-  for (int j = 0; j < 4; ++j) y[j] = x[j] * r * w[j];
+  for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float r = 1.f / sqrtf(ss / static_cast<float>(kHeadDim) + p.eps);
+  float y[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    y[2 * q] = x[2 * q] * r * bf16_lo(ww[q]);
+    y[2 * q + 1] = x[2 * q + 1] * r * bf16_hi(ww[q]);
+  }
   if (p.rope) {
     const int pos = p.positions[t];
     const bool bad = pos < 0 || pos >= p.max_pos;
     if (bad && lane == 0 && p.status != nullptr) atomicOr(p.status, FLINT_DEVCHECK_INDEX);
-    // pair index c = element mod 64: lanes 0..15 hold the first halves,
-    // lanes 16..31 the second halves of the same pairs
-    const int c = 4 * (lane & 15);
-    float4 cs = make_float4(1.f, 1.f, 1.f, 1.f), sn = make_float4(0.f, 0.f, 0.f, 0.f);
+    // pair index c = element mod 64: lanes 0..7 of a half hold the first
+    // halves, lanes 8..15 the second halves of the same pairs
+    const int c = 8 * (lane & 7);
+    float cc[8], sn[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      cc[j] = 1.f;
+      sn[j] = 0.f;
+    }
     if (!bad) {
       const float* row = p.cos_sin + static_cast<size_t>(pos) * kHeadDim;
-      cs = __ldg(reinterpret_cast<const float4*>(row + c));
-      sn = __ldg(reinterpret_cast<const float4*>(row + 64 + c));
+      const float4 c0 = __ldg(reinterpret_cast<const float4*>(row + c));
+      const float4 c1 = __ldg(reinterpret_cast<const float4*>(row + c + 4));
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(row + 64 + c));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(row + 64 + c + 4));
+      cc[0] = c0.x; cc[1] = c0.y; cc[2] = c0.z; cc[3] = c0.w;
+      cc[4] = c1.x; cc[5] = c1.y; cc[6] = c1.z; cc[7] = c1.w;
+      sn[0] = s0.x; sn[1] = s0.y; sn[2] = s0.z; sn[3] = s0.w;
+      sn[4] = s1.x; sn[5] = s1.y; sn[6] = s1.z; sn[7] = s1.w;
     }
-    const float cc[4] = {cs.x, cs.y, cs.z, cs.w}, ssn[4] = {sn.x, sn.y, sn.z, sn.w};
-    const bool first = lane < 16;
+    const bool first = lane < 8;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float partner = __shfl_xor_sync(0xffffffffu, y[j], 16);
+    for (int j = 0; j < 8; ++j) {
+      const float partner = __shfl_xor_sync(0xffffffffu, y[j], 8);
       // first half: y cos - partner sin; second half: y cos + partner sin
-      y[j] = first ? fmaf(y[j], cc[j], -partner * ssn[j]) : fmaf(y[j], cc[j], partner * ssn[j]);
+      y[j] = first ? fmaf(y[j], cc[j], -partner * sn[j]) : fmaf(y[j], cc[j], partner * sn[j]);
     }
   }
-  const uint2 o = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+  const uint4 o = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                             pack_bf16x2(y[6], y[7]));
   uint16_t* dst = h < p.Hq ? p.q_out + (static_cast<size_t>(t) * p.Hq + h) * kHeadDim
                            : p.k_cache + (slot * p.Hkv + (h - p.Hq)) * kHeadDim;
-  reinterpret_cast<uint2*>(dst)[lane] = o;
+  reinterpret_cast<uint4*>(dst)[lane] = o;
 }
 
-bool aligned8(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 7u) == 0; }
+bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
+
 
 }  // namespace
 }  // namespace flint
@@ -130,8 +154,8 @@ extern "C" int flint_qk_norm_rope_kv(const uint16_t* qkv, int32_t T, int32_t n_q
   if (!qkv || !q_norm_w || !k_norm_w || !slots || !q_out || !k_cache || !v_cache ||
       (rope && (!cos_sin || !positions || max_pos < 1)))
     return flint_fail_external(FLINT_ERR_INVALID_ARG, "flint_qk_norm_rope_kv: NULL pointer");
-  if (!aligned8(qkv) || !aligned8(q_norm_w) || !aligned8(k_norm_w) || !aligned8(q_out) || !aligned8(k_cache) ||
-      !aligned8(v_cache) || (rope && (reinterpret_cast<uintptr_t>(cos_sin) & 15u)))
+  if (!aligned16(qkv) || !aligned16(q_norm_w) || !aligned16(k_norm_w) || !aligned16(q_out) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || (rope && !aligned16(cos_sin)))
     return flint_fail_external(FLINT_ERR_MISALIGNED, "flint_qk_norm_rope_kv: misaligned pointer");
   AttnPrologueParams p{};
   p.qkv = qkv;
@@ -151,9 +175,9 @@ extern "C" int flint_qk_norm_rope_kv(const uint16_t* qkv, int32_t T, int32_t n_q
   p.rope = rope ? 1 : 0;
   p.n_slots = n_slots;
   p.eps = eps;
-  const long long warps = static_cast<long long>(T) * (n_q_heads + 2 * n_kv_heads);
-  const long long blocks = (warps + 7) / 8;
-  if (blocks > 0x7fffffffLL) return flint_fail_external(FLINT_ERR_UNSUPPORTED_SHAPE, "too many tokens");
+  const long long tasks = static_cast<long long>(T) * (n_q_heads + 2 * n_kv_heads);
+  if (tasks > 0x7fffffffLL) return flint_fail_external(FLINT_ERR_UNSUPPORTED_SHAPE, "too many tokens");
+  const long long blocks = (tasks + 15) / 16;
   k_qk_norm_rope_kv<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return flint_fail_external(FLINT_ERR_CUDA, cudaGetErrorString(e));
