@@ -543,6 +543,109 @@ def run_decode_attention(seed: int, calls: int = 40):
     return res
 
 
+def run_ep(seed: int, R: int = 8, T: int = 64, reps: int = 20):
+    """Expert-parallel layer step (config 1's layer, NVFP4, T tokens per rank),
+    R ranks emulated on one GPU: every rank's weights (E/R routed experts +
+    the shared one) resident, each phase run for every rank in turn, the
+    all-to-all replaced by copies between the ranks' buffers (not timed: on a
+    node it is NCCL over NVLink). Timed per rank and call with CUDA events:
+    route + dispatch, the routed expert call over the received rows, the
+    combine (each phase a CUDA graph of all ranks' calls). Reported beside
+    them: the bytes a rank sends and receives over NVLink per step and their
+    time at the measured 770 GB/s per direction."""
+    import torch
+    import nvfp4_weight_only_flint_b200 as fm
+    from nvfp4_weight_only_flint_b200 import ep
+    w = synth.CONFIGS["cfg1"]
+    shape = fm.Shape(w.d, w.inter, w.E, w.k, w.S, fm.FLINT_W_NVFP4)
+    pshape = ep.packing_shape(shape, R)
+    wr = _bits_to_cuda(synth.to_bf16_bits(synth.router_plain(seed, w.d, w.E, 0)))
+    full = synth.layer_weights_torch(seed, 0, w.E + w.S, w.d, w.inter, w.std, device="cuda")
+    pack_ws = torch.empty(fm.flint_moe_workspace_bytes(pshape, 1), dtype=torch.uint8, device="cuda")
+    fm.flint_moe_workspace_init(pack_ws)
+    layers, keep = [], []
+    for r in range(R):
+        wl = ep.slice_rank_weights(full, shape, r, R)
+        packed = torch.empty(fm.flint_packed_bytes(pshape), dtype=torch.uint8, device="cuda")
+        scales = torch.empty(fm.flint_block_scale_bytes(pshape), dtype=torch.uint8, device="cuda")
+        tsc = torch.empty((pshape.n_experts + pshape.n_shared) * 3, dtype=torch.float32, device="cuda")
+        fm.flint_pack_nvfp4(wl, 0, pshape, packed, scales, tsc, pack_ws)
+        keep.append((packed, scales, tsc))
+        layers.append(ep.ExpertParallelLayer(shape, r, R, fm.Weights(packed.data_ptr(), scales.data_ptr(),
+                                                                        tsc.data_ptr()), wr, max_tokens=T))
+        del wl
+    del full
+    torch.cuda.synchronize()
+    xs = [_bits_to_cuda(synth.x_bits(seed + 900 + r, T, w.d)) for r in range(R)]
+    outs = [torch.empty_like(x) for x in xs]
+    # one step with the loopback exchange, so every buffer holds real rows
+    sc = [l.send(x, T).cpu().tolist() for l, x in zip(layers, xs)]
+    n_recv = []
+    for dst in range(R):
+        n = 0
+        for src in range(R):
+            off, c = sum(sc[src][:dst]), sc[src][dst]
+            layers[dst].recv_x[n:n + c].copy_(layers[src].send_x[off:off + c])
+            layers[dst].recv_ids[n:n + c].copy_(layers[src].send_ids[off:off + c])
+            layers[dst].recv_gates[n:n + c].copy_(layers[src].send_gates[off:off + c])
+            n += c
+        n_recv.append(n)
+        layers[dst].experts(n)
+    for src in range(R):
+        n = 0
+        for dst in range(R):
+            c, at = sc[src][dst], sum(sc[s2][dst] for s2 in range(src))
+            layers[src].y_back[n:n + c].copy_(layers[dst].y[at:at + c])
+            n += c
+        layers[src].finish(T, outs[src])
+    torch.cuda.synchronize()
+    for l in layers:
+        if int(l.status.item()) != 0:
+            raise RuntimeError("expert-parallel step: device check flags")
+
+    st = torch.cuda.Stream()
+
+    def timed(fn):
+        """Device time per rank and call: a CUDA graph of reps x R calls."""
+        with torch.cuda.stream(st):
+            for _ in range(3):
+                for r in range(R):
+                    fn(r)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=st):
+            for _ in range(reps):
+                for r in range(R):
+                    fn(r)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(st):
+            graph.replay()
+            torch.cuda.synchronize()
+            e0.record()
+            graph.replay()
+            e1.record()
+        torch.cuda.synchronize()
+        del graph
+        return e0.elapsed_time(e1) / (reps * R) * 1e3
+    us_send = timed(lambda r: layers[r].send(xs[r], T))
+    us_exp = timed(lambda r: layers[r].experts(n_recv[r]))
+    us_fin = timed(lambda r: layers[r].finish(T, outs[r]))
+    row = w.d * 2
+    remote_out = [sum(c for dst, c in enumerate(sc[r]) if dst != r) for r in range(R)]
+    remote_in = [sum(sc[src][r] for src in range(R) if src != r) for r in range(R)]
+    # out: rows + ids + gates there, rows back; the larger direction sets the time
+    b_out = max(remote_out[r] * (row + 8) + remote_in[r] * row for r in range(R))
+    b_in = max(remote_in[r] * (row + 8) + remote_out[r] * row for r in range(R))
+    link = 770.0
+    return {"workload": f"cfg1 layer, NVFP4, {T} tokens per rank, {R} ranks emulated on one GPU "
+                        "(E/R = 32 routed + the shared expert per rank)",
+            "us_route_dispatch": us_send, "us_expert_call": us_exp, "us_combine": us_fin,
+            "rows_received_mean": float(np.mean(n_recv)), "rows_received_max": int(max(n_recv)),
+            "nvlink_bytes_per_rank_max": int(max(b_out, b_in)),
+            "us_exchange_at_770GBs": max(b_out, b_in) / (link * 1e3),
+            "note": "the all-to-all itself is not measured: one GPU per run"}
+
+
 def cpu_baseline(n_tokens: int = 3, seed: int = 0):
     """The fp64 oracle as it stands, on host cores: T=1 layer decodes of the
     default workload (quantisation of the needed experts is untimed set-up),
@@ -735,6 +838,7 @@ def main():
         extras["prefill"] = run_prefill(world, args.seed)
         extras["attn_prologue"] = run_attn_prologue(args.seed)
         extras["decode_attention"] = run_decode_attention(args.seed)
+        extras["ep_emulated"] = run_ep(args.seed)
         extras["stack47"] = {
             "workload": "cfg3: 47 resident layers (21.4 GB NVFP4), residual chain, no attention",
             "batch1_tokens_per_s": tok_s / N_LAYERS, "batch1_us_per_layer": ms_step * 1e3,

@@ -633,6 +633,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
   const int tiles = EPI == kEpiGateUp ? p.I / 64 : p.d / 128;
   const int n_sub = K / kMmaSliceK;
   const int KS = p.k + p.S;
+  // With two accumulators, issuer i takes the slices s = i (mod 2), all eight
+  // K steps of each: one commit per slice (a commit costs the issuing thread
+  // about as much as four MMAs). With a single slice both take alternate K
+  // steps of it.
+  const bool SLICE_SPLIT = NI == 2 && n_sub >= 2;
 
   if (tid == 0) {
     for (int i = 0; i < kMmaMaxStages; ++i) {
@@ -640,7 +645,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
       mbar_init(&raw_empty[i], 8);
       mbar_init(&a_full[i], fp4 ? 4 : 1);
       mbar_init(&b_full[i], 1);
-      mbar_init(&ab_empty[i], NI);
+      mbar_init(&ab_empty[i], SLICE_SPLIT ? 1 : NI);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], NI);
@@ -734,7 +739,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
   } else if (warp == 1 || (warp == 3 && NI == 2)) {
     // ------------------------------------------------ MMA issuers
     if (lane == 0) {
-      const int iss = warp == 1 ? 0 : 1;  // accumulator (K steps iss, iss + NI, ...)
+      const int iss = warp == 1 ? 0 : 1;  // accumulator (its slices, or alternate K steps of one)
       int sc = 0, icount = 0;
       bool ok = true;
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++icount) {
@@ -747,22 +752,32 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
         // the NI accumulators of an item are kMmaMaxTokens / NI columns apart;
         // independent accumulation chains, summed in the epilogue
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * kMmaMaxTokens + iss * (kMmaMaxTokens / NI));
+        const int k0 = SLICE_SPLIT ? 0 : iss, kstep = SLICE_SPLIT ? 1 : NI;
+        bool first = true;  // the accumulator's first MMA of the item overwrites it
         for (int s = 0; s < n_sub; ++s) {
           const int as = sc % NA;
+          if (SLICE_SPLIT && (s & 1) != iss) {  // the other issuer's slice
+            ++sc;
+            continue;
+          }
           if (!(ok = mma_wait(&a_full[as], (sc / NA) & 1, abort_flag, p.status))) break;
           if (!(ok = mma_wait(&b_full[as], (sc / NA) & 1, abort_flag, p.status))) break;
           tc_fence_after();
           const uint32_t baddr = smem_addr(bbuf + as * BB);
           if (fp4) {
             const uint32_t a_tmem = tmem + kAccCols + static_cast<uint32_t>(64 * as);
-            for (int kk = iss; kk < 8; kk += NI)
+            for (int kk = k0; kk < 8; kk += kstep) {
               mma_f16_ts(d_tmem, a_tmem + 8 * kk, sw128_desc(baddr + (kk >> 2) * (BB / 2) + 32 * (kk & 3)), idesc,
-                         (s > 0 || kk >= NI) ? 1u : 0u);
+                         first ? 0u : 1u);
+              first = false;
+            }
           } else {
             const uint32_t aaddr = smem_addr(abuf + as * kMmaABytes);
-            for (int kk = iss; kk < 8; kk += NI)
+            for (int kk = k0; kk < 8; kk += kstep) {
               mma_f16(d_tmem, sw128_desc(aaddr + (kk >> 2) * (kMmaABytes / 2) + 32 * (kk & 3)),
-                      sw128_desc(baddr + (kk >> 2) * (BB / 2) + 32 * (kk & 3)), idesc, (s > 0 || kk >= NI) ? 1u : 0u);
+                      sw128_desc(baddr + (kk >> 2) * (BB / 2) + 32 * (kk & 3)), idesc, first ? 0u : 1u);
+              first = false;
+            }
           }
           mma_commit(&ab_empty[as]);
           ++sc;
