@@ -149,5 +149,37 @@ def test_decode_attention_host_validation(L):
     assert call(ws=None) == -4
 
 
+def test_expert_parallel_host_validation(L):
+    a = 0x100000
+    # dispatch: sizes, rank counts, alignment; T = 0 still writes the counts (needs the pointer)
+    def disp(T=4, k=6, S=1, E=256, R=8, rank=0, d=2048, x=a, counts=a):
+        return L.flint_ep_dispatch(a, a, T, k, S, E, R, rank, x, d, a, a, a, a, counts, a, None, None)
+    assert disp(R=9) == -2            # more than 8 ranks
+    assert disp(E=250) == -2          # experts not a multiple of the ranks
+    assert disp(rank=8) == -1
+    assert disp(k=9) == -1
+    assert disp(S=2) == -1
+    assert disp(d=2044) == -1         # rows of whole 16-byte vectors
+    assert disp(counts=None) == -1
+    assert disp(x=a + 8) == -3
+    # combine
+    assert L.flint_ep_combine(a, a, 4, 10, 2048, None, a, None) == -1   # at most 9 slots
+    assert L.flint_ep_combine(a, a, 0, 7, 2048, None, a, None) == 0     # no-op
+    assert L.flint_ep_combine(a + 8, a, 4, 7, 2048, None, a, None) == -3
+    assert L.flint_ep_combine(None, a, 4, 7, 2048, None, a, None) == -1
+    # routed forward: the tensor-core path's limits
+    s = _shape()
+    w = _weights()
+    ws_need = fm.flint_moe_workspace_bytes(s, 4)
+    assert L.flint_moe_forward_routed(a, 4, None, a, ctypes.byref(w), ctypes.byref(s), None, a, a, ws_need,
+                                      None) == -1
+    assert L.flint_moe_forward_routed(a, 4, a + 2, a, ctypes.byref(w), ctypes.byref(s), None, a, a, ws_need,
+                                      None) == -3
+    assert L.flint_moe_forward_routed(a, 4, a, a, ctypes.byref(w), ctypes.byref(s), None, a, a, 64, None) == -4
+    assert L.flint_moe_forward_routed(a, 0, a, a, ctypes.byref(w), ctypes.byref(s), None, a, a, ws_need, None) == 0
+    assert L.flint_moe_forward_routed(a, 20000, a, a, ctypes.byref(w), ctypes.byref(s), None, a, a, ws_need,
+                                      None) == -2
+
+
 def test_version(L):
     assert "sm_100a" in fm.flint_version()
