@@ -51,8 +51,11 @@ struct AttnPrologueParams {
 };
 
 __global__ void __launch_bounds__(256) k_qk_norm_rope_kv(AttnPrologueParams p) {
-  // half-warp per (token, head): lane l of the half holds elements 8l .. 8l+7
+  // half-warp per (token, head): lane l of the half holds elements 8l .. 8l+7.
+  // The two halves of a warp may take different branches (a value head returns
+  // early beside a query or key head), so shuffles name only this half's lanes.
   const int lane = threadIdx.x & 15;
+  const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
   const int H = p.Hq + 2 * p.Hkv;
   const int task = blockIdx.x * 16 + (threadIdx.x >> 4);
   if (task >= p.T * H) return;
@@ -86,7 +89,7 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope_kv(AttnPrologueParams p) {
   for (int j = 0; j < 8; ++j) ss = fmaf(x[j], x[j], ss);
   // sum over the 16 lanes of this half-warp (xor offsets below 16 stay in it)
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(hmask, ss, o);
   const float r = 1.f / sqrtf(ss / static_cast<float>(kHeadDim) + p.eps);
   float y[8];
 #pragma unroll
@@ -121,7 +124,7 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope_kv(AttnPrologueParams p) {
     const bool first = lane < 8;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const float partner = __shfl_xor_sync(0xffffffffu, y[j], 8);
+      const float partner = __shfl_xor_sync(hmask, y[j], 8);
       // first half: y cos - partner sin; second half: y cos + partner sin
       y[j] = first ? fmaf(y[j], cc[j], -partner * sn[j]) : fmaf(y[j], cc[j], partner * sn[j]);
     }

@@ -24,9 +24,9 @@ def _table(max_pos, theta=10000.0):
     return np.concatenate([np.cos(ang), np.sin(ang)], axis=1).astype(np.float32)
 
 
-def _case(T, rope, seed, n_slots=1000, max_pos=4096, scale=1.0):
+def _case(T, rope, seed, n_slots=1000, max_pos=4096, scale=1.0, hq=HQ, hkv=HKV):
     rng = np.random.default_rng(seed)
-    qkv = synth.to_bf16_bits((rng.standard_normal((T, HQ + 2 * HKV, DH)) * scale).astype(np.float32))
+    qkv = synth.to_bf16_bits((rng.standard_normal((T, hq + 2 * hkv, DH)) * scale).astype(np.float32))
     qw = synth.to_bf16_bits((1.0 + 0.1 * rng.standard_normal(DH)).astype(np.float32))
     kw = synth.to_bf16_bits((1.0 + 0.1 * rng.standard_normal(DH)).astype(np.float32))
     cs = _table(max_pos)
@@ -35,14 +35,14 @@ def _case(T, rope, seed, n_slots=1000, max_pos=4096, scale=1.0):
     return qkv, qw, kw, cs, pos, slots
 
 
-def _run(qkv, qw, kw, cs, pos, slots, rope, n_slots=1000, eps=1e-6):
+def _run(qkv, qw, kw, cs, pos, slots, rope, n_slots=1000, eps=1e-6, hq=HQ, hkv=HKV):
     T = qkv.shape[0]
     d = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a).view(dt)).cuda()
-    q_out = torch.zeros((T, HQ, DH), dtype=torch.int16, device="cuda")
-    kc = torch.full((n_slots, HKV, DH), SENTINEL, dtype=torch.int16, device="cuda")
-    vc = torch.full((n_slots, HKV, DH), SENTINEL, dtype=torch.int16, device="cuda")
+    q_out = torch.zeros((T, hq, DH), dtype=torch.int16, device="cuda")
+    kc = torch.full((n_slots, hkv, DH), SENTINEL, dtype=torch.int16, device="cuda")
+    vc = torch.full((n_slots, hkv, DH), SENTINEL, dtype=torch.int16, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    fm.flint_qk_norm_rope_kv(d(qkv, np.int16), T, HQ, HKV, d(qw, np.int16), d(kw, np.int16), d(cs, np.float32),
+    fm.flint_qk_norm_rope_kv(d(qkv, np.int16), T, hq, hkv, d(qw, np.int16), d(kw, np.int16), d(cs, np.float32),
                              cs.shape[0], d(pos, np.int32), rope, eps, d(slots, np.int32), n_slots, q_out, kc, vc,
                              status)
     torch.cuda.synchronize()
@@ -72,6 +72,19 @@ def test_attn_prologue_matches_oracle(T, rope):
     assert np.array_equal(vc[slots], qkv[:, HQ + HKV:])
     untouched = np.setdiff1d(np.arange(kc.shape[0]), slots)
     assert (kc[untouched] == SENTINEL).all() and (vc[untouched] == SENTINEL).all()
+
+
+@pytest.mark.parametrize("hq,hkv,T", [(7, 3, 37), (5, 1, 3), (1, 2, 11)])
+def test_attn_prologue_odd_head_counts(hq, hkv, T):
+    # odd head counts put a value head and a query/key head in the two halves
+    # of one warp, and an odd task count leaves the last half-warp alone
+    qkv, qw, kw, cs, pos, slots = _case(T, True, seed=hq * 100 + hkv, hq=hq, hkv=hkv)
+    q_g, kc, vc, st = _run(qkv, qw, kw, cs, pos, slots, True, hq=hq, hkv=hkv)
+    assert st == 0
+    q_r, k_r, v_r = oracle.qk_norm_rope_kv(qkv, hq, hkv, qw, kw, cs, pos, rope=True)
+    _close(q_g, q_r, "q")
+    _close(kc[slots], k_r, "k cache rows")
+    assert np.array_equal(vc[slots], qkv[:, hq + hkv:])
 
 
 def test_attn_prologue_large_and_small_magnitudes():
