@@ -415,11 +415,9 @@ extern "C" int flint_decode_attention(const uint16_t* q, const uint16_t* k_cache
     p.po = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256(units * 2 * sizeof(float)));
   }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(k_attn_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return flint_fail_external(FLINT_ERR_CUDA, cudaGetErrorString(e));
-    attr_set = true;
+  {
+    const cudaError_t ea = flint_ensure_smem(reinterpret_cast<const void*>(k_attn_partial));
+    if (ea != cudaSuccess) return flint_fail_external(FLINT_ERR_CUDA, cudaGetErrorString(ea));
   }
   k_attn_partial<<<dim3(p.n_chunks, n_kv_heads, T), kWarps * 32, kSmemBytes, st>>>(p);
   cudaError_t e = cudaGetLastError();

@@ -16,6 +16,10 @@ namespace flint {
 // code; defined in flint_moe.cu.
 int flint_fail_external(int code, const char* msg);
 
+// Raises a kernel's dynamic shared-memory limit to the device's opt-in maximum,
+// once per (kernel, current device); defined in flint_moe.cu.
+cudaError_t flint_ensure_smem(const void* kern);
+
 // A bounded device wait gives up after this many SM clock cycles (about one
 // second at the B200's boost clock) and records FLINT_DEVCHECK_WAIT.
 constexpr long long kWaitCycles = 2000000000LL;

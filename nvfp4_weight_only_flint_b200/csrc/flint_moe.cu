@@ -1078,6 +1078,10 @@ int run_mma_path(LayerParams& p, const Dims& s, const WsLayout& w, uint8_t* ws, 
 }
 
 }  // namespace
+
+// Raises a kernel's dynamic shared-memory limit on the current device, once per
+// (kernel, device): for the kernels of the other translation units.
+cudaError_t flint_ensure_smem(const void* kern) { return ensure_smem(kern); }
 }  // namespace flint
 
 using namespace flint;
