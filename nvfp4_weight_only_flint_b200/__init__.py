@@ -23,6 +23,8 @@ __all__ = [
     "flint_moe_get_status", "flint_last_error", "flint_debug_noalloc_scratch",
     "flint_pack_nvfp4_dense", "flint_lm_head",
     "flint_debug_dequant", "flint_debug_decode", "flint_debug_group", "flint_debug_wait_timeout", "flint_version",
+    "flint_qk_norm_rope_kv", "flint_decode_attention", "flint_decode_attention_workspace_bytes",
+    "flint_moe_forward_routed", "flint_ep_dispatch", "flint_ep_combine",
 ]
 
 FLINT_W_NVFP4, FLINT_W_BF16 = 0, 1
@@ -30,6 +32,7 @@ FLINT_PATH_AUTO, FLINT_PATH_GEMV, FLINT_PATH_MMA = 0, 1, 2
 FLINT_LAYER_AUTO, FLINT_LAYER_FMA, FLINT_LAYER_MMA, FLINT_LAYER_CLUSTER = 0, 1, 2, 3
 FLINT_DEVCHECK_EXPERT_ID, FLINT_DEVCHECK_NONFINITE, FLINT_DEVCHECK_WAIT, FLINT_DEVCHECK_MMA = 1, 2, 4, 8
 FLINT_DEVCHECK_INDEX = 16
+FLINT_ERR_DEVICE_CHECK, FLINT_ERR_TIMEOUT = -6, -7
 STATUS_NAMES = {0: "FLINT_OK", -1: "FLINT_ERR_INVALID_ARG", -2: "FLINT_ERR_UNSUPPORTED_SHAPE",
                 -3: "FLINT_ERR_MISALIGNED", -4: "FLINT_ERR_WORKSPACE", -5: "FLINT_ERR_CUDA",
                 -6: "FLINT_ERR_DEVICE_CHECK", -7: "FLINT_ERR_TIMEOUT"}

@@ -26,8 +26,9 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import (Shape, Weights, flint_ep_combine, flint_ep_dispatch, flint_moe_forward_routed, flint_moe_route,
-               flint_moe_workspace_bytes, flint_moe_workspace_init)
+from . import (FLINT_ERR_DEVICE_CHECK, FlintError, Shape, Weights, flint_ep_combine, flint_ep_dispatch,
+               flint_moe_forward_routed, flint_moe_get_status, flint_moe_route, flint_moe_workspace_bytes,
+               flint_moe_workspace_init)
 
 
 class AllToAll:
@@ -126,6 +127,21 @@ class ExpertParallelLayer:
     def finish(self, T: int, out: torch.Tensor, residual=None) -> torch.Tensor:
         flint_ep_combine(self.y_back, self.pair_pos, T, self.slots, self.shape.d, residual, out)
         return out
+
+    def check(self) -> None:
+        """Synchronises and raises FlintError if a kernel of the last steps
+        recorded a failed check: an out-of-range id in the dispatch or the
+        router (FLINT_DEVCHECK_* bits of this rank's status words), or a
+        bounded wait that gave up in the expert call. Clears the flags."""
+        flags = int(self.status.item())
+        self.status.zero_()
+        rc_r, f_r = flint_moe_get_status(self.route_ws)
+        rc_e, f_e = flint_moe_get_status(self.expert_ws)
+        flags |= f_r | f_e
+        rc = rc_e or rc_r
+        if flags or rc:
+            raise FlintError(rc or FLINT_ERR_DEVICE_CHECK,
+                             f"expert-parallel step on rank {self.rank}: device check flags {flags:#x}")
 
     # --------------------------------------------------------------- one step
     def forward(self, x: torch.Tensor, T: int, out: torch.Tensor, residual=None, exchange: AllToAll | None = None):

@@ -179,7 +179,7 @@ def test_ep_layer_emulated_ranks(w, R, T):
     outs = _emulated_step(layers, [bits_to_cuda(b) for b in xbs], T,
                           [bits_to_cuda(b) if b is not None else None for b in resb])
     for r in range(R):
-        assert int(layers[r].status.item()) == 0
+        layers[r].check()  # raises on any device check flag of the step
         _check_ep(outs[r], layer, xbs[r], wrb, layers[r].ids[:T].cpu().numpy(), resb[r], f"rank {r} of {R}")
 
 
