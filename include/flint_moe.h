@@ -420,7 +420,7 @@ int flint_qk_norm_rope_kv(const uint16_t* qkv, int32_t T, int32_t n_q_heads, int
  *            a range outside [0, n_rows) or len < 0 (that token's output is
  *            zeros) sets FLINT_DEVCHECK_INDEX.
  * head_dim must be 128, n_q_heads a multiple of n_kv_heads with at most 8
- * query heads per kv head, T <= 65535, scale > 0 (1/sqrt(128) for the
+ * query heads per kv head, T <= 65535, max_len <= 2^30, scale > 0 (1/sqrt(128) for the
  * model). q, caches, out: 16-byte aligned. The caller owns all buffers. One or
  * two kernels, asynchronous on `stream`; T = 0 launches nothing. */
 size_t flint_decode_attention_workspace_bytes(int32_t T, int32_t n_kv_heads, int32_t max_len);

@@ -48,6 +48,7 @@ constexpr int kStageElems = 2 * kBlock * kRow;              // key rows, then va
 constexpr int kSmemBytes = kWarps * kStages * kStageElems * 2;  // 104,448
 constexpr int kChunkQuantum = kWarps * kBlock;              // 64 keys
 constexpr int kCtaSlots = 2 * 148;    // resident CTAs: 2 per SM on 148 SMs
+constexpr int kMaxLen = 1 << 30;      // context rows per token (chunk arithmetic stays in int)
 
 struct Params {
   const uint16_t* q;        // [T][Hq][128]
@@ -361,7 +362,7 @@ size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 using namespace flint;
 
 extern "C" size_t flint_decode_attention_workspace_bytes(int32_t T, int32_t n_kv_heads, int32_t max_len) {
-  if (T < 1 || n_kv_heads < 1 || max_len < 1) return 0;
+  if (T < 1 || n_kv_heads < 1 || max_len < 1 || max_len > kMaxLen) return 0;
   const int chunk = pick_chunk(T, n_kv_heads, max_len);
   const long long nch = (max_len + chunk - 1) / chunk;
   if (nch <= 1) return 0;
@@ -381,6 +382,7 @@ extern "C" int flint_decode_attention(const uint16_t* q, const uint16_t* k_cache
     return flint_fail_external(FLINT_ERR_UNSUPPORTED_SHAPE, "n_q_heads / n_kv_heads must be an integer <= 8");
   if (T > 65535 || n_kv_heads > 65535)
     return flint_fail_external(FLINT_ERR_UNSUPPORTED_SHAPE, "at most 65535 tokens and kv heads");
+  if (max_len > kMaxLen) return flint_fail_external(FLINT_ERR_UNSUPPORTED_SHAPE, "max_len above 2^30 rows");
   if (T == 0) return FLINT_OK;
   if (!q || !out || !start || !len || (n_rows > 0 && (!k_cache || !v_cache)))
     return flint_fail_external(FLINT_ERR_INVALID_ARG, "flint_decode_attention: NULL pointer");

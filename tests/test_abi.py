@@ -147,6 +147,8 @@ def test_decode_attention_host_validation(L):
     assert call(q=a + 8) == -3
     assert call(ws_bytes=need - 16) == -4
     assert call(ws=None) == -4
+    assert call(max_len=(1 << 30) + 1) == -2
+    assert fm.flint_decode_attention_workspace_bytes(1, 4, (1 << 30) + 1) == 0
 
 
 def test_expert_parallel_host_validation(L):
